@@ -1,0 +1,154 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+Every mutant replaces one oracle function with a subtly wrong variant (a dropped
+term, a wrong sign, a wrong index or orientation); the named pin tests must then
+fail.  This shows the pins constrain the oracle rather than restate it.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import kva_ref as R
+from tests import test_oracle_pins as P
+
+
+def _rope_wrong_sign(x, positions, rope_dims, theta):
+    return R_orig["rope_apply"](x, -np.asarray(positions), rope_dims, theta)
+
+
+def _rope_interleaved(x, positions, rope_dims, theta):
+    # rotates adjacent pairs (2i, 2i+1) instead of the half split
+    x = np.array(x, dtype=np.float64, copy=True)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * R.rope_inv_freq(rope_dims, theta)[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    xi, xj = x[:, :, 0:rope_dims:2].copy(), x[:, :, 1:rope_dims:2].copy()
+    x[:, :, 0:rope_dims:2] = xi * c - xj * s
+    x[:, :, 1:rope_dims:2] = xj * c + xi * s
+    return x
+
+
+def _inv_freq_wrong_theta(rope_dims, theta):
+    return R_orig["rope_inv_freq"](rope_dims, 1.0e6)
+
+
+def _conv_flipped(X, tail, w):
+    return R_orig["causal_conv_silu"](X, tail, w[:, ::-1])
+
+
+def _scan_decay_outside(S0, k, v, g, beta):
+    # decay also applied to the write term: e^g (S(I - b k k^T) + b v k^T)
+    S = np.array(S0, dtype=np.float64, copy=True)
+    grp = S.shape[0] // k.shape[1]
+    kmap = np.arange(S.shape[0]) // grp
+    for t in range(k.shape[0]):
+        kt = k[t, kmap]
+        Sk = np.einsum("hij,hj->hi", S, kt)
+        bt = beta[t][:, None, None]
+        S = np.exp(g[t])[:, None, None] * (S - bt * Sk[:, :, None] * kt[:, None, :]
+                                           + bt * v[t][:, :, None] * kt[:, None, :])
+    return S
+
+
+def _scan_gqa_modulo(S0, k, v, g, beta):
+    # v head h reads k head h % n_k instead of h // (n_v / n_k)
+    n_v, n_k = S0.shape[0], k.shape[1]
+    perm = np.arange(n_v) % n_k
+    kk = k[:, perm]                                   # expand to one k per v head
+    return R_orig["delta_scan_sequential"](S0, kk, v, g, beta)
+
+
+def _scan_variant_no_beta(S0, k, v, g, beta):
+    S = np.array(S0, dtype=np.float64, copy=True)
+    grp = S.shape[0] // k.shape[1]
+    kmap = np.arange(S.shape[0]) // grp
+    for t in range(k.shape[0]):
+        kt = k[t, kmap]
+        Sk = np.einsum("hij,hj->hi", S, kt)
+        bt = beta[t][:, None, None]
+        S = np.exp(g[t])[:, None, None] * (S - Sk[:, :, None] * kt[:, None, :]) \
+            + bt * v[t][:, :, None] * kt[:, None, :]
+    return S
+
+
+def _attn_no_scale(Q, K, V, window):
+    return R_orig["block_causal_attention"](Q * math.sqrt(Q.shape[-1]), K, V, window)
+
+
+def _attn_mask_off_by_one(Q, K, V, window):
+    T = Q.shape[0]
+    S = np.einsum("thd,shd->hts", Q, K) / math.sqrt(Q.shape[-1])
+    i, j = np.arange(T)[:, None], np.arange(T)[None, :]
+    m = (j < i) | (i == 0) & (j == 0)
+    S = np.where(m[None], S, -np.inf)
+    S = S - S.max(-1, keepdims=True)
+    Pm = np.exp(S)
+    Pm /= Pm.sum(-1, keepdims=True)
+    return np.einsum("hts,shd->thd", Pm, V)
+
+
+def _rms_eps_outside(x, g, eps=R.EPS):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps) * g
+
+
+def _gates_exp_not_softplus(a, b, A_log, dt_bias):
+    return -np.exp(A_log)[None, :] * np.exp(a + dt_bias[None, :]), R.sigmoid(b)
+
+
+def _chunked_no_decay_mask(S0, k, v, g, beta, chunk=64):
+    # forgets the per-pair decay inside the chunk (uses e^gam_t only)
+    S = np.array(S0, dtype=np.float64, copy=True)
+    grp = S.shape[0] // k.shape[1]
+    kmap = np.arange(S.shape[0]) // grp
+    T = k.shape[0]
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        C = c1 - c0
+        for h in range(S.shape[0]):
+            K, V = k[c0:c1, kmap[h]], v[c0:c1, h]
+            gam, bt = np.cumsum(g[c0:c1, h]), beta[c0:c1, h]
+            L = np.tril(bt[:, None] * (K @ K.T), -1)
+            rhs = bt[:, None] * V - (bt * np.exp(gam))[:, None] * (K @ S[h].T)
+            U = np.linalg.solve(np.eye(C) + L, rhs)
+            S[h] = np.exp(gam[-1]) * S[h] + (U * np.exp(gam[-1] - gam)[:, None]).T @ K
+    return S
+
+
+R_orig = {name: getattr(R, name) for name in (
+    "rope_apply", "rope_inv_freq", "causal_conv_silu", "delta_scan_sequential",
+    "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked")}
+
+MUTANTS = [
+    ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
+    ("rope_apply", _rope_interleaved, [P.test_rope_equals_complex_rotation]),
+    ("rope_inv_freq", _inv_freq_wrong_theta, [P.test_rope_low_frequency_angles_match_mla_card]),
+    ("causal_conv_silu", _conv_flipped, [P.test_conv_matches_numpy_convolve_per_channel]),
+    ("delta_scan_sequential", _scan_decay_outside, [P.test_scan_matches_dense_matrix_brute_force]),
+    ("delta_scan_sequential", _scan_gqa_modulo, [P.test_scan_matches_dense_matrix_brute_force]),
+    ("delta_scan_sequential", _scan_variant_no_beta, [P.test_scan_matches_dense_matrix_brute_force]),
+    ("block_causal_attention", _attn_no_scale, [P.test_attention_brute_force_loops]),
+    ("block_causal_attention", _attn_mask_off_by_one, [P.test_attention_equal_keys_gives_prefix_mean]),
+    ("rmsnorm", _rms_eps_outside, [P.test_rmsnorm_closed_forms]),
+    ("gdn_gates", _gates_exp_not_softplus, [P.test_gates_special_values]),
+    ("delta_scan_chunked", _chunked_no_decay_mask, [lambda: P.test_scan_chunked_equals_sequential(150, 64)]),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(MUTANTS)))
+def test_planted_mistake_is_caught(idx, monkeypatch):
+    name, bad, pins = MUTANTS[idx]
+    monkeypatch.setattr(R, name, bad)
+    caught = False
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            caught = True
+    assert caught, f"no pin caught the mutant of {name} ({bad.__name__})"
+
+
+def test_unmutated_oracle_passes_the_same_pins():
+    for _, _, pins in MUTANTS:
+        for pin in pins:
+            pin()

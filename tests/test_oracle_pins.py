@@ -1,0 +1,374 @@
+"""Pins of the float64 oracle against facts fixed by the pages and by mathematics.
+
+None of these re-type the oracle's own formula: each compares it with a value the
+pages print, a closed form, a different formulation (dense matrices, complex
+numbers, numpy.convolve, brute-force loops), or an invariant.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kva_inputs as KI
+from oracle import kva_ref as R
+from tests.conftest import read_golden
+
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------- geometry
+def test_param_counts_match_model_card():
+    """Printed millions = bias-free linear counts rounded up to 1M (all six)."""
+    for variant, part, printed in read_golden("param_counts.txt"):
+        geom = KI.GEOMETRIES[variant]
+        pc = geom.param_counts()
+        if part == "total":
+            # the printed r3 total counts the drafter heads, r2 has none
+            n = pc["total"]
+        else:
+            n = pc[part]
+        assert math.ceil(n / 1e6) == int(printed), (variant, part, n)
+    # the opening paragraph's '1.24B' for r3
+    assert round(KI.R3.param_counts()["total"] / 1e9, 2) == 1.24
+
+
+def test_param_counts_reject_other_shapes():
+    """The pin discriminates: extra matrices or another FFN width break it."""
+    g = KI.R3
+    bad = KI.with_changes(g, ffn=g.ffn + 256)
+    assert math.ceil(bad.param_counts()["trunk"] / 1e6) != 363
+    # an attention block with separate q/k/v of width 2d (not d) breaks it too
+    d, H, F = g.d_model, g.hidden, g.ffn
+    wrong = H * d + 3 * (6 * d * d + 3 * d * F)
+    assert math.ceil(wrong / 1e6) != 363
+
+
+def test_mixer_widths_match_model_card():
+    gw = dict((k, int(v)) for k, v in read_golden("mixer_widths.txt"))
+    for geom in (KI.R2, KI.R3):
+        assert 2 * geom.gdn_n_k * geom.gdn_d_k + geom.gdn_n_v * geom.gdn_d_v == gw["gdn_qkv"]
+        assert geom.gdn_n_v == gw["gdn_a"] == gw["gdn_b"]
+        assert geom.attn_n_kv * geom.attn_d_h == gw["attn_k"] == gw["attn_v"]
+        assert geom.n_gdn == gw["late_gdn_layers"]
+        assert geom.n_attn == gw["late_attn_layers"]
+        assert geom.n_mix == 24 * (10240 + 96) + 8 * 2048
+
+
+# ---------------------------------------------------------------- RoPE
+def test_rope_low_frequency_angles_match_mla_card():
+    """theta = 1e7 and omega_i = theta^(-2i/64) reproduce 3.4 / 2.1 / 1.2 degrees."""
+    inv = R.rope_inv_freq(64, 1.0e7)
+    for pair, deg in read_golden("rope_low_freq_angles.txt"):
+        got = math.degrees(inv[int(pair)] * 131072)
+        assert abs(got - float(deg)) < 0.05, (pair, got, deg)
+        got2 = math.degrees(inv[int(pair)] * 131000)
+        assert abs(got2 - float(deg)) < 0.05
+    # other common bases do not fit the printed values
+    for theta in (1.0e6, 5.0e6, 1.0e4):
+        inv = R.rope_inv_freq(64, theta)
+        assert abs(math.degrees(inv[31] * 131072) - 1.2) > 0.1
+
+
+def test_rope_equals_complex_rotation():
+    """Each pair (i, i+r/2) as a complex number is multiplied by e^{i p w_i}."""
+    T, n, d, r, theta = 7, 3, 256, 64, 1.0e7
+    x = RNG.standard_normal((T, n, d))
+    pos = np.array([0, 1, 5, 1023, 4096, 32767, 131071])
+    y = R.rope_apply(x, pos, r, theta)
+    w = theta ** (-np.arange(r // 2) * 2.0 / r)
+    z = x[:, :, : r // 2] + 1j * x[:, :, r // 2 : r]
+    zr = z * np.exp(1j * pos[:, None, None] * w[None, None, :])
+    np.testing.assert_allclose(y[:, :, : r // 2], zr.real, atol=1e-12)
+    np.testing.assert_allclose(y[:, :, r // 2 : r], zr.imag, atol=1e-12)
+    np.testing.assert_array_equal(y[:, :, r:], x[:, :, r:])
+
+
+def test_rope_dot_product_depends_on_relative_position_only():
+    d, r, theta = 256, 64, 1.0e7
+    q = RNG.standard_normal((1, 1, d))
+    k = RNG.standard_normal((1, 1, d))
+    vals = []
+    for m, nn in [(10, 3), (1010, 1003), (32767, 32760)]:
+        qm = R.rope_apply(q, np.array([m]), r, theta)
+        kn = R.rope_apply(k, np.array([nn]), r, theta)
+        vals.append(float(np.sum(qm * kn)))
+    np.testing.assert_allclose(vals, vals[0], rtol=1e-10)
+    # and it does depend on the offset
+    qm = R.rope_apply(q, np.array([10]), r, theta)
+    kn = R.rope_apply(k, np.array([9]), r, theta)
+    assert abs(float(np.sum(qm * kn)) - vals[0]) > 1e-6
+
+
+# ---------------------------------------------------------------- norms, gates
+def test_rmsnorm_closed_forms():
+    x = RNG.standard_normal((5, 512)) * 30
+    y = R.rmsnorm(x, np.ones(512))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), math.sqrt(512), rtol=1e-8)
+    np.testing.assert_allclose(R.rmsnorm(3.5 * x, np.ones(512)), y, rtol=1e-8)
+    g = RNG.uniform(0.5, 1.5, 512)
+    np.testing.assert_allclose(R.rmsnorm(x, g), y * g, rtol=1e-12)
+    # eps sits inside the root: a zero row stays zero, a tiny row is damped
+    assert np.all(R.rmsnorm(np.zeros((1, 8)), np.ones(8)) == 0)
+    small = np.full((1, 4), 1e-3)
+    np.testing.assert_allclose(R.rmsnorm(small, np.ones(4)), 1e-3 / math.sqrt(1e-6 + 1e-6))
+
+
+def test_l2norm_unit_rows():
+    x = RNG.standard_normal((9, 4 * 64)) * 7
+    y = R.l2norm_heads(x, 4, 64)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), 1.0, rtol=1e-9)
+    xs = x.reshape(9, 4, 64)
+    np.testing.assert_allclose(y * np.linalg.norm(xs, axis=-1, keepdims=True), xs, rtol=1e-8)
+
+
+def test_gates_special_values():
+    A_log = np.array([0.0, 1.0, 2.7])
+    dt = np.array([0.3, -0.2, 0.0])
+    a = -dt[None, :]                          # a + dt_bias = 0 -> softplus = ln 2
+    b = np.zeros((1, 3))
+    g, beta = R.gdn_gates(a, b, A_log, dt)
+    np.testing.assert_allclose(g[0], -np.exp(A_log) * math.log(2.0), rtol=1e-14)
+    np.testing.assert_allclose(beta[0], 0.5)
+    big = np.array([[50.0, -50.0, 700.0]])
+    g2, beta2 = R.gdn_gates(big, big, A_log, np.zeros(3))
+    np.testing.assert_allclose(g2[0, 0], -50.0, rtol=1e-14)          # softplus(x) -> x
+    np.testing.assert_allclose(g2[0, 1], -math.exp(1.0) * math.exp(-50.0), rtol=1e-10)
+    assert np.all(np.isfinite(g2)) and np.all(g2 <= 0)
+    np.testing.assert_allclose(beta2[0], [1.0, math.exp(-50.0), 1.0], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- conv
+def test_conv_matches_numpy_convolve_per_channel():
+    T, C, K = 37, 6, 4
+    X = RNG.standard_normal((T, C))
+    tail = RNG.standard_normal((K - 1, C))
+    w = RNG.standard_normal((C, K))
+    Z, new_tail = R.causal_conv_silu(X, tail, w)
+    for c in range(C):
+        ext = np.concatenate([tail[:, c], X[:, c]])
+        # np.convolve flips its kernel: tap K-1 must meet the current token
+        full = np.convolve(ext, w[c, ::-1], mode="valid")
+        np.testing.assert_allclose(Z[:, c], full / (1 + np.exp(-full)), rtol=1e-12)
+    np.testing.assert_array_equal(new_tail, X[-(K - 1):])
+
+
+def test_conv_delta_weights_are_shifts():
+    T, C, K = 10, 3, 4
+    X = RNG.standard_normal((T, C))
+    tail = RNG.standard_normal((K - 1, C))
+    ext = np.concatenate([tail, X])
+    for lag in range(K):
+        w = np.zeros((C, K))
+        w[:, K - 1 - lag] = 1.0                         # picks the token `lag` steps back
+        Z, _ = R.causal_conv_silu(X, tail, w)
+        pre = ext[K - 1 - lag:K - 1 - lag + T]
+        np.testing.assert_allclose(Z, pre / (1 + np.exp(-pre)), rtol=1e-12)
+
+
+def test_conv_tail_carry_equals_one_long_sequence():
+    T1, T2, C, K = 2, 9, 5, 4                          # T1 < K-1: tail mixes old and new
+    X = RNG.standard_normal((T1 + T2, C))
+    tail = RNG.standard_normal((K - 1, C))
+    w = RNG.standard_normal((C, K))
+    Z, t_end = R.causal_conv_silu(X, tail, w)
+    Za, ta = R.causal_conv_silu(X[:T1], tail, w)
+    Zb, tb = R.causal_conv_silu(X[T1:], ta, w)
+    np.testing.assert_allclose(np.concatenate([Za, Zb]), Z, rtol=1e-13)
+    np.testing.assert_array_equal(tb, t_end)
+    np.testing.assert_array_equal(ta, np.concatenate([tail[T1:], X[:T1]]))
+
+
+# ---------------------------------------------------------------- scan
+def _rand_scan(T, n_k, n_v, d_k, d_v, seed=0, beta_lo=0.0):
+    r = np.random.default_rng(seed)
+    k = r.standard_normal((T, n_k, d_k))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = r.standard_normal((T, n_v, d_v))
+    g = -r.uniform(0.0, 2.0, (T, n_v))
+    beta = r.uniform(beta_lo, 1.0, (T, n_v))
+    S0 = r.standard_normal((n_v, d_v, d_k)) * 0.3
+    return S0, k, v, g, beta
+
+
+def test_scan_matches_dense_matrix_brute_force():
+    """The stated recurrence with explicit d_k x d_k matrices, GQA map h // 2."""
+    S0, k, v, g, beta = _rand_scan(11, 2, 4, 5, 3, seed=1)
+    got = R.delta_scan_sequential(S0, k, v, g, beta)
+    for h in range(4):
+        S = S0[h].copy()
+        kh = h // 2
+        for t in range(11):
+            kt = k[t, kh][:, None]
+            A = math.exp(g[t, h]) * (np.eye(5) - beta[t, h] * (kt @ kt.T))
+            S = S @ A + beta[t, h] * (v[t, h][:, None] @ kt.T)
+        np.testing.assert_allclose(got[h], S, rtol=1e-12, atol=1e-12)
+
+
+def test_scan_beta_zero_is_pure_decay_and_identity():
+    S0, k, v, g, beta = _rand_scan(13, 2, 4, 6, 6, seed=2)
+    z = np.zeros_like(beta)
+    got = R.delta_scan_sequential(S0, k, v, g, z)
+    np.testing.assert_allclose(got, np.exp(g.sum(0))[:, None, None] * S0, rtol=1e-12)
+    got0 = R.delta_scan_sequential(S0, k, v, np.zeros_like(g), z)
+    np.testing.assert_array_equal(got0, S0)
+    for fn in (R.delta_scan_chunked,):
+        np.testing.assert_allclose(fn(S0, k, v, g, z, chunk=4),
+                                   np.exp(g.sum(0))[:, None, None] * S0, rtol=1e-12)
+        np.testing.assert_allclose(fn(S0, k, v, np.zeros_like(g), z, chunk=4), S0,
+                                   rtol=1e-13, atol=1e-15)
+
+
+def test_scan_delta_rule_write_property():
+    """beta = 1, unit k, no decay: the new state maps k_t exactly to v_t."""
+    S0, k, v, g, beta = _rand_scan(6, 1, 2, 8, 4, seed=3)
+    for t in range(1, 7):
+        S = R.delta_scan_sequential(S0, k[:t], v[:t], np.zeros((t, 2)), np.ones((t, 2)))
+        for h in range(2):
+            np.testing.assert_allclose(S[h] @ k[t - 1, 0], v[t - 1, h], atol=1e-12)
+
+
+def test_scan_orthonormal_keys_closed_form():
+    """Orthonormal keys, beta = 1, g = 0: S_T = S0 (I - sum k k^T) + sum v k^T."""
+    d = 8
+    Qm, _ = np.linalg.qr(RNG.standard_normal((d, d)))
+    T = 5
+    k = Qm[:, :T].T[:, None, :]                       # [T, 1, d]
+    v = RNG.standard_normal((T, 1, 3))
+    S0 = RNG.standard_normal((1, 3, d))
+    got = R.delta_scan_sequential(S0, k, v, np.zeros((T, 1)), np.ones((T, 1)))
+    P = sum(np.outer(k[t, 0], k[t, 0]) for t in range(T))
+    want = S0[0] @ (np.eye(d) - P) + sum(np.outer(v[t, 0], k[t, 0]) for t in range(T))
+    np.testing.assert_allclose(got[0], want, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,chunk", [(1, 64), (63, 64), (64, 64), (150, 64), (130, 16)])
+def test_scan_chunked_equals_sequential(T, chunk):
+    S0, k, v, g, beta = _rand_scan(T, 2, 6, 16, 8, seed=T)
+    g[: T // 3] *= 20.0                              # strong decay, e^(sum g) underflows
+    a = R.delta_scan_sequential(S0, k, v, g, beta)
+    b = R.delta_scan_chunked(S0, k, v, g, beta, chunk=chunk)
+    np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- attention
+def test_attention_equal_keys_gives_prefix_mean():
+    T, n, d = 12, 2, 16
+    Q = RNG.standard_normal((T, n, d))
+    K = np.broadcast_to(RNG.standard_normal((1, n, d)), (T, n, d)).copy()
+    V = RNG.standard_normal((T, n, d))
+    O = R.block_causal_attention(Q, K, V, 0)
+    want = np.cumsum(V, axis=0) / np.arange(1, T + 1)[:, None, None]
+    np.testing.assert_allclose(O, want, rtol=1e-12)
+    O4 = R.block_causal_attention(Q, K, V, 4)        # blocks of 4: mean restarts
+    for t in range(T):
+        b0 = (t // 4) * 4
+        np.testing.assert_allclose(O4[t], V[b0:t + 1].mean(0), rtol=1e-12)
+
+
+def test_attention_brute_force_loops():
+    T, n, d = 9, 2, 8
+    Q, K, V = (RNG.standard_normal((T, n, d)) for _ in range(3))
+    O = R.block_causal_attention(Q, K, V, 4)
+    for h in range(n):
+        for i in range(T):
+            js = [j for j in range(T) if j <= i and j // 4 == i // 4]
+            s = [sum(Q[i, h, e] * K[j, h, e] for e in range(d)) / math.sqrt(d) for j in js]
+            m = max(s)
+            p = [math.exp(x - m) for x in s]
+            tot = sum(p)
+            o = [sum(p[a] * V[js[a], h, e] for a in range(len(js))) / tot for e in range(d)]
+            np.testing.assert_allclose(O[i, h], o, rtol=1e-10)
+
+
+def test_block_causal_equals_causal_within_window():
+    T, n, d = 40, 2, 8
+    Q, K, V = (RNG.standard_normal((T, n, d)) for _ in range(3))
+    np.testing.assert_allclose(R.block_causal_attention(Q, K, V, 64),
+                               R.block_causal_attention(Q, K, V, 0), rtol=1e-13)
+    np.testing.assert_allclose(R.block_causal_attention(Q, K, V, 40),
+                               R.block_causal_attention(Q, K, V, 0), rtol=1e-13)
+    # blocks do not see each other: block 2 alone gives the same rows
+    Ob = R.block_causal_attention(Q, K, V, 16)
+    np.testing.assert_allclose(Ob[16:32], R.block_causal_attention(Q[16:32], K[16:32], V[16:32], 0),
+                               rtol=1e-13)
+
+
+# ---------------------------------------------------------------- projector
+def _tiny_f64(seed=7, random_gains=True):
+    geom = KI.TINY
+    W = R.weights_to_f64(KI.make_projector_weights(geom, seed, random_gains=random_gains))
+    return geom, W
+
+
+def test_projector_with_zero_output_projections_is_linear_chain():
+    geom, W = _tiny_f64()
+    for b in W["blocks"]:
+        b["Wo"] = np.zeros_like(b["Wo"])
+        b["Wd"] = np.zeros_like(b["Wd"])
+    res = RNG.standard_normal((16, geom.hidden))
+    Y = R.projector(res, W, geom)
+    h = R.rmsnorm(res, W["g_in"]) @ W["W_in"].T
+    np.testing.assert_allclose(Y, R.rmsnorm(h, W["g_out"]) @ W["W_heads"].T, rtol=1e-10)
+
+
+def test_projector_is_causal_and_position_free():
+    geom, W = _tiny_f64()
+    res = RNG.standard_normal((20, geom.hidden))
+    Y = R.projector(res, W, geom)
+    res2 = res.copy()
+    res2[12:] = RNG.standard_normal((8, geom.hidden))
+    Y2 = R.projector(res2, W, geom)
+    np.testing.assert_allclose(Y2[:12], Y[:12], rtol=1e-12)
+    assert np.abs(Y2[12:] - Y[12:]).max() > 1e-3
+    # ubatch-local: the first k tokens alone give the same rows
+    np.testing.assert_allclose(R.projector(res[:7], W, geom), Y[:7], rtol=1e-12)
+
+
+def test_concatenated_heads_equal_per_layer_heads():
+    geom, W = _tiny_f64()
+    z = RNG.standard_normal((5, geom.d_model))
+    Y = R.projector_heads(z, W["W_heads"])
+    for li, off in enumerate(geom.layer_offsets):
+        w = geom.layer_width(li)
+        Wl = W["W_heads"][off:off + w]
+        np.testing.assert_allclose(Y[:, off:off + w],
+                                   np.einsum("td,nd->tn", z, Wl), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- cache, carry
+def test_paged_slots_are_a_bijection_through_the_page_table():
+    pt = KI.make_page_table(1, 8, seed=3).numpy()[0]
+    s = R.kv_slots(0, 8 * 16, pt, 16)
+    assert sorted(s.tolist()) == list(range(8 * 16))
+    for p in (0, 15, 16, 100, 127):
+        assert s[p] == pt[p // 16] * 16 + p % 16
+
+
+def test_update_states_two_ubatches_equal_one():
+    geom = KI.TINY
+    P = {k: v.double().numpy() for k, v in KI.make_layer_params(geom, 5, random_k_gain=True).items()}
+    st = KI.make_states(geom, 1, 6, std=0.1)
+    S0 = st["state"][0].double().numpy()
+    tail0 = st["conv_tail"][0].double().numpy()
+    T = 50
+    Y = RNG.standard_normal((T, geom.n_mix))
+    mk = lambda: ([np.full((geom.attn_n_kv, 64, geom.attn_d_h), -7.0)],
+                  [np.full((geom.attn_n_kv, 64, geom.attn_d_h), -7.0)])
+    k1, v1 = mk()
+    S1, t1 = R.update_states(Y, geom, P, S0, tail0, k1, v1, 3)
+    k2, v2 = mk()
+    Sa, ta = R.update_states(Y[:2], geom, P, S0, tail0, k2, v2, 3)
+    Sb, tb = R.update_states(Y[2:], geom, P, Sa, ta, k2, v2, 5, scan="chunked")
+    np.testing.assert_allclose(Sb, S1, rtol=1e-10, atol=1e-12)
+    np.testing.assert_array_equal(tb, t1)
+    np.testing.assert_allclose(k2[0], k1[0], rtol=1e-12)
+    np.testing.assert_allclose(v2[0], v1[0], rtol=1e-12)
+    # rows outside 3..52 untouched
+    assert np.all(k1[0][:, :3] == -7.0) and np.all(k1[0][:, 53:] == -7.0)
+    # rotation keeps the k-norm of each head: |k| = sqrt(d) * gain-weighted rms
+    K = k1[0][:, 3:53].transpose(1, 0, 2)
+    Yk = Y[:, geom.layer_offsets[2]:geom.layer_offsets[2] + geom.attn_n_kv * geom.attn_d_h]
+    kn = R.rmsnorm(Yk.reshape(T, geom.attn_n_kv, geom.attn_d_h), P["k_norm_g"][0])
+    np.testing.assert_allclose(np.linalg.norm(K, axis=-1), np.linalg.norm(kn, axis=-1), rtol=1e-12)
+    np.testing.assert_array_equal(K[:, :, geom.rope_dims:], kn[:, :, geom.rope_dims:])
