@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the KVA prefill path on B200: tokens/s per 1024-token ubatch.
+
+One step = one kva_prefill_ubatch call over a 1024-token ubatch of the r3
+projector (d 3072, 24 heads block-causal within 1024, FFN 8448, 32 late-layer
+heads + 4 drafter heads) followed by every state update (24 gated-DeltaNet
+layers: conv, norms, gates, chunked scan; 8 attention layers: k norm, RoPE,
+KV-cache write).  The DeltaNet state, conv tail and KV caches carry from step to
+step; positions advance through a 32768-row cache (32 ubatches, then wrap).
+
+Inputs are synthetic and seeded (random bf16 weights of the r3 shapes, residual
+N(0,1) with 8 outlier channels x20), resident in HBM before timing.  The 2.48 GB
+of weights are larger than L2 and stream from HBM every step.
+
+Multi-GPU (torchrun): each rank runs its own independent sequence on its own GPU
+(weak scaling); the only collectives are the barrier and the max-over-ranks of
+the device time.  `--impl reference` times the float64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kva_inputs as KI  # noqa: E402
+
+T_UB = 1024
+CACHE_POS = 32768
+METRIC = "KVA prefill tokens/s on 1 B200 (1024-tok ubatch) and % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def geometry(name):
+    return KI.R3 if name == "r3" else KI.R2
+
+
+def algorithmic(geom, T=T_UB):
+    """FLOPs and HBM bytes the method must spend on one ubatch (see the accounting
+    in the design notes): every linear 2*params*T, causal attention over unmasked
+    pairs, the recurrence 4*d_k*d_v per token per v head; bytes = weights once,
+    residual in, state read+write, conv tail, KV rows written, drafter outputs."""
+    d, H, F = geom.d_model, geom.hidden, geom.ffn
+    lin = H * d + geom.n_blocks * (4 * d * d + 3 * d * F) + geom.n_total * d
+    W = geom.window if geom.window else T
+    pairs = sum(min(i % W, i) + 1 for i in range(T))
+    attn = geom.n_blocks * 4 * geom.head_dim * geom.n_heads * pairs
+    scan = geom.n_gdn * geom.gdn_n_v * T * 4 * geom.gdn_d_k * geom.gdn_d_v
+    flops = 2 * lin * T + attn + scan
+    state = geom.n_gdn * geom.gdn_n_v * geom.gdn_d_k * geom.gdn_d_v * 4
+    tail = geom.n_gdn * (geom.conv_k - 1) * geom.gdn_conv_ch * 2
+    kv = geom.n_attn * 2 * geom.attn_n_kv * geom.attn_d_h * T * 2
+    weights = lin * 2 + 4 * (H + d * (2 * geom.n_blocks + 1))
+    bytes_ = weights + T * H * 2 + 2 * state + 2 * tail + kv + T * geom.n_draft_cols * 2
+    return flops, bytes_
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def heads_traffic(geom_name):
+    """dram bytes per launch of the heads GEMM from the committed ncu summary, or None
+    when the summary is missing or the GEMM source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"gemm_heads_{geom_name}_T1024.md")
+    src = os.path.join(ROOT, "hybrid_deltanet_attention_kva_b200", "csrc", "kva_gemm.cu")
+    if not os.path.exists(path):
+        return None
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel source sha256[:16]") != h:
+        return None
+    try:
+        return float(vals["traffic bytes per launch (full size)"])
+    except (KeyError, ValueError):
+        return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        uuid = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        sel = uuid if uuid else str(device_index)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import hybrid_deltanet_attention_kva_b200 as K
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    geom = geometry(args.workload)
+    seed = 1003 if args.workload == "r3" else 1002
+    W = KI.make_projector_weights(geom, seed, device="cuda")
+    P = KI.make_layer_params(geom, seed + 1, device="cuda")
+    st = KI.make_states(geom, 1, seed + 2, device="cuda")
+    n_pool = 4
+    res = [KI.make_residual(geom, T_UB, seed + 100 + rank * n_pool + i, device="cuda")
+           for i in range(n_pool)]
+    kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h, dtype=torch.bfloat16, device=dev)
+          for _ in range(geom.n_attn)]
+    vc = [torch.zeros_like(k) for k in kc]
+    kv = K.KvCache(kc, vc, max_pos=CACHE_POS)
+    Wt = K.Weights(proj=W, layer=P)
+    S = st["state"][0]
+    tail = st["conv_tail"][0]
+    draft = (torch.empty(T_UB, geom.n_draft_cols, dtype=torch.bfloat16, device=dev)
+             if geom.n_draft else None)
+    h = K.kva_init(K.make_dims(geom, T_UB, 1))
+    stream = torch.cuda.current_stream()
+    n_ub = CACHE_POS // T_UB
+
+    def step(i, resid=None):
+        K.kva_prefill_ubatch(h, res[i % n_pool] if resid is None else resid, Wt, S, tail, kv,
+                             (i % n_ub) * T_UB, draft_out=draft, stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert K.kva_get_device_status(h) == 0, "device status set during warm-up"
+    K.kva_profile_enable(h, args.steps * 40 + 64)
+
+    # ---------------- timed region (device time, max over ranks)
+    clocks = Clocks(local_rank)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    prof = K.kva_profile_read(h)
+    status = K.kva_get_device_status(h)
+    K.kva_profile_enable(h, 0)
+
+    # ---------------- end to end: host residual in (pinned), drafter row out
+    e2e = None
+    if not args.no_e2e:
+        host_res = [r.cpu().pin_memory() for r in res]
+        dres = torch.empty_like(res[0])
+        out_host = torch.empty(geom.n_draft_cols if geom.n_draft else geom.d_model,
+                               dtype=torch.bfloat16).pin_memory()
+        steps_e2e = max(3, min(args.steps, 200))
+        for i in range(3):
+            dres.copy_(host_res[i % n_pool], non_blocking=True)
+            step(i, dres)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(steps_e2e):
+            dres.copy_(host_res[i % n_pool], non_blocking=True)
+            step(i, dres)
+            src = draft[-1] if draft is not None else None
+            if src is not None:
+                out_host.copy_(src, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(f0.elapsed_time(f1))
+        e2e = {"value": world * steps_e2e * T_UB / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": res[0].numel() * 2,
+               "d2h_bytes_per_step": out_host.numel() * 2 if draft is not None else 0,
+               "steps": steps_e2e,
+               "what": "kva_prefill_ubatch through the binding; residual copied from pinned host "
+                       "memory each step, last token's drafter outputs copied back"}
+    K.kva_free(h)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    flops, bytes_ = algorithmic(geom)
+    peaks, src = load_peaks()
+    ms_step = ms / args.steps
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    gh = prof["gemm_heads"]
+    heads_flops = 2.0 * T_UB * geom.n_total * geom.d_model
+    heads_ms = gh["ms"] / max(gh["timed"], 1)
+    achieved = heads_flops / (heads_ms / 1e3) / 1e12
+    peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    launches = int(sum(v["launches"] for v in prof.values()))
+    line = {
+        "metric": METRIC,
+        "value": world * args.steps * T_UB / (ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random bf16 weights of the projector shapes, N(0,1) residual "
+                "with 8 outlier channels x20)",
+        "config": {
+            "workload": f"{geom.name} projector + state updates, 1024-token ubatch, state / conv "
+                        f"tail / KV cache carried, positions 0..{CACHE_POS - 1}",
+            "geometry": geom.name, "tokens_per_step": T_UB, "d_model": geom.d_model,
+            "heads": geom.n_heads, "ffn": geom.ffn, "late_layers": f"{geom.n_gdn} gdn + {geom.n_attn} attn",
+            "drafter_cols": geom.n_draft_cols, "parallelism": f"independent sequence per GPU x{world}",
+            "l2": "weights (2.48 GB) exceed L2 and stream from HBM every step" if geom.name == "r3"
+                  else "weights exceed L2 and stream from HBM every step",
+        },
+        "roofline": {
+            "bound": "tensor", "kernel": "gemm_heads (one wide GEMM over all per-layer and drafter heads)",
+            "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
+            "peak_kind": f"{src} bf16 sustained (kernel timed inside a long step loop)",
+            "frac_of_burst": achieved / peaks["bf16_tflops"],
+            "flops_per_launch": heads_flops, "avg_launch_ms": heads_ms,
+            "traffic": heads_traffic(geom.name),
+        },
+        "path_roofline": {
+            "flops_alg": flops, "bytes_alg": bytes_, "t_roof_ms": t_roof * 1e3,
+            "frac": t_roof / (ms_step / 1e3), "peaks": f"{src}: {peaks['bf16_tflops']} TFLOP/s bf16, "
+                                                     f"{peaks['hbm_gbs']} GB/s",
+        },
+        "stages_ms_per_step": {k: v["ms"] / args.steps for k, v in prof.items()},
+        "gpu_launches": launches,
+        "device_status": status,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(geom, seed, tokens=512)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- oracle
+class OracleSample:
+    """The float64 oracle on `tokens` tokens of the same workload (projector + all
+    state updates).  Weights are drawn on the host with the same recipe and widened
+    to float64 once, outside the timed calls."""
+
+    def __init__(self, geom, seed, tokens):
+        from oracle import kva_ref as R
+        self.R, self.geom = R, geom
+        W = KI.make_projector_weights(geom, seed)
+        P = KI.make_layer_params(geom, seed + 1)
+        Wh = W.pop("W_heads")
+        self.Wn = R.weights_to_f64(W)
+        self.Whb = [Wh[c:c + 16384].double().numpy() for c in range(0, geom.n_total, 16384)]
+        del Wh
+        self.Pn = {k: v.double().numpy() for k, v in P.items()}
+        self.res = KI.make_residual(geom, tokens, seed + 100).double().numpy()
+        g = geom
+        self.S = np.zeros((g.n_gdn, g.gdn_n_v, g.gdn_d_v, g.gdn_d_k))
+        self.tail = np.zeros((g.n_gdn, g.conv_k - 1, g.gdn_conv_ch))
+        self.kc = [np.zeros((g.attn_n_kv, tokens, g.attn_d_h)) for _ in range(g.n_attn)]
+        self.vc = [np.zeros_like(k) for k in self.kc]
+
+    def run(self):
+        R = self.R
+        t0 = time.perf_counter()
+        z = R.projector_trunk(self.res, self.Wn, self.geom)
+        Y = np.concatenate([R.projector_heads(z, b) for b in self.Whb], axis=1)
+        R.update_states(Y, self.geom, self.Pn, self.S, self.tail, self.kc, self.vc, 0, scan="chunked")
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(geom, seed, tokens):
+    cores = len(os.sched_getaffinity(0))
+    t = OracleSample(geom, seed, tokens).run()
+    return {"value": tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{tokens} tokens of one {geom.name} ubatch through the float64 numpy oracle "
+                      f"(projector + every state update, chunked scan), one pass, {t:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: rank 0 only, each step a small sample of the
+    workload so that the whole --steps/--warmup run stays within a few minutes."""
+    if rank != 0:
+        return
+    geom = geometry(args.workload)
+    seed = 1003 if args.workload == "r3" else 1002
+    tokens = 8
+    osmp = OracleSample(geom, seed, tokens)
+    times = [osmp.run() for _ in range(args.warmup + args.steps)]
+    total = sum(times[args.warmup:])
+    cores = len(os.sched_getaffinity(0))
+    value = args.steps * tokens / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{geom.name} projector + state updates, {tokens} tokens per step",
+                   "geometry": geom.name, "tokens_per_step": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{tokens} tokens of one {geom.name} ubatch per step through the "
+                                   "float64 numpy oracle (projector + every state update)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,463 @@
+// Persistent bf16 GEMM on the 5th-generation tensor cores (tcgen05 / TMEM),
+// D = A * B^T with fused epilogues.  It serves every linear layer of the KVA
+// projector ("Qwen3.8-27B-KVA" model card, architecture: Linear{5120 -> d},
+// the q/k/v/o and SwiGLU projections of the 3 causal blocks, and the one wide
+// GEMM over all per-layer heads concatenated).
+//
+// Design (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per stage,
+//               128-byte swizzle, into a STAGES-deep shared-memory ring.
+//   warp 1      TMEM allocator + single-thread MMA issuer: 4 x tcgen05.mma
+//               (M=128, N=BN, K=16) per stage into one of two TMEM accumulators
+//               (2 x BN fp32 columns), tcgen05.commit frees the stage.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, fused store /
+//               residual add / SwiGLU, while the MMA warp already accumulates
+//               the next tile in the other TMEM buffer.
+// Tiles are visited M-fastest so the 8 M tiles of a 1024-token ubatch that
+// share one weight tile run together and read it from HBM once.
+#include <cuda.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "kva_common.cuh"
+
+namespace kva {
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+};
+
+struct GemmParams {
+  int M, N, K;
+  int b_mode;
+  int seg_rows;
+  void* D;
+  int64_t ldd;
+  void* D1;
+  int64_t ldd1;
+  int64_t n_split;
+  int* err;
+};
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v, int valid) {
+  if (valid >= 32) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 pk;
+      pk.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+      pk.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+      pk.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+      pk.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      reinterpret_cast<uint4*>(dst)[q] = pk;
+    }
+  } else {
+    for (int i = 0; i < valid; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
+                   const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
+                   const GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * Cfg::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mA);
+    tma_prefetch_desc(&mB0);
+    if (p.b_mode != B_SINGLE) tma_prefetch_desc(&mB1);
+    if (p.b_mode == B_SEGMENTS) tma_prefetch_desc(&mB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (p.M + Cfg::BM - 1) / Cfg::BM;
+  const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
+  const int num_n = (p.N + n_per_tile - 1) / n_per_tile;
+  const int num_k = (p.K + Cfg::BK - 1) / Cfg::BK;
+  const int tiles = num_m * num_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol_a = l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;  // stages with a load issued and not yet seen consumed
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % num_m;
+        const int n_blk = tile / num_m;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          armed |= 1u << stage;
+          const int kc = kb * Cfg::BK;
+          tma_load_2d(sA + stage * Cfg::A_BYTES, &mA, &full[stage], kc, m_blk * Cfg::BM, pol_a);
+          uint8_t* b = sB + stage * Cfg::B_BYTES;
+          if (p.b_mode == B_PAIRED) {
+            const int r = n_blk * (BN / 2);
+            tma_load_2d(b, &mB0, &full[stage], kc, r, pol_b);
+            tma_load_2d(b + (BN / 2) * 128, &mB1, &full[stage], kc, r, pol_b);
+          } else if (p.b_mode == B_SEGMENTS) {
+            const int n0 = n_blk * BN;
+            const int seg = n0 / p.seg_rows;
+            const int r = n0 - seg * p.seg_rows;
+            const CUtensorMap* m = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
+            tma_load_2d(b, m, &full[stage], kc, r, pol_b);
+          } else {
+            tma_load_2d(b, &mB0, &full[stage], kc, n_blk * BN, pol_b);
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      // Wait for the copies this thread issued to land before the CTA can exit.
+      // The last phase armed on stage s has parity (phase of s at arm time);
+      // waiting on it returns at once when it already completed.
+      (void)armed;
+      {
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < S; ++i) {
+          // step back one stage
+          if (st == 0) {
+            st = S - 1;
+            ph ^= 1u;
+          } else {
+            --st;
+          }
+          if (armed & (1u << st)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[st], ph)) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int j = 0; j < Cfg::BK / 16; ++j) {
+            umma_f16_ss(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
+                        idesc, (kb | j) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      // Drain: every MMA issued by this thread completes before TMEM is freed.
+      umma_commit(&tfull[acc]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&tfull[acc], acc_phase)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue warps 2..5
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      const int m_blk = tile % num_m;
+      const int n_blk = tile / num_m;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int row = m_blk * Cfg::BM + q * 32 + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t taddr =
+          tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (EPI == EPI_SWIGLU_BF16) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_ld_32x32b_x32(taddr + c, gr);
+          tmem_ld_32x32b_x32(taddr + BN / 2 + c, ur);
+          tmem_ld_wait();
+          const int col = n_blk * (BN / 2) + c;
+          if (row_ok && col < p.N) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col;
+            store_bf16x32(dst, v, p.N - col);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c, r);
+          tmem_ld_wait();
+          int col = n_blk * BN + c;
+          if (row_ok && col < p.N) {
+            const int valid = min(32, p.N - col);
+            void* base = p.D;
+            int64_t ld = p.ldd;
+            if (p.n_split > 0 && col >= p.n_split) {
+              base = p.D1;
+              ld = p.ldd1;
+              col -= static_cast<int>(p.n_split);
+            }
+            if constexpr (EPI == EPI_STORE_BF16) {
+              float v[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+              store_bf16x32(reinterpret_cast<__nv_bfloat16*>(base) + row * ld + col, v, valid);
+            } else {
+              float* dst = reinterpret_cast<float*>(base) + row * ld + col;
+              if (valid == 32) {
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                  float4 o;
+                  if constexpr (EPI == EPI_ADD_F32) o = reinterpret_cast<float4*>(dst)[q4];
+                  else o = make_float4(0.f, 0.f, 0.f, 0.f);
+                  o.x += __uint_as_float(r[4 * q4 + 0]);
+                  o.y += __uint_as_float(r[4 * q4 + 1]);
+                  o.z += __uint_as_float(r[4 * q4 + 2]);
+                  o.w += __uint_as_float(r[4 * q4 + 3]);
+                  reinterpret_cast<float4*>(dst)[q4] = o;
+                }
+              } else {
+                for (int i = 0; i < valid; ++i) {
+                  if constexpr (EPI == EPI_ADD_F32) dst[i] += __uint_as_float(r[i]);
+                  else dst[i] = __uint_as_float(r[i]);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 row-major [rows, inner] with row stride `ld` elements; box [box_rows, 64].
+static bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld,
+                     int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+template <int BN, int EPI>
+static int launch_instance(const GemmArgs& a, cudaStream_t s) {
+  using Cfg = GemmCfg<BN>;
+  const bool paired = a.b_mode == B_PAIRED;
+  const int box_b = paired ? BN / 2 : BN;
+  CUtensorMap mA, mB[3];
+  if (!make_map(&mA, a.A, a.K, a.M, a.lda, Cfg::BM)) return KVA_ERR_CUDA;
+  const int nb = a.b_mode == B_SINGLE ? 1 : (paired ? 2 : 3);
+  const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
+  for (int i = 0; i < 3; ++i) {
+    const void* src = a.B[i < nb ? i : 0];
+    if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, box_b)) return KVA_ERR_CUDA;
+  }
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.b_mode = a.b_mode;
+  p.seg_rows = static_cast<int>(a.seg_rows);
+  p.D = a.D;
+  p.ldd = a.ldd;
+  p.D1 = a.D1;
+  p.ldd1 = a.ldd1;
+  p.n_split = a.n_split;
+  p.err = a.err;
+  const int n_per_tile = paired ? BN / 2 : BN;
+  const int tiles = ((a.M + Cfg::BM - 1) / Cfg::BM) * ((a.N + n_per_tile - 1) / n_per_tile);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  auto kern = gemm_tc_kernel<BN, EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+      cudaSuccess)
+    return KVA_ERR_CUDA;
+  kern<<<grid, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+int launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0) return a.M == 0 ? KVA_OK : KVA_ERR_INVALID_ARG;
+  if (!a.A || !a.B[0] || !a.D) return KVA_ERR_INVALID_ARG;
+  if (!aligned16(a.A) || !aligned16(a.B[0]) || !aligned16(a.D)) return KVA_ERR_ALIGNMENT;
+  if ((a.lda % 8) || (a.ldb % 8) || (a.K % 8)) return KVA_ERR_ALIGNMENT;
+  const bool f32out = a.epilogue == EPI_STORE_F32 || a.epilogue == EPI_ADD_F32;
+  if (a.ldd % (f32out ? 4 : 8)) return KVA_ERR_ALIGNMENT;
+  if (a.n_split > 0) {
+    if (!a.D1 || !aligned16(a.D1) || (a.n_split % 32) || (a.ldd1 % (f32out ? 4 : 8)))
+      return KVA_ERR_ALIGNMENT;
+  }
+  if (a.b_mode == B_PAIRED && (a.epilogue != EPI_SWIGLU_BF16 || !a.B[1] || !aligned16(a.B[1])))
+    return KVA_ERR_INVALID_ARG;
+  if (a.epilogue == EPI_SWIGLU_BF16 && a.b_mode != B_PAIRED) return KVA_ERR_INVALID_ARG;
+  int bn = a.block_n;
+  if (bn == 0) {
+    if (a.b_mode == B_PAIRED) {
+      bn = 256;
+    } else {
+      const long tiles256 = ((a.M + 127) / 128) * (long)((a.N + 255) / 256);
+      bn = tiles256 >= 2L * num_sms() ? 256 : 128;
+    }
+  }
+  if (a.b_mode == B_SEGMENTS) {
+    if (!a.B[1] || !a.B[2] || !aligned16(a.B[1]) || !aligned16(a.B[2])) return KVA_ERR_INVALID_ARG;
+    if (a.seg_rows <= 0 || a.seg_rows % bn || a.N != 3 * a.seg_rows) return KVA_ERR_UNSUPPORTED;
+  }
+  if (bn != 128 && bn != 256) return KVA_ERR_UNSUPPORTED;
+  switch (a.epilogue) {
+    case EPI_STORE_BF16:
+      return bn == 256 ? launch_instance<256, EPI_STORE_BF16>(a, s)
+                       : launch_instance<128, EPI_STORE_BF16>(a, s);
+    case EPI_STORE_F32:
+      return bn == 256 ? launch_instance<256, EPI_STORE_F32>(a, s)
+                       : launch_instance<128, EPI_STORE_F32>(a, s);
+    case EPI_ADD_F32:
+      return bn == 256 ? launch_instance<256, EPI_ADD_F32>(a, s)
+                       : launch_instance<128, EPI_ADD_F32>(a, s);
+    case EPI_SWIGLU_BF16:
+      return bn == 256 ? launch_instance<256, EPI_SWIGLU_BF16>(a, s)
+                       : launch_instance<128, EPI_SWIGLU_BF16>(a, s);
+    default:
+      return KVA_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace kva

@@ -1,0 +1,91 @@
+// Internal launchers shared by the translation units of libkva.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kva.h"
+
+namespace kva {
+
+enum GemmEpilogue {
+  EPI_STORE_BF16 = 0,   // D = acc (bf16)
+  EPI_STORE_F32 = 1,    // D = acc (fp32)
+  EPI_ADD_F32 = 2,      // D += acc (fp32 residual stream)
+  EPI_SWIGLU_BF16 = 3,  // D[:, j] = silu(gate_j) * up_j (bf16), gate/up rows from B0/B1
+};
+
+enum GemmBMode {
+  B_SINGLE = 0,    // B0 is [N, K]
+  B_SEGMENTS = 1,  // B0,B1,B2 stacked along N, each [seg_rows, K] (q, k, v projections)
+  B_PAIRED = 2,    // B0 (gate) and B1 (up), each [N, K]; output N columns
+};
+
+struct GemmArgs {
+  const void* A = nullptr;  // bf16 [M, K], row stride lda elements
+  int64_t lda = 0;
+  const void* B[3] = {nullptr, nullptr, nullptr};
+  int b_mode = B_SINGLE;
+  int64_t ldb = 0;          // row stride of every B matrix (elements)
+  int64_t seg_rows = 0;     // rows of each segment (B_SEGMENTS)
+  void* D = nullptr;        // output columns [0, n_split)
+  int64_t ldd = 0;
+  void* D1 = nullptr;       // output columns [n_split, N), column index shifted by n_split
+  int64_t ldd1 = 0;
+  int64_t n_split = 0;      // 0: everything goes to D
+  int M = 0, N = 0, K = 0;
+  int epilogue = EPI_STORE_BF16;
+  int block_n = 0;          // 0: choose
+  int* err = nullptr;       // device status word
+};
+
+int num_sms();
+int launch_gemm(const GemmArgs& a, cudaStream_t s);
+int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
+                   int64_t ldo, int rows, int n, float eps, cudaStream_t s);
+int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
+                     int window, cudaStream_t s);
+
+struct GdnLaunch {
+  const void* mix = nullptr;    // bf16 [n_seq, T, mix_ld]
+  int64_t mix_ld = 0;
+  int64_t mix_seq_stride = 0;   // elements between sequences
+  int n_seq = 0, T = 0;
+  int n_gdn = 0;
+  int layer_col[KVA_MAX_LATE] = {0};
+  int n_k = 0, n_v = 0, d_k = 0, d_v = 0, C = 0;
+  const float* conv_w = nullptr;
+  const float* A_log = nullptr;
+  const float* dt_bias = nullptr;
+  void* conv_state = nullptr;   // bf16 [n_seq, n_gdn, 3, C]
+  float* state = nullptr;       // fp32 [n_seq, n_gdn, n_v, d_v, d_k]
+  void* kbuf = nullptr;         // bf16 [n_seq, n_gdn, T, n_k*d_k]
+  void* vbuf = nullptr;         // bf16 [n_seq, n_gdn, T, n_v*d_v]
+  float* gbuf = nullptr;        // fp32 [n_seq, n_gdn, 2, n_v, T] (g then beta)
+  void* debug_qkv = nullptr;    // bf16 [n_seq, n_gdn, T, C] or null
+  float eps = 1e-6f;
+  int* err = nullptr;
+};
+int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s);
+int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s);
+int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s);
+
+constexpr int kMaxSeqPos = 256;
+struct KvLaunch {
+  const void* mix = nullptr;
+  int64_t mix_ld = 0;
+  int64_t mix_seq_stride = 0;
+  int n_seq = 0, T = 0;
+  int n_attn = 0;
+  int layer_col[KVA_MAX_LATE] = {0};
+  int n_kv = 0, d_h = 0, rope_dims = 0;
+  double rope_theta = 1e7;
+  const float* k_gain = nullptr;  // [n_attn, d_h]
+  int64_t pos[kMaxSeqPos] = {0};
+  kva_kv_cache cache;
+  float eps = 1e-6f;
+  int* err = nullptr;
+};
+int launch_kv_write(const KvLaunch& k, cudaStream_t s);
+
+}  // namespace kva

@@ -1,0 +1,134 @@
+// Full-attention late layers: k RMSNorm per KV head, partial RoPE and the KV
+// cache write ("Qwen3.8-27B-KVA" model card, table "late layer type": k_proj /
+// v_proj outputs before k_norm / rope; "Qwen3.8-27B-MLA" model card, "What this
+// is": 4 KV heads of dim 256 with 64 rotary dims, whose lowest pairs turn
+// 3.4 / 2.1 / 1.2 degrees across 131k tokens, i.e. theta = 1e7).
+//
+// One warp per (token, KV head): each lane holds d_h/32 consecutive dims as one
+// 16- (or 8-) byte vector; the RMS is a warp reduction; RoPE pairs (i, i+r/2)
+// meet through one xor shuffle; the angle (pos * theta^(-2i/r)) is formed and
+// range-reduced in fp64 before sincosf, so it stays exact at 32k+ positions.
+// K and V rows are written with one vector store per lane (coalesced rows of
+// 512 bytes); V is copied bit for bit.  Paged caches go through the page table,
+// an out-of-range entry skips the write and sets the device status word.
+#include "kva_common.cuh"
+
+namespace kva {
+
+template <int EPL>
+struct VecT;
+template <>
+struct VecT<8> {
+  using T = uint4;
+};
+template <>
+struct VecT<4> {
+  using T = uint2;
+};
+
+template <int EPL>
+__global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
+  using V = typename VecT<EPL>::T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= p.T) return;
+  const int seq = blockIdx.z;
+  const int ai = blockIdx.y / p.n_kv, hh = blockIdx.y % p.n_kv;
+  const int d_h = p.d_h;
+  const __nv_bfloat16* row = static_cast<const __nv_bfloat16*>(p.mix) + seq * p.mix_seq_stride +
+                             static_cast<int64_t>(t) * p.mix_ld + p.layer_col[ai];
+  const int dim0 = lane * EPL;
+  V kv = *reinterpret_cast<const V*>(row + hh * d_h + dim0);
+  const V vv = *reinterpret_cast<const V*>(row + p.n_kv * d_h + hh * d_h + dim0);
+  float k[EPL];
+  {
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(&kv);
+#pragma unroll
+    for (int i = 0; i < EPL / 2; ++i) {
+      const float2 f = unpack_bf16(u[i]);
+      k[2 * i] = f.x;
+      k[2 * i + 1] = f.y;
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) ss += k[i] * k[i];
+  ss = warp_sum(ss);
+  const float scale = rsqrtf(ss / static_cast<float>(d_h) + p.eps);
+  const float* gain = p.k_gain + ai * d_h + dim0;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) k[i] *= scale * gain[i];
+
+  const int64_t pos = p.pos[seq] + t;
+  const int half = p.rope_dims / 2;
+  const int off = half / EPL;  // lane distance between the two dims of a pair
+  float partner[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, k[i], off);
+  if (dim0 < p.rope_dims) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double lt = log2(p.rope_theta);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int d = dim0 + i;
+      const int pi = d < half ? d : d - half;
+      const double inv = exp2(-(2.0 * pi / p.rope_dims) * lt);
+      const double ang = static_cast<double>(pos) * inv;
+      const double q = rint(ang / two_pi);
+      const float red = static_cast<float>(fma(-q, two_pi, ang));
+      float sn, cs;
+      sincosf(red, &sn, &cs);
+      k[i] = d < half ? k[i] * cs - partner[i] * sn : k[i] * cs + partner[i] * sn;
+    }
+  }
+  V ko;
+  {
+    uint32_t* u = reinterpret_cast<uint32_t*>(&ko);
+#pragma unroll
+    for (int i = 0; i < EPL / 2; ++i) u[i] = pack_bf16(k[2 * i], k[2 * i + 1]);
+  }
+
+  int64_t rowidx;
+  const kva_kv_cache& cc = p.cache;
+  if (cc.layout == KVA_KV_PAGED) {
+    const int64_t pg_i = pos / cc.page_size;
+    if (pg_i < 0 || pg_i >= cc.pages_per_seq) {
+      if (lane == 0) set_device_error(p.err, KVA_DEV_PAGE_OOB);
+      return;
+    }
+    const int page = cc.page_table[static_cast<int64_t>(seq) * cc.pages_per_seq + pg_i];
+    if (page < 0 || page >= cc.n_pages) {
+      if (lane == 0) set_device_error(p.err, KVA_DEV_PAGE_OOB);
+      return;
+    }
+    rowidx = (static_cast<int64_t>(page) * p.n_kv + hh) * cc.page_size + pos % cc.page_size;
+  } else {
+    rowidx = (static_cast<int64_t>(seq) * p.n_kv + hh) * cc.max_pos + pos;
+  }
+  __nv_bfloat16* kd = static_cast<__nv_bfloat16*>(cc.k[ai]) + rowidx * d_h + dim0;
+  __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(cc.v[ai]) + rowidx * d_h + dim0;
+  *reinterpret_cast<V*>(kd) = ko;
+  *reinterpret_cast<V*>(vd) = vv;
+}
+
+int launch_kv_write(const KvLaunch& k, cudaStream_t s) {
+  if (k.T == 0 || k.n_attn == 0 || k.n_seq == 0) return KVA_OK;
+  if (!k.mix || !k.k_gain) return KVA_ERR_INVALID_ARG;
+  if (k.d_h != 128 && k.d_h != 256) return KVA_ERR_UNSUPPORTED;
+  const int epl = k.d_h / 32;
+  const int half = k.rope_dims / 2;
+  if (k.rope_dims < 0 || k.rope_dims % 2 || k.rope_dims > k.d_h) return KVA_ERR_UNSUPPORTED;
+  if (k.rope_dims > 0) {
+    if (half % epl) return KVA_ERR_UNSUPPORTED;
+    const int off = half / epl;
+    if (off & (off - 1)) return KVA_ERR_UNSUPPORTED;  // xor pairing needs a power of two
+  }
+  dim3 grid((k.T + 7) / 8, k.n_kv * k.n_attn, k.n_seq);
+  if (epl == 8)
+    kv_write_kernel<8><<<grid, 256, 0, s>>>(k);
+  else
+    kv_write_kernel<4><<<grid, 256, 0, s>>>(k);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+}  // namespace kva

@@ -1,0 +1,77 @@
+// RMSNorm rows -> bf16 ("Qwen3.8-27B-KVA" model card, architecture:
+// RMSNorm before the input Linear, before each attention and FFN sub-block, and
+// once before all heads).  out = x / sqrt(mean(x^2) + eps) * g, stats in fp32.
+// HBM-bound: one read of x (fp32 or bf16), one bf16 write; the second pass over
+// the row hits L1.
+#include "kva_common.cuh"
+
+namespace kva {
+
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, int64_t ldx,
+                                                      const float* __restrict__ g,
+                                                      __nv_bfloat16* __restrict__ out,
+                                                      int64_t ldo, int n, float eps) {
+  const int row = blockIdx.x;
+  const T* xr = x + row * ldx;
+  __nv_bfloat16* orow = out + row * ldo;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < n; i += blockDim.x * 4) {
+    float4 v = load4<T>(xr + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(n) + eps);
+  for (int i = threadIdx.x * 4; i < n; i += blockDim.x * 4) {
+    float4 v = load4<T>(xr + i);
+    float4 gg = *reinterpret_cast<const float4*>(g + i);
+    uint2 o;
+    o.x = pack_bf16(v.x * scale * gg.x, v.y * scale * gg.y);
+    o.y = pack_bf16(v.z * scale * gg.z, v.w * scale * gg.w);
+    *reinterpret_cast<uint2*>(orow + i) = o;
+  }
+}
+
+int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
+                   int64_t ldo, int rows, int n, float eps, cudaStream_t s) {
+  if (rows == 0) return KVA_OK;
+  if (!x || !g || !out || rows < 0 || n <= 0) return KVA_ERR_INVALID_ARG;
+  if (n % 4 || ldx % 4 || ldo % 4) return KVA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(g) |
+       reinterpret_cast<uintptr_t>(out)) & 15u)
+    return KVA_ERR_ALIGNMENT;
+  if (x_dtype == KVA_F32)
+    rmsnorm_kernel<float><<<rows, 256, 0, s>>>(static_cast<const float*>(x), ldx, g,
+                                                static_cast<__nv_bfloat16*>(out), ldo, n, eps);
+  else if (x_dtype == KVA_BF16)
+    rmsnorm_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                        ldx, g, static_cast<__nv_bfloat16*>(out),
+                                                        ldo, n, eps);
+  else
+    return KVA_ERR_INVALID_ARG;
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+}  // namespace kva

@@ -1,0 +1,73 @@
+/*
+ * kva_ops.h -- per-step entry points of libkva.
+ *
+ * Each call runs exactly one step of the path (one kernel) on caller buffers.
+ * They exist so every step can be checked on its own against the float64
+ * oracle, and for callers that compose the path themselves.  Conventions
+ * (device pointers, row-major, async on `stream`, host-side validation,
+ * kva_status return) are those of kva.h.  `err` is an optional device int
+ * that receives device status bits (KVA_DEV_*); NULL disables reporting.
+ */
+#ifndef KVA_OPS_H_
+#define KVA_OPS_H_
+
+#include <stdint.h>
+
+#include "kva.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kva_epilogue {
+  KVA_EPI_STORE_BF16 = 0,  /* D = A B^T, bf16 */
+  KVA_EPI_STORE_F32 = 1,   /* D = A B^T, fp32 */
+  KVA_EPI_ADD_F32 = 2,     /* D += A B^T, fp32 (the projector's residual stream) */
+  KVA_EPI_SWIGLU_BF16 = 3  /* D = silu(A Bg^T) * (A Bu^T), bf16 (SwiGLU FFN, model card table) */
+} kva_epilogue;
+
+typedef enum kva_b_mode {
+  KVA_B_SINGLE = 0,   /* B[0] is [N, K] */
+  KVA_B_SEGMENTS = 1, /* B[0..2] each [seg_rows, K], stacked along N (q | k | v) */
+  KVA_B_PAIRED = 2    /* B[0] gate, B[1] up, each [N, K]; only with KVA_EPI_SWIGLU_BF16 */
+} kva_b_mode;
+
+/* RMSNorm of `rows` rows of width n ("Qwen3.8-27B-KVA" model card, architecture):
+ * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out bf16 [rows, ldo].
+ * x is [rows, ldx] in x_dtype.  n, ldx, ldo multiples of 4; pointers 16-byte aligned. */
+int kva_op_rmsnorm(const void* x, int32_t x_dtype, int64_t ldx, const float* g, void* out,
+                   int64_t ldo, int32_t rows, int32_t n, float eps, void* stream);
+
+/* D = A B^T with an epilogue on tcgen05 tensor cores (the projector's linears).
+ *   A     bf16 [M, K], row stride lda
+ *   B     HOST array of 1..3 device pointers per b_mode, each with row stride ldb
+ *   D     output [M, ldd] (bf16 or fp32 per epilogue); with n_split > 0 columns
+ *         >= n_split go to D1 [M, ldd1] at column - n_split (n_split % 32 == 0)
+ *   block_n 0 (choose), 128 or 256
+ * K, lda, ldb multiples of 8; seg_rows a multiple of the chosen block_n. */
+int kva_op_gemm(const void* A, int64_t lda, const void* const* B, int32_t b_mode, int64_t ldb,
+                int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1, int64_t n_split,
+                int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t block_n, int32_t* err,
+                void* stream);
+
+/* Block-causal multi-head attention of the projector (model card table row
+ * "attention"): qkv bf16 [T, ldq] holds q | k | v, each n_heads x 128 wide;
+ * out bf16 [T, ldo] gets the n_heads x 128 head outputs.  Key j is visible to
+ * query i iff j <= i and i / window == j / window (window 0: plain causal). */
+int kva_op_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int32_t T,
+                     int32_t n_heads, int32_t window, void* stream);
+
+/* Gated delta-rule scan alone, for n_seq x n_layers independent problems of T tokens:
+ *   k     bf16 [n_seq*n_layers, T, n_k*d]  (unit-norm keys)
+ *   v     bf16 [n_seq*n_layers, T, n_v*d]
+ *   gb    fp32 [n_seq*n_layers, 2, n_v, T] (g then beta per v head)
+ *   state fp32 [n_seq*n_layers, n_v, d, d] read and updated in place
+ * v head h reads k head h / (n_v / n_k).  d = 64 or 128. */
+int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state, int32_t n_seq,
+                    int32_t n_layers, int32_t T, int32_t n_k, int32_t n_v, int32_t d,
+                    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVA_OPS_H_ */

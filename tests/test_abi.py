@@ -1,0 +1,119 @@
+"""The C ABI library loads and exports every symbol the headers declare; host-side
+validation rejects bad arguments before touching the GPU (no compute calls here)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import kva_inputs as KI
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in ("kva.h", "kva_ops.h"):
+        with open(os.path.join(ROOT, "include", h)) as f:
+            txt = f.read()
+        names |= set(re.findall(r"^\s*(?:int|void|size_t|const char\*)\s+(kva_\w+)\s*\(", txt, re.M))
+    return names
+
+
+def test_headers_declare_the_boundary():
+    names = _declared()
+    for n in ("kva_init", "kva_prefill_ubatch", "kva_update_states", "kva_free",
+              "kva_get_device_status", "kva_strerror", "kva_stats", "kva_workspace_bytes",
+              "kva_op_gemm", "kva_op_attention", "kva_op_rmsnorm", "kva_op_gdn_scan"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import hybrid_deltanet_attention_kva_b200 as K
+    out = subprocess.run(["nm", "-D", "--defined-only", K.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(kva_\w+)$", out, re.M))
+    missing = _declared() - exported
+    assert not missing, missing
+    assert set(K.EXPORTED) <= exported
+
+
+def test_binding_names_match_c_names():
+    import hybrid_deltanet_attention_kva_b200 as K
+    for n in _declared():
+        assert hasattr(K, n), n
+
+
+def test_struct_layouts_match_the_c_compiler(tmp_path):
+    """sizeof / offsetof of every ABI struct, from gcc compiling the header, equal ctypes'."""
+    import hybrid_deltanet_attention_kva_b200 as K
+    fields = {"kva_dims": (K.KvaDims, ["rope_theta", "norm_eps", "max_seq", "layer_type"]),
+              "kva_weights": (K.KvaWeights, ["blocks", "W_heads", "k_norm_g"]),
+              "kva_block_weights": (K.KvaBlockWeights, ["Wd"]),
+              "kva_kv_cache": (K.KvaKvCache, ["v", "max_pos", "page_table"])}
+    src = ["#include <stdio.h>", "#include <stddef.h>", '#include "kva.h"', "int main(void){"]
+    for st, (_, fs) in fields.items():
+        src.append(f'printf("{st} %zu\\n", sizeof({st}));')
+        for f in fs:
+            src.append(f'printf("{st}.{f} %zu\\n", offsetof({st}, {f}));')
+    src.append("return 0;}")
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(src))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    for st, (cls, fs) in fields.items():
+        assert int(got[st]) == C.sizeof(cls), st
+        for f in fs:
+            assert int(got[f"{st}.{f}"]) == getattr(cls, f).offset, (st, f)
+
+
+def test_workspace_and_strerror_without_gpu():
+    import hybrid_deltanet_attention_kva_b200 as K
+    for g in (KI.TINY, KI.R2, KI.R3):
+        assert K.kva_workspace_bytes(K.make_dims(g, 1024, 1)) > 0
+    bad = K.make_dims(KI.R3, 1024, 1)
+    bad.head_dim = 64
+    assert K.kva_workspace_bytes(bad) == 0
+    bad = K.make_dims(KI.R3, 1024, 1)
+    bad.conv_k = 3
+    assert K.kva_workspace_bytes(bad) == 0
+    bad = K.make_dims(KI.R3, 1024, 1)
+    bad.layer_type[0] = 7
+    assert K.kva_workspace_bytes(bad) == 0
+    assert K.kva_strerror(K.KVA_ERR_TOO_LARGE).startswith("size beyond")
+    assert K.kva_strerror(12345) == "unknown status"
+
+
+def test_host_validation_rejects_before_any_launch():
+    import hybrid_deltanet_attention_kva_b200 as K
+    L = K.lib()
+    h = C.c_void_p()
+    assert L.kva_init(None, C.byref(h)) == K.KVA_ERR_INVALID_ARG
+    d = K.make_dims(KI.R3, 1024, 1)
+    d.n_late = 0
+    assert L.kva_init(C.byref(d), C.byref(h)) == K.KVA_ERR_INVALID_ARG
+    assert h.value is None
+    # entry points refuse a null handle
+    assert L.kva_prefill_ubatch(None, None, 0, 1, None, None, None, None, 0, None, None, None) \
+        == K.KVA_ERR_INVALID_ARG
+    assert L.kva_update_states(None, None, 0, 1, 1, None, None, None, None, None, None, None,
+                               None) == K.KVA_ERR_INVALID_ARG
+    n = C.c_int64()
+    assert L.kva_stats(None, C.byref(n)) == K.KVA_ERR_INVALID_ARG
+    s = C.c_int32()
+    assert L.kva_get_device_status(None, C.byref(s)) == K.KVA_ERR_INVALID_ARG
+    # per-step ops: misaligned / invalid shapes are refused on the host
+    assert L.kva_op_rmsnorm(C.c_void_p(16), 1, 6, C.c_void_p(16), C.c_void_p(16), 6, 2, 6, 1e-6,
+                            None) == K.KVA_ERR_ALIGNMENT
+    arr = (C.c_void_p * 3)(16, None, None)
+    assert L.kva_op_gemm(C.c_void_p(16), 12, arr, 0, 12, 0, C.c_void_p(16), 64, None, 0, 0,
+                         64, 64, 12, 0, 0, None, None) == K.KVA_ERR_ALIGNMENT
+    assert L.kva_op_gemm(C.c_void_p(16), 64, arr, 5, 64, 0, C.c_void_p(16), 64, None, 0, 0,
+                         64, 64, 64, 0, 0, None, None) == K.KVA_ERR_INVALID_ARG
+    assert L.kva_op_attention(C.c_void_p(16), 384, C.c_void_p(16), 128, 16, 1, -1, None) \
+        == K.KVA_ERR_INVALID_ARG
+    assert L.kva_op_gdn_scan(C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), 1,
+                             1, 8, 1, 1, 96, None) == K.KVA_ERR_UNSUPPORTED

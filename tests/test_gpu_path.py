@@ -1,0 +1,322 @@
+"""End-to-end parity of kva_update_states and kva_prefill_ubatch against the oracle.
+
+Bit-exact: conv tails (equal to the raw mixer rows they come from), V cache rows
+(copies of the predicted v), the set of written cache rows (sentinel elsewhere).
+Within tolerance: mixer / drafter outputs, q/k/v after conv and norms, g and
+beta, K cache rows, final DeltaNet states.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kva_inputs as KI
+from oracle import kva_ref as R
+from tests.parity import BF16_ELEM, assert_rms_close, assert_state_close, f64
+
+pytestmark = pytest.mark.gpu
+SENT = -7.0  # sentinel of untouched cache rows (exact in bf16)
+
+
+@pytest.fixture(scope="module")
+def K():
+    import hybrid_deltanet_attention_kva_b200 as K
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return K
+
+
+class Caches:
+    """Caches on the device and their float64 oracle twins (sentinel-filled)."""
+
+    def __init__(self, K, geom, n_seq, max_pos, paged=False, page_size=256, seed=77):
+        self.geom, self.n_seq, self.paged = geom, n_seq, paged
+        self.page_size = page_size
+        na, nkv, dh = geom.n_attn, geom.attn_n_kv, geom.attn_d_h
+        if paged:
+            pps = (max_pos + page_size - 1) // page_size
+            self.n_pages = n_seq * pps + 3                      # a few spare pages
+            self.pt = KI.make_page_table(n_seq, pps, seed, n_pages=self.n_pages)
+            shape = (self.n_pages, nkv, page_size, dh)
+        else:
+            shape = (n_seq, nkv, max_pos, dh)
+        self.k = [torch.full(shape, SENT, dtype=torch.bfloat16, device="cuda") for _ in range(na)]
+        self.v = [torch.full(shape, SENT, dtype=torch.bfloat16, device="cuda") for _ in range(na)]
+        self.ok = [np.full(shape, SENT) for _ in range(na)]
+        self.ov = [np.full(shape, SENT) for _ in range(na)]
+        if paged:
+            self.c = K.KvCache(self.k, self.v, page_table=self.pt.cuda(), page_size=page_size,
+                               n_pages=self.n_pages)
+        else:
+            self.c = K.KvCache(self.k, self.v, max_pos=max_pos)
+
+    def oracle_views(self, s):
+        """Per-sequence cache views for the oracle's update_states."""
+        if self.paged:
+            return self.ok, self.ov, self.pt.numpy()[s], self.page_size
+        return [k[s] for k in self.ok], [v[s] for v in self.ov], None, 0
+
+    def compare(self, v_exact=True):
+        """v_exact: the oracle read the same bf16 mixer values (state-update tests), so
+        V rows must match bit for bit; after a projector pass V is compared within
+        tolerance here and bitwise against the GPU's own mixer by the caller."""
+        for a in range(len(self.k)):
+            gk, gv = f64(self.k[a]), f64(self.v[a])
+            ok, ov = self.ok[a], self.ov[a]
+            written = ok != SENT
+            # the same rows were written (sentinel elsewhere, bit for bit)
+            np.testing.assert_array_equal(gk == SENT, ~written)
+            np.testing.assert_array_equal(gv[~written], ov[~written])
+            assert_rms_close(gk[written], ok[written], what=f"K cache layer {a}", elem=BF16_ELEM)
+            if v_exact:
+                np.testing.assert_array_equal(gv[written], ov[written])   # V is a bit copy
+            else:
+                assert_rms_close(gv[written], ov[written], what=f"V cache layer {a}", elem=BF16_ELEM)
+
+
+def _gpu(t):
+    return t.cuda() if isinstance(t, torch.Tensor) else t
+
+
+def _proj_to_gpu(W):
+    return {"g_in": W["g_in"].cuda(), "W_in": W["W_in"].cuda(), "g_out": W["g_out"].cuda(),
+            "W_heads": W["W_heads"].cuda(),
+            "blocks": [{k: v.cuda() for k, v in b.items()} for b in W["blocks"]]}
+
+
+# ------------------------------------------------------------------ state updates
+@pytest.mark.parametrize("geom_name,n_seq,T,paged", [("tiny", 2, 100, False), ("tiny", 3, 2, True),
+                                                     ("r3", 2, 200, True)])
+def test_update_states_matches_oracle(K, geom_name, n_seq, T, paged):
+    geom = KI.GEOMETRIES[geom_name]
+    if geom_name == "r3":
+        geom = KI.with_changes(geom, n_draft=0)
+    P = KI.make_layer_params(geom, 11, random_k_gain=True)
+    st = KI.make_states(geom, n_seq, 12, std=0.1)
+    mix = KI.make_mixer_inputs(geom, n_seq, T, 13)
+    pos = [5 + 301 * s for s in range(n_seq)]
+    max_pos = max(pos) + T + 7
+    caches = Caches(K, geom, n_seq, max_pos, paged=paged, page_size=64)
+    h = K.kva_init(K.make_dims(geom, max(T, 16), n_seq))
+    try:
+        S = st["state"].cuda()
+        tail = st["conv_tail"].cuda()
+        dbg = torch.zeros(n_seq, geom.n_gdn, T, geom.gdn_conv_ch, dtype=torch.bfloat16, device="cuda")
+        dgb = torch.zeros(n_seq, geom.n_gdn, 2, geom.gdn_n_v, T, device="cuda")
+        Wt = K.Weights(layer={k: v.cuda() for k, v in P.items()})
+        K.kva_update_states(h, mix.cuda(), pos, Wt, S, tail, caches.c, debug_qkv=dbg, debug_gb=dgb)
+        assert K.kva_get_device_status(h) == 0
+        assert K.kva_stats(h) == n_seq * T
+    finally:
+        K.kva_free(h)
+    Pn = {k: f64(v) for k, v in P.items()}
+    for s in range(n_seq):
+        debug = {}
+        kc, vc, pt, ps = caches.oracle_views(s)
+        S_o, tail_o = R.update_states(f64(mix[s]), geom, Pn, f64(st["state"][s]),
+                                      f64(st["conv_tail"][s]), kc, vc, pos[s], page_table=pt,
+                                      page_size=ps, scan="chunked", debug=debug)
+        assert_state_close(S[s], S_o, what=f"state seq {s}")
+        # the conv tail is a bit copy of raw mixer rows
+        np.testing.assert_array_equal(f64(tail[s]), tail_o)
+        nk = geom.gdn_n_k * geom.gdn_d_k
+        for gi, pr in enumerate(debug["gdn"]):
+            got = f64(dbg[s, gi])
+            assert_rms_close(got[:, :nk], pr["q"].reshape(T, -1), what="q_hat", elem=BF16_ELEM)
+            assert_rms_close(got[:, nk:2 * nk], pr["k"].reshape(T, -1), what="k_hat", elem=BF16_ELEM)
+            assert_rms_close(got[:, 2 * nk:], pr["v"].reshape(T, -1), what="v", elem=BF16_ELEM)
+            assert_rms_close(dgb[s, gi, 0].T, pr["g"], what="g", elem=1e-5)
+            assert_rms_close(dgb[s, gi, 1].T, pr["beta"], what="beta", elem=1e-5)
+    caches.compare()
+
+
+def test_update_states_rejects_oob_page_table_on_device(K):
+    geom = KI.TINY
+    P = KI.make_layer_params(geom, 1)
+    st = KI.make_states(geom, 1, 2)
+    mix = KI.make_mixer_inputs(geom, 1, 8, 3)
+    caches = Caches(K, geom, 1, 64, paged=True, page_size=16)
+    bad = caches.pt.clone()
+    bad[0, 0] = caches.n_pages + 5                      # out of the pool: write skipped, flagged
+    c = K.KvCache(caches.k, caches.v, page_table=bad.cuda(), page_size=16, n_pages=caches.n_pages)
+    h = K.kva_init(K.make_dims(geom, 16, 1))
+    try:
+        K.kva_update_states(h, mix.cuda(), [0], K.Weights(layer={k: v.cuda() for k, v in P.items()}),
+                            st["state"].cuda(), st["conv_tail"].cuda(), c)
+        status = K.kva_get_device_status(h)
+        assert status & K.KVA_DEV_PAGE_OOB
+        assert K.kva_get_device_status(h) == 0           # cleared by the read
+        for t in caches.k + caches.v:
+            assert bool((t == SENT).all())               # nothing written anywhere
+        # host-side: a position beyond the page table is refused before launch
+        with pytest.raises(K.KvaError) as ei:
+            K.kva_update_states(h, mix.cuda(), [60], K.Weights(layer={k: v.cuda() for k, v in P.items()}),
+                                st["state"].cuda(), st["conv_tail"].cuda(), c)
+        assert ei.value.status == K.KVA_ERR_TOO_LARGE
+    finally:
+        K.kva_free(h)
+
+
+# ------------------------------------------------------------------ full ubatch
+def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outliers=8):
+    """Run consecutive ubatches of one sequence on the GPU; return GPU results + inputs."""
+    W = KI.make_projector_weights(geom, seed)
+    P = KI.make_layer_params(geom, seed + 1)
+    st = KI.make_states(geom, 1, seed + 2)
+    total = sum(ubatches)
+    res = KI.make_residual(geom, total, seed + 3, dtype=residual_dtype, n_outliers=n_outliers)
+    caches = Caches(K, geom, 1, total + 16)
+    h = K.kva_init(K.make_dims(geom, max(ubatches), 1))
+    Wg = K.Weights(proj=_proj_to_gpu(W), layer={k: v.cuda() for k, v in P.items()})
+    S = st["state"][0].cuda()
+    tail = st["conv_tail"][0].cuda()
+    mixers, drafts = [], []
+    pos = 0
+    try:
+        for T in ubatches:
+            mo = torch.empty(T, geom.n_mix, dtype=torch.bfloat16, device="cuda")
+            do = (torch.empty(T, geom.n_draft_cols, dtype=torch.bfloat16, device="cuda")
+                  if draft and geom.n_draft else None)
+            K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wg, S, tail, caches.c, pos,
+                                 draft_out=do, mixer_out=mo)
+            mixers.append(mo)
+            drafts.append(do)
+            pos += T
+        torch.cuda.synchronize()
+        assert K.kva_get_device_status(h) == 0
+    finally:
+        K.kva_free(h)
+    return dict(W=W, P=P, st=st, res=res, caches=caches, S=S, tail=tail, mixers=mixers,
+                drafts=drafts)
+
+
+def _v_rows_are_mixer_copies(r, geom):
+    """Every written V row is bitwise the v part of the GPU's own mixer row."""
+    pos = 0
+    offs = geom.layer_offsets
+    nkd = geom.attn_n_kv * geom.attn_d_h
+    for mo in r["mixers"]:
+        T = mo.shape[0]
+        for ai, li in enumerate(geom.attn_layers()):
+            v = mo[:, offs[li] + nkd:offs[li] + 2 * nkd].reshape(T, geom.attn_n_kv, geom.attn_d_h)
+            got = r["caches"].v[ai][0][:, pos:pos + T].transpose(0, 1)
+            assert torch.equal(got, v)
+        pos += T
+
+
+def test_prefill_tiny_matches_oracle_everywhere(K):
+    """Tiny workload (T=128, fp32 residual): every output compared."""
+    geom = KI.TINY
+    r = _run_prefill(K, geom, [128], torch.float32, 1001, n_outliers=0)
+    Wn = R.weights_to_f64(r["W"])
+    Pn = {k: f64(v) for k, v in r["P"].items()}
+    kc, vc, _, _ = r["caches"].oracle_views(0)
+    Y, S_o, tail_o = R.prefill_ubatch(f64(r["res"]), Wn, geom, Pn, f64(r["st"]["state"][0]),
+                                      f64(r["st"]["conv_tail"][0]), kc, vc, 0)
+    assert_rms_close(r["mixers"][0], Y[:, :geom.n_mix], what="mixer")
+    assert_state_close(r["S"], S_o)
+    assert_rms_close(r["tail"], tail_o, what="conv tail")
+    # the tail is bitwise the GPU's own last raw mixer rows
+    mo = r["mixers"][0]
+    for gi, li in enumerate(geom.gdn_layers()):
+        off = geom.layer_offsets[li]
+        assert torch.equal(r["tail"][gi], mo[-3:, off:off + geom.gdn_conv_ch])
+    r["caches"].compare(v_exact=False)
+    _v_rows_are_mixer_copies(r, geom)
+
+
+@pytest.mark.parametrize("T", [1, 2, 77, 300])
+def test_prefill_tiny_ragged_and_carry(K, T):
+    """Ragged ubatches carried across calls equal the oracle run on the same split."""
+    geom = KI.TINY
+    splits = [T, 128 - T] if T < 128 else [T]
+    r = _run_prefill(K, geom, splits, torch.float32, 2000 + T, n_outliers=0)
+    Wn = R.weights_to_f64(r["W"])
+    Pn = {k: f64(v) for k, v in r["P"].items()}
+    kc, vc, _, _ = r["caches"].oracle_views(0)
+    S_o, tail_o = f64(r["st"]["state"][0]), f64(r["st"]["conv_tail"][0])
+    pos = 0
+    res = f64(r["res"])
+    for i, t in enumerate(splits):
+        Y, S_o, tail_o = R.prefill_ubatch(res[pos:pos + t], Wn, geom, Pn, S_o, tail_o, kc, vc, pos)
+        assert_rms_close(r["mixers"][i], Y[:, :geom.n_mix], what=f"mixer ubatch {i}")
+        pos += t
+    assert_state_close(r["S"], S_o)
+    assert_rms_close(r["tail"], tail_o, what="conv tail")
+    r["caches"].compare(v_exact=False)
+    _v_rows_are_mixer_copies(r, geom)
+
+
+def _err(got, want):
+    got = f64(got) if isinstance(got, torch.Tensor) else np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(want * want)))
+    e = np.abs(got - want)
+    return {"max_over_rms": float(e.max() / rms), "rms_err_over_rms": float(np.sqrt(np.mean(e * e)) / rms),
+            "n": int(e.size)}
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_prefill_full_size_sampled(K, cfg):
+    """r2 T=1024 and r3 1024+512 (carry, drafter heads) at full size.
+
+    The oracle runs the whole projector in float64 for every ubatch, the scan of
+    three sampled GDN layers across the ubatches, and every attention layer."""
+    import json
+    wl = KI.workload(cfg)
+    geom = wl.geom
+    r = _run_prefill(K, geom, wl.ubatches, wl.residual_dtype, wl.seed, draft=True)
+    Wh = r["W"].pop("W_heads")                      # bf16; widened block by block below
+    Wn = R.weights_to_f64(r["W"])
+
+    def heads(zz, lo, hi, step=16384):
+        return np.concatenate([R.projector_heads(zz, f64(Wh[c:min(hi, c + step)]))
+                               for c in range(lo, hi, step)], axis=1)
+
+    Pn = {k: f64(v) for k, v in r["P"].items()}
+    res = f64(r["res"])
+    gsel = [0, geom.n_gdn // 2, geom.n_gdn - 1]
+    S_o = f64(r["st"]["state"][0])
+    tail_o = f64(r["st"]["conv_tail"][0])
+    kc, vc, _, _ = r["caches"].oracle_views(0)
+    offs = geom.layer_offsets
+    metrics = {}
+    pos = 0
+    for i, T in enumerate(wl.ubatches):
+        z = R.projector_trunk(res[pos:pos + T], Wn, geom)
+        rows = np.unique(np.linspace(0, T - 1, 16).astype(int))
+        Yr = heads(z[rows], 0, geom.n_total)
+        metrics[f"mixer_{i}"] = _err(f64(r["mixers"][i])[rows], Yr[:, :geom.n_mix])
+        if r["drafts"][i] is not None:
+            metrics[f"drafter_{i}"] = _err(f64(r["drafts"][i])[rows], Yr[:, geom.n_mix:])
+        for gi in gsel:
+            li = geom.gdn_layers()[gi]
+            Yl = heads(z, offs[li], offs[li] + geom.gdn_width)
+            pr = R.gdn_prepare(Yl, tail_o[gi], Pn["conv_w"][gi], Pn["A_log"][gi], Pn["dt_bias"][gi], geom)
+            tail_o[gi] = pr["tail"]
+            S_o[gi] = R.delta_scan_chunked(S_o[gi], pr["k"], pr["v"], pr["g"], pr["beta"])
+        for ai, li in enumerate(geom.attn_layers()):
+            Yl = heads(z, offs[li], offs[li] + geom.attn_width)
+            Kx, Vx = R.attn_kv(Yl, Pn["k_norm_g"][ai], pos, geom)
+            kc[ai][:, pos:pos + T] = Kx.transpose(1, 0, 2)
+            vc[ai][:, pos:pos + T] = Vx.transpose(1, 0, 2)
+        pos += T
+    for gi in gsel:
+        metrics[f"state_{gi}"] = {"rel_frob": assert_state_close(r["S"][gi], S_o[gi], what=f"state layer {gi}")}
+        metrics[f"tail_{gi}"] = _err(r["tail"][gi], tail_o[gi])
+    gk_all, ok_all, gv_all, ov_all = [], [], [], []
+    for a in range(geom.n_attn):
+        gk = f64(r["caches"].k[a][0])
+        written = kc[a] != SENT
+        np.testing.assert_array_equal(gk == SENT, ~written)
+        gk_all.append(gk[written]); ok_all.append(kc[a][written])
+        gv_all.append(f64(r["caches"].v[a][0])[written]); ov_all.append(vc[a][written])
+    metrics["K_cache"] = _err(np.concatenate(gk_all), np.concatenate(ok_all))
+    metrics["V_cache"] = _err(np.concatenate(gv_all), np.concatenate(ov_all))
+    print("PARITY_METRICS", cfg, json.dumps(metrics))
+    # conv tails equal the GPU's own last raw rows (bitwise), V rows are mixer copies
+    last = r["mixers"][-1]
+    for gi, li in enumerate(geom.gdn_layers()):
+        assert torch.equal(r["tail"][gi], last[-3:, offs[li]:offs[li] + geom.gdn_conv_ch])
+    _v_rows_are_mixer_copies(r, geom)
+    for name, m in metrics.items():
+        if "max_over_rms" in m:
+            assert m["max_over_rms"] <= 2e-2, (name, m)

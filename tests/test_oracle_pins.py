@@ -333,7 +333,7 @@ def test_concatenated_heads_equal_per_layer_heads():
         w = geom.layer_width(li)
         Wl = W["W_heads"][off:off + w]
         np.testing.assert_allclose(Y[:, off:off + w],
-                                   np.einsum("td,nd->tn", z, Wl), rtol=1e-12)
+                                   np.einsum("td,nd->tn", z, Wl), rtol=1e-12, atol=1e-13)
 
 
 # ---------------------------------------------------------------- cache, carry
