@@ -24,7 +24,9 @@ def f64(t: torch.Tensor) -> np.ndarray:
 BF16_ELEM = 2.0 ** -8
 
 
-def assert_rms_close(got, want, tol=TOL_RMS, what="", elem=0.0):
+def assert_rms_close(got, want, tol=TOL_RMS, what="", elem=0.0, scale=None):
+    """max over elements of |got - want| - elem * scale <= tol * RMS(want);
+    scale defaults to |want| (the magnitude the stored value is rounded at)."""
     got = f64(got) if isinstance(got, torch.Tensor) else np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape, (what, got.shape, want.shape)
@@ -32,7 +34,8 @@ def assert_rms_close(got, want, tol=TOL_RMS, what="", elem=0.0):
     rms = float(np.sqrt(np.mean(want * want)))
     if not got.size:
         return 0.0
-    excess = np.abs(got - want) - elem * np.abs(want)
+    sc = np.abs(want) if scale is None else np.asarray(scale, dtype=np.float64)
+    excess = np.abs(got - want) - elem * sc
     i = int(np.argmax(excess))
     err = float(np.abs(got - want).flat[i])
     assert excess.flat[i] <= tol * rms, (

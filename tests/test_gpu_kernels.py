@@ -133,7 +133,10 @@ def test_attention(K, T, heads, window):
     Kk = q[:, d:2 * d].reshape(T, heads, 128)
     V = q[:, 2 * d:].reshape(T, heads, 128)
     want = R.block_causal_attention(Q, Kk, V, window).reshape(T, d)
-    assert_rms_close(out, want, what="attention", elem=BF16_ELEM)
+    # the softmax weights are rounded to bf16 before P V: each output element may move
+    # by 2^-8 of the weighted sum of |v| it averages (the oracle's attention over |V|)
+    scale = R.block_causal_attention(Q, Kk, np.abs(V), window).reshape(T, d)
+    assert_rms_close(out, want, what="attention", elem=BF16_ELEM, scale=scale)
 
 
 # ------------------------------------------------------------------ scan
