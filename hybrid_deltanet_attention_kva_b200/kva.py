@@ -110,6 +110,7 @@ def _load() -> C.CDLL:
                               I32, I32, I32, I32, P, P]),
         "kva_op_attention": (I32, [P, I64, P, I64, I32, I32, I32, P]),
         "kva_op_gdn_scan": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, P]),
+        "kva_gdn_layer_update_noalloc": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, F32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -122,7 +123,8 @@ _lib = _load()
 EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update_states",
             "kva_get_device_status", "kva_stats", "kva_free", "kva_strerror",
             "kva_profile_enable", "kva_profile_read",
-            "kva_op_rmsnorm", "kva_op_gemm", "kva_op_attention", "kva_op_gdn_scan")
+            "kva_op_rmsnorm", "kva_op_gemm", "kva_op_attention", "kva_op_gdn_scan",
+            "kva_gdn_layer_update_noalloc")
 
 
 def lib() -> C.CDLL:
@@ -318,3 +320,15 @@ def kva_op_gdn_scan(k: torch.Tensor, v: torch.Tensor, gb: torch.Tensor, state: t
     T = k.shape[-2]
     _check(_lib.kva_op_gdn_scan(_ptr(k), _ptr(v), _ptr(gb), _ptr(state), n_seq, n_layers, T, n_k,
                                 n_v, d, _stream(stream)), "kva_op_gdn_scan")
+
+
+def kva_gdn_layer_update_noalloc(mixer_in: torch.Tensor, n_k: int, n_v: int, d: int,
+                                 conv_w: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+                                 state: torch.Tensor, conv_state: torch.Tensor, eps: float = 1e-6,
+                                 stream=None) -> None:
+    """One gated-DeltaNet layer's state update without any device allocation (see
+    include/kva_ops.h): for callers that may not allocate device memory."""
+    T, ld = mixer_in.shape
+    _check(_lib.kva_gdn_layer_update_noalloc(
+        _ptr(mixer_in), ld, T, n_k, n_v, d, _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(state),
+        _ptr(conv_state), float(eps), _stream(stream)), "kva_gdn_layer_update_noalloc")

@@ -67,6 +67,38 @@ int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state,
                     int32_t n_layers, int32_t T, int32_t n_k, int32_t n_v, int32_t d,
                     void* stream);
 
+/* Limits of kva_gdn_layer_update_noalloc's fixed scratch (about 4.4 MB per GPU). */
+#define KVA_NOALLOC_MAX_T 256    /* tokens per call */
+#define KVA_NOALLOC_MAX_QK 2048  /* n_k * d */
+#define KVA_NOALLOC_MAX_V 6144   /* n_v * d */
+#define KVA_NOALLOC_MAX_NV 64    /* n_v */
+
+/* State update of ONE gated-DeltaNet layer of one sequence that allocates nothing.
+ *
+ * For callers that may not call cudaMalloc (or create a kva_handle, which does): an
+ * engine that has reserved nearly all device memory for its own cache pool and
+ * routes every allocation through its own allocator, or a plugin whose host program
+ * owns device memory.  The method described by the model card has no counterpart to
+ * this entry point; it exists only so such callers can run the layer update.
+ *
+ * It runs the same kernels as kva_update_states for that layer (conv + SiLU,
+ * L2 norms, gates, chunked scan, tail shift), keeping the intermediates in a
+ * fixed array compiled into the library (every GPU that loads the library holds it
+ * until the process exits).  The caller still passes every input and output:
+ *   mixer_in   bf16 [T, mixer_ld]: this layer's columns [q | k | v | a | b] from column 0
+ *   conv_w     fp32 [C, 4], A_log / dt_bias fp32 [n_v]
+ *   state      fp32 [n_v, d, d], conv_state bf16 [3, C]: read and updated in place
+ * Sizes beyond the KVA_NOALLOC_* limits return KVA_ERR_TOO_LARGE before any launch.
+ * The first call on a device looks up the array's device address (once per device,
+ * with that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose work overlaps on the GPU (different
+ * streams, or different host threads) race on it and must be serialised by the
+ * caller.  Returns kva_status. */
+int kva_gdn_layer_update_noalloc(const void* mixer_in, int64_t mixer_ld, int32_t T, int32_t n_k,
+                                 int32_t n_v, int32_t d, const float* conv_w, const float* A_log,
+                                 const float* dt_bias, float* state, void* conv_state, float eps,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif
