@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
+    ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16",
+                    help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -174,9 +176,15 @@ def run_ours(args, rank, world, local_rank):
                                 device_id=dev)
     geom = geometry(args.workload)
     seed = 1003 if args.workload == "r3" else 1002
+    dt = torch.float16 if args.dtype == "f16" else torch.bfloat16
     W = KI.make_projector_weights(geom, seed, device="cuda")
+    if dt != torch.bfloat16:
+        W = {k: (v if k.startswith("g_") or k == "blocks" else v.to(dt)) for k, v in W.items()}
+        W["blocks"] = [{k: (v if k.startswith("g_") else v.to(dt)) for k, v in b.items()}
+                       for b in W["blocks"]]
     P = KI.make_layer_params(geom, seed + 1, device="cuda")
     st = KI.make_states(geom, 1, seed + 2, device="cuda")
+    st["conv_tail"] = st["conv_tail"].to(dt)
     n_pool = 4
     res = [KI.make_residual(geom, T_UB, seed + 100 + rank * n_pool + i, device="cuda")
            for i in range(n_pool)]
@@ -187,9 +195,9 @@ def run_ours(args, rank, world, local_rank):
     Wt = K.Weights(proj=W, layer=P)
     S = st["state"][0]
     tail = st["conv_tail"][0]
-    draft = (torch.empty(T_UB, geom.n_draft_cols, dtype=torch.bfloat16, device=dev)
+    draft = (torch.empty(T_UB, geom.n_draft_cols, dtype=dt, device=dev)
              if geom.n_draft else None)
-    h = K.kva_init(K.make_dims(geom, T_UB, 1))
+    h = K.kva_init(K.make_dims(geom, T_UB, 1, dtype=dt))
     stream = torch.cuda.current_stream()
     n_ub = CACHE_POS // T_UB
 
@@ -241,7 +249,7 @@ def run_ours(args, rank, world, local_rank):
         host_res = [r.cpu().pin_memory() for r in res]
         dres = torch.empty_like(res[0])
         out_host = torch.empty(geom.n_draft_cols if geom.n_draft else geom.d_model,
-                               dtype=torch.bfloat16).pin_memory()
+                               dtype=dt).pin_memory()
         steps_e2e = max(3, min(args.steps, 200))
         for i in range(3):
             dres.copy_(host_res[i % n_pool], non_blocking=True)
@@ -297,9 +305,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded random bf16 weights of the projector shapes, N(0,1) residual "
-                "with 8 outlier channels x20)",
+        "dtype": args.dtype,
+        "data": "synthetic (seeded random N(0,0.02) weights of the projector shapes drawn in bf16"
+                + (" and converted to fp16" if dt == torch.float16 else "")
+                + ", bf16 N(0,1) residual with 8 outlier channels x20)",
         "config": {
             "workload": f"{geom.name} projector + state updates, 1024-token ubatch, state / conv "
                         f"tail / KV cache carried, positions 0..{CACHE_POS - 1}",

@@ -83,6 +83,7 @@ int derive(const kva_dims* d, int* n_gdn, int* n_attn, int64_t* n_mix) {
   if (d->hidden % 64 || d->d_model % 256 || d->ffn % 64) return KVA_ERR_UNSUPPORTED;
   if (d->conv_k != 4) return KVA_ERR_UNSUPPORTED;
   if (d->max_seq > kMaxSeqPos) return KVA_ERR_UNSUPPORTED;
+  if (d->compute_dtype != KVA_BF16 && d->compute_dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   int ng = 0, na = 0;
   for (int i = 0; i < d->n_late; ++i) {
     if (d->layer_type[i] == KVA_LAYER_GDN) ++ng;
@@ -217,6 +218,7 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     g.debug_qkv = debug_qkv;
     g.eps = d.norm_eps;
     g.err = h->status;
+    g.mix_dtype = d.compute_dtype;
     if ((e = staged(h, KVA_ST_GDN_PREPARE, s, [&] { return launch_gdn_prepare(g, s); }))) return e;
     if ((e = staged(h, KVA_ST_GDN_TAIL, s, [&] { return launch_gdn_tail(g, s); }))) return e;
     if ((e = staged(h, KVA_ST_GDN_SCAN, s, [&] { return launch_gdn_scan(g, s); }))) return e;
@@ -239,6 +241,7 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     k.cache = *kv;
     k.eps = d.norm_eps;
     k.err = h->status;
+    k.mix_dtype = d.compute_dtype;
     if ((e = staged(h, KVA_ST_KV_WRITE, s, [&] { return launch_kv_write(k, s); }))) return e;
   }
   return KVA_OK;
@@ -406,7 +409,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   if (T < 0) return KVA_ERR_INVALID_ARG;
   if (T > d.max_T) return KVA_ERR_TOO_LARGE;
   if (T == 0) return KVA_OK;
-  if (!residual || (residual_dtype != KVA_BF16 && residual_dtype != KVA_F32))
+  if (!residual ||
+      (residual_dtype != KVA_BF16 && residual_dtype != KVA_F32 && residual_dtype != KVA_F16))
     return KVA_ERR_INVALID_ARG;
   if (!a16(residual)) return KVA_ERR_ALIGNMENT;
   int e = check_weights(h, w, true);
@@ -426,10 +430,11 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   h->last_stream = s;
 
   const int H = d.hidden, dm = d.d_model, F = d.ffn;
+  const int cd = d.compute_dtype;
   const float eps = d.norm_eps;
   // 1. RMSNorm(residual) -> Linear{H -> d} into the fp32 residual stream x
   if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
-         return launch_rmsnorm(residual, residual_dtype, H, w->g_in, h->u_in, H, T, H, eps, s);
+         return launch_rmsnorm(residual, residual_dtype, H, w->g_in, h->u_in, H, T, H, eps, s, cd);
        })))
     goto done;
   {
@@ -445,13 +450,14 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     a.K = H;
     a.epilogue = EPI_STORE_F32;
     a.err = h->status;
+    a.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(a, s); }))) goto done;
   }
   // 2. the causal transformer blocks (pre-norm, residual adds fused in the GEMM epilogues)
   for (int b = 0; b < d.n_blocks; ++b) {
     const kva_block_weights& B = w->blocks[b];
     if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
-           return launch_rmsnorm(h->x, KVA_F32, dm, B.g_attn, h->u, dm, T, dm, eps, s);
+           return launch_rmsnorm(h->x, KVA_F32, dm, B.g_attn, h->u, dm, T, dm, eps, s, cd);
          })))
       goto done;
     GemmArgs q;
@@ -471,9 +477,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     q.epilogue = EPI_STORE_BF16;
     q.block_n = 128;
     q.err = h->status;
+    q.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(q, s); }))) goto done;
     if ((e = staged(h, KVA_ST_ATTENTION, s, [&] {
-           return launch_attention(h->qkv, 3 * dm, h->o, dm, T, d.n_heads, d.attn_window, s);
+           return launch_attention(h->qkv, 3 * dm, h->o, dm, T, d.n_heads, d.attn_window, s, cd);
          })))
       goto done;
     GemmArgs o;
@@ -488,9 +495,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     o.K = dm;
     o.epilogue = EPI_ADD_F32;
     o.err = h->status;
+    o.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(o, s); }))) goto done;
     if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
-           return launch_rmsnorm(h->x, KVA_F32, dm, B.g_ffn, h->u, dm, T, dm, eps, s);
+           return launch_rmsnorm(h->x, KVA_F32, dm, B.g_ffn, h->u, dm, T, dm, eps, s, cd);
          })))
       goto done;
     GemmArgs gu;
@@ -507,6 +515,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     gu.K = dm;
     gu.epilogue = EPI_SWIGLU_BF16;
     gu.err = h->status;
+    gu.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(gu, s); }))) goto done;
     GemmArgs dn;
     dn.A = h->qkv;
@@ -520,11 +529,12 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     dn.K = F;
     dn.epilogue = EPI_ADD_F32;
     dn.err = h->status;
+    dn.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(dn, s); }))) goto done;
   }
   // 3. RMSNorm -> all per-layer heads (+ drafter heads) in one wide GEMM
   if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
-         return launch_rmsnorm(h->x, KVA_F32, dm, w->g_out, h->u, dm, T, dm, eps, s);
+         return launch_rmsnorm(h->x, KVA_F32, dm, w->g_out, h->u, dm, T, dm, eps, s, cd);
        })))
     goto done;
   {
@@ -546,6 +556,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
       hd.n_split = h->n_mix;
     }
     hd.err = h->status;
+    hd.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] { return launch_gemm(hd, s); }))) goto done;
     // 4. state updates on the mixer inputs
     e = update_states_impl(h, mix, h->n_mix, 1, T, &pos, w, deltanet_state, conv_state, kv,
@@ -623,15 +634,16 @@ const char* kva_strerror(int32_t status) {
 
 // ------------------------------------------------------------ per-step ops
 int kva_op_rmsnorm(const void* x, int32_t x_dtype, int64_t ldx, const float* g, void* out,
-                   int64_t ldo, int32_t rows, int32_t n, float eps, void* stream) {
+                   int32_t out_dtype, int64_t ldo, int32_t rows, int32_t n, float eps,
+                   void* stream) {
   return launch_rmsnorm(x, x_dtype, ldx, g, out, ldo, rows, n, eps,
-                        static_cast<cudaStream_t>(stream));
+                        static_cast<cudaStream_t>(stream), out_dtype);
 }
 
-int kva_op_gemm(const void* A, int64_t lda, const void* const* B, int32_t b_mode, int64_t ldb,
-                int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1, int64_t n_split,
-                int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t block_n, int32_t* err,
-                void* stream) {
+int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B, int32_t b_mode,
+                int64_t ldb, int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1,
+                int64_t n_split, int32_t M, int32_t N, int32_t K, int32_t epilogue,
+                int32_t block_n, int32_t* err, void* stream) {
   if (!B) return KVA_ERR_INVALID_ARG;
   if (b_mode < KVA_B_SINGLE || b_mode > KVA_B_PAIRED) return KVA_ERR_INVALID_ARG;
   GemmArgs a;
@@ -653,14 +665,15 @@ int kva_op_gemm(const void* A, int64_t lda, const void* const* B, int32_t b_mode
   a.epilogue = epilogue;
   a.block_n = block_n;
   a.err = err;
+  a.dtype = dtype;
   if (M < 0 || N < 0 || K < 0) return KVA_ERR_INVALID_ARG;
   return launch_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
-int kva_op_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int32_t T,
-                     int32_t n_heads, int32_t window, void* stream) {
+int kva_op_attention(int32_t dtype, const void* qkv, int64_t ldq, void* out, int64_t ldo,
+                     int32_t T, int32_t n_heads, int32_t window, void* stream) {
   return launch_attention(qkv, ldq, out, ldo, T, n_heads, window,
-                          static_cast<cudaStream_t>(stream));
+                          static_cast<cudaStream_t>(stream), dtype);
 }
 
 int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state, int32_t n_seq,

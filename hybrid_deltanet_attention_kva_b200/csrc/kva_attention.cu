@@ -6,9 +6,9 @@
 // local to the ubatch (W = window, or the whole ubatch when window = 0).
 // Flash-style: one CTA per (128-query tile, head), 8 warps x 16 query rows,
 // 64-key tiles double-buffered in shared memory with cp.async, S = Q K^T and
-// O += P V on mma.sync (bf16 in, fp32 accumulate), online softmax in fp32 with
-// exp2.  qkv is [T, 3d] bf16 (q | k | v, head h at columns h*128 of each part),
-// output [T, d] bf16.
+// O += P V on mma.sync (16-bit in, fp32 accumulate), online softmax in fp32 with
+// exp2.  qkv is [T, 3d] 16-bit (q | k | v, head h at columns h*128 of each
+// part), output [T, d] in the same format (bf16 or fp16).
 #include <cmath>
 
 #include "kva_common.cuh"
@@ -21,27 +21,28 @@ constexpr int ATT_D = 128;
 constexpr int ATT_THREADS = 256;
 constexpr int ATT_SMEM = (ATT_BQ + 4 * ATT_BKV) * ATT_D * 2;  // Q + 2 x (K, V)
 
-// byte offset of (row, 16-byte chunk) in a [rows][128] bf16 tile, XOR swizzled
+// byte offset of (row, 16-byte chunk) in a [rows][128] 16-bit tile, XOR swizzled
 __device__ __forceinline__ uint32_t att_off(int row, int chunk) {
   return static_cast<uint32_t>(row * 256 + ((chunk ^ (row & 7)) << 4));
 }
 
-__device__ __forceinline__ void att_load_tile(uint32_t dst, const __nv_bfloat16* src, int64_t ld,
+template <typename E>
+__device__ __forceinline__ void att_load_tile(uint32_t dst, const E* src, int64_t ld,
                                               int row0, int rows, int T, int tid) {
   // rows x 16 chunks of 16 bytes; rows at or beyond T are zero-filled
   for (int i = tid; i < rows * 16; i += ATT_THREADS) {
     const int r = i >> 4, c = i & 15;
     const int gr = row0 + r;
     const bool ok = gr < T;
-    const __nv_bfloat16* g = src + static_cast<int64_t>(ok ? gr : 0) * ld + c * 8;
+    const E* g = src + static_cast<int64_t>(ok ? gr : 0) * ld + c * 8;
     cp_async16(dst + att_off(r, c), g, ok ? 16u : 0u);
   }
 }
 
+template <typename E>
 __global__ void __launch_bounds__(ATT_THREADS)
-    attention_kernel(const __nv_bfloat16* __restrict__ qkv, int64_t ldq,
-                     __nv_bfloat16* __restrict__ out, int64_t ldo, int T, int d_model,
-                     int window, float scale_log2) {
+    attention_kernel(const E* __restrict__ qkv, int64_t ldq, E* __restrict__ out, int64_t ldo,
+                     int T, int d_model, int window, float scale_log2) {
   extern __shared__ __align__(128) uint8_t att_smem[];
   const uint32_t sQ = smem_u32(att_smem);
   const uint32_t sK0 = sQ + ATT_BQ * 256;
@@ -53,9 +54,9 @@ __global__ void __launch_bounds__(ATT_THREADS)
   const int h = blockIdx.y;
   const int W = window > 0 ? window : 0x3fffffff;
 
-  const __nv_bfloat16* Qg = qkv + h * ATT_D;
-  const __nv_bfloat16* Kg = qkv + d_model + h * ATT_D;
-  const __nv_bfloat16* Vg = qkv + 2 * d_model + h * ATT_D;
+  const E* Qg = qkv + h * ATT_D;
+  const E* Kg = qkv + d_model + h * ATT_D;
+  const E* Vg = qkv + 2 * d_model + h * ATT_D;
 
   const int q_last = min(T, q0 + ATT_BQ) - 1;
   const int kv_lo = (q0 / W) * W;             // first key any row of the tile may see
@@ -118,8 +119,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
         const int ch = ks * 2 + (mi & 1);
         ldmatrix_x4(kb, sK + att_off(row, ch));
         uint32_t b0[2] = {kb[0], kb[1]}, b1[2] = {kb[2], kb[3]};
-        mma_bf16_16816(s[nt], qf[ks], b0);
-        mma_bf16_16816(s[nt + 1], qf[ks], b1);
+        F16<E>::mma(s[nt], qf[ks], b0);
+        F16<E>::mma(s[nt + 1], qf[ks], b1);
       }
     }
     // mask + row max
@@ -176,10 +177,10 @@ __global__ void __launch_bounds__(ATT_THREADS)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t a[4];
-      a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      a[0] = F16<E>::pack(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = F16<E>::pack(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = F16<E>::pack(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = F16<E>::pack(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int dt = 0; dt < 16; dt += 2) {
         uint32_t vb[4];
@@ -188,8 +189,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
         const int ch = dt + (mi >> 1);
         ldmatrix_x4_trans(vb, sV + att_off(row, ch));
         uint32_t b0[2] = {vb[0], vb[1]}, b1[2] = {vb[2], vb[3]};
-        mma_bf16_16816(o[dt], a, b0);
-        mma_bf16_16816(o[dt + 1], a, b1);
+        F16<E>::mma(o[dt], a, b0);
+        F16<E>::mma(o[dt + 1], a, b1);
       }
     }
     __syncthreads();  // buffer `buf` is refilled two iterations later
@@ -202,30 +203,40 @@ __global__ void __launch_bounds__(ATT_THREADS)
     const int col = h * ATT_D + dt * 8 + 2 * c;
     if (r0 < T)
       *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(r0) * ldo + col) =
-          pack_bf16(o[dt][0] * inv0, o[dt][1] * inv0);
+          F16<E>::pack(o[dt][0] * inv0, o[dt][1] * inv0);
     if (r1 < T)
       *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(r1) * ldo + col) =
-          pack_bf16(o[dt][2] * inv1, o[dt][3] * inv1);
+          F16<E>::pack(o[dt][2] * inv1, o[dt][3] * inv1);
   }
 }
 
 int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
-                     int window, cudaStream_t s) {
+                     int window, cudaStream_t s, int dtype) {
   if (T == 0) return KVA_OK;
   if (!qkv || !out || T < 0 || n_heads <= 0 || window < 0) return KVA_ERR_INVALID_ARG;
+  if (dtype != KVA_BF16 && dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   if ((ldq % 8) || (ldo % 8) ||
       ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15u))
     return KVA_ERR_ALIGNMENT;
   const int d_model = n_heads * ATT_D;
   if (ldq < 3 * d_model || ldo < d_model) return KVA_ERR_INVALID_ARG;
-  if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           ATT_SMEM) != cudaSuccess)
-    return KVA_ERR_CUDA;
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ATT_D));
   dim3 grid((T + ATT_BQ - 1) / ATT_BQ, n_heads);
-  attention_kernel<<<grid, ATT_THREADS, ATT_SMEM, s>>>(
-      static_cast<const __nv_bfloat16*>(qkv), ldq, static_cast<__nv_bfloat16*>(out), ldo, T,
-      d_model, window, scale_log2);
+  if (dtype == KVA_F16) {
+    if (cudaFuncSetAttribute(attention_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ATT_SMEM) != cudaSuccess)
+      return KVA_ERR_CUDA;
+    attention_kernel<__half><<<grid, ATT_THREADS, ATT_SMEM, s>>>(
+        static_cast<const __half*>(qkv), ldq, static_cast<__half*>(out), ldo, T, d_model, window,
+        scale_log2);
+  } else {
+    if (cudaFuncSetAttribute(attention_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) != cudaSuccess)
+      return KVA_ERR_CUDA;
+    attention_kernel<__nv_bfloat16><<<grid, ATT_THREADS, ATT_SMEM, s>>>(
+        static_cast<const __nv_bfloat16*>(qkv), ldq, static_cast<__nv_bfloat16*>(out), ldo, T,
+        d_model, window, scale_log2);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 

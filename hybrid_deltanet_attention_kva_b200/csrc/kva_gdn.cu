@@ -16,83 +16,109 @@
 //    One CTA per (sequence, layer, v head); warp w owns state rows
 //    [16w, 16w+16) as mma.sync accumulators, so the state-dependent products
 //    (U and the update) are warp-local; K K^T, Tm and W = Tm diag(beta e^gam) K
-//    are shared per chunk.  Chunk contractions run on tensor cores with bf16
-//    operands and fp32 accumulation; the state stays fp32.
+//    are shared per chunk.  Chunk contractions run on tensor cores with fp16
+//    operands (every operand is bounded: unit keys, SiLU values, the inverse,
+//    the state) and fp32 accumulation; the state stays fp32.
 #include "kva_common.cuh"
 
 namespace kva {
 
 // ------------------------------------------------------------------ prepare
-constexpr int PREP_TT = 32;
-constexpr int PREP_THREADS = 128;
+// Each thread owns 8 consecutive channels (one 16-byte vector per token row) for
+// PREP_TT tokens: all raw rows are loaded up front, the conv runs in registers,
+// and the L2 norm of a q/k head is a shuffle reduction over the d_k/8 lanes that
+// hold it.  Blocks along x cover 2048 channels of one row, the last x-block of a
+// token group computes the gates.
+constexpr int PREP_TT = 16;
+constexpr int PREP_THREADS = 256;
+constexpr int PREP_CH = PREP_THREADS * 8;
 
-__device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
-
+template <typename TM>
 __global__ void __launch_bounds__(PREP_THREADS) gdn_prepare_kernel(const GdnLaunch p) {
   const int slot = blockIdx.z;  // seq * n_gdn + layer
   const int seq = slot / p.n_gdn, layer = slot % p.n_gdn;
   const int T = p.T;
-  const int t0 = blockIdx.x * PREP_TT;
+  const int t0 = blockIdx.y * PREP_TT;
   const int nt = min(PREP_TT, T - t0);
   const int C = p.C;
   const int nkdk = p.n_k * p.d_k;
-  const __nv_bfloat16* mix = static_cast<const __nv_bfloat16*>(p.mix) +
-                             seq * p.mix_seq_stride + p.layer_col[layer];
+  const TM* mix = static_cast<const TM*>(p.mix) + seq * p.mix_seq_stride + p.layer_col[layer];
   const int64_t ld = p.mix_ld;
+  const int n_cblk = (C + PREP_CH - 1) / PREP_CH;
 
-  if (blockIdx.y < C / 128) {
-    const int c = blockIdx.y * 128 + threadIdx.x;
-    const float* w = p.conv_w + (static_cast<int64_t>(layer) * C + c) * 4;
-    const float w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3];
-    const __nv_bfloat16* tail =
-        static_cast<const __nv_bfloat16*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * C + c;
-    auto raw = [&](int t) -> float {
-      return t >= 0 ? bf2f(mix[t * ld + c]) : bf2f(tail[(t + 3) * C]);
-    };
-    float e0 = raw(t0 - 3), e1 = raw(t0 - 2), e2 = raw(t0 - 1);
-    float z[PREP_TT];
+  if (static_cast<int>(blockIdx.x) < n_cblk) {
+    const int c0 = blockIdx.x * PREP_CH + threadIdx.x * 8;
+    const bool active = c0 < C;
+    const int cc = active ? c0 : 0;
+    const TM* tail = static_cast<const TM*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * C + cc;
+    // raw rows t0-3 .. t0+PREP_TT-1 of [tail; X] for these 8 channels
+    uint4 raw[PREP_TT + 3];
 #pragma unroll
-    for (int i = 0; i < PREP_TT; ++i) {
-      const float xv = i < nt ? bf2f(mix[(t0 + i) * ld + c]) : 0.f;
-      const float cv = w0 * e0 + w1 * e1 + w2 * e2 + w3 * xv;
-      z[i] = silu_f(cv);
-      e0 = e1;
-      e1 = e2;
-      e2 = xv;
+    for (int i = 0; i < PREP_TT + 3; ++i) {
+      const int t = t0 - 3 + i;
+      if (t < 0)
+        raw[i] = *reinterpret_cast<const uint4*>(tail + (t + 3) * C);
+      else if (t < T)
+        raw[i] = *reinterpret_cast<const uint4*>(mix + t * ld + cc);
+      else
+        raw[i] = make_uint4(0u, 0u, 0u, 0u);
     }
-    const bool is_qk = blockIdx.y * 128 < 2 * nkdk;
-    if (is_qk) {
-      __shared__ float red[PREP_TT][PREP_THREADS / 32];
-      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float w[8][4];
 #pragma unroll
-      for (int i = 0; i < PREP_TT; ++i) {
-        const float ss = warp_sum(z[i] * z[i]);
-        if (lane == 0) red[i][warp] = ss;
-      }
-      __syncthreads();
-      const int wph = p.d_k / 32;                 // warps per head
-      const int hw = (threadIdx.x / p.d_k) * wph;  // first warp of this head
-#pragma unroll
-      for (int i = 0; i < PREP_TT; ++i) {
-        float tot = 0.f;
-        for (int k = 0; k < wph; ++k) tot += red[i][hw + k];
-        z[i] *= rsqrtf(tot + p.eps);
-      }
+    for (int e = 0; e < 8; ++e) {
+      const float4 wv = *reinterpret_cast<const float4*>(p.conv_w + (static_cast<int64_t>(layer) * C + cc + e) * 4);
+      w[e][0] = wv.x;
+      w[e][1] = wv.y;
+      w[e][2] = wv.z;
+      w[e][3] = wv.w;
     }
+    const bool is_qk = c0 < 2 * nkdk;
+    const int hl = p.d_k / 8;  // lanes per q/k head
     const int64_t tbase = static_cast<int64_t>(slot) * T;
     __nv_bfloat16* dbg = static_cast<__nv_bfloat16*>(p.debug_qkv);
 #pragma unroll
     for (int i = 0; i < PREP_TT; ++i) {
-      if (i < nt) {
+      float z[8];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float2 x0 = F16<TM>::unpack((&raw[i].x)[e / 2]);
+        float2 x1 = F16<TM>::unpack((&raw[i + 1].x)[e / 2]);
+        float2 x2 = F16<TM>::unpack((&raw[i + 2].x)[e / 2]);
+        float2 x3 = F16<TM>::unpack((&raw[i + 3].x)[e / 2]);
+        z[e] = silu_f(w[e][0] * x0.x + w[e][1] * x1.x + w[e][2] * x2.x + w[e][3] * x3.x);
+        z[e + 1] = silu_f(w[e + 1][0] * x0.y + w[e + 1][1] * x1.y + w[e + 1][2] * x2.y +
+                          w[e + 1][3] * x3.y);
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += z[e] * z[e];
+      for (int o = 1; o < hl; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (is_qk) {
+        const float sc = rsqrtf(ss + p.eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] *= sc;
+      }
+      if (active && i < nt) {
         const int64_t t = tbase + t0 + i;
-        const __nv_bfloat16 zb = __float2bfloat16_rn(z[i]);
-        if (c >= 2 * nkdk) {
+        uint4 hv;
+        hv.x = pack_f16(z[0], z[1]);
+        hv.y = pack_f16(z[2], z[3]);
+        hv.z = pack_f16(z[4], z[5]);
+        hv.w = pack_f16(z[6], z[7]);
+        if (c0 >= 2 * nkdk) {
           const int nvdv = C - 2 * nkdk;
-          static_cast<__nv_bfloat16*>(p.vbuf)[t * nvdv + (c - 2 * nkdk)] = zb;
-        } else if (c >= nkdk) {
-          static_cast<__nv_bfloat16*>(p.kbuf)[t * nkdk + (c - nkdk)] = zb;
+          *reinterpret_cast<uint4*>(static_cast<__half*>(p.vbuf) + t * nvdv + (c0 - 2 * nkdk)) = hv;
+        } else if (c0 >= nkdk) {
+          *reinterpret_cast<uint4*>(static_cast<__half*>(p.kbuf) + t * nkdk + (c0 - nkdk)) = hv;
         }
-        if (dbg) dbg[t * C + c] = zb;
+        if (dbg) {
+          uint4 bv;
+          bv.x = pack_bf16(z[0], z[1]);
+          bv.y = pack_bf16(z[2], z[3]);
+          bv.z = pack_bf16(z[4], z[5]);
+          bv.w = pack_bf16(z[6], z[7]);
+          *reinterpret_cast<uint4*>(dbg + t * C + c0) = bv;
+        }
       }
     }
   } else {
@@ -104,8 +130,8 @@ __global__ void __launch_bounds__(PREP_THREADS) gdn_prepare_kernel(const GdnLaun
     for (int idx = threadIdx.x; idx < nt * n_v; idx += PREP_THREADS) {
       const int i = idx / n_v, h = idx - i * n_v;
       const int t = t0 + i;
-      const float a = bf2f(mix[t * ld + C + h]);
-      const float b = bf2f(mix[t * ld + C + n_v + h]);
+      const float a = F16<TM>::to(mix[t * ld + C + h]);
+      const float b = F16<TM>::to(mix[t * ld + C + n_v + h]);
       const float x = a + dt_bias[h];
       const float sp = x > 20.f ? x : log1pf(expf(x));
       gb[h * T + t] = -expf(A_log[h]) * sp;
@@ -114,19 +140,19 @@ __global__ void __launch_bounds__(PREP_THREADS) gdn_prepare_kernel(const GdnLaun
   }
 }
 
+// The tail holds raw 16-bit values: a bit copy, whatever their format.
 __global__ void gdn_tail_kernel(const GdnLaunch p) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= p.C) return;
   const int slot = blockIdx.y;
   const int seq = slot / p.n_gdn, layer = slot % p.n_gdn;
-  const __nv_bfloat16* mix = static_cast<const __nv_bfloat16*>(p.mix) +
-                             seq * p.mix_seq_stride + p.layer_col[layer] + c;
-  __nv_bfloat16* tail =
-      static_cast<__nv_bfloat16*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * p.C + c;
+  const uint16_t* mix = static_cast<const uint16_t*>(p.mix) + seq * p.mix_seq_stride +
+                        p.layer_col[layer] + c;
+  uint16_t* tail = static_cast<uint16_t*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * p.C + c;
   // new tail row i is row T+i of [old tail; X]; ascending i reads only rows > i
   for (int i = 0; i < 3; ++i) {
     const int src = p.T + i;
-    const __nv_bfloat16 v = src >= 3 ? mix[static_cast<int64_t>(src - 3) * p.mix_ld] : tail[src * p.C];
+    const uint16_t v = src >= 3 ? mix[static_cast<int64_t>(src - 3) * p.mix_ld] : tail[src * p.C];
     tail[i * p.C] = v;
   }
 }
@@ -187,10 +213,10 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
   const int T = p.T;
   const int slot = seq * p.n_gdn + layer;
   const int nkdk = p.n_k * D, nvdv = n_v * D;
-  const __nv_bfloat16* kg =
-      static_cast<const __nv_bfloat16*>(p.kbuf) + static_cast<int64_t>(slot) * T * nkdk + kh * D;
-  const __nv_bfloat16* vg =
-      static_cast<const __nv_bfloat16*>(p.vbuf) + static_cast<int64_t>(slot) * T * nvdv + h * D;
+  const __half* kg =
+      static_cast<const __half*>(p.kbuf) + static_cast<int64_t>(slot) * T * nkdk + kh * D;
+  const __half* vg =
+      static_cast<const __half*>(p.vbuf) + static_cast<int64_t>(slot) * T * nvdv + h * D;
   const float* gg = p.gbuf + static_cast<int64_t>(slot) * 2 * n_v * T + h * T;
   const float* bg = gg + static_cast<int64_t>(n_v) * T;
   float* Sg = p.state + (static_cast<int64_t>(slot) * n_v + h) * D * D;
@@ -248,8 +274,8 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
         uint32_t b[4];
         ldmatrix_x4(b, sK + sw_off((nb_a + j) * 8 + (mi >> 1) * 8 + lr, ks * 2 + (mi & 1), RB));
         uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
-        mma_bf16_16816(acc[j], a, b0);
-        mma_bf16_16816(acc[j + 1], a, b1);
+        mma_f16_16816(acc[j], a, b0);
+        mma_f16_16816(acc[j + 1], a, b1);
       }
     }
     if (warp == 0) {
@@ -331,9 +357,9 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
       const float x1 = upper ? 0.f : Tf[t * LD + s + 1];
       const float b0 = bs[s], b1 = bs[s + 1];
       const uint32_t off = static_cast<uint32_t>(t * 128 + (((s >> 3) ^ (t & 7)) << 4) + (s & 7) * 2);
-      *reinterpret_cast<uint32_t*>(sm + SM::OFF_TB + off) = pack_bf16(x0 * b0, x1 * b1);
+      *reinterpret_cast<uint32_t*>(sm + SM::OFF_TB + off) = pack_f16(x0 * b0, x1 * b1);
       *reinterpret_cast<uint32_t*>(sm + SM::OFF_TBG + off) =
-          pack_bf16(x0 * b0 * Gam[s], x1 * b1 * Gam[s + 1]);
+          pack_f16(x0 * b0 * Gam[s], x1 * b1 * Gam[s + 1]);
     }
     __syncthreads();
 
@@ -363,10 +389,10 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
           const uint32_t off = sw_off(m * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), 128);
           ldmatrix_x4(a, sTB + off);
           ldmatrix_x4(ag, sTBG + off);
-          mma_bf16_16816(U[m][0], a, bv0);
-          mma_bf16_16816(U[m][1], a, bv1);
-          mma_bf16_16816(Wt[m][0], ag, bk0);
-          mma_bf16_16816(Wt[m][1], ag, bk1);
+          mma_f16_16816(U[m][0], a, bv0);
+          mma_f16_16816(U[m][1], a, bv1);
+          mma_f16_16816(Wt[m][0], ag, bk0);
+          mma_f16_16816(Wt[m][1], ag, bk1);
         }
       }
 #pragma unroll
@@ -376,9 +402,9 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
           const int ch = warp * 2 + n;
           const int r0 = m * 16 + g;
           *reinterpret_cast<uint32_t*>(sm + SM::OFF_W + sw_off(r0, ch, RB) + 4 * c) =
-              pack_bf16(-Wt[m][n][0], -Wt[m][n][1]);
+              pack_f16(-Wt[m][n][0], -Wt[m][n][1]);
           *reinterpret_cast<uint32_t*>(sm + SM::OFF_W + sw_off(r0 + 8, ch, RB) + 4 * c) =
-              pack_bf16(-Wt[m][n][2], -Wt[m][n][3]);
+              pack_f16(-Wt[m][n][2], -Wt[m][n][3]);
         }
     }
     __syncthreads();
@@ -388,8 +414,8 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
       uint32_t sb[D / 8][2];
 #pragma unroll
       for (int nt = 0; nt < D / 8; ++nt) {
-        sb[nt][0] = pack_bf16(S[nt][0], S[nt][1]);
-        sb[nt][1] = pack_bf16(S[nt][2], S[nt][3]);
+        sb[nt][0] = pack_f16(S[nt][0], S[nt][1]);
+        sb[nt][1] = pack_f16(S[nt][2], S[nt][3]);
       }
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -399,8 +425,8 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
         for (int m = 0; m < 4; ++m) {
           uint32_t a[4];
           ldmatrix_x4(a, sW + sw_off(m * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), RB));
-          mma_bf16_16816(U[m][0], a, b0);
-          mma_bf16_16816(U[m][1], a, b1);
+          mma_f16_16816(U[m][0], a, b0);
+          mma_f16_16816(U[m][1], a, b1);
         }
       }
     }
@@ -416,17 +442,17 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
       for (int m = 0; m < 4; ++m) {
         const float d0 = dec[m * 16 + g], d1 = dec[m * 16 + 8 + g];
         uint32_t a[4];
-        a[0] = movmatrix_trans(pack_bf16(U[m][0][0] * d0, U[m][0][1] * d0));
-        a[1] = movmatrix_trans(pack_bf16(U[m][1][0] * d0, U[m][1][1] * d0));
-        a[2] = movmatrix_trans(pack_bf16(U[m][0][2] * d1, U[m][0][3] * d1));
-        a[3] = movmatrix_trans(pack_bf16(U[m][1][2] * d1, U[m][1][3] * d1));
+        a[0] = movmatrix_trans(pack_f16(U[m][0][0] * d0, U[m][0][1] * d0));
+        a[1] = movmatrix_trans(pack_f16(U[m][1][0] * d0, U[m][1][1] * d0));
+        a[2] = movmatrix_trans(pack_f16(U[m][0][2] * d1, U[m][0][3] * d1));
+        a[3] = movmatrix_trans(pack_f16(U[m][1][2] * d1, U[m][1][3] * d1));
 #pragma unroll
         for (int nt = 0; nt < D / 8; nt += 2) {
           uint32_t b[4];
           ldmatrix_x4_trans(b, sK + sw_off(m * 16 + (mi & 1) * 8 + lr, nt + (mi >> 1), RB));
           uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
-          mma_bf16_16816(S[nt], a, b0);
-          mma_bf16_16816(S[nt + 1], a, b1);
+          mma_f16_16816(S[nt], a, b0);
+          mma_f16_16816(S[nt + 1], a, b1);
         }
       }
     }
@@ -452,6 +478,10 @@ static int check_gdn(const GdnLaunch& g) {
   if (g.d_k != g.d_v || (g.d_k != 64 && g.d_k != 128)) return KVA_ERR_UNSUPPORTED;
   if (g.n_k <= 0 || g.n_v % g.n_k) return KVA_ERR_UNSUPPORTED;
   if (g.C % 128 || (g.n_k * g.d_k) % 128) return KVA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(g.mix) | reinterpret_cast<uintptr_t>(g.conv_state) |
+       reinterpret_cast<uintptr_t>(g.conv_w)) & 15u)
+    return KVA_ERR_ALIGNMENT;
+  if (g.mix_ld % 8) return KVA_ERR_ALIGNMENT;
   return KVA_OK;
 }
 
@@ -459,8 +489,14 @@ int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s) {
   if (g.T == 0 || g.n_gdn == 0 || g.n_seq == 0) return KVA_OK;
   int e = check_gdn(g);
   if (e) return e;
-  dim3 grid((g.T + PREP_TT - 1) / PREP_TT, g.C / 128 + 1, g.n_seq * g.n_gdn);
-  gdn_prepare_kernel<<<grid, PREP_THREADS, 0, s>>>(g);
+  // channel blocks vary fastest, so the blocks in flight read whole row segments
+  dim3 grid((g.C + PREP_CH - 1) / PREP_CH + 1, (g.T + PREP_TT - 1) / PREP_TT, g.n_seq * g.n_gdn);
+  if (g.mix_dtype == KVA_F16)
+    gdn_prepare_kernel<__half><<<grid, PREP_THREADS, 0, s>>>(g);
+  else if (g.mix_dtype == KVA_BF16)
+    gdn_prepare_kernel<__nv_bfloat16><<<grid, PREP_THREADS, 0, s>>>(g);
+  else
+    return KVA_ERR_INVALID_ARG;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 

@@ -19,6 +19,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 
 #include "kva_common.cuh"
 
@@ -49,23 +50,24 @@ struct GemmParams {
   int* err;
 };
 
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v, int valid) {
+template <typename T>
+__device__ __forceinline__ void store16x32(T* dst, const float* v, int valid) {
   if (valid >= 32) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 pk;
-      pk.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-      pk.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-      pk.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-      pk.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      pk.x = F16<T>::pack(v[8 * q + 0], v[8 * q + 1]);
+      pk.y = F16<T>::pack(v[8 * q + 2], v[8 * q + 3]);
+      pk.z = F16<T>::pack(v[8 * q + 4], v[8 * q + 5]);
+      pk.w = F16<T>::pack(v[8 * q + 6], v[8 * q + 7]);
       reinterpret_cast<uint4*>(dst)[q] = pk;
     }
   } else {
-    for (int i = 0; i < valid; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+    for (int i = 0; i < valid; ++i) dst[i] = F16<T>::from(v[i]);
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, typename T>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                    const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, BN);
+      constexpr uint32_t idesc = idesc_f16kind_f32(Cfg::BM, BN, F16<T>::umma_fmt);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -272,8 +274,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + row * p.ldd + col;
-            store_bf16x32(dst, v, p.N - col);
+            T* dst = reinterpret_cast<T*>(p.D) + row * p.ldd + col;
+            store16x32<T>(dst, v, p.N - col);
           }
         }
       } else {
@@ -296,7 +298,7 @@ __global__ void __launch_bounds__(192, 1)
               float v[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-              store_bf16x32(reinterpret_cast<__nv_bfloat16*>(base) + row * ld + col, v, valid);
+              store16x32<T>(reinterpret_cast<T*>(base) + row * ld + col, v, valid);
             } else {
               float* dst = reinterpret_cast<float*>(base) + row * ld + col;
               if (valid == 32) {
@@ -354,16 +356,16 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// bf16 row-major [rows, inner] with row stride `ld` elements; box [box_rows, 64].
+// 16-bit row-major [rows, inner] with row stride `ld` elements; box [box_rows, 64].
 static bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld,
-                     int box_rows) {
+                     int box_rows, CUtensorMapDataType dt) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -376,18 +378,20 @@ int num_sms() {
   return n;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, typename T>
 static int launch_instance(const GemmArgs& a, cudaStream_t s) {
+  const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   using Cfg = GemmCfg<BN>;
   const bool paired = a.b_mode == B_PAIRED;
   const int box_b = paired ? BN / 2 : BN;
   CUtensorMap mA, mB[3];
-  if (!make_map(&mA, a.A, a.K, a.M, a.lda, Cfg::BM)) return KVA_ERR_CUDA;
+  if (!make_map(&mA, a.A, a.K, a.M, a.lda, Cfg::BM, dt)) return KVA_ERR_CUDA;
   const int nb = a.b_mode == B_SINGLE ? 1 : (paired ? 2 : 3);
   const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
   for (int i = 0; i < 3; ++i) {
     const void* src = a.B[i < nb ? i : 0];
-    if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, box_b)) return KVA_ERR_CUDA;
+    if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, box_b, dt)) return KVA_ERR_CUDA;
   }
   GemmParams p;
   p.M = a.M;
@@ -404,7 +408,7 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
   const int n_per_tile = paired ? BN / 2 : BN;
   const int tiles = ((a.M + Cfg::BM - 1) / Cfg::BM) * ((a.N + n_per_tile - 1) / n_per_tile);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  auto kern = gemm_tc_kernel<BN, EPI>;
+  auto kern = gemm_tc_kernel<BN, EPI, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
@@ -442,22 +446,23 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s) {
     if (a.seg_rows <= 0 || a.seg_rows % bn || a.N != 3 * a.seg_rows) return KVA_ERR_UNSUPPORTED;
   }
   if (bn != 128 && bn != 256) return KVA_ERR_UNSUPPORTED;
+  if (a.dtype != KVA_BF16 && a.dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
+  const bool h = a.dtype == KVA_F16;
+#define KVA_GEMM_CASE(E)                                                                   \
+  case E:                                                                                  \
+    if (h) return bn == 256 ? launch_instance<256, E, __half>(a, s)                        \
+                            : launch_instance<128, E, __half>(a, s);                       \
+    return bn == 256 ? launch_instance<256, E, __nv_bfloat16>(a, s)                        \
+                     : launch_instance<128, E, __nv_bfloat16>(a, s);
   switch (a.epilogue) {
-    case EPI_STORE_BF16:
-      return bn == 256 ? launch_instance<256, EPI_STORE_BF16>(a, s)
-                       : launch_instance<128, EPI_STORE_BF16>(a, s);
-    case EPI_STORE_F32:
-      return bn == 256 ? launch_instance<256, EPI_STORE_F32>(a, s)
-                       : launch_instance<128, EPI_STORE_F32>(a, s);
-    case EPI_ADD_F32:
-      return bn == 256 ? launch_instance<256, EPI_ADD_F32>(a, s)
-                       : launch_instance<128, EPI_ADD_F32>(a, s);
-    case EPI_SWIGLU_BF16:
-      return bn == 256 ? launch_instance<256, EPI_SWIGLU_BF16>(a, s)
-                       : launch_instance<128, EPI_SWIGLU_BF16>(a, s);
+    KVA_GEMM_CASE(EPI_STORE_BF16)
+    KVA_GEMM_CASE(EPI_STORE_F32)
+    KVA_GEMM_CASE(EPI_ADD_F32)
+    KVA_GEMM_CASE(EPI_SWIGLU_BF16)
     default:
       return KVA_ERR_INVALID_ARG;
   }
+#undef KVA_GEMM_CASE
 }
 
 }  // namespace kva

@@ -9,10 +9,10 @@
 namespace kva {
 
 enum GemmEpilogue {
-  EPI_STORE_BF16 = 0,   // D = acc (bf16)
+  EPI_STORE_BF16 = 0,   // D = acc (in the 16-bit operand format)
   EPI_STORE_F32 = 1,    // D = acc (fp32)
   EPI_ADD_F32 = 2,      // D += acc (fp32 residual stream)
-  EPI_SWIGLU_BF16 = 3,  // D[:, j] = silu(gate_j) * up_j (bf16), gate/up rows from B0/B1
+  EPI_SWIGLU_BF16 = 3,  // D[:, j] = silu(gate_j) * up_j (16-bit), gate/up rows from B0/B1
 };
 
 enum GemmBMode {
@@ -36,18 +36,21 @@ struct GemmArgs {
   int M = 0, N = 0, K = 0;
   int epilogue = EPI_STORE_BF16;
   int block_n = 0;          // 0: choose
+  int dtype = KVA_BF16;     // 16-bit format of A, B and 16-bit outputs: KVA_BF16 or KVA_F16
   int* err = nullptr;       // device status word
 };
 
 int num_sms();
 int launch_gemm(const GemmArgs& a, cudaStream_t s);
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
-                   int64_t ldo, int rows, int n, float eps, cudaStream_t s);
+                   int64_t ldo, int rows, int n, float eps, cudaStream_t s,
+                   int out_dtype = KVA_BF16);
 int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
-                     int window, cudaStream_t s);
+                     int window, cudaStream_t s, int dtype = KVA_BF16);
 
 struct GdnLaunch {
-  const void* mix = nullptr;    // bf16 [n_seq, T, mix_ld]
+  int mix_dtype = KVA_BF16;     // format of the mixer inputs and of the conv tail
+  const void* mix = nullptr;    // 16-bit [n_seq, T, mix_ld]
   int64_t mix_ld = 0;
   int64_t mix_seq_stride = 0;   // elements between sequences
   int n_seq = 0, T = 0;
@@ -57,10 +60,10 @@ struct GdnLaunch {
   const float* conv_w = nullptr;
   const float* A_log = nullptr;
   const float* dt_bias = nullptr;
-  void* conv_state = nullptr;   // bf16 [n_seq, n_gdn, 3, C]
+  void* conv_state = nullptr;   // 16-bit [n_seq, n_gdn, 3, C]
   float* state = nullptr;       // fp32 [n_seq, n_gdn, n_v, d_v, d_k]
-  void* kbuf = nullptr;         // bf16 [n_seq, n_gdn, T, n_k*d_k]
-  void* vbuf = nullptr;         // bf16 [n_seq, n_gdn, T, n_v*d_v]
+  void* kbuf = nullptr;         // fp16 [n_seq, n_gdn, T, n_k*d_k]
+  void* vbuf = nullptr;         // fp16 [n_seq, n_gdn, T, n_v*d_v]
   float* gbuf = nullptr;        // fp32 [n_seq, n_gdn, 2, n_v, T] (g then beta)
   void* debug_qkv = nullptr;    // bf16 [n_seq, n_gdn, T, C] or null
   float eps = 1e-6f;
@@ -72,6 +75,7 @@ int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s);
 
 constexpr int kMaxSeqPos = 256;
 struct KvLaunch {
+  int mix_dtype = KVA_BF16;
   const void* mix = nullptr;
   int64_t mix_ld = 0;
   int64_t mix_seq_stride = 0;

@@ -11,6 +11,8 @@
 // K and V rows are written with one vector store per lane (coalesced rows of
 // 512 bytes); V is copied bit for bit.  Paged caches go through the page table,
 // an out-of-range entry skips the write and sets the device status word.
+#include <type_traits>
+
 #include "kva_common.cuh"
 
 namespace kva {
@@ -26,7 +28,7 @@ struct VecT<4> {
   using T = uint2;
 };
 
-template <int EPL>
+template <int EPL, typename TM, typename TC>
 __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
   using V = typename VecT<EPL>::T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -35,19 +37,28 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
   const int seq = blockIdx.z;
   const int ai = blockIdx.y / p.n_kv, hh = blockIdx.y % p.n_kv;
   const int d_h = p.d_h;
-  const __nv_bfloat16* row = static_cast<const __nv_bfloat16*>(p.mix) + seq * p.mix_seq_stride +
-                             static_cast<int64_t>(t) * p.mix_ld + p.layer_col[ai];
+  const TM* row = static_cast<const TM*>(p.mix) + seq * p.mix_seq_stride +
+                  static_cast<int64_t>(t) * p.mix_ld + p.layer_col[ai];
   const int dim0 = lane * EPL;
   V kv = *reinterpret_cast<const V*>(row + hh * d_h + dim0);
-  const V vv = *reinterpret_cast<const V*>(row + p.n_kv * d_h + hh * d_h + dim0);
+  V vv = *reinterpret_cast<const V*>(row + p.n_kv * d_h + hh * d_h + dim0);
   float k[EPL];
   {
     const uint32_t* u = reinterpret_cast<const uint32_t*>(&kv);
 #pragma unroll
     for (int i = 0; i < EPL / 2; ++i) {
-      const float2 f = unpack_bf16(u[i]);
+      const float2 f = F16<TM>::unpack(u[i]);
       k[2 * i] = f.x;
       k[2 * i + 1] = f.y;
+    }
+  }
+  if constexpr (!std::is_same<TM, TC>::value) {
+    // v is stored in the cache's format (a bit copy when the formats agree)
+    uint32_t* u = reinterpret_cast<uint32_t*>(&vv);
+#pragma unroll
+    for (int i = 0; i < EPL / 2; ++i) {
+      const float2 f = F16<TM>::unpack(u[i]);
+      u[i] = F16<TC>::pack(f.x, f.y);
     }
   }
   float ss = 0.f;
@@ -85,7 +96,7 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
   {
     uint32_t* u = reinterpret_cast<uint32_t*>(&ko);
 #pragma unroll
-    for (int i = 0; i < EPL / 2; ++i) u[i] = pack_bf16(k[2 * i], k[2 * i + 1]);
+    for (int i = 0; i < EPL / 2; ++i) u[i] = F16<TC>::pack(k[2 * i], k[2 * i + 1]);
   }
 
   int64_t rowidx;
@@ -105,8 +116,8 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
   } else {
     rowidx = (static_cast<int64_t>(seq) * p.n_kv + hh) * cc.max_pos + pos;
   }
-  __nv_bfloat16* kd = static_cast<__nv_bfloat16*>(cc.k[ai]) + rowidx * d_h + dim0;
-  __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(cc.v[ai]) + rowidx * d_h + dim0;
+  TC* kd = static_cast<TC*>(cc.k[ai]) + rowidx * d_h + dim0;
+  TC* vd = static_cast<TC*>(cc.v[ai]) + rowidx * d_h + dim0;
   *reinterpret_cast<V*>(kd) = ko;
   *reinterpret_cast<V*>(vd) = vv;
 }
@@ -123,11 +134,24 @@ int launch_kv_write(const KvLaunch& k, cudaStream_t s) {
     const int off = half / epl;
     if (off & (off - 1)) return KVA_ERR_UNSUPPORTED;  // xor pairing needs a power of two
   }
+  if ((k.mix_dtype != KVA_BF16 && k.mix_dtype != KVA_F16) ||
+      (k.cache.dtype != KVA_BF16 && k.cache.dtype != KVA_F16))
+    return KVA_ERR_INVALID_ARG;
   dim3 grid((k.T + 7) / 8, k.n_kv * k.n_attn, k.n_seq);
-  if (epl == 8)
-    kv_write_kernel<8><<<grid, 256, 0, s>>>(k);
-  else
-    kv_write_kernel<4><<<grid, 256, 0, s>>>(k);
+  const bool mh = k.mix_dtype == KVA_F16, ch = k.cache.dtype == KVA_F16;
+#define KVA_KV_LAUNCH(EPL, TM, TC) kv_write_kernel<EPL, TM, TC><<<grid, 256, 0, s>>>(k)
+  if (epl == 8) {
+    if (mh && ch) KVA_KV_LAUNCH(8, __half, __half);
+    else if (mh) KVA_KV_LAUNCH(8, __half, __nv_bfloat16);
+    else if (ch) KVA_KV_LAUNCH(8, __nv_bfloat16, __half);
+    else KVA_KV_LAUNCH(8, __nv_bfloat16, __nv_bfloat16);
+  } else {
+    if (mh && ch) KVA_KV_LAUNCH(4, __half, __half);
+    else if (mh) KVA_KV_LAUNCH(4, __half, __nv_bfloat16);
+    else if (ch) KVA_KV_LAUNCH(4, __nv_bfloat16, __half);
+    else KVA_KV_LAUNCH(4, __nv_bfloat16, __nv_bfloat16);
+  }
+#undef KVA_KV_LAUNCH
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 

@@ -1,4 +1,4 @@
-// RMSNorm rows -> bf16 ("Qwen3.8-27B-KVA" model card, architecture:
+// RMSNorm rows -> bf16 or fp16 ("Qwen3.8-27B-KVA" model card, architecture:
 // RMSNorm before the input Linear, before each attention and FFN sub-block, and
 // once before all heads).  out = x / sqrt(mean(x^2) + eps) * g, stats in fp32.
 // HBM-bound: one read of x (fp32 or bf16), one bf16 write; the second pass over
@@ -19,15 +19,21 @@ __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
   float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
   return make_float4(a.x, a.y, b.x, b.y);
 }
+template <>
+__device__ __forceinline__ float4 load4<__half>(const __half* p) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  float2 a = F16<__half>::unpack(u.x), b = F16<__half>::unpack(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, int64_t ldx,
                                                       const float* __restrict__ g,
-                                                      __nv_bfloat16* __restrict__ out,
-                                                      int64_t ldo, int n, float eps) {
+                                                      TO* __restrict__ out, int64_t ldo, int n,
+                                                      float eps) {
   const int row = blockIdx.x;
   const T* xr = x + row * ldx;
-  __nv_bfloat16* orow = out + row * ldo;
+  TO* orow = out + row * ldo;
   float ss = 0.f;
   for (int i = threadIdx.x * 4; i < n; i += blockDim.x * 4) {
     float4 v = load4<T>(xr + i);
@@ -48,29 +54,40 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, i
     float4 v = load4<T>(xr + i);
     float4 gg = *reinterpret_cast<const float4*>(g + i);
     uint2 o;
-    o.x = pack_bf16(v.x * scale * gg.x, v.y * scale * gg.y);
-    o.y = pack_bf16(v.z * scale * gg.z, v.w * scale * gg.w);
+    o.x = F16<TO>::pack(v.x * scale * gg.x, v.y * scale * gg.y);
+    o.y = F16<TO>::pack(v.z * scale * gg.z, v.w * scale * gg.w);
     *reinterpret_cast<uint2*>(orow + i) = o;
   }
 }
 
+template <typename TO>
+static void rms_dispatch(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
+                         int64_t ldo, int rows, int n, float eps, cudaStream_t s) {
+  TO* o = static_cast<TO*>(out);
+  if (x_dtype == KVA_F32)
+    rmsnorm_kernel<float, TO><<<rows, 256, 0, s>>>(static_cast<const float*>(x), ldx, g, o, ldo, n, eps);
+  else if (x_dtype == KVA_BF16)
+    rmsnorm_kernel<__nv_bfloat16, TO><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                            ldx, g, o, ldo, n, eps);
+  else
+    rmsnorm_kernel<__half, TO><<<rows, 256, 0, s>>>(static_cast<const __half*>(x), ldx, g, o, ldo,
+                                                     n, eps);
+}
+
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
-                   int64_t ldo, int rows, int n, float eps, cudaStream_t s) {
+                   int64_t ldo, int rows, int n, float eps, cudaStream_t s, int out_dtype) {
   if (rows == 0) return KVA_OK;
   if (!x || !g || !out || rows < 0 || n <= 0) return KVA_ERR_INVALID_ARG;
+  if (x_dtype != KVA_F32 && x_dtype != KVA_BF16 && x_dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
+  if (out_dtype != KVA_BF16 && out_dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   if (n % 4 || ldx % 4 || ldo % 4) return KVA_ERR_ALIGNMENT;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(g) |
        reinterpret_cast<uintptr_t>(out)) & 15u)
     return KVA_ERR_ALIGNMENT;
-  if (x_dtype == KVA_F32)
-    rmsnorm_kernel<float><<<rows, 256, 0, s>>>(static_cast<const float*>(x), ldx, g,
-                                                static_cast<__nv_bfloat16*>(out), ldo, n, eps);
-  else if (x_dtype == KVA_BF16)
-    rmsnorm_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                        ldx, g, static_cast<__nv_bfloat16*>(out),
-                                                        ldo, n, eps);
+  if (out_dtype == KVA_F16)
+    rms_dispatch<__half>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s);
   else
-    return KVA_ERR_INVALID_ARG;
+    rms_dispatch<__nv_bfloat16>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s);
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 

@@ -30,7 +30,8 @@ KVA_DEV_PAGE_OOB = 0x1
 KVA_DEV_WAIT_TIMEOUT = 0x2
 
 KVA_LAYER_GDN, KVA_LAYER_ATTN = 0, 1
-KVA_BF16, KVA_F32 = 0, 1
+KVA_BF16, KVA_F32, KVA_F16 = 0, 1, 2
+_DT = {torch.bfloat16: KVA_BF16, torch.float32: KVA_F32, torch.float16: KVA_F16}
 KVA_KV_CONTIGUOUS, KVA_KV_PAGED = 0, 1
 EPI_STORE_BF16, EPI_STORE_F32, EPI_ADD_F32, EPI_SWIGLU_BF16 = 0, 1, 2, 3
 B_SINGLE, B_SEGMENTS, B_PAIRED = 0, 1, 2
@@ -46,7 +47,7 @@ class KvaDims(C.Structure):
         ("gdn_d_v", C.c_int32), ("conv_k", C.c_int32), ("attn_n_kv", C.c_int32),
         ("attn_d_h", C.c_int32), ("rope_dims", C.c_int32), ("rope_theta", C.c_double),
         ("norm_eps", C.c_float), ("n_draft_cols", C.c_int32), ("max_T", C.c_int32),
-        ("max_seq", C.c_int32),
+        ("max_seq", C.c_int32), ("compute_dtype", C.c_int32),
     ]
 
 
@@ -66,7 +67,7 @@ class KvaKvCache(C.Structure):
     _fields_ = [("layout", C.c_int32), ("n_layers", C.c_int32),
                 ("k", C.c_void_p * MAX_LATE), ("v", C.c_void_p * MAX_LATE),
                 ("max_pos", C.c_int64), ("page_size", C.c_int32), ("n_pages", C.c_int32),
-                ("pages_per_seq", C.c_int32), ("page_table", C.c_void_p)]
+                ("pages_per_seq", C.c_int32), ("page_table", C.c_void_p), ("dtype", C.c_int32)]
 
 
 ST_NAMES = ("rmsnorm", "gemm_trunk", "attention", "gemm_heads", "gdn_prepare", "gdn_tail",
@@ -105,10 +106,10 @@ def _load() -> C.CDLL:
         "kva_profile_enable": (I32, [P, I32]),
         "kva_profile_read": (I32, [P, C.POINTER(KvaProfile)]),
         "kva_strerror": (C.c_char_p, [I32]),
-        "kva_op_rmsnorm": (I32, [P, I32, I64, P, P, I64, I32, I32, F32, P]),
-        "kva_op_gemm": (I32, [P, I64, C.POINTER(P), I32, I64, I64, P, I64, P, I64, I64, I32,
+        "kva_op_rmsnorm": (I32, [P, I32, I64, P, P, I32, I64, I32, I32, F32, P]),
+        "kva_op_gemm": (I32, [I32, P, I64, C.POINTER(P), I32, I64, I64, P, I64, P, I64, I64, I32,
                               I32, I32, I32, I32, P, P]),
-        "kva_op_attention": (I32, [P, I64, P, I64, I32, I32, I32, P]),
+        "kva_op_attention": (I32, [I32, P, I64, P, I64, I32, I32, I32, P]),
         "kva_op_gdn_scan": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "kva_gdn_layer_update_noalloc": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, F32, P]),
     }
@@ -157,8 +158,9 @@ def _check(status: int, what: str) -> None:
 
 
 # ----------------------------------------------------------------- structs
-def make_dims(geom, max_T: int, max_seq: int = 1) -> KvaDims:
-    """kva_dims from any object carrying the geometry attributes."""
+def make_dims(geom, max_T: int, max_seq: int = 1, dtype=torch.float16) -> KvaDims:
+    """kva_dims from any object carrying the geometry attributes; dtype is the
+    16-bit operand format of the projector (torch.float16 or torch.bfloat16)."""
     d = KvaDims()
     d.hidden, d.d_model, d.n_heads = geom.hidden, geom.d_model, geom.n_heads
     d.head_dim, d.ffn, d.n_blocks = geom.head_dim, geom.ffn, geom.n_blocks
@@ -173,6 +175,7 @@ def make_dims(geom, max_T: int, max_seq: int = 1) -> KvaDims:
     d.norm_eps = geom.norm_eps
     d.n_draft_cols = geom.n_draft * geom.hidden
     d.max_T, d.max_seq = max_T, max_seq
+    d.compute_dtype = _DT[dtype]
     return d
 
 
@@ -208,6 +211,7 @@ class KvCache:
                  page_size: int = 0, n_pages: int = 0):
         self._keep = list(k) + list(v)
         self.c = KvaKvCache()
+        self.c.dtype = _DT[k[0].dtype] if len(k) else KVA_BF16
         self.c.n_layers = len(k)
         for i, (kk, vv) in enumerate(zip(k, v)):
             self.c.k[i] = _ptr(kk)
@@ -243,7 +247,7 @@ def kva_prefill_ubatch(handle: int, residual: torch.Tensor, weights: Weights,
                        deltanet_state: torch.Tensor, conv_state: torch.Tensor,
                        kv: Optional[KvCache], pos: int, draft_out: Optional[torch.Tensor] = None,
                        mixer_out: Optional[torch.Tensor] = None, stream=None) -> None:
-    dt = KVA_F32 if residual.dtype == torch.float32 else KVA_BF16
+    dt = _DT[residual.dtype]
     _check(_lib.kva_prefill_ubatch(
         handle, _ptr(residual), dt, residual.shape[0], C.byref(weights.c), _ptr(deltanet_state),
         _ptr(conv_state), C.byref(kv.c) if kv is not None else None, int(pos), _ptr(draft_out),
@@ -291,9 +295,9 @@ def kva_profile_read(handle: int) -> Dict[str, Dict[str, float]]:
 def kva_op_rmsnorm(x: torch.Tensor, g: torch.Tensor, out: torch.Tensor, eps: float = 1e-6,
                    stream=None) -> None:
     rows, n = x.shape
-    dt = KVA_F32 if x.dtype == torch.float32 else KVA_BF16
-    _check(_lib.kva_op_rmsnorm(_ptr(x), dt, n, _ptr(g), _ptr(out), out.shape[1], rows, n,
-                               float(eps), _stream(stream)), "kva_op_rmsnorm")
+    _check(_lib.kva_op_rmsnorm(_ptr(x), _DT[x.dtype], n, _ptr(g), _ptr(out), _DT[out.dtype],
+                               out.shape[1], rows, n, float(eps), _stream(stream)),
+           "kva_op_rmsnorm")
 
 
 def kva_op_gemm(A: torch.Tensor, B: Sequence[torch.Tensor], D: torch.Tensor, *, N: int,
@@ -303,7 +307,7 @@ def kva_op_gemm(A: torch.Tensor, B: Sequence[torch.Tensor], D: torch.Tensor, *, 
     M, K = A.shape
     arr = (C.c_void_p * 3)(*([_ptr(b) for b in B] + [None] * (3 - len(B))))
     _check(_lib.kva_op_gemm(
-        _ptr(A), K, arr, b_mode, B[0].shape[1], seg_rows, _ptr(D), D.shape[1], _ptr(D1),
+        _DT[A.dtype], _ptr(A), K, arr, b_mode, B[0].shape[1], seg_rows, _ptr(D), D.shape[1], _ptr(D1),
         D1.shape[1] if D1 is not None else 0, n_split, M, N, K, epilogue, block_n, _ptr(err),
         _stream(stream)), "kva_op_gemm")
 
@@ -311,8 +315,8 @@ def kva_op_gemm(A: torch.Tensor, B: Sequence[torch.Tensor], D: torch.Tensor, *, 
 def kva_op_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, window: int,
                      stream=None) -> None:
     T = qkv.shape[0]
-    _check(_lib.kva_op_attention(_ptr(qkv), qkv.shape[1], _ptr(out), out.shape[1], T, n_heads,
-                                 window, _stream(stream)), "kva_op_attention")
+    _check(_lib.kva_op_attention(_DT[qkv.dtype], _ptr(qkv), qkv.shape[1], _ptr(out), out.shape[1],
+                                 T, n_heads, window, _stream(stream)), "kva_op_attention")
 
 
 def kva_op_gdn_scan(k: torch.Tensor, v: torch.Tensor, gb: torch.Tensor, state: torch.Tensor,

@@ -62,7 +62,7 @@ typedef enum kva_status {
 #define KVA_DEV_WAIT_TIMEOUT 0x2  /* a pipeline wait inside a kernel gave up */
 
 typedef enum kva_layer_type { KVA_LAYER_GDN = 0, KVA_LAYER_ATTN = 1 } kva_layer_type;
-typedef enum kva_dtype { KVA_BF16 = 0, KVA_F32 = 1 } kva_dtype;
+typedef enum kva_dtype { KVA_BF16 = 0, KVA_F32 = 1, KVA_F16 = 2 } kva_dtype;
 typedef enum kva_kv_layout { KVA_KV_CONTIGUOUS = 0, KVA_KV_PAGED = 1 } kva_kv_layout;
 
 /* Geometry.  The r3 projector of the model card is
@@ -92,28 +92,32 @@ typedef struct kva_dims {
   int32_t n_draft_cols; /* drafter output columns after the mixer columns (0 if none) */
   int32_t max_T;        /* largest ubatch the handle accepts */
   int32_t max_seq;      /* largest n_seq for kva_update_states */
+  int32_t compute_dtype;/* 16-bit operand format of the projector: KVA_BF16 or KVA_F16.  The
+                           projector matrices, every activation fed to a GEMM, the mixer
+                           inputs (mixer_out / mixer_in), the drafter outputs and the conv
+                           state are in this format; accumulation is fp32 throughout. */
 } kva_dims;
 
 /* Weights of one projector block (device pointers). */
 typedef struct kva_block_weights {
   const float* g_attn;  /* [d] RMSNorm gain before attention (effective gain, no +1) */
-  const void* Wq;       /* bf16 [d, d] */
-  const void* Wk;       /* bf16 [d, d] */
-  const void* Wv;       /* bf16 [d, d] */
-  const void* Wo;       /* bf16 [d, d] */
+  const void* Wq;       /* [d, d] in compute_dtype (bf16 or fp16), like every matrix below */
+  const void* Wk;       /* [d, d] */
+  const void* Wv;       /* [d, d] */
+  const void* Wo;       /* [d, d] */
   const float* g_ffn;   /* [d] RMSNorm gain before the FFN */
-  const void* Wg;       /* bf16 [ffn, d] gate */
-  const void* Wu;       /* bf16 [ffn, d] up */
-  const void* Wd;       /* bf16 [d, ffn] down */
+  const void* Wg;       /* [ffn, d] gate */
+  const void* Wu;       /* [ffn, d] up */
+  const void* Wd;       /* [d, ffn] down */
 } kva_block_weights;
 
 /* Projector weights and the late layers' own parameters (device pointers). */
 typedef struct kva_weights {
   const float* g_in;    /* [H] input RMSNorm gain */
-  const void* W_in;     /* bf16 [d, H] */
+  const void* W_in;     /* [d, H], compute_dtype */
   kva_block_weights blocks[KVA_MAX_BLOCKS];
   const float* g_out;   /* [d] output RMSNorm gain */
-  const void* W_heads;  /* bf16 [n_mix + n_draft_cols, d]: the heads of all late layers
+  const void* W_heads;  /* [n_mix + n_draft_cols, d], compute_dtype: the heads of all late layers
                            concatenated in layer order, then the drafter heads.  Per GDN
                            layer the rows are [q (n_k*d_k) | k (n_k*d_k) | v (n_v*d_v) |
                            a (n_v) | b (n_v)], per attention layer [k (n_kv*d_h) | v (n_kv*d_h)]. */
@@ -139,6 +143,7 @@ typedef struct kva_kv_cache {
   int32_t n_pages;           /* PAGED: pages in each layer's pool */
   int32_t pages_per_seq;     /* PAGED: columns of page_table */
   const int32_t* page_table; /* PAGED: [n_seq, pages_per_seq] */
+  int32_t dtype;             /* element format of the caches: KVA_BF16 or KVA_F16 */
 } kva_kv_cache;
 
 typedef struct kva_handle kva_handle;
@@ -151,15 +156,15 @@ int kva_init(const kva_dims* dims, kva_handle** out);
 size_t kva_workspace_bytes(const kva_dims* dims);
 
 /* One ubatch of one sequence: projector + all state updates.
- *   residual       [T, H] in residual_dtype (KVA_BF16 or KVA_F32)
+ *   residual       [T, H] in residual_dtype (KVA_BF16, KVA_F16 or KVA_F32)
  *   T              1..max_T tokens
  *   deltanet_state fp32 [n_gdn, n_v, d_v, d_k], read and updated in place
- *   conv_state     bf16 [n_gdn, conv_k-1, C], the last raw conv inputs (oldest
+ *   conv_state     compute_dtype [n_gdn, conv_k-1, C], the last raw conv inputs (oldest
  *                  first), read and updated in place
  *   kv             caches written at positions pos .. pos+T-1 (sequence 0)
  *   pos            absolute position of the first token (RoPE angle and cache row)
- *   draft_out      bf16 [T, n_draft_cols] or NULL (drafter outputs)
- *   mixer_out      bf16 [T, n_mix] or NULL: when given, the mixer inputs are written
+ *   draft_out      compute_dtype [T, n_draft_cols] or NULL (drafter outputs)
+ *   mixer_out      compute_dtype [T, n_mix] or NULL: when given, the mixer inputs are written
  *                  there (and read back by the state updates) instead of the workspace */
 int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dtype,
                        int32_t T, const kva_weights* w, float* deltanet_state,
@@ -167,10 +172,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
                        void* draft_out, void* mixer_out, void* stream);
 
 /* State updates only, for n_seq independent sequences of T tokens each.
- *   mixer_in  bf16 [n_seq, T, mixer_ld] (the first n_mix columns are used)
+ *   mixer_in  compute_dtype [n_seq, T, mixer_ld] (the first n_mix columns are used)
  *   pos       HOST int64 [n_seq], first position of each sequence's ubatch
  *   state     fp32 [n_seq, n_gdn, n_v, d_v, d_k], in place
- *   conv_state bf16 [n_seq, n_gdn, conv_k-1, C], in place
+ *   conv_state compute_dtype [n_seq, n_gdn, conv_k-1, C], in place
  *   debug_qkv bf16 [n_seq, n_gdn, T, 2*n_k*d_k + n_v*d_v] or NULL: when given,
  *             receives [q_hat | k_hat | v] after conv, SiLU and the L2 norms
  *   debug_gb  fp32 [n_seq, n_gdn, 2, n_v, T] or NULL: receives g then beta */

@@ -20,10 +20,10 @@ extern "C" {
 #endif
 
 typedef enum kva_epilogue {
-  KVA_EPI_STORE_BF16 = 0,  /* D = A B^T, bf16 */
+  KVA_EPI_STORE_BF16 = 0,  /* D = A B^T, in the operands' 16-bit format */
   KVA_EPI_STORE_F32 = 1,   /* D = A B^T, fp32 */
   KVA_EPI_ADD_F32 = 2,     /* D += A B^T, fp32 (the projector's residual stream) */
-  KVA_EPI_SWIGLU_BF16 = 3  /* D = silu(A Bg^T) * (A Bu^T), bf16 (SwiGLU FFN, model card table) */
+  KVA_EPI_SWIGLU_BF16 = 3  /* D = silu(A Bg^T) * (A Bu^T), 16-bit (SwiGLU FFN, model card table) */
 } kva_epilogue;
 
 typedef enum kva_b_mode {
@@ -33,33 +33,36 @@ typedef enum kva_b_mode {
 } kva_b_mode;
 
 /* RMSNorm of `rows` rows of width n ("Qwen3.8-27B-KVA" model card, architecture):
- * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out bf16 [rows, ldo].
+ * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out [rows, ldo] in out_dtype (bf16 / fp16).
  * x is [rows, ldx] in x_dtype.  n, ldx, ldo multiples of 4; pointers 16-byte aligned. */
 int kva_op_rmsnorm(const void* x, int32_t x_dtype, int64_t ldx, const float* g, void* out,
-                   int64_t ldo, int32_t rows, int32_t n, float eps, void* stream);
+                   int32_t out_dtype, int64_t ldo, int32_t rows, int32_t n, float eps,
+                   void* stream);
 
 /* D = A B^T with an epilogue on tcgen05 tensor cores (the projector's linears).
- *   A     bf16 [M, K], row stride lda
+ *   dtype 16-bit format of A, B and of 16-bit outputs: KVA_BF16 or KVA_F16
+ *   A     [M, K], row stride lda
  *   B     HOST array of 1..3 device pointers per b_mode, each with row stride ldb
  *   D     output [M, ldd] (bf16 or fp32 per epilogue); with n_split > 0 columns
  *         >= n_split go to D1 [M, ldd1] at column - n_split (n_split % 32 == 0)
  *   block_n 0 (choose), 128 or 256
  * K, lda, ldb multiples of 8; seg_rows a multiple of the chosen block_n. */
-int kva_op_gemm(const void* A, int64_t lda, const void* const* B, int32_t b_mode, int64_t ldb,
-                int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1, int64_t n_split,
-                int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t block_n, int32_t* err,
-                void* stream);
+int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B, int32_t b_mode,
+                int64_t ldb, int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1,
+                int64_t n_split, int32_t M, int32_t N, int32_t K, int32_t epilogue,
+                int32_t block_n, int32_t* err, void* stream);
 
 /* Block-causal multi-head attention of the projector (model card table row
- * "attention"): qkv bf16 [T, ldq] holds q | k | v, each n_heads x 128 wide;
- * out bf16 [T, ldo] gets the n_heads x 128 head outputs.  Key j is visible to
- * query i iff j <= i and i / window == j / window (window 0: plain causal). */
-int kva_op_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int32_t T,
-                     int32_t n_heads, int32_t window, void* stream);
+ * "attention"): qkv [T, ldq] holds q | k | v, each n_heads x 128 wide;
+ * out [T, ldo] gets the n_heads x 128 head outputs, both in dtype (bf16 / fp16).
+ * Key j is visible to query i iff j <= i and i / window == j / window (window 0:
+ * plain causal). */
+int kva_op_attention(int32_t dtype, const void* qkv, int64_t ldq, void* out, int64_t ldo,
+                     int32_t T, int32_t n_heads, int32_t window, void* stream);
 
 /* Gated delta-rule scan alone, for n_seq x n_layers independent problems of T tokens:
- *   k     bf16 [n_seq*n_layers, T, n_k*d]  (unit-norm keys)
- *   v     bf16 [n_seq*n_layers, T, n_v*d]
+ *   k     fp16 [n_seq*n_layers, T, n_k*d]  (unit-norm keys)
+ *   v     fp16 [n_seq*n_layers, T, n_v*d]
  *   gb    fp32 [n_seq*n_layers, 2, n_v, T] (g then beta per v head)
  *   state fp32 [n_seq*n_layers, n_v, d, d] read and updated in place
  * v head h reads k head h / (n_v / n_k).  d = 64 or 128. */

@@ -83,6 +83,9 @@ def test_workspace_and_strerror_without_gpu():
     bad = K.make_dims(KI.R3, 1024, 1)
     bad.layer_type[0] = 7
     assert K.kva_workspace_bytes(bad) == 0
+    bad = K.make_dims(KI.R3, 1024, 1)
+    bad.compute_dtype = K.KVA_F32                     # operands must be 16-bit
+    assert K.kva_workspace_bytes(bad) == 0
     assert K.kva_strerror(K.KVA_ERR_TOO_LARGE).startswith("size beyond")
     assert K.kva_strerror(12345) == "unknown status"
 
@@ -106,14 +109,18 @@ def test_host_validation_rejects_before_any_launch():
     s = C.c_int32()
     assert L.kva_get_device_status(None, C.byref(s)) == K.KVA_ERR_INVALID_ARG
     # per-step ops: misaligned / invalid shapes are refused on the host
-    assert L.kva_op_rmsnorm(C.c_void_p(16), 1, 6, C.c_void_p(16), C.c_void_p(16), 6, 2, 6, 1e-6,
-                            None) == K.KVA_ERR_ALIGNMENT
+    assert L.kva_op_rmsnorm(C.c_void_p(16), 1, 6, C.c_void_p(16), C.c_void_p(16), 0, 6, 2, 6,
+                            1e-6, None) == K.KVA_ERR_ALIGNMENT
+    assert L.kva_op_rmsnorm(C.c_void_p(16), 1, 8, C.c_void_p(16), C.c_void_p(16), 1, 8, 2, 8,
+                            1e-6, None) == K.KVA_ERR_INVALID_ARG          # fp32 out: refused
     arr = (C.c_void_p * 3)(16, None, None)
-    assert L.kva_op_gemm(C.c_void_p(16), 12, arr, 0, 12, 0, C.c_void_p(16), 64, None, 0, 0,
+    assert L.kva_op_gemm(0, C.c_void_p(16), 12, arr, 0, 12, 0, C.c_void_p(16), 64, None, 0, 0,
                          64, 64, 12, 0, 0, None, None) == K.KVA_ERR_ALIGNMENT
-    assert L.kva_op_gemm(C.c_void_p(16), 64, arr, 5, 64, 0, C.c_void_p(16), 64, None, 0, 0,
+    assert L.kva_op_gemm(0, C.c_void_p(16), 64, arr, 5, 64, 0, C.c_void_p(16), 64, None, 0, 0,
                          64, 64, 64, 0, 0, None, None) == K.KVA_ERR_INVALID_ARG
-    assert L.kva_op_attention(C.c_void_p(16), 384, C.c_void_p(16), 128, 16, 1, -1, None) \
+    assert L.kva_op_gemm(1, C.c_void_p(16), 64, arr, 0, 64, 0, C.c_void_p(16), 64, None, 0, 0,
+                         64, 64, 64, 0, 0, None, None) == K.KVA_ERR_INVALID_ARG  # fp32 operands
+    assert L.kva_op_attention(0, C.c_void_p(16), 384, C.c_void_p(16), 128, 16, 1, -1, None) \
         == K.KVA_ERR_INVALID_ARG
     assert L.kva_op_gdn_scan(C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), 1,
                              1, 8, 1, 1, 96, None) == K.KVA_ERR_UNSUPPORTED

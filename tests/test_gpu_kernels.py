@@ -29,12 +29,13 @@ def _gen(seed):
 
 # ------------------------------------------------------------------ RMSNorm
 @pytest.mark.parametrize("dtype,rows,n", [(torch.float32, 37, 512), (torch.bfloat16, 129, 5120),
-                                          (torch.float32, 1024, 3072)])
-def test_rmsnorm(K, dtype, rows, n):
+                                          (torch.float32, 1024, 3072), (torch.float16, 64, 256)])
+@pytest.mark.parametrize("odt", [torch.bfloat16, torch.float16])
+def test_rmsnorm(K, dtype, rows, n, odt):
     g = _gen(rows)
     x = (torch.randn(rows, n, generator=g) * 3).to(dtype)
     gain = torch.rand(n, generator=g) + 0.5
-    out = torch.empty(rows, n, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(rows, n, dtype=odt, device="cuda")
     K.kva_op_rmsnorm(x.cuda(), gain.cuda(), out)
     torch.cuda.synchronize()
     want = R.rmsnorm(f64(x), f64(gain))
@@ -45,13 +46,14 @@ def test_rmsnorm(K, dtype, rows, n):
 @pytest.mark.parametrize("M,N,K_,bn", [(128, 256, 64, 256), (200, 1296, 520, 0), (1024, 3072, 3072, 128),
                                        (77, 512, 256, 256), (1024, 2560, 5120, 0)])
 @pytest.mark.parametrize("epi", [0, 1, 2])
-def test_gemm_epilogues(K, M, N, K_, bn, epi):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_gemm_epilogues(K, M, N, K_, bn, epi, dt):
     g = _gen(M * 7 + N + epi)
-    A = torch.randn(M, K_, generator=g).to(torch.bfloat16)
-    B = (torch.randn(N, K_, generator=g) * 0.05).to(torch.bfloat16)
+    A = torch.randn(M, K_, generator=g).to(dt)
+    B = (torch.randn(N, K_, generator=g) * 0.05).to(dt)
     want = R.projector_heads(f64(A), f64(B))
     if epi == K.EPI_STORE_BF16:
-        D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        D = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
     else:
         D = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
     D0 = None
@@ -65,12 +67,13 @@ def test_gemm_epilogues(K, M, N, K_, bn, epi):
 
 
 @pytest.mark.parametrize("M,F,K_", [(128, 704, 256), (1000, 1024, 512), (1024, 8448, 3072)])
-def test_gemm_swiglu_paired(K, M, F, K_):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_gemm_swiglu_paired(K, M, F, K_, dt):
     g = _gen(F)
-    A = torch.randn(M, K_, generator=g).to(torch.bfloat16)
-    Bg = (torch.randn(F, K_, generator=g) * 0.05).to(torch.bfloat16)
-    Bu = (torch.randn(F, K_, generator=g) * 0.05).to(torch.bfloat16)
-    D = torch.full((M, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    A = torch.randn(M, K_, generator=g).to(dt)
+    Bg = (torch.randn(F, K_, generator=g) * 0.05).to(dt)
+    Bu = (torch.randn(F, K_, generator=g) * 0.05).to(dt)
+    D = torch.full((M, F), float("nan"), dtype=dt, device="cuda")
     K.kva_op_gemm(A.cuda(), [Bg.cuda(), Bu.cuda()], D, N=F, epilogue=K.EPI_SWIGLU_BF16,
                   b_mode=K.B_PAIRED)
     torch.cuda.synchronize()
@@ -80,11 +83,12 @@ def test_gemm_swiglu_paired(K, M, F, K_):
 
 
 @pytest.mark.parametrize("M,d", [(300, 256), (1024, 3072)])
-def test_gemm_qkv_segments(K, M, d):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_gemm_qkv_segments(K, M, d, dt):
     g = _gen(d)
-    A = torch.randn(M, d, generator=g).to(torch.bfloat16)
-    Ws = [(torch.randn(d, d, generator=g) * 0.05).to(torch.bfloat16) for _ in range(3)]
-    D = torch.full((M, 3 * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    A = torch.randn(M, d, generator=g).to(dt)
+    Ws = [(torch.randn(d, d, generator=g) * 0.05).to(dt) for _ in range(3)]
+    D = torch.full((M, 3 * d), float("nan"), dtype=dt, device="cuda")
     K.kva_op_gemm(A.cuda(), [w.cuda() for w in Ws], D, N=3 * d, b_mode=K.B_SEGMENTS,
                   seg_rows=d, block_n=128)
     torch.cuda.synchronize()
@@ -121,11 +125,12 @@ def test_gemm_rejects_misaligned(K):
 # ------------------------------------------------------------------ attention
 @pytest.mark.parametrize("T,heads,window", [(128, 2, 0), (300, 3, 0), (1024, 4, 1024), (1024, 2, 256),
                                             (700, 2, 200), (1, 1, 0)])
-def test_attention(K, T, heads, window):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_attention(K, T, heads, window, dt):
     g = _gen(T + heads)
     d = heads * 128
-    qkv = torch.randn(T, 3 * d, generator=g).to(torch.bfloat16)
-    out = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qkv = torch.randn(T, 3 * d, generator=g).to(dt)
+    out = torch.full((T, d), float("nan"), dtype=dt, device="cuda")
     K.kva_op_attention(qkv.cuda(), out, heads, window)
     torch.cuda.synchronize()
     q = f64(qkv)
@@ -144,8 +149,8 @@ def _scan_inputs(seed, n_layers, T, n_k, n_v, d, g_scale=1.0, beta=None, gzero=F
     g = _gen(seed)
     k = torch.randn(n_layers, T, n_k, d, generator=g, dtype=torch.float64)
     k = k / k.norm(dim=-1, keepdim=True)
-    k = k.to(torch.bfloat16)
-    v = torch.randn(n_layers, T, n_v, d, generator=g).to(torch.bfloat16)
+    k = k.to(torch.float16)
+    v = torch.randn(n_layers, T, n_v, d, generator=g).to(torch.float16)
     gg = -torch.rand(n_layers, n_v, T, generator=g) * g_scale
     if gzero:
         gg.zero_()

