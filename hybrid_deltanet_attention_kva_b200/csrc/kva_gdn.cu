@@ -13,10 +13,11 @@
 //        L[t,s] = beta_t e^(gam_t-gam_s) k_t.k_s (s < t),  Tm = (I + L)^-1,
 //        U      = Tm diag(beta) V - Tm diag(beta e^gam) K S^T,
 //        S     <- e^gam_last S + (diag(e^(gam_last-gam)) U)^T K.
-//    One CTA per (sequence, layer, v head); warp w owns state rows
+//    One CTA per (sequence, layer, v head); state warp w owns state rows
 //    [16w, 16w+16) as mma.sync accumulators, so the state-dependent products
-//    (U and the update) are warp-local; K K^T, Tm and W = Tm diag(beta e^gam) K
-//    are shared per chunk.  Chunk contractions run on tensor cores with fp16
+//    (U and the update) are warp-local, while 4 prep warps build the chunk-local
+//    K K^T, Tm and W = Tm diag(beta e^gam) K one chunk ahead.  Chunk
+//    contractions run on tensor cores with fp16
 //    operands (every operand is bounded: unit keys, SiLU values, the inverse,
 //    the state) and fp32 accumulation; the state stays fp32.
 #include "kva_common.cuh"
@@ -34,7 +35,7 @@ constexpr int PREP_THREADS = 256;
 constexpr int PREP_CH = PREP_THREADS * 8;
 
 template <typename TM>
-__global__ void __launch_bounds__(PREP_THREADS) gdn_prepare_kernel(const GdnLaunch p) {
+__global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnLaunch p) {
   const int slot = blockIdx.z;  // seq * n_gdn + layer
   const int seq = slot / p.n_gdn, layer = slot % p.n_gdn;
   const int T = p.T;
@@ -52,17 +53,18 @@ __global__ void __launch_bounds__(PREP_THREADS) gdn_prepare_kernel(const GdnLaun
     const int cc = active ? c0 : 0;
     const TM* tail = static_cast<const TM*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * C + cc;
     // raw rows t0-3 .. t0+PREP_TT-1 of [tail; X] for these 8 channels
+    // every load is unconditional (pointer select, zero mask after) so that all
+    // PREP_TT + 3 of them are in flight together
     uint4 raw[PREP_TT + 3];
 #pragma unroll
     for (int i = 0; i < PREP_TT + 3; ++i) {
       const int t = t0 - 3 + i;
-      if (t < 0)
-        raw[i] = *reinterpret_cast<const uint4*>(tail + (t + 3) * C);
-      else if (t < T)
-        raw[i] = *reinterpret_cast<const uint4*>(mix + t * ld + cc);
-      else
-        raw[i] = make_uint4(0u, 0u, 0u, 0u);
+      const TM* src = t < 0 ? tail + (t + 3) * C : mix + static_cast<int64_t>(min(t, T - 1)) * ld + cc;
+      raw[i] = __ldg(reinterpret_cast<const uint4*>(src));
     }
+#pragma unroll
+    for (int i = 0; i < PREP_TT + 3; ++i)
+      if (t0 - 3 + i >= T) raw[i] = make_uint4(0u, 0u, 0u, 0u);
     float w[8][4];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -159,52 +161,72 @@ __global__ void gdn_tail_kernel(const GdnLaunch p) {
 
 // ------------------------------------------------------------------ scan
 constexpr int SCAN_CH = 64;
+constexpr int SCAN_PREP_WARPS = 4;
+constexpr int SCAN_PREP_THREADS = SCAN_PREP_WARPS * 32;
+constexpr uint64_t kScanWaitNs = 200000000ull;  // a chunk hand-off takes microseconds
 
-// byte offset of (row, 16-byte chunk) in a bf16 tile whose rows are `rb` bytes
+// byte offset of (row, 16-byte chunk) in a 16-bit tile whose rows are `rb` bytes
 __device__ __forceinline__ uint32_t sw_off(int row, int chunk, int rb) {
   return static_cast<uint32_t>(row * rb + ((chunk ^ (row & 7)) << 4));
 }
 
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit) return false;
+  }
+}
+
+__device__ __forceinline__ void prep_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(SCAN_PREP_THREADS) : "memory");
+}
+
 template <int D>
-struct ScanSmem {
-  static constexpr int KV_BYTES = SCAN_CH * D * 2;
-  static constexpr int TB_BYTES = SCAN_CH * SCAN_CH * 2;
-  static constexpr int LD = SCAN_CH + 1;
-  static constexpr int F_BYTES = SCAN_CH * LD * 4;
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_W = OFF_V + KV_BYTES;
-  static constexpr int OFF_TB = OFF_W + KV_BYTES;
-  static constexpr int OFF_TBG = OFF_TB + TB_BYTES;
-  static constexpr int OFF_L = OFF_TBG + TB_BYTES;
-  static constexpr int OFF_T = OFF_L + F_BYTES;
-  static constexpr int OFF_M = OFF_T + F_BYTES;
-  static constexpr int OFF_VEC = OFF_M + 3 * 256 * 4;
-  static constexpr int BYTES = OFF_VEC + 5 * SCAN_CH * 4;
+struct ScanLayout {
+  static constexpr int NSW = D / 16;  // state warps: 16 state rows each
+  static constexpr int NT = (NSW + SCAN_PREP_WARPS) * 32;
+  static constexpr int KVB = SCAN_CH * D * 2;        // one [64][D] fp16 tile
+  static constexpr int TBB = SCAN_CH * SCAN_CH * 2;  // one [64][64] fp16 tile
+  // one chunk buffer (prep -> state): K, -W = -Tm diag(beta e^gam) K, U0 = Tm diag(beta) V,
+  // decay vector and e^(gam_last)
+  static constexpr int B_K = 0;
+  static constexpr int B_W = KVB;
+  static constexpr int B_U = 2 * KVB;
+  static constexpr int B_DEC = 3 * KVB;
+  static constexpr int BUF = ((B_DEC + SCAN_CH * 4 + 16) + 127) / 128 * 128;
+  // prep-private
+  static constexpr int OFF_V = 2 * BUF;                // V of the chunk in preparation
+  static constexpr int OFF_LN = OFF_V + KVB;           // -L, fp16 [64][64]
+  static constexpr int OFF_TD = OFF_LN + TBB;          // diagonal blocks of Tm, fp16 [64][64]
+  static constexpr int OFF_LD = OFF_TD + TBB;          // diagonal blocks of L, fp32 [4][16][17]
+  static constexpr int OFF_G = OFF_LD + 4 * 16 * 17 * 4;  // g, beta, gam, e^gam
+  static constexpr int OFF_BAR = OFF_G + 4 * SCAN_CH * 4;
+  static constexpr int BYTES = OFF_BAR + 64;
 };
 
-template <int D>
-__global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
-  constexpr int NW = D / 16;
-  constexpr int NT = NW * 32;
-  constexpr int RB = 2 * D;  // bytes per K/V/W row
-  using SM = ScanSmem<D>;
-  extern __shared__ __align__(128) uint8_t sm[];
-  const uint32_t sK = smem_u32(sm + SM::OFF_K);
-  const uint32_t sV = smem_u32(sm + SM::OFF_V);
-  const uint32_t sW = smem_u32(sm + SM::OFF_W);
-  const uint32_t sTB = smem_u32(sm + SM::OFF_TB);
-  const uint32_t sTBG = smem_u32(sm + SM::OFF_TBG);
-  float* Lf = reinterpret_cast<float*>(sm + SM::OFF_L);
-  float* Tf = reinterpret_cast<float*>(sm + SM::OFF_T);
-  float* Mf = reinterpret_cast<float*>(sm + SM::OFF_M);
-  float* gs = reinterpret_cast<float*>(sm + SM::OFF_VEC);
-  float* bs = gs + SCAN_CH;
-  float* gam = bs + SCAN_CH;
-  float* Gam = gam + SCAN_CH;
-  float* dec = Gam + SCAN_CH;
-  constexpr int LD = SM::LD;
+__device__ __forceinline__ uint32_t ld_smem_u32(const uint8_t* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
 
+// One CTA per (sequence, layer, v head).  Warps [0, NSW) are state warps: warp w
+// holds state rows [16w, 16w+16) as mma.sync accumulators and, per chunk, forms
+// U = U0 + (-W) S^T for its rows and the update S <- e^gam_last S + (dec U)^T K.
+// The 4 prep warps run one chunk ahead: cumulative decays, L = beta e^(gam_t -
+// gam_s) K K^T (s < t), the 16x16 diagonal blocks of Tm = (I + L)^-1 by substitution
+// in registers, and then (I + L) X = [diag(beta) V | diag(beta e^gam) K] by block-row
+// forward substitution on tensor cores, each prep warp owning a quarter of the
+// columns (so the solve needs no cross-warp synchronisation).  Buffers change
+// hands through mbarriers (ready: prep -> state, free: state -> prep) with
+// time-bounded waits.
+template <int D>
+__global__ void __launch_bounds__(ScanLayout<D>::NT, 1) gdn_scan_kernel(const GdnLaunch p) {
+  using L = ScanLayout<D>;
+  constexpr int NSW = L::NSW;
+  constexpr int RB = 2 * D;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);  // ready[2], free[2]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3, mi = lane >> 3, lr = lane & 7;
   const int h = blockIdx.x, layer = blockIdx.y, seq = blockIdx.z;
@@ -213,259 +235,292 @@ __global__ void __launch_bounds__(2 * D) gdn_scan_kernel(const GdnLaunch p) {
   const int T = p.T;
   const int slot = seq * p.n_gdn + layer;
   const int nkdk = p.n_k * D, nvdv = n_v * D;
-  const __half* kg =
-      static_cast<const __half*>(p.kbuf) + static_cast<int64_t>(slot) * T * nkdk + kh * D;
-  const __half* vg =
-      static_cast<const __half*>(p.vbuf) + static_cast<int64_t>(slot) * T * nvdv + h * D;
-  const float* gg = p.gbuf + static_cast<int64_t>(slot) * 2 * n_v * T + h * T;
-  const float* bg = gg + static_cast<int64_t>(n_v) * T;
-  float* Sg = p.state + (static_cast<int64_t>(slot) * n_v + h) * D * D;
-
-  // state rows r0 = 16w + g and r0 + 8, as m16n8 accumulator fragments
-  float S[D / 8][4];
-  {
-    const float* s0 = Sg + (16 * warp + g) * D + 2 * c;
-    const float* s1 = s0 + 8 * D;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      const float2 a = *reinterpret_cast<const float2*>(s0 + 8 * nt);
-      const float2 b = *reinterpret_cast<const float2*>(s1 + 8 * nt);
-      S[nt][0] = a.x;
-      S[nt][1] = a.y;
-      S[nt][2] = b.x;
-      S[nt][3] = b.y;
-    }
-  }
-
   const int n_chunks = (T + SCAN_CH - 1) / SCAN_CH;
-  for (int ci = 0; ci < n_chunks; ++ci) {
-    const int c0 = ci * SCAN_CH;
-    // (1) K, V rows of the chunk (zero past T), g and beta (0 past T: identity steps)
-    for (int i = tid; i < SCAN_CH * (D / 8); i += NT) {
-      const int r = i / (D / 8), ch = i % (D / 8);
-      const int t = c0 + r;
-      const bool ok = t < T;
-      const int64_t tt = ok ? t : 0;
-      cp_async16(sK + sw_off(r, ch, RB), kg + tt * nkdk + ch * 8, ok ? 16u : 0u);
-      cp_async16(sV + sw_off(r, ch, RB), vg + tt * nvdv + ch * 8, ok ? 16u : 0u);
-    }
-    cp_async_commit();
-    if (tid < SCAN_CH) {
-      const int t = c0 + tid;
-      gs[tid] = t < T ? gg[t] : 0.f;
-      bs[tid] = t < T ? bg[t] : 0.f;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
 
-    // (2) A = K K^T tiles of this warp; warp 0 also forms the cumulative decays
-    constexpr int NPW = 32 / NW;  // n-tiles (of 8) per warp
-    const int mt_a = warp & 3;
-    const int nb_a = (warp >> 2) * NPW;
-    float acc[NPW][4];
-#pragma unroll
-    for (int j = 0; j < NPW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      uint32_t a[4];
-      ldmatrix_x4(a, sK + sw_off(mt_a * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), RB));
-#pragma unroll
-      for (int j = 0; j < NPW; j += 2) {
-        uint32_t b[4];
-        ldmatrix_x4(b, sK + sw_off((nb_a + j) * 8 + (mi >> 1) * 8 + lr, ks * 2 + (mi & 1), RB));
-        uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
-        mma_f16_16816(acc[j], a, b0);
-        mma_f16_16816(acc[j + 1], a, b1);
-      }
-    }
-    if (warp == 0) {
-      const float v0 = gs[2 * lane], v1 = gs[2 * lane + 1];
-      const float pair = v0 + v1;
-      float sc = pair;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, sc, o);
-        if (lane >= o) sc += y;
-      }
-      const float ex = sc - pair;
-      const float total = __shfl_sync(0xffffffffu, sc, 31);
-      const float ga = ex + v0, gb2 = ex + pair;
-      gam[2 * lane] = ga;
-      gam[2 * lane + 1] = gb2;
-      Gam[2 * lane] = expf(ga);
-      Gam[2 * lane + 1] = expf(gb2);
-      dec[2 * lane] = expf(total - ga);
-      dec[2 * lane + 1] = expf(total - gb2);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < NPW; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = mt_a * 16 + g + (e >> 1) * 8;
-        const int s = (nb_a + j) * 8 + 2 * c + (e & 1);
-        Lf[t * LD + s] = s < t ? bs[t] * expf(gam[t] - gam[s]) * acc[j][e] : 0.f;
-      }
-    }
-    __syncthreads();
+  if (tid == 0) {
+    mbar_init(&bars[0], SCAN_PREP_THREADS);
+    mbar_init(&bars[1], SCAN_PREP_THREADS);
+    mbar_init(&bars[2], NSW * 32);
+    mbar_init(&bars[3], NSW * 32);
+    fence_mbar_init();
+  }
+  __syncthreads();
 
-    // (3) Tm = (I + L)^-1 by 16x16 blocks: diagonal blocks by substitution ...
-    if (tid < 64) {
-      const int base = (tid >> 4) * 16, col = tid & 15;
-      for (int r = 0; r < 16; ++r) {
-        float v;
-        if (r < col) {
-          v = 0.f;
-        } else if (r == col) {
-          v = 1.f;
-        } else {
-          float s = 0.f;
-          for (int q = col; q < r; ++q) s += Lf[(base + r) * LD + base + q] * Tf[(base + q) * LD + base + col];
-          v = -s;
-        }
-        Tf[(base + r) * LD + base + col] = v;
-      }
-    }
-    __syncthreads();
-    // ... then block rows i = 1..3: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj
-    for (int i = 1; i < 4; ++i) {
-      for (int o = tid; o < i * 256; o += NT) {
-        const int j = o >> 8, e = o & 255, r = e >> 4, cc = e & 15;
-        float s = 0.f;
-        for (int k = j; k < i; ++k)
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            s += Lf[(16 * i + r) * LD + 16 * k + q] * Tf[(16 * k + q) * LD + 16 * j + cc];
-        Mf[o] = s;
-      }
-      __syncthreads();
-      for (int o = tid; o < i * 256; o += NT) {
-        const int j = o >> 8, e = o & 255, r = e >> 4, cc = e & 15;
-        float s = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) s += Tf[(16 * i + r) * LD + 16 * i + q] * Mf[(j << 8) + q * 16 + cc];
-        Tf[(16 * i + r) * LD + 16 * j + cc] = -s;
-      }
-      __syncthreads();
-    }
-
-    // (4) TB = Tm diag(beta), TBG = Tm diag(beta e^gam) as bf16 (zero above the block diagonal)
-    for (int o = tid; o < SCAN_CH * SCAN_CH / 2; o += NT) {
-      const int t = o >> 5, s = (o & 31) * 2;
-      const bool upper = (s >> 4) > (t >> 4);
-      const float x0 = upper ? 0.f : Tf[t * LD + s];
-      const float x1 = upper ? 0.f : Tf[t * LD + s + 1];
-      const float b0 = bs[s], b1 = bs[s + 1];
-      const uint32_t off = static_cast<uint32_t>(t * 128 + (((s >> 3) ^ (t & 7)) << 4) + (s & 7) * 2);
-      *reinterpret_cast<uint32_t*>(sm + SM::OFF_TB + off) = pack_f16(x0 * b0, x1 * b1);
-      *reinterpret_cast<uint32_t*>(sm + SM::OFF_TBG + off) =
-          pack_f16(x0 * b0 * Gam[s], x1 * b1 * Gam[s + 1]);
-    }
-    __syncthreads();
-
-    // (5) this warp's columns [16w, 16w+16): U = TB V (initial value of U) and
-    //     W = TBG K, stored negated for everyone
-    float U[4][2][4];
+  if (warp < NSW) {
+    // ===================================================== state warps
+    float* Sg = p.state + (static_cast<int64_t>(slot) * n_v + h) * D * D;
+    float S[D / 8][4];
     {
-      float Wt[4][2][4];
+      const float* s0 = Sg + (16 * warp + g) * D + 2 * c;
+      const float* s1 = s0 + 8 * D;
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) U[m][n][e] = Wt[m][n][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t bv[4], bk[4];
-        const int row = ks * 16 + (mi & 1) * 8 + lr;
-        const int ch = warp * 2 + (mi >> 1);
-        ldmatrix_x4_trans(bv, sV + sw_off(row, ch, RB));
-        ldmatrix_x4_trans(bk, sK + sw_off(row, ch, RB));
-        uint32_t bv0[2] = {bv[0], bv[1]}, bv1[2] = {bv[2], bv[3]};
-        uint32_t bk0[2] = {bk[0], bk[1]}, bk1[2] = {bk[2], bk[3]};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          uint32_t a[4], ag[4];
-          const uint32_t off = sw_off(m * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), 128);
-          ldmatrix_x4(a, sTB + off);
-          ldmatrix_x4(ag, sTBG + off);
-          mma_f16_16816(U[m][0], a, bv0);
-          mma_f16_16816(U[m][1], a, bv1);
-          mma_f16_16816(Wt[m][0], ag, bk0);
-          mma_f16_16816(Wt[m][1], ag, bk1);
-        }
+      for (int nt = 0; nt < D / 8; ++nt) {
+        const float2 a = *reinterpret_cast<const float2*>(s0 + 8 * nt);
+        const float2 b = *reinterpret_cast<const float2*>(s1 + 8 * nt);
+        S[nt][0] = a.x;
+        S[nt][1] = a.y;
+        S[nt][2] = b.x;
+        S[nt][3] = b.y;
       }
+    }
+    for (int ci = 0; ci < n_chunks; ++ci) {
+      const int b = ci & 1;
+      if (!mbar_wait_ns(&bars[b], (ci >> 1) & 1, kScanWaitNs)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      const uint8_t* buf = sm + b * L::BUF;
+      const uint32_t sK = smem_u32(buf + L::B_K), sW = smem_u32(buf + L::B_W);
+      const float* dec = reinterpret_cast<const float*>(buf + L::B_DEC);
+      // U starts from U0 = Tm diag(beta) V, this warp's columns [16w, 16w+16)
+      float U[4][2][4];
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
-          const int ch = warp * 2 + n;
-          const int r0 = m * 16 + g;
-          *reinterpret_cast<uint32_t*>(sm + SM::OFF_W + sw_off(r0, ch, RB) + 4 * c) =
-              pack_f16(-Wt[m][n][0], -Wt[m][n][1]);
-          *reinterpret_cast<uint32_t*>(sm + SM::OFF_W + sw_off(r0 + 8, ch, RB) + 4 * c) =
-              pack_f16(-Wt[m][n][2], -Wt[m][n][3]);
+          const int t = m * 16 + g;
+          const float2 u0 = F16<__half>::unpack(ld_smem_u32(buf + L::B_U + sw_off(t, warp * 2 + n, RB) + 4 * c));
+          const float2 u1 = F16<__half>::unpack(ld_smem_u32(buf + L::B_U + sw_off(t + 8, warp * 2 + n, RB) + 4 * c));
+          U[m][n][0] = u0.x;
+          U[m][n][1] = u0.y;
+          U[m][n][2] = u1.x;
+          U[m][n][3] = u1.y;
         }
-    }
-    __syncthreads();
-
-    // (6) U += (-W) S^T, the B operand taken straight from this warp's state rows
-    {
-      uint32_t sb[D / 8][2];
+      // U += (-W) S^T, the B operand straight from this warp's state rows
+      {
+        uint32_t sb[D / 8][2];
 #pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        sb[nt][0] = pack_f16(S[nt][0], S[nt][1]);
-        sb[nt][1] = pack_f16(S[nt][2], S[nt][3]);
+        for (int nt = 0; nt < D / 8; ++nt) {
+          sb[nt][0] = pack_f16(S[nt][0], S[nt][1]);
+          sb[nt][1] = pack_f16(S[nt][2], S[nt][3]);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t b0[2] = {sb[2 * ks][0], sb[2 * ks + 1][0]};
+          uint32_t b1[2] = {sb[2 * ks][1], sb[2 * ks + 1][1]};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            uint32_t a[4];
+            ldmatrix_x4(a, sW + sw_off(m * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), RB));
+            mma_f16_16816(U[m][0], a, b0);
+            mma_f16_16816(U[m][1], a, b1);
+          }
+        }
       }
+      // S <- e^gam_last S + (dec U)^T K
+      {
+        const float gl = dec[SCAN_CH];
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        uint32_t b0[2] = {sb[2 * ks][0], sb[2 * ks + 1][0]};
-        uint32_t b1[2] = {sb[2 * ks][1], sb[2 * ks + 1][1]};
+        for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) S[nt][e] *= gl;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
+          const float d0 = dec[m * 16 + g], d1 = dec[m * 16 + 8 + g];
           uint32_t a[4];
-          ldmatrix_x4(a, sW + sw_off(m * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), RB));
-          mma_f16_16816(U[m][0], a, b0);
-          mma_f16_16816(U[m][1], a, b1);
+          a[0] = movmatrix_trans(pack_f16(U[m][0][0] * d0, U[m][0][1] * d0));
+          a[1] = movmatrix_trans(pack_f16(U[m][1][0] * d0, U[m][1][1] * d0));
+          a[2] = movmatrix_trans(pack_f16(U[m][0][2] * d1, U[m][0][3] * d1));
+          a[3] = movmatrix_trans(pack_f16(U[m][1][2] * d1, U[m][1][3] * d1));
+#pragma unroll
+          for (int nt = 0; nt < D / 8; nt += 2) {
+            uint32_t bk[4];
+            ldmatrix_x4_trans(bk, sK + sw_off(m * 16 + (mi & 1) * 8 + lr, nt + (mi >> 1), RB));
+            uint32_t b0[2] = {bk[0], bk[1]}, b1[2] = {bk[2], bk[3]};
+            mma_f16_16816(S[nt], a, b0);
+            mma_f16_16816(S[nt + 1], a, b1);
+          }
         }
       }
+      mbar_arrive(&bars[2 + b]);
     }
-
-    // (7) S <- e^gam_last S + (dec U)^T K
-    {
-      const float gl = Gam[SCAN_CH - 1];
-#pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) S[nt][e] *= gl;
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float d0 = dec[m * 16 + g], d1 = dec[m * 16 + 8 + g];
-        uint32_t a[4];
-        a[0] = movmatrix_trans(pack_f16(U[m][0][0] * d0, U[m][0][1] * d0));
-        a[1] = movmatrix_trans(pack_f16(U[m][1][0] * d0, U[m][1][1] * d0));
-        a[2] = movmatrix_trans(pack_f16(U[m][0][2] * d1, U[m][0][3] * d1));
-        a[3] = movmatrix_trans(pack_f16(U[m][1][2] * d1, U[m][1][3] * d1));
-#pragma unroll
-        for (int nt = 0; nt < D / 8; nt += 2) {
-          uint32_t b[4];
-          ldmatrix_x4_trans(b, sK + sw_off(m * 16 + (mi & 1) * 8 + lr, nt + (mi >> 1), RB));
-          uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
-          mma_f16_16816(S[nt], a, b0);
-          mma_f16_16816(S[nt + 1], a, b1);
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  {
     float* s0 = Sg + (16 * warp + g) * D + 2 * c;
     float* s1 = s0 + 8 * D;
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
       *reinterpret_cast<float2*>(s0 + 8 * nt) = make_float2(S[nt][0], S[nt][1]);
       *reinterpret_cast<float2*>(s1 + 8 * nt) = make_float2(S[nt][2], S[nt][3]);
+    }
+  } else {
+    // ===================================================== prep warps
+    constexpr int NTW = D / 16;  // 8-column tiles per prep warp (a quarter of 2D columns)
+    const int pt = tid - NSW * 32;  // 0..127
+    const int pw = warp - NSW;      // 0..3
+    const bool kpart = pw >= 2;     // warps 0,1: U0 columns (V); warps 2,3: -W columns (K)
+    const int col0 = (pw & 1) * (D / 2);
+    const __half* kg =
+        static_cast<const __half*>(p.kbuf) + static_cast<int64_t>(slot) * T * nkdk + kh * D;
+    const __half* vg =
+        static_cast<const __half*>(p.vbuf) + static_cast<int64_t>(slot) * T * nvdv + h * D;
+    const float* gg = p.gbuf + static_cast<int64_t>(slot) * 2 * n_v * T + h * T;
+    const float* bg = gg + static_cast<int64_t>(n_v) * T;
+    float* Ld = reinterpret_cast<float*>(sm + L::OFF_LD);
+    float* gs = reinterpret_cast<float*>(sm + L::OFF_G);
+    float* bs = gs + SCAN_CH;
+    float* gam = bs + SCAN_CH;
+    float* Gam = gam + SCAN_CH;
+    const uint32_t sV = smem_u32(sm + L::OFF_V);
+    const uint32_t sLN = smem_u32(sm + L::OFF_LN);
+    const uint32_t sTD = smem_u32(sm + L::OFF_TD);
+
+    for (int ci = 0; ci < n_chunks; ++ci) {
+      const int b = ci & 1;
+      if (ci >= 2 && !mbar_wait_ns(&bars[2 + b], ((ci >> 1) - 1) & 1, kScanWaitNs))
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      uint8_t* buf = sm + b * L::BUF;
+      const uint32_t sK = smem_u32(buf + L::B_K);
+      float* dec = reinterpret_cast<float*>(buf + L::B_DEC);
+      const int c0 = ci * SCAN_CH;
+      // (1) K, V rows of the chunk (zero past T: identity steps with g = beta = 0)
+      for (int i = pt; i < SCAN_CH * (D / 8); i += SCAN_PREP_THREADS) {
+        const int r = i / (D / 8), ch = i % (D / 8);
+        const int t = c0 + r;
+        const bool ok = t < T;
+        const int64_t tt = ok ? t : 0;
+        cp_async16(sK + sw_off(r, ch, RB), kg + tt * nkdk + ch * 8, ok ? 16u : 0u);
+        cp_async16(sV + sw_off(r, ch, RB), vg + tt * nvdv + ch * 8, ok ? 16u : 0u);
+      }
+      cp_async_commit();
+      if (pt < SCAN_CH) {
+        const int t = c0 + pt;
+        gs[pt] = t < T ? gg[t] : 0.f;
+        bs[pt] = t < T ? bg[t] : 0.f;
+      }
+      cp_async_wait<0>();
+      prep_sync();
+      // (2) cumulative decays (warp 0) and K K^T for m-tile pw
+      if (pw == 0) {
+        const float v0 = gs[2 * lane], v1 = gs[2 * lane + 1];
+        const float pair = v0 + v1;
+        float sc = pair;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, sc, o);
+          if (lane >= o) sc += y;
+        }
+        const float ex = sc - pair;
+        const float total = __shfl_sync(0xffffffffu, sc, 31);
+        const float ga = ex + v0, gb2 = ex + pair;
+        gam[2 * lane] = ga;
+        gam[2 * lane + 1] = gb2;
+        Gam[2 * lane] = expf(ga);
+        Gam[2 * lane + 1] = expf(gb2);
+        dec[2 * lane] = expf(total - ga);
+        dec[2 * lane + 1] = expf(total - gb2);
+        if (lane == 0) dec[SCAN_CH] = expf(total);
+      }
+      {
+        float acc[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t a[4];
+          ldmatrix_x4(a, sK + sw_off(pw * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1), RB));
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            uint32_t bb[4];
+            ldmatrix_x4(bb, sK + sw_off(j * 8 + (mi >> 1) * 8 + lr, ks * 2 + (mi & 1), RB));
+            uint32_t b0[2] = {bb[0], bb[1]}, b1[2] = {bb[2], bb[3]};
+            mma_f16_16816(acc[j], a, b0);
+            mma_f16_16816(acc[j + 1], a, b1);
+          }
+        }
+        prep_sync();  // gam ready
+        // -L (fp16, all blocks) and the diagonal blocks of L (fp32)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float lv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = pw * 16 + g + (e >> 1) * 8;
+            const int s2 = j * 8 + 2 * c + (e & 1);
+            lv[e] = s2 < t ? bs[t] * expf(gam[t] - gam[s2]) * acc[j][e] : 0.f;
+            if ((s2 >> 4) == pw) Ld[(pw * 16 + (t & 15)) * 17 + (s2 & 15)] = lv[e];
+          }
+          const int t0 = pw * 16 + g;
+          const uint32_t o0 = static_cast<uint32_t>(t0 * 128 + ((j ^ (t0 & 7)) << 4) + 4 * c);
+          const uint32_t o1 = static_cast<uint32_t>((t0 + 8) * 128 + ((j ^ ((t0 + 8) & 7)) << 4) + 4 * c);
+          *reinterpret_cast<uint32_t*>(sm + L::OFF_LN + o0) = pack_f16(-lv[0], -lv[1]);
+          *reinterpret_cast<uint32_t*>(sm + L::OFF_LN + o1) = pack_f16(-lv[2], -lv[3]);
+        }
+      }
+      prep_sync();
+      // (3) diagonal blocks of Tm = (I + L)^-1, one column per thread, in registers
+      if (pt < 64) {
+        const int blk = pt >> 4, col = pt & 15;
+        const float* Lb = Ld + blk * 16 * 17;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+          float sacc = 0.f;
+#pragma unroll
+          for (int q = 0; q < r; ++q) sacc += Lb[r * 17 + q] * x[q];
+          if (r > col) x[r] = -sacc;
+        }
+        // Tm block into the fp16 tile at rows/cols [16 blk, 16 blk + 16)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int t = blk * 16 + r, s2 = blk * 16 + col;
+          *reinterpret_cast<__half*>(sm + L::OFF_TD + t * 128 + (((s2 >> 3) ^ (t & 7)) << 4) + (s2 & 7) * 2) =
+              __float2half_rn(x[r]);
+        }
+      }
+      prep_sync();
+      // (4) block rows i = 0..3: X_i = Tm_ii (B_i - sum_{j<i} L_ij X_j), for this warp's
+      //     2D/4 columns of B = [diag(beta) V | diag(beta e^gam) K]
+      {
+        const uint32_t srcB = kpart ? sK : sV;
+        const uint8_t* srcBp = kpart ? buf + L::B_K : sm + L::OFF_V;
+        uint8_t* dst = kpart ? buf + L::B_W : buf + L::B_U;
+        const float sgn = kpart ? -1.f : 1.f;
+        (void)srcB;
+        uint32_t xb[3][NTW][2];  // X_0..X_2 as B fragments (k = rows of the block)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float y[NTW][4];
+          const int t0 = i * 16 + g, t1 = t0 + 8;
+          const float f0 = bs[t0] * (kpart ? Gam[t0] : 1.f);
+          const float f1 = bs[t1] * (kpart ? Gam[t1] : 1.f);
+#pragma unroll
+          for (int n = 0; n < NTW; ++n) {
+            const int ch = (col0 >> 3) + n;
+            const float2 v0 = F16<__half>::unpack(ld_smem_u32(srcBp + sw_off(t0, ch, RB) + 4 * c));
+            const float2 v1 = F16<__half>::unpack(ld_smem_u32(srcBp + sw_off(t1, ch, RB) + 4 * c));
+            y[n][0] = f0 * v0.x;
+            y[n][1] = f0 * v0.y;
+            y[n][2] = f1 * v1.x;
+            y[n][3] = f1 * v1.y;
+          }
+#pragma unroll
+          for (int j = 0; j < i; ++j) {
+            uint32_t a[4];
+            ldmatrix_x4(a, sLN + sw_off(i * 16 + (mi & 1) * 8 + lr, j * 2 + (mi >> 1), 128));
+#pragma unroll
+            for (int n = 0; n < NTW; ++n) mma_f16_16816(y[n], a, xb[j][n]);
+          }
+          uint32_t yb[NTW][2];
+#pragma unroll
+          for (int n = 0; n < NTW; ++n) {
+            yb[n][0] = movmatrix_trans(pack_f16(y[n][0], y[n][1]));
+            yb[n][1] = movmatrix_trans(pack_f16(y[n][2], y[n][3]));
+          }
+          uint32_t a[4];
+          ldmatrix_x4(a, sTD + sw_off(i * 16 + (mi & 1) * 8 + lr, i * 2 + (mi >> 1), 128));
+#pragma unroll
+          for (int n = 0; n < NTW; ++n) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_f16_16816(x, a, yb[n]);
+            if (i < 3) {
+              xb[i < 3 ? i : 0][n][0] = movmatrix_trans(pack_f16(x[0], x[1]));
+              xb[i < 3 ? i : 0][n][1] = movmatrix_trans(pack_f16(x[2], x[3]));
+            }
+            const int ch = (col0 >> 3) + n;
+            *reinterpret_cast<uint32_t*>(dst + sw_off(t0, ch, RB) + 4 * c) = pack_f16(sgn * x[0], sgn * x[1]);
+            *reinterpret_cast<uint32_t*>(dst + sw_off(t1, ch, RB) + 4 * c) = pack_f16(sgn * x[2], sgn * x[3]);
+          }
+        }
+      }
+      mbar_arrive(&bars[b]);
     }
   }
 }
@@ -511,12 +566,12 @@ int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s) {
 
 template <int D>
 static int launch_scan_d(const GdnLaunch& g, cudaStream_t s) {
-  constexpr int bytes = ScanSmem<D>::BYTES;
+  constexpr int bytes = ScanLayout<D>::BYTES;
   if (cudaFuncSetAttribute(gdn_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            bytes) != cudaSuccess)
     return KVA_ERR_CUDA;
   dim3 grid(g.n_v, g.n_gdn, g.n_seq);
-  gdn_scan_kernel<D><<<grid, 2 * D, bytes, s>>>(g);
+  gdn_scan_kernel<D><<<grid, ScanLayout<D>::NT, bytes, s>>>(g);
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
