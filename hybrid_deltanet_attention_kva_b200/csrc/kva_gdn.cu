@@ -189,20 +189,23 @@ struct ScanLayout {
   static constexpr int NT = (NSW + SCAN_PREP_WARPS) * 32;
   static constexpr int KVB = SCAN_CH * D * 2;        // one [64][D] fp16 tile
   static constexpr int TBB = SCAN_CH * SCAN_CH * 2;  // one [64][64] fp16 tile
-  // one chunk buffer (prep -> state): K, -W = -Tm diag(beta e^gam) K, U0 = Tm diag(beta) V,
+  // one chunk buffer (prep -> state): -W = -Tm diag(beta e^gam) K, U0 = Tm diag(beta) V,
   // decay vector and e^(gam_last)
-  static constexpr int B_K = 0;
-  static constexpr int B_W = KVB;
-  static constexpr int B_U = 2 * KVB;
-  static constexpr int B_DEC = 3 * KVB;
+  static constexpr int B_W = 0;
+  static constexpr int B_U = KVB;
+  static constexpr int B_DEC = 2 * KVB;
   static constexpr int BUF = ((B_DEC + SCAN_CH * 4 + 16) + 127) / 128 * 128;
+  // K ring of 3 slots: the state warps read chunk c's slot while the prep warps
+  // solve chunk c+1 and prefetch chunk c+2
+  static constexpr int OFF_K = 2 * BUF;
   // prep-private
-  static constexpr int OFF_V = 2 * BUF;                // V of the chunk in preparation
-  static constexpr int OFF_LN = OFF_V + KVB;           // -L, fp16 [64][64]
+  static constexpr int OFF_V = OFF_K + 3 * KVB;               // V, double buffered
+  static constexpr int OFF_GB = OFF_V + 2 * KVB;              // raw g, beta, double buffered
+  static constexpr int OFF_LN = OFF_GB + 2 * 2 * SCAN_CH * 4;  // -L, fp16 [64][64]
   static constexpr int OFF_TD = OFF_LN + TBB;          // diagonal blocks of Tm, fp16 [64][64]
   static constexpr int OFF_LD = OFF_TD + TBB;          // diagonal blocks of L, fp32 [4][16][17]
-  static constexpr int OFF_G = OFF_LD + 4 * 16 * 17 * 4;  // g, beta, gam, e^gam
-  static constexpr int OFF_BAR = OFF_G + 4 * SCAN_CH * 4;
+  static constexpr int OFF_G = OFF_LD + 4 * 16 * 17 * 4;  // gam, e^gam
+  static constexpr int OFF_BAR = OFF_G + 2 * SCAN_CH * 4;
   static constexpr int BYTES = OFF_BAR + 64;
 };
 
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(ScanLayout<D>::NT, 1) gdn_scan_kernel(const Gd
       const int b = ci & 1;
       if (!mbar_wait_ns(&bars[b], (ci >> 1) & 1, kScanWaitNs)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
       const uint8_t* buf = sm + b * L::BUF;
-      const uint32_t sK = smem_u32(buf + L::B_K), sW = smem_u32(buf + L::B_W);
+      const uint32_t sK = smem_u32(sm + L::OFF_K + (ci % 3) * L::KVB), sW = smem_u32(buf + L::B_W);
       const float* dec = reinterpret_cast<const float*>(buf + L::B_DEC);
       // U starts from U0 = Tm diag(beta) V, this warp's columns [16w, 16w+16)
       float U[4][2][4];
@@ -352,38 +355,55 @@ __global__ void __launch_bounds__(ScanLayout<D>::NT, 1) gdn_scan_kernel(const Gd
     const float* gg = p.gbuf + static_cast<int64_t>(slot) * 2 * n_v * T + h * T;
     const float* bg = gg + static_cast<int64_t>(n_v) * T;
     float* Ld = reinterpret_cast<float*>(sm + L::OFF_LD);
-    float* gs = reinterpret_cast<float*>(sm + L::OFF_G);
-    float* bs = gs + SCAN_CH;
-    float* gam = bs + SCAN_CH;
+    float* gam = reinterpret_cast<float*>(sm + L::OFF_G);
     float* Gam = gam + SCAN_CH;
-    const uint32_t sV = smem_u32(sm + L::OFF_V);
     const uint32_t sLN = smem_u32(sm + L::OFF_LN);
     const uint32_t sTD = smem_u32(sm + L::OFF_TD);
 
+    // K, V rows of chunk cj into their ring slots and its raw g, beta into the
+    // chunk's g/beta slot, all with cp.async (zero past T: identity steps)
+    auto issue_chunk = [&](int cj) {
+      const uint32_t dK = smem_u32(sm + L::OFF_K + (cj % 3) * L::KVB);
+      const uint32_t dV = smem_u32(sm + L::OFF_V + (cj & 1) * L::KVB);
+      const uint32_t dG = smem_u32(sm + L::OFF_GB + (cj & 1) * 2 * SCAN_CH * 4);
+      const int cb = cj * SCAN_CH;
+      for (int i = pt; i < SCAN_CH * (D / 8); i += SCAN_PREP_THREADS) {
+        const int r = i / (D / 8), ch = i % (D / 8);
+        const int t = cb + r;
+        const bool ok = t < T;
+        const int64_t tt = ok ? t : 0;
+        cp_async16(dK + sw_off(r, ch, RB), kg + tt * nkdk + ch * 8, ok ? 16u : 0u);
+        cp_async16(dV + sw_off(r, ch, RB), vg + tt * nvdv + ch * 8, ok ? 16u : 0u);
+      }
+      if (pt < SCAN_CH) {
+        const int t = cb + pt;
+        const bool ok = t < T;
+        cp_async4(dG + pt * 4, gg + (ok ? t : 0), ok ? 4u : 0u);
+        cp_async4(dG + (SCAN_CH + pt) * 4, bg + (ok ? t : 0), ok ? 4u : 0u);
+      }
+      cp_async_commit();
+    };
+
+    issue_chunk(0);
     for (int ci = 0; ci < n_chunks; ++ci) {
       const int b = ci & 1;
       if (ci >= 2 && !mbar_wait_ns(&bars[2 + b], ((ci >> 1) - 1) & 1, kScanWaitNs))
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      // chunk ci + 1's K slot was last read by the state warps for chunk ci - 2 (done)
+      if (ci + 1 < n_chunks) {
+        issue_chunk(ci + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
       uint8_t* buf = sm + b * L::BUF;
-      const uint32_t sK = smem_u32(buf + L::B_K);
+      const uint8_t* kp = sm + L::OFF_K + (ci % 3) * L::KVB;
+      const uint8_t* vp = sm + L::OFF_V + (ci & 1) * L::KVB;
+      const uint32_t sK = smem_u32(kp);
+      const uint32_t sV = smem_u32(vp);
+      const float* gs = reinterpret_cast<const float*>(sm + L::OFF_GB + (ci & 1) * 2 * SCAN_CH * 4);
+      const float* bs = gs + SCAN_CH;
       float* dec = reinterpret_cast<float*>(buf + L::B_DEC);
-      const int c0 = ci * SCAN_CH;
-      // (1) K, V rows of the chunk (zero past T: identity steps with g = beta = 0)
-      for (int i = pt; i < SCAN_CH * (D / 8); i += SCAN_PREP_THREADS) {
-        const int r = i / (D / 8), ch = i % (D / 8);
-        const int t = c0 + r;
-        const bool ok = t < T;
-        const int64_t tt = ok ? t : 0;
-        cp_async16(sK + sw_off(r, ch, RB), kg + tt * nkdk + ch * 8, ok ? 16u : 0u);
-        cp_async16(sV + sw_off(r, ch, RB), vg + tt * nvdv + ch * 8, ok ? 16u : 0u);
-      }
-      cp_async_commit();
-      if (pt < SCAN_CH) {
-        const int t = c0 + pt;
-        gs[pt] = t < T ? gg[t] : 0.f;
-        bs[pt] = t < T ? bg[t] : 0.f;
-      }
-      cp_async_wait<0>();
       prep_sync();
       // (2) cumulative decays (warp 0) and K K^T for m-tile pw
       if (pw == 0) {
@@ -470,7 +490,7 @@ __global__ void __launch_bounds__(ScanLayout<D>::NT, 1) gdn_scan_kernel(const Gd
       //     2D/4 columns of B = [diag(beta) V | diag(beta e^gam) K]
       {
         const uint32_t srcB = kpart ? sK : sV;
-        const uint8_t* srcBp = kpart ? buf + L::B_K : sm + L::OFF_V;
+        const uint8_t* srcBp = kpart ? kp : vp;
         uint8_t* dst = kpart ? buf + L::B_W : buf + L::B_U;
         const float sgn = kpart ? -1.f : 1.f;
         (void)srcB;
