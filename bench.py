@@ -104,7 +104,7 @@ def heads_traffic(geom_name):
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel source sha256[:16]") != h:
+    if vals.get("kernel source sha256 prefix") != h:
         return None
     try:
         return float(vals["traffic bytes per launch (full size)"])
