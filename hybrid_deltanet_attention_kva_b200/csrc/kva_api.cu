@@ -433,6 +433,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   const int cd = d.compute_dtype;
   const float eps = d.norm_eps;
   // 1. RMSNorm(residual) -> Linear{H -> d} into the fp32 residual stream x
+  if (cudaMemsetAsync(h->x, 0, static_cast<size_t>(T) * dm * sizeof(float), s) != cudaSuccess) {
+    e = KVA_ERR_CUDA;
+    goto done;
+  }
   if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
          return launch_rmsnorm(residual, residual_dtype, H, w->g_in, h->u_in, H, T, H, eps, s, cd);
        })))
@@ -448,7 +452,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     a.M = T;
     a.N = dm;
     a.K = H;
-    a.epilogue = EPI_STORE_F32;
+    a.epilogue = EPI_ADD_F32;  // into a zeroed x, so the K range can be split
     a.err = h->status;
     a.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(a, s); }))) goto done;

@@ -47,6 +47,7 @@ struct GemmParams {
   void* D1;
   int64_t ldd1;
   int64_t n_split;
+  int splits;  // K ranges per tile (ADD_F32 only; partial sums added atomically)
   int* err;
 };
 
@@ -121,21 +122,24 @@ __global__ void __launch_bounds__(192, 1)
   const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
   const int num_n = (p.N + n_per_tile - 1) / n_per_tile;
   const int num_k = (p.K + Cfg::BK - 1) / Cfg::BK;
-  const int tiles = num_m * num_n;
+  const int splits = p.splits;
+  const int tiles = num_m * num_n * splits;  // work items: (n tile, K range, m tile), m fastest
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       const uint64_t pol_a = l2_policy_evict_last();
-      const uint64_t pol_b = l2_policy_evict_first();
+      const uint64_t pol_b = l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0;  // stages with a load issued and not yet seen consumed
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int m_blk = tile % num_m;
-        const int n_blk = tile / num_m;
-        for (int kb = 0; kb < num_k; ++kb) {
+        const int ns = tile / num_m;
+        const int n_blk = ns / splits, sp = ns % splits;
+        const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -208,7 +212,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < num_k; ++kb) {
+        const int sp = (tile / num_m) % splits;
+        const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < Cfg::BK / 16; ++j) {
             umma_f16_ss(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
-                        idesc, (kb | j) != 0 ? 1u : 0u);
+                        idesc, (kb != kb0 || j != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == S) {
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
       const int m_blk = tile % num_m;
-      const int n_blk = tile / num_m;
+      const int n_blk = (tile / num_m) / splits;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
         *abort_flag = 1;
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
@@ -301,7 +307,18 @@ __global__ void __launch_bounds__(192, 1)
               store16x32<T>(reinterpret_cast<T*>(base) + row * ld + col, v, valid);
             } else {
               float* dst = reinterpret_cast<float*>(base) + row * ld + col;
-              if (valid == 32) {
+              if (EPI == EPI_ADD_F32 && splits > 1) {
+                // partial sums of one K range: added atomically (16-byte vector adds)
+                if (valid == 32) {
+#pragma unroll
+                  for (int q4 = 0; q4 < 8; ++q4)
+                    atomicAdd(reinterpret_cast<float4*>(dst) + q4,
+                              make_float4(__uint_as_float(r[4 * q4 + 0]), __uint_as_float(r[4 * q4 + 1]),
+                                          __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3])));
+                } else {
+                  for (int i = 0; i < valid; ++i) atomicAdd(dst + i, __uint_as_float(r[i]));
+                }
+              } else if (valid == 32) {
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
                   float4 o;
@@ -406,8 +423,22 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
   p.n_split = a.n_split;
   p.err = a.err;
   const int n_per_tile = paired ? BN / 2 : BN;
-  const int tiles = ((a.M + Cfg::BM - 1) / Cfg::BM) * ((a.N + n_per_tile - 1) / n_per_tile);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const int num_m = (a.M + Cfg::BM - 1) / Cfg::BM;
+  const int num_k = (a.K + Cfg::BK - 1) / Cfg::BK;
+  int splits = 1;
+  if (EPI == EPI_ADD_F32) {
+    // fill about two waves with partial-K work items when the output has few tiles
+    const int t = num_m * ((a.N + n_per_tile - 1) / n_per_tile);
+    splits = a.splits > 0 ? a.splits : (2 * num_sms() + t - 1) / t;
+    splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
+    while (splits > 1 && num_k / splits < 4) --splits;
+  }
+  p.splits = splits;
+  const int tiles = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
+  int grid = tiles < num_sms() ? tiles : num_sms();
+  // whole groups of num_m CTAs: a CTA keeps its M tile, and the num_m CTAs that share
+  // a weight tile run side by side
+  if (tiles > grid && num_m > 1 && grid >= num_m && num_m <= 16) grid -= grid % num_m;
   auto kern = gemm_tc_kernel<BN, EPI, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
@@ -434,8 +465,8 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.epilogue == EPI_SWIGLU_BF16 && a.b_mode != B_PAIRED) return KVA_ERR_INVALID_ARG;
   int bn = a.block_n;
   if (bn == 0) {
-    if (a.b_mode == B_PAIRED) {
-      bn = 256;
+    if (a.b_mode == B_PAIRED || a.epilogue == EPI_ADD_F32) {
+      bn = 256;  // residual-add GEMMs fill the machine with split K instead of narrow tiles
     } else {
       const long tiles256 = ((a.M + 127) / 128) * (long)((a.N + 255) / 256);
       bn = tiles256 >= 2L * num_sms() ? 256 : 128;

@@ -37,6 +37,7 @@ struct GemmArgs {
   int epilogue = EPI_STORE_BF16;
   int block_n = 0;          // 0: choose
   int dtype = KVA_BF16;     // 16-bit format of A, B and 16-bit outputs: KVA_BF16 or KVA_F16
+  int splits = 0;           // ADD_F32 only: K ranges per tile (0: choose)
   int* err = nullptr;       // device status word
 };
 
