@@ -166,14 +166,11 @@ class Clocks:
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import hybrid_deltanet_attention_kva_b200 as K
+    from hybrid_deltanet_attention_kva_b200 import multi
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    multi.init("nccl", timeout_s=120, device=dev)
     geom = geometry(args.workload)
     seed = 1003 if args.workload == "r3" else 1002
     dt = torch.float16 if args.dtype == "f16" else torch.bfloat16
@@ -186,7 +183,7 @@ def run_ours(args, rank, world, local_rank):
     st = KI.make_states(geom, 1, seed + 2, device="cuda")
     st["conv_tail"] = st["conv_tail"].to(dt)
     n_pool = 4
-    res = [KI.make_residual(geom, T_UB, seed + 100 + rank * n_pool + i, device="cuda")
+    res = [KI.make_residual(geom, T_UB, multi.rank_seed(seed + 100 + i, rank), device="cuda")
            for i in range(n_pool)]
     kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h, dtype=torch.bfloat16, device=dev)
           for _ in range(geom.n_attn)]
@@ -205,18 +202,10 @@ def run_ours(args, rank, world, local_rank):
         K.kva_prefill_ubatch(h, res[i % n_pool] if resid is None else resid, Wt, S, tail, kv,
                              (i % n_ub) * T_UB, draft_out=draft, stream=stream)
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    barrier = multi.barrier
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return multi.max_over_ranks(x, dev)
 
     for i in range(args.warmup):
         step(i)
@@ -279,9 +268,7 @@ def run_ours(args, rank, world, local_rank):
     K.kva_free(h)
 
     if rank != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        multi.finish()
         return
 
     flops, bytes_ = algorithmic(geom)
@@ -340,9 +327,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(geom, seed, tokens=512)
     print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    multi.finish()
 
 
 # ----------------------------------------------------------------------------- oracle

@@ -479,7 +479,6 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     q.N = 3 * dm;
     q.K = dm;
     q.epilogue = EPI_STORE_BF16;
-    q.block_n = 128;
     q.err = h->status;
     q.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(q, s); }))) goto done;

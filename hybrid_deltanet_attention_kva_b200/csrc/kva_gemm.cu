@@ -68,6 +68,89 @@ __device__ __forceinline__ void store16x32(T* dst, const float* v, int valid) {
   }
 }
 
+// One accumulator tile (128 TMEM lanes x BN fp32 columns) to global memory with the
+// fused epilogue.  Warp q of the epilogue group reads TMEM lanes [32q, 32q+32).
+template <int BN, int EPI, typename T>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tmem_acc, int row0,
+                                              int n_blk, int q, int lane) {
+  const int row = row0 + q * 32 + lane;
+  const bool row_ok = row < p.M;
+  const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
+  if constexpr (EPI == EPI_SWIGLU_BF16) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_ld_32x32b_x32(taddr + c, gr);
+      tmem_ld_32x32b_x32(taddr + BN / 2 + c, ur);
+      tmem_ld_wait();
+      const int col = n_blk * (BN / 2) + c;
+      if (row_ok && col < p.N) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+        T* dst = reinterpret_cast<T*>(p.D) + row * p.ldd + col;
+        store16x32<T>(dst, v, p.N - col);
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(taddr + c, r);
+      tmem_ld_wait();
+      int col = n_blk * BN + c;
+      if (row_ok && col < p.N) {
+        const int valid = min(32, p.N - col);
+        void* base = p.D;
+        int64_t ld = p.ldd;
+        if (p.n_split > 0 && col >= p.n_split) {
+          base = p.D1;
+          ld = p.ldd1;
+          col -= static_cast<int>(p.n_split);
+        }
+        if constexpr (EPI == EPI_STORE_BF16) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          store16x32<T>(reinterpret_cast<T*>(base) + row * ld + col, v, valid);
+        } else {
+          float* dst = reinterpret_cast<float*>(base) + row * ld + col;
+          if (EPI == EPI_ADD_F32 && p.splits > 1) {
+            // partial sums of one K range: added atomically (16-byte vector adds)
+            if (valid == 32) {
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                atomicAdd(reinterpret_cast<float4*>(dst) + q4,
+                          make_float4(__uint_as_float(r[4 * q4 + 0]), __uint_as_float(r[4 * q4 + 1]),
+                                      __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3])));
+            } else {
+              for (int i = 0; i < valid; ++i) atomicAdd(dst + i, __uint_as_float(r[i]));
+            }
+          } else if (valid == 32) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              float4 o;
+              if constexpr (EPI == EPI_ADD_F32) o = reinterpret_cast<float4*>(dst)[q4];
+              else o = make_float4(0.f, 0.f, 0.f, 0.f);
+              o.x += __uint_as_float(r[4 * q4 + 0]);
+              o.y += __uint_as_float(r[4 * q4 + 1]);
+              o.z += __uint_as_float(r[4 * q4 + 2]);
+              o.w += __uint_as_float(r[4 * q4 + 3]);
+              reinterpret_cast<float4*>(dst)[q4] = o;
+            }
+          } else {
+            for (int i = 0; i < valid; ++i) {
+              if constexpr (EPI == EPI_ADD_F32) dst[i] += __uint_as_float(r[i]);
+              else dst[i] = __uint_as_float(r[i]);
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int BN, int EPI, typename T>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
@@ -263,83 +346,8 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
-      const int row = m_blk * Cfg::BM + q * 32 + lane;
-      const bool row_ok = row < p.M;
-      const uint32_t taddr =
-          tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (EPI == EPI_SWIGLU_BF16) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld_32x32b_x32(taddr + c, gr);
-          tmem_ld_32x32b_x32(taddr + BN / 2 + c, ur);
-          tmem_ld_wait();
-          const int col = n_blk * (BN / 2) + c;
-          if (row_ok && col < p.N) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
-            T* dst = reinterpret_cast<T*>(p.D) + row * p.ldd + col;
-            store16x32<T>(dst, v, p.N - col);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c, r);
-          tmem_ld_wait();
-          int col = n_blk * BN + c;
-          if (row_ok && col < p.N) {
-            const int valid = min(32, p.N - col);
-            void* base = p.D;
-            int64_t ld = p.ldd;
-            if (p.n_split > 0 && col >= p.n_split) {
-              base = p.D1;
-              ld = p.ldd1;
-              col -= static_cast<int>(p.n_split);
-            }
-            if constexpr (EPI == EPI_STORE_BF16) {
-              float v[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-              store16x32<T>(reinterpret_cast<T*>(base) + row * ld + col, v, valid);
-            } else {
-              float* dst = reinterpret_cast<float*>(base) + row * ld + col;
-              if (EPI == EPI_ADD_F32 && splits > 1) {
-                // partial sums of one K range: added atomically (16-byte vector adds)
-                if (valid == 32) {
-#pragma unroll
-                  for (int q4 = 0; q4 < 8; ++q4)
-                    atomicAdd(reinterpret_cast<float4*>(dst) + q4,
-                              make_float4(__uint_as_float(r[4 * q4 + 0]), __uint_as_float(r[4 * q4 + 1]),
-                                          __uint_as_float(r[4 * q4 + 2]), __uint_as_float(r[4 * q4 + 3])));
-                } else {
-                  for (int i = 0; i < valid; ++i) atomicAdd(dst + i, __uint_as_float(r[i]));
-                }
-              } else if (valid == 32) {
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                  float4 o;
-                  if constexpr (EPI == EPI_ADD_F32) o = reinterpret_cast<float4*>(dst)[q4];
-                  else o = make_float4(0.f, 0.f, 0.f, 0.f);
-                  o.x += __uint_as_float(r[4 * q4 + 0]);
-                  o.y += __uint_as_float(r[4 * q4 + 1]);
-                  o.z += __uint_as_float(r[4 * q4 + 2]);
-                  o.w += __uint_as_float(r[4 * q4 + 3]);
-                  reinterpret_cast<float4*>(dst)[q4] = o;
-                }
-              } else {
-                for (int i = 0; i < valid; ++i) {
-                  if constexpr (EPI == EPI_ADD_F32) dst[i] += __uint_as_float(r[i]);
-                  else dst[i] = __uint_as_float(r[i]);
-                }
-              }
-            }
-          }
-        }
-      }
+      epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN), m_blk * Cfg::BM,
+                                n_blk, q, lane);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
@@ -351,6 +359,245 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+
+// ------------------------------------------------------------------ CTA-pair variant
+// The same pipeline on a pair of CTAs (a cluster of 2) sharing one 256 x 256 tile
+// through tcgen05.mma.cta_group::2: each CTA loads its 128 rows of A and its 128 rows
+// of B (B rows 0-127 of the tile in the leader, 128-255 in the peer), the leader's
+// single thread issues M = 256 MMAs that read both CTAs' operands, and each CTA's
+// TMEM receives its own 128 rows of the accumulator.  Per CTA this halves the B
+// bytes that the tensor core reads from shared memory per MMA, the limit of the
+// one-CTA 128 x 256 tile.  TMA loads of both CTAs complete on the leader's barrier
+// (no multicast loads); MMA completion is committed to both CTAs' barriers.
+struct PairCfg {
+  static constexpr int BM = 128;  // rows per CTA (256 per pair)
+  static constexpr int BN = 256;  // tile columns (128 B rows held by each CTA)
+  static constexpr int BK = 64;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+template <int EPI, typename T>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
+                     const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
+                     const GemmParams p) {
+  using Cfg = PairCfg;
+  constexpr int S = Cfg::STAGES;
+  constexpr int BN = Cfg::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * Cfg::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES);
+  uint64_t* full = bars;            // leader: both CTAs' bytes of a stage
+  uint64_t* empty = bars + S;       // both: the pair's MMAs on a stage completed
+  uint64_t* tfull = bars + 2 * S;   // both: the pair's accumulator is ready
+  uint64_t* tempty = bars + 2 * S + 2;  // leader: both CTAs' epilogues released it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 256);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mA);
+    tma_prefetch_desc(&mB0);
+    if (p.b_mode != B_SINGLE) tma_prefetch_desc(&mB1);
+    if (p.b_mode == B_SEGMENTS) tma_prefetch_desc(&mB2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before anything arrives on them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (p.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
+  const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
+  const int num_n = (p.N + n_per_tile - 1) / n_per_tile;
+  const int num_k = (p.K + Cfg::BK - 1) / Cfg::BK;
+  const int splits = p.splits;
+  const int items = num_m * num_n * splits;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      const uint64_t pol_a = l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;
+      bool ok = true;
+      for (int it = cid; it < items && ok; it += ncl) {
+        const int m_blk = it % num_m;
+        const int ns = it / num_m;
+        const int n_blk = ns / splits, sp = ns % splits;
+        const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+            armed |= 1u << stage;
+          }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          const int kc = kb * Cfg::BK;
+          tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
+                           m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
+          uint8_t* b = sB + stage * Cfg::B_BYTES;
+          if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
+            tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
+          } else if (p.b_mode == B_SEGMENTS) {
+            const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
+            const int seg = n0 / p.seg_rows;
+            const int r = n0 - seg * p.seg_rows;
+            const CUtensorMap* m = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
+            tma_load_2d_pair(b, m, fb, kc, r, pol_b);
+          } else {
+            tma_load_2d_pair(b, &mB0, fb, kc, n_blk * BN + static_cast<int>(rank) * (BN / 2), pol_b);
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      if (leader) {  // every stage armed here has landed (both CTAs' bytes) before exit
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < S; ++i) {
+          if (st == 0) {
+            st = S - 1;
+            ph ^= 1u;
+          } else {
+            --st;
+          }
+          if (armed & (1u << st)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[st], ph)) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader only)
+      constexpr uint32_t idesc = idesc_f16kind_f32(2 * Cfg::BM, BN, F16<T>::umma_fmt);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int it = cid; it < items && ok; it += ncl) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const int sp = (it / num_m) % splits;
+        const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int j = 0; j < Cfg::BK / 16; ++j) {
+            umma_f16_ss_pair(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
+                             idesc, (kb != kb0 || j != 0) ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      // Drain: the pair's MMAs complete before either CTA releases TMEM or exits.
+      umma_commit_pair(&tfull[acc], 0x3);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&tfull[acc], acc_phase)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue warps 2..5 (both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
+                                     mapa_shared(smem_u32(&tempty[1]), 0)};
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int it = cid; it < items; it += ncl) {
+      const int m_blk = it % num_m;
+      const int n_blk = (it / num_m) / splits;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
+                                m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
+                                lane);
+      tc_fence_before();
+      if (leader) mbar_arrive(&tempty[acc]);
+      else mbar_arrive_remote(tempty_lead[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the leader's MMAs (reading the peer's shared memory) are done
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host side
@@ -447,6 +694,56 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
+
+template <int EPI, typename T>
+static int launch_pair(const GemmArgs& a, cudaStream_t s) {
+  using Cfg = PairCfg;
+  const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool paired = a.b_mode == B_PAIRED;
+  CUtensorMap mA, mB[3];
+  if (!make_map(&mA, a.A, a.K, a.M, a.lda, Cfg::BM, dt)) return KVA_ERR_CUDA;
+  const int nb = a.b_mode == B_SINGLE ? 1 : (paired ? 2 : 3);
+  const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
+  for (int i = 0; i < 3; ++i) {
+    const void* src = a.B[i < nb ? i : 0];
+    if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, Cfg::BN / 2, dt)) return KVA_ERR_CUDA;
+  }
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.b_mode = a.b_mode;
+  p.seg_rows = static_cast<int>(a.seg_rows);
+  p.D = a.D;
+  p.ldd = a.ldd;
+  p.D1 = a.D1;
+  p.ldd1 = a.ldd1;
+  p.n_split = a.n_split;
+  p.err = a.err;
+  const int n_per_tile = paired ? Cfg::BN / 2 : Cfg::BN;
+  const int num_m = (a.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
+  const int num_k = (a.K + Cfg::BK - 1) / Cfg::BK;
+  const int max_cl = num_sms() / 2;
+  int splits = 1;
+  if (EPI == EPI_ADD_F32) {
+    const int t = num_m * ((a.N + n_per_tile - 1) / n_per_tile);
+    splits = a.splits > 0 ? a.splits : (2 * max_cl + t - 1) / t;
+    splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
+    while (splits > 1 && num_k / splits < 4) --splits;
+  }
+  p.splits = splits;
+  const int items = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
+  int ncl = items < max_cl ? items : max_cl;
+  if (items > ncl && num_m > 1 && ncl >= num_m && num_m <= 16) ncl -= ncl % num_m;
+  auto kern = gemm_pair_kernel<EPI, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+      cudaSuccess)
+    return KVA_ERR_CUDA;
+  kern<<<2 * ncl, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 int launch_gemm(const GemmArgs& a, cudaStream_t s) {
@@ -463,24 +760,21 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.b_mode == B_PAIRED && (a.epilogue != EPI_SWIGLU_BF16 || !a.B[1] || !aligned16(a.B[1])))
     return KVA_ERR_INVALID_ARG;
   if (a.epilogue == EPI_SWIGLU_BF16 && a.b_mode != B_PAIRED) return KVA_ERR_INVALID_ARG;
+  // block_n: 128 / 256 one-CTA tiles of that width, 512 a CTA pair on a 256 x 256 tile
+  // (the default wherever the B layout allows it)
   int bn = a.block_n;
-  if (bn == 0) {
-    if (a.b_mode == B_PAIRED || a.epilogue == EPI_ADD_F32) {
-      bn = 256;  // residual-add GEMMs fill the machine with split K instead of narrow tiles
-    } else {
-      const long tiles256 = ((a.M + 127) / 128) * (long)((a.N + 255) / 256);
-      bn = tiles256 >= 2L * num_sms() ? 256 : 128;
-    }
-  }
+  if (bn == 0) bn = (a.b_mode != B_SEGMENTS || (a.seg_rows > 0 && a.seg_rows % 256 == 0)) ? 512 : 128;
   if (a.b_mode == B_SEGMENTS) {
     if (!a.B[1] || !a.B[2] || !aligned16(a.B[1]) || !aligned16(a.B[2])) return KVA_ERR_INVALID_ARG;
-    if (a.seg_rows <= 0 || a.seg_rows % bn || a.N != 3 * a.seg_rows) return KVA_ERR_UNSUPPORTED;
+    const int seg_tile = bn == 512 ? 256 : bn;
+    if (a.seg_rows <= 0 || a.seg_rows % seg_tile || a.N != 3 * a.seg_rows) return KVA_ERR_UNSUPPORTED;
   }
-  if (bn != 128 && bn != 256) return KVA_ERR_UNSUPPORTED;
+  if (bn != 128 && bn != 256 && bn != 512) return KVA_ERR_UNSUPPORTED;
   if (a.dtype != KVA_BF16 && a.dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   const bool h = a.dtype == KVA_F16;
 #define KVA_GEMM_CASE(E)                                                                   \
   case E:                                                                                  \
+    if (bn == 512) return h ? launch_pair<E, __half>(a, s) : launch_pair<E, __nv_bfloat16>(a, s); \
     if (h) return bn == 256 ? launch_instance<256, E, __half>(a, s)                        \
                             : launch_instance<128, E, __half>(a, s);                       \
     return bn == 256 ? launch_instance<256, E, __nv_bfloat16>(a, s)                        \

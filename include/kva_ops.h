@@ -45,8 +45,9 @@ int kva_op_rmsnorm(const void* x, int32_t x_dtype, int64_t ldx, const float* g, 
  *   B     HOST array of 1..3 device pointers per b_mode, each with row stride ldb
  *   D     output [M, ldd] (bf16 or fp32 per epilogue); with n_split > 0 columns
  *         >= n_split go to D1 [M, ldd1] at column - n_split (n_split % 32 == 0)
- *   block_n 0 (choose), 128 or 256
- * K, lda, ldb multiples of 8; seg_rows a multiple of the chosen block_n. */
+ *   block_n 0 (choose), 128 or 256 (one CTA per tile of that width), 512 (a CTA pair on
+ *           a 256 x 256 tile, the default when the B layout allows it)
+ * K, lda, ldb multiples of 8; seg_rows a multiple of the tile width (256 for the pair). */
 int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B, int32_t b_mode,
                 int64_t ldb, int64_t seg_rows, void* D, int64_t ldd, void* D1, int64_t ldd1,
                 int64_t n_split, int32_t M, int32_t N, int32_t K, int32_t epilogue,

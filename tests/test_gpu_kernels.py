@@ -44,7 +44,8 @@ def test_rmsnorm(K, dtype, rows, n, odt):
 
 # ------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("M,N,K_,bn", [(128, 256, 64, 256), (200, 1296, 520, 0), (1024, 3072, 3072, 128),
-                                       (77, 512, 256, 256), (1024, 2560, 5120, 0)])
+                                       (77, 512, 256, 256), (1024, 2560, 5120, 0), (600, 1040, 704, 512),
+                                       (1024, 3072, 3072, 256)])
 @pytest.mark.parametrize("epi", [0, 1, 2])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 def test_gemm_epilogues(K, M, N, K_, bn, epi, dt):
@@ -84,13 +85,14 @@ def test_gemm_swiglu_paired(K, M, F, K_, dt):
 
 @pytest.mark.parametrize("M,d", [(300, 256), (1024, 3072)])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
-def test_gemm_qkv_segments(K, M, d, dt):
+@pytest.mark.parametrize("bn", [128, 512])
+def test_gemm_qkv_segments(K, M, d, dt, bn):
     g = _gen(d)
     A = torch.randn(M, d, generator=g).to(dt)
     Ws = [(torch.randn(d, d, generator=g) * 0.05).to(dt) for _ in range(3)]
     D = torch.full((M, 3 * d), float("nan"), dtype=dt, device="cuda")
     K.kva_op_gemm(A.cuda(), [w.cuda() for w in Ws], D, N=3 * d, b_mode=K.B_SEGMENTS,
-                  seg_rows=d, block_n=128)
+                  seg_rows=d, block_n=bn)
     torch.cuda.synchronize()
     want = np.concatenate([f64(A) @ f64(w).T for w in Ws], axis=1)
     assert_rms_close(D, want, what="qkv", elem=BF16_ELEM)
