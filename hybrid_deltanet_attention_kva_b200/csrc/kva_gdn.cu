@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
   const int n_cblk = (C + PREP_CH - 1) / PREP_CH;
 
   if (static_cast<int>(blockIdx.x) < n_cblk) {
+    // q is only an optional debug output (the state update reads k, v and the gates):
+    // without a debug buffer, blocks whose channels are all q have nothing to do
+    if (!p.debug_qkv && (blockIdx.x + 1) * PREP_CH <= nkdk) return;
     const int c0 = blockIdx.x * PREP_CH + threadIdx.x * 8;
     const bool active = c0 < C;
     const int cc = active ? c0 : 0;
@@ -170,12 +173,16 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk, int rb) {
   return static_cast<uint32_t>(row * rb + ((chunk ^ (row & 7)) << 4));
 }
 
+// Bounded wait; the clock is read only every 64 polls (a %globaltimer read is slow).
 __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit) return false;
+    if ((i & 63u) == 0) {
+      const uint64_t t = globaltimer_ns();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > limit) return false;
+    }
   }
 }
 
