@@ -607,7 +607,7 @@ int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s) {
   int e = check_gdn(g);
   if (e) return e;
   if (!g.state) return KVA_ERR_INVALID_ARG;
-  return g.d_k == 128 ? launch_scan_d<128>(g, s) : launch_scan_d<64>(g, s);
+  return g.d_k == 128 ? launch_gdn_scan_tc(g, s) : launch_scan_d<64>(g, s);
 }
 
 }  // namespace kva

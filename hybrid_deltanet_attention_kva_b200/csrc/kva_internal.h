@@ -42,6 +42,12 @@ struct GemmArgs {
 };
 
 int num_sms();
+// Tiled TMA descriptor (128-byte swizzle, zero fill out of range) of a 16-bit
+// array with three dimensions: d0 contiguous, d1 rows of d0 elements, d2 blocks of
+// d1 rows; box [box1 rows][box0 elements], one block deep.  False when the driver
+// entry point is missing or rejects the arguments.
+bool make_map_3d_16bit(void* map, const void* base, bool fp16, int64_t d0, int64_t d1,
+                       int64_t d2, int box0, int box1);
 int launch_gemm(const GemmArgs& a, cudaStream_t s);
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
                    int64_t ldo, int rows, int n, float eps, cudaStream_t s,
@@ -73,6 +79,7 @@ struct GdnLaunch {
 int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s);
+int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s);  // d_k = d_v = 128
 
 constexpr int kMaxSeqPos = 256;
 struct KvLaunch {
