@@ -38,6 +38,7 @@ struct kva_handle {
   __nv_bfloat16* vbuf = nullptr;  // [max_seq, n_gdn, max_T, n_v d_v]
   float* gbuf = nullptr;          // [max_seq, n_gdn, 2, n_v, max_T]
   int* status = nullptr;          // device status word
+  void* chunk = nullptr;          // per-chunk B1 and scalars of the 128-dimensional scan
   cudaStream_t last_stream = nullptr;
   int64_t tokens = 0;
   // profiling: event pairs around launches, launch counters per stage kind
@@ -130,7 +131,7 @@ Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
   sz[7] = S * ng * T * (size_t)d->gdn_n_v * d->gdn_d_v * 2;           // vbuf
   sz[8] = S * ng * 2 * (size_t)d->gdn_n_v * T * 4;                    // gbuf
   sz[9] = 256;                                                        // status
-  sz[10] = 0;
+  sz[10] = d->gdn_d_k == 128 ? gdn_chunk_bytes((int)S, ng, d->gdn_n_v, (int)T) : 0;  // B1, scalars
   (void)C;
   Layout L;
   size_t o = 0;
@@ -215,6 +216,7 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     g.kbuf = h->kbuf;
     g.vbuf = h->vbuf;
     g.gbuf = debug_gb ? static_cast<float*>(debug_gb) : h->gbuf;
+    gdn_chunk_split(h->chunk, n_seq, h->n_gdn, d.gdn_n_v, T, &g.b1buf, &g.scbuf);
     g.debug_qkv = debug_qkv;
     g.eps = d.norm_eps;
     g.err = h->status;
@@ -306,6 +308,7 @@ int kva_init(const kva_dims* dims, kva_handle** out) {
   h->vbuf = reinterpret_cast<__nv_bfloat16*>(b + L.off[7]);
   h->gbuf = reinterpret_cast<float*>(b + L.off[8]);
   h->status = reinterpret_cast<int*>(b + L.off[9]);
+  h->chunk = b + L.off[10];
   if (cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->ws);
     delete h;
@@ -704,7 +707,17 @@ int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state,
   g.conv_w = gb;
   g.A_log = gb;
   g.dt_bias = gb;
-  return launch_gdn_scan(g, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the 128-dimensional scan stages B1 and the chunk scalars in stream-ordered scratch
+  void* chunk = nullptr;
+  if (d == 128 && T > 0 && n_seq > 0 && n_layers > 0) {
+    if (cudaMallocAsync(&chunk, gdn_chunk_bytes(n_seq, n_layers, n_v, T), st) != cudaSuccess)
+      return KVA_ERR_NO_MEMORY;
+    gdn_chunk_split(chunk, n_seq, n_layers, n_v, T, &g.b1buf, &g.scbuf);
+  }
+  const int e = launch_gdn_scan(g, st);
+  if (chunk && cudaFreeAsync(chunk, st) != cudaSuccess) return KVA_ERR_CUDA;
+  return e;
 }
 
 }  // extern "C"

@@ -72,6 +72,8 @@ struct GdnLaunch {
   void* kbuf = nullptr;         // fp16 [n_seq, n_gdn, T, n_k*d_k]
   void* vbuf = nullptr;         // fp16 [n_seq, n_gdn, T, n_v*d_v]
   float* gbuf = nullptr;        // fp32 [n_seq, n_gdn, 2, n_v, T] (g then beta)
+  void* b1buf = nullptr;        // d_k = 128: fp16 [n_seq, n_gdn, n_v, chunks, 64, 64]
+  float* scbuf = nullptr;       // d_k = 128: fp32 [n_seq, n_gdn, n_v, chunks, 80]
   void* debug_qkv = nullptr;    // bf16 [n_seq, n_gdn, T, C] or null
   float eps = 1e-6f;
   int* err = nullptr;
@@ -80,6 +82,10 @@ int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s);  // d_k = d_v = 128
+// bytes of the per-chunk buffers (b1buf, then scbuf) the 128-dimensional scan needs
+size_t gdn_chunk_bytes(int n_seq, int n_gdn, int n_v, int T);
+// b1buf and scbuf inside a region of gdn_chunk_bytes(...) bytes at `base`
+void gdn_chunk_split(void* base, int n_seq, int n_gdn, int n_v, int T, void** b1, float** sc);
 
 constexpr int kMaxSeqPos = 256;
 struct KvLaunch {

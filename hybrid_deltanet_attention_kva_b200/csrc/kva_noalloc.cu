@@ -26,8 +26,11 @@ constexpr int kMaxT = KVA_NOALLOC_MAX_T;
 constexpr size_t kKBytes = static_cast<size_t>(kMaxT) * KVA_NOALLOC_MAX_QK * 2;
 constexpr size_t kVBytes = static_cast<size_t>(kMaxT) * KVA_NOALLOC_MAX_V * 2;
 constexpr size_t kGBytes = static_cast<size_t>(2) * KVA_NOALLOC_MAX_NV * kMaxT * 4;
-constexpr size_t kScratchBytes = kKBytes + kVBytes + kGBytes;
-static_assert(kKBytes % 256 == 0 && kVBytes % 256 == 0, "scratch parts stay 256-byte aligned");
+// per-chunk B1 tiles and scalars of the 128-dimensional scan
+constexpr size_t kCBytes = static_cast<size_t>((kMaxT + 63) / 64) * KVA_NOALLOC_MAX_NV * (64 * 64 * 2 + 80 * 4);
+constexpr size_t kScratchBytes = kKBytes + kVBytes + kGBytes + kCBytes;
+static_assert(kKBytes % 256 == 0 && kVBytes % 256 == 0 && kGBytes % 256 == 0,
+              "scratch parts stay 256-byte aligned");
 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -103,6 +106,10 @@ extern "C" int kva_gdn_layer_update_noalloc(const void* mixer_in, int64_t mixer_
   g.kbuf = b;                      // every row < T is written before the scan reads it,
   g.vbuf = b + kKBytes;            // so nothing in the scratch has to start at zero
   g.gbuf = reinterpret_cast<float*>(b + kKBytes + kVBytes);
+  if (d == 128) {
+    // every chunk's B1 and scalars are written before the scan reads them
+    kva::gdn_chunk_split(b + kKBytes + kVBytes + kGBytes, 1, 1, n_v, T, &g.b1buf, &g.scbuf);
+  }
   g.eps = eps;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((e = kva::launch_gdn_prepare(g, s))) return e;

@@ -66,12 +66,14 @@ int kva_op_attention(int32_t dtype, const void* qkv, int64_t ldq, void* out, int
  *   v     fp16 [n_seq*n_layers, T, n_v*d]
  *   gb    fp32 [n_seq*n_layers, 2, n_v, T] (g then beta per v head)
  *   state fp32 [n_seq*n_layers, n_v, d, d] read and updated in place
- * v head h reads k head h / (n_v / n_k).  d = 64 or 128. */
+ * v head h reads k head h / (n_v / n_k).  d = 64 or 128.  With d = 128 the call
+ * stages per-chunk intermediates in stream-ordered scratch (cudaMallocAsync and
+ * cudaFreeAsync on `stream`); KVA_ERR_NO_MEMORY if that fails. */
 int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state, int32_t n_seq,
                     int32_t n_layers, int32_t T, int32_t n_k, int32_t n_v, int32_t d,
                     void* stream);
 
-/* Limits of kva_gdn_layer_update_noalloc's fixed scratch (about 4.4 MB per GPU). */
+/* Limits of kva_gdn_layer_update_noalloc's fixed scratch (about 6.6 MB per GPU). */
 #define KVA_NOALLOC_MAX_T 256    /* tokens per call */
 #define KVA_NOALLOC_MAX_QK 2048  /* n_k * d */
 #define KVA_NOALLOC_MAX_V 6144   /* n_v * d */
