@@ -211,7 +211,7 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
     assert K.kva_get_device_status(h) == 0, "device status set during warm-up"
-    K.kva_profile_enable(h, args.steps * 40 + 64)
+    K.kva_profile_read(h)  # resets the launch counters (no events: nothing is timed per launch)
 
     # ---------------- timed region (device time, max over ranks)
     clocks = Clocks(local_rank)
@@ -228,9 +228,19 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1))
-    prof = K.kva_profile_read(h)
+    launches = int(sum(v["launches"] for v in K.kva_profile_read(h).values()))
     status = K.kva_get_device_status(h)
+
+    # ---------------- stage breakdown: a separate pass with an event pair around every
+    # launch (all launches then stay on the caller's stream, each timed alone)
+    n_prof = max(1, min(args.steps, 50))
+    K.kva_profile_enable(h, n_prof * 40 + 64)
+    for i in range(n_prof):
+        step(args.warmup + args.steps + i)
+    torch.cuda.synchronize()
+    prof = K.kva_profile_read(h)
     K.kva_profile_enable(h, 0)
+    status |= K.kva_get_device_status(h)
 
     # ---------------- end to end: host residual in (pinned), drafter row out
     e2e = None
@@ -280,7 +290,6 @@ def run_ours(args, rank, world, local_rank):
     heads_ms = gh["ms"] / max(gh["timed"], 1)
     achieved = heads_flops / (heads_ms / 1e3) / 1e12
     peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    launches = int(sum(v["launches"] for v in prof.values()))
     line = {
         "metric": METRIC,
         "value": world * args.steps * T_UB / (ms / 1e3),
@@ -318,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
             "frac": t_roof / (ms_step / 1e3), "peaks": f"{src}: {peaks['bf16_tflops']} TFLOP/s bf16, "
                                                      f"{peaks['hbm_gbs']} GB/s",
         },
-        "stages_ms_per_step": {k: v["ms"] / args.steps for k, v in prof.items()},
+        "stages_ms_per_step": {k: v["ms"] / n_prof for k, v in prof.items()},
         "gpu_launches": launches,
         "device_status": status,
         "clocks": clk,

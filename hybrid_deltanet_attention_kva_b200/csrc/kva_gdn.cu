@@ -90,8 +90,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
         float2 x1 = F16<TM>::unpack((&raw[i + 1].x)[e / 2]);
         float2 x2 = F16<TM>::unpack((&raw[i + 2].x)[e / 2]);
         float2 x3 = F16<TM>::unpack((&raw[i + 3].x)[e / 2]);
-        z[e] = silu_f(w[e][0] * x0.x + w[e][1] * x1.x + w[e][2] * x2.x + w[e][3] * x3.x);
-        z[e + 1] = silu_f(w[e + 1][0] * x0.y + w[e + 1][1] * x1.y + w[e + 1][2] * x2.y +
+        z[e] = silu_tanh(w[e][0] * x0.x + w[e][1] * x1.x + w[e][2] * x2.x + w[e][3] * x3.x);
+        z[e + 1] = silu_tanh(w[e + 1][0] * x0.y + w[e + 1][1] * x1.y + w[e + 1][2] * x2.y +
                           w[e + 1][3] * x3.y);
       }
       float ss = 0.f;

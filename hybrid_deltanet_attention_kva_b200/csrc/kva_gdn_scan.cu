@@ -73,18 +73,19 @@ struct Cp {
   static constexpr int ALLOC = BYTES + 1024;       // slack for 1024-byte alignment (TMA tile)
 };
 
-// grid (value head, chunk, sequence x layer): the value heads that share a key head
+// grid (value head, chunk, sequence x layer in [l0, l0 + nl)): the value heads that share a key head
 // are neighbours, so their K tile is read from L2.  4 warps; warp w owns the 16
 // rows [16 w, 16 w + 16) of K K^T and L.
 __global__ void __launch_bounds__(Cp::THREADS, 6)
-    gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap mK, const GdnLaunch p) {
+    gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap mK, const GdnLaunch p, int l0, int nl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* kbar = reinterpret_cast<uint64_t*>(sm + Cp::BAR);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, lr = lane & 7;
-  const int h = blockIdx.x, c = blockIdx.y, slot = blockIdx.z;
+  const int h = blockIdx.x, c = blockIdx.y;
+  const int slot = (blockIdx.z / nl) * p.n_gdn + l0 + blockIdx.z % nl;  // layers [l0, l0 + nl)
   const int T = p.T, n_v = p.n_v;
   const int kh = h / (n_v / p.n_k);
   const int n_chunks = (T + SCH - 1) / SCH;
@@ -341,7 +342,7 @@ constexpr uint32_t ID_S = idesc_f16kind_f32_major(128, 128, 0, false, true);   /
 
 __global__ void __launch_bounds__(NTHREADS, 2)
     gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
-                       const __grid_constant__ CUtensorMap mB, const GdnLaunch p) {
+                       const __grid_constant__ CUtensorMap mB, const GdnLaunch p, int l0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, hc = warp >> 2;  // TMEM lane quarter, column half
-  const int h = blockIdx.x, layer = blockIdx.y, seq = blockIdx.z;
+  const int h = blockIdx.x, layer = l0 + blockIdx.y, seq = blockIdx.z;
   const int n_v = p.n_v;
   const int kh = h / (n_v / p.n_k);
   const int T = p.T;
@@ -588,35 +589,58 @@ void gdn_chunk_split(void* base, int n_seq, int n_gdn, int n_v, int T, void** b1
   *sc = base ? reinterpret_cast<float*>(static_cast<uint8_t*>(base) + units * B1_BYTES) : nullptr;
 }
 
-int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s) {
+static int check_scan_tc(const GdnLaunch& g) {
   if (g.d_k != SD || g.d_v != SD) return KVA_ERR_UNSUPPORTED;
   if (!g.b1buf || !g.scbuf) return KVA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(g.kbuf) | reinterpret_cast<uintptr_t>(g.vbuf) |
        reinterpret_cast<uintptr_t>(g.b1buf) | reinterpret_cast<uintptr_t>(g.scbuf)) & 15u)
     return KVA_ERR_ALIGNMENT;
+  return KVA_OK;
+}
+
+int launch_gdn_chunk_prep(const GdnLaunch& g, int l0, int nl, cudaStream_t s) {
+  if (g.T == 0 || nl <= 0 || g.n_seq == 0) return KVA_OK;
+  int e = check_scan_tc(g);
+  if (e) return e;
+  if (l0 < 0 || l0 + nl > g.n_gdn) return KVA_ERR_INVALID_ARG;
   const int n_chunks = (g.T + SCH - 1) / SCH;
   const int64_t slots = static_cast<int64_t>(g.n_seq) * g.n_gdn;
-  // chunk preparation
-  CUtensorMap mK, mV, mB;
+  CUtensorMap mK;
   if (!make_map_3d_16bit(&mK, g.kbuf, true, static_cast<int64_t>(g.n_k) * SD, g.T, slots, 64, SCH))
     return KVA_ERR_CUDA;
   if (cudaFuncSetAttribute(gdn_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cp::ALLOC) != cudaSuccess)
     return KVA_ERR_CUDA;
-  dim3 gp(g.n_v, n_chunks, static_cast<unsigned>(slots));
-  gdn_chunk_prep_kernel<<<gp, Cp::THREADS, Cp::ALLOC, s>>>(mK, g);
-  if (cudaPeekAtLastError() != cudaSuccess) return KVA_ERR_CUDA;
-  // state chain
-  if (!make_map_3d_16bit(&mV, g.vbuf, true, static_cast<int64_t>(g.n_v) * SD, g.T, slots, 64, SCH) ||
+  dim3 gp(g.n_v, n_chunks, static_cast<unsigned>(g.n_seq * nl));
+  gdn_chunk_prep_kernel<<<gp, Cp::THREADS, Cp::ALLOC, s>>>(mK, g, l0, nl);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+int launch_gdn_chain(const GdnLaunch& g, int l0, int nl, cudaStream_t s) {
+  if (g.T == 0 || nl <= 0 || g.n_seq == 0) return KVA_OK;
+  int e = check_scan_tc(g);
+  if (e) return e;
+  if (l0 < 0 || l0 + nl > g.n_gdn || !g.state) return KVA_ERR_INVALID_ARG;
+  const int n_chunks = (g.T + SCH - 1) / SCH;
+  const int64_t slots = static_cast<int64_t>(g.n_seq) * g.n_gdn;
+  CUtensorMap mK, mV, mB;
+  if (!make_map_3d_16bit(&mK, g.kbuf, true, static_cast<int64_t>(g.n_k) * SD, g.T, slots, 64, SCH) ||
+      !make_map_3d_16bit(&mV, g.vbuf, true, static_cast<int64_t>(g.n_v) * SD, g.T, slots, 64, SCH) ||
       !make_map_3d_16bit(&mB, g.b1buf, true, SCH, static_cast<int64_t>(n_chunks) * SCH,
                          slots * g.n_v, 64, SCH))
     return KVA_ERR_CUDA;
   if (cudaFuncSetAttribute(gdn_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Sc::ALLOC) != cudaSuccess)
     return KVA_ERR_CUDA;
-  dim3 grid(g.n_v, g.n_gdn, g.n_seq);
-  gdn_scan_tc_kernel<<<grid, NTHREADS, Sc::ALLOC, s>>>(mK, mV, mB, g);
+  dim3 grid(g.n_v, nl, g.n_seq);
+  gdn_scan_tc_kernel<<<grid, NTHREADS, Sc::ALLOC, s>>>(mK, mV, mB, g, l0);
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s) {
+  int e = launch_gdn_chunk_prep(g, 0, g.n_gdn, s);
+  if (e) return e;
+  return launch_gdn_chain(g, 0, g.n_gdn, s);
 }
 
 }  // namespace kva

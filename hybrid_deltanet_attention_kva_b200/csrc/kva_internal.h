@@ -82,6 +82,10 @@ int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s);
 int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s);  // d_k = d_v = 128
+// the two halves of launch_gdn_scan_tc for the layers [l0, l0 + nl): B1 and scalars
+// (no state), then the state chain (reads what the first wrote for those layers)
+int launch_gdn_chunk_prep(const GdnLaunch& g, int l0, int nl, cudaStream_t s);
+int launch_gdn_chain(const GdnLaunch& g, int l0, int nl, cudaStream_t s);
 // bytes of the per-chunk buffers (b1buf, then scbuf) the 128-dimensional scan needs
 size_t gdn_chunk_bytes(int n_seq, int n_gdn, int n_v, int T);
 // b1buf and scbuf inside a region of gdn_chunk_bytes(...) bytes at `base`
