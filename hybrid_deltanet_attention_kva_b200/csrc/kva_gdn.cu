@@ -25,14 +25,28 @@
 namespace kva {
 
 // ------------------------------------------------------------------ prepare
-// Each thread owns 8 consecutive channels (one 16-byte vector per token row) for
-// PREP_TT tokens: all raw rows are loaded up front, the conv runs in registers,
-// and the L2 norm of a q/k head is a shuffle reduction over the d_k/8 lanes that
-// hold it.  Blocks along x cover 2048 channels of one row, the last x-block of a
-// token group computes the gates.
-constexpr int PREP_TT = 16;
+// Each thread owns 8 consecutive channels (one 16-byte vector per token row) and
+// streams PREP_TT tokens: a window of the 3 previous rows (unpacked) and
+// PREP_AHEAD raw rows in flight, so every input row is loaded and unpacked once
+// and the loads of later rows overlap the arithmetic of earlier ones.  The L2 norm
+// of a q/k head is a shuffle reduction over the d_k/8 lanes that hold it.  Blocks
+// along x cover 2048 channels of the token range, the last x-block computes the
+// gates.
+constexpr int PREP_TT = 64;
+constexpr int PREP_AHEAD = 8;
 constexpr int PREP_THREADS = 256;
 constexpr int PREP_CH = PREP_THREADS * 8;
+
+template <typename TM>
+__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
+  const uint32_t* u = &v.x;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = F16<TM>::unpack(u[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
 
 template <typename TM>
 __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnLaunch p) {
@@ -40,7 +54,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
   const int seq = slot / p.n_gdn, layer = slot % p.n_gdn;
   const int T = p.T;
   const int t0 = blockIdx.y * PREP_TT;
-  const int nt = min(PREP_TT, T - t0);
+  const int tend = min(T, t0 + PREP_TT);
+  const int nt = tend - t0;
   const int C = p.C;
   const int nkdk = p.n_k * p.d_k;
   const TM* mix = static_cast<const TM*>(p.mix) + seq * p.mix_seq_stride + p.layer_col[layer];
@@ -55,19 +70,18 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
     const bool active = c0 < C;
     const int cc = active ? c0 : 0;
     const TM* tail = static_cast<const TM*>(p.conv_state) + static_cast<int64_t>(slot) * 3 * C + cc;
-    // raw rows t0-3 .. t0+PREP_TT-1 of [tail; X] for these 8 channels
-    // every load is unconditional (pointer select, zero mask after) so that all
-    // PREP_TT + 3 of them are in flight together
-    uint4 raw[PREP_TT + 3];
-#pragma unroll
-    for (int i = 0; i < PREP_TT + 3; ++i) {
-      const int t = t0 - 3 + i;
+    // raw row t of [tail; X] for these 8 channels (t >= -3; rows past T re-read row
+    // T - 1, whose values are then not used)
+    auto row = [&](int t) {
       const TM* src = t < 0 ? tail + (t + 3) * C : mix + static_cast<int64_t>(min(t, T - 1)) * ld + cc;
-      raw[i] = __ldg(reinterpret_cast<const uint4*>(src));
-    }
+      return __ldg(reinterpret_cast<const uint4*>(src));
+    };
+    uint4 q[PREP_AHEAD];
 #pragma unroll
-    for (int i = 0; i < PREP_TT + 3; ++i)
-      if (t0 - 3 + i >= T) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < PREP_AHEAD; ++j) q[j] = row(t0 + j);
+    float win[3][8];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) unpack8<TM>(row(t0 - 3 + r), win[r]);
     float w[8][4];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -81,48 +95,55 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
     const int hl = p.d_k / 8;  // lanes per q/k head
     const int64_t tbase = static_cast<int64_t>(slot) * T;
     __nv_bfloat16* dbg = static_cast<__nv_bfloat16*>(p.debug_qkv);
+    // the token loop is uniform over the block (the norm shuffles need every lane)
+    for (int tb = 0; tb < nt; tb += PREP_AHEAD) {
 #pragma unroll
-    for (int i = 0; i < PREP_TT; ++i) {
-      float z[8];
+      for (int j = 0; j < PREP_AHEAD; ++j) {
+        const int i = tb + j;
+        float x[8];
+        unpack8<TM>(q[j], x);
+        q[j] = row(t0 + i + PREP_AHEAD);
+        float z[8];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        float2 x0 = F16<TM>::unpack((&raw[i].x)[e / 2]);
-        float2 x1 = F16<TM>::unpack((&raw[i + 1].x)[e / 2]);
-        float2 x2 = F16<TM>::unpack((&raw[i + 2].x)[e / 2]);
-        float2 x3 = F16<TM>::unpack((&raw[i + 3].x)[e / 2]);
-        z[e] = silu_tanh(w[e][0] * x0.x + w[e][1] * x1.x + w[e][2] * x2.x + w[e][3] * x3.x);
-        z[e + 1] = silu_tanh(w[e + 1][0] * x0.y + w[e + 1][1] * x1.y + w[e + 1][2] * x2.y +
-                          w[e + 1][3] * x3.y);
-      }
-      float ss = 0.f;
+        for (int e = 0; e < 8; ++e)
+          z[e] = silu_tanh(w[e][0] * win[0][e] + w[e][1] * win[1][e] + w[e][2] * win[2][e] +
+                           w[e][3] * x[e]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss += z[e] * z[e];
-      for (int o = 1; o < hl; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (is_qk) {
-        const float sc = rsqrtf(ss + p.eps);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] *= sc;
-      }
-      if (active && i < nt) {
-        const int64_t t = tbase + t0 + i;
-        uint4 hv;
-        hv.x = pack_f16(z[0], z[1]);
-        hv.y = pack_f16(z[2], z[3]);
-        hv.z = pack_f16(z[4], z[5]);
-        hv.w = pack_f16(z[6], z[7]);
-        if (c0 >= 2 * nkdk) {
-          const int nvdv = C - 2 * nkdk;
-          *reinterpret_cast<uint4*>(static_cast<__half*>(p.vbuf) + t * nvdv + (c0 - 2 * nkdk)) = hv;
-        } else if (c0 >= nkdk) {
-          *reinterpret_cast<uint4*>(static_cast<__half*>(p.kbuf) + t * nkdk + (c0 - nkdk)) = hv;
+        for (int e = 0; e < 8; ++e) {
+          win[0][e] = win[1][e];
+          win[1][e] = win[2][e];
+          win[2][e] = x[e];
         }
-        if (dbg) {
-          uint4 bv;
-          bv.x = pack_bf16(z[0], z[1]);
-          bv.y = pack_bf16(z[2], z[3]);
-          bv.z = pack_bf16(z[4], z[5]);
-          bv.w = pack_bf16(z[6], z[7]);
-          *reinterpret_cast<uint4*>(dbg + t * C + c0) = bv;
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += z[e] * z[e];
+        for (int o = 1; o < hl; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (is_qk) {
+          const float sc = rsqrtf(ss + p.eps);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) z[e] *= sc;
+        }
+        if (active && i < nt) {
+          const int64_t t = tbase + t0 + i;
+          uint4 hv;
+          hv.x = pack_f16(z[0], z[1]);
+          hv.y = pack_f16(z[2], z[3]);
+          hv.z = pack_f16(z[4], z[5]);
+          hv.w = pack_f16(z[6], z[7]);
+          if (c0 >= 2 * nkdk) {
+            const int nvdv = C - 2 * nkdk;
+            *reinterpret_cast<uint4*>(static_cast<__half*>(p.vbuf) + t * nvdv + (c0 - 2 * nkdk)) = hv;
+          } else if (c0 >= nkdk) {
+            *reinterpret_cast<uint4*>(static_cast<__half*>(p.kbuf) + t * nkdk + (c0 - nkdk)) = hv;
+          }
+          if (dbg) {
+            uint4 bv;
+            bv.x = pack_bf16(z[0], z[1]);
+            bv.y = pack_bf16(z[2], z[3]);
+            bv.z = pack_bf16(z[4], z[5]);
+            bv.w = pack_bf16(z[6], z[7]);
+            *reinterpret_cast<uint4*>(dbg + t * C + c0) = bv;
+          }
         }
       }
     }

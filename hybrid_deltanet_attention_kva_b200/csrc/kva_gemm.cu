@@ -652,6 +652,25 @@ bool make_map_3d_16bit(void* map, const void* base, bool fp16, int64_t d0, int64
   return r == CUDA_SUCCESS;
 }
 
+// Split-K factor for the residual-add GEMMs (whose partial sums are added
+// atomically): the number of K ranges s in [1, 8] (each at least 4 K blocks) that
+// minimises the waves of work items per unit of K work, ceil(tiles * s / slots) / s,
+// with a small charge per extra split for its atomic traffic.
+static int choose_splits(int tiles, int slots, int num_k) {
+  int best = 1;
+  double best_cost = 1e30;
+  for (int sp = 1; sp <= 8; ++sp) {
+    if (sp > 1 && num_k / sp < 4) break;
+    const int waves = (tiles * sp + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) / sp + 0.02 * (sp - 1);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -691,11 +710,8 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
   const int num_k = (a.K + Cfg::BK - 1) / Cfg::BK;
   int splits = 1;
   if (EPI == EPI_ADD_F32) {
-    // fill about two waves with partial-K work items when the output has few tiles
     const int t = num_m * ((a.N + n_per_tile - 1) / n_per_tile);
-    splits = a.splits > 0 ? a.splits : (2 * num_sms() + t - 1) / t;
-    splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
-    while (splits > 1 && num_k / splits < 4) --splits;
+    splits = a.splits > 0 ? a.splits : choose_splits(t, num_sms(), num_k);
   }
   p.splits = splits;
   const int tiles = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
@@ -745,9 +761,7 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   int splits = 1;
   if (EPI == EPI_ADD_F32) {
     const int t = num_m * ((a.N + n_per_tile - 1) / n_per_tile);
-    splits = a.splits > 0 ? a.splits : (2 * max_cl + t - 1) / t;
-    splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
-    while (splits > 1 && num_k / splits < 4) --splits;
+    splits = a.splits > 0 ? a.splits : choose_splits(t, max_cl, num_k);
   }
   p.splits = splits;
   const int items = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
