@@ -53,6 +53,9 @@ def parse():
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kernel-case", choices=["heads", "gdn", "attention"], default=None,
+                    help="run a small case of one hot kernel three times and exit (for ncu "
+                         "captures; prints no JSON line)")
     return ap.parse_args()
 
 
@@ -407,8 +410,53 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_case(case):
+    """Small cases of the hot kernels, each above L2 in size where the kernel streams HBM:
+    heads   - the heads GEMM's CTA-pair kernel on M = 1024, K = 3072, N = 49 152 (302 MB of
+              weights, 1/5.8 of the r3 head matrix)
+    gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
+              T = 1024, every launch on the caller's stream
+    attention - one block-causal attention of the r3 trunk (T = 1024, 24 heads, window 1024)"""
+    import hybrid_deltanet_attention_kva_b200 as K
+    torch.manual_seed(0)
+    if case == "heads":
+        M, Kd, N = 1024, 3072, 49152
+        A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+        B = (torch.randn(N, Kd, device="cuda") * 0.02).half()
+        D = torch.empty(M, N, dtype=torch.half, device="cuda")
+        for _ in range(3):
+            K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512)
+    elif case == "gdn":
+        geom = KI.with_changes(KI.R3, layer_types=KI.R3.layer_types[:8], n_draft=0)
+        P = KI.make_layer_params(geom, 2)
+        st = KI.make_states(geom, 1, 3, std=0.1)
+        mix = KI.make_mixer_inputs(geom, 1, T_UB, 4, device="cuda").half()
+        S, tail = st["state"].cuda(), st["conv_tail"].cuda().half()
+        kc = [torch.zeros(1, geom.attn_n_kv, 4096, geom.attn_d_h, dtype=torch.bfloat16, device="cuda")
+              for _ in range(geom.n_attn)]
+        kv = K.KvCache(kc, [torch.zeros_like(k) for k in kc], max_pos=4096)
+        Wt = K.Weights(layer={k: x.cuda() for k, x in P.items()})
+        h = K.kva_init(K.make_dims(geom, T_UB, 1, dtype=torch.float16))
+        K.kva_profile_enable(h, 64)
+        for _ in range(3):
+            K.kva_update_states(h, mix, [0], Wt, S, tail, kv)
+        torch.cuda.synchronize()
+        K.kva_profile_read(h)
+        K.kva_free(h)
+    else:
+        T, heads = T_UB, KI.R3.n_heads
+        qkv = torch.randn(T, 3 * heads * 128, device="cuda").half()
+        out = torch.empty(T, heads * 128, dtype=torch.half, device="cuda")
+        for _ in range(3):
+            K.kva_op_attention(qkv, out, heads, KI.R3.window)
+    torch.cuda.synchronize()
+
+
 def main():
     args = parse()
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case)
+        return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
