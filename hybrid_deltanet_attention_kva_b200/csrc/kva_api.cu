@@ -40,10 +40,6 @@ struct kva_handle {
   int* status = nullptr;          // device status word
   void* chunk = nullptr;          // per-chunk B1 and scalars of the 128-dimensional scan
   cudaStream_t last_stream = nullptr;
-  // a second stream on which the 128-dimensional state chains of one group of layers
-  // run while the caller's stream prepares the next group (ordered by events)
-  cudaStream_t aux = nullptr;
-  cudaEvent_t ov[9] = {nullptr};  // [0, 8): group prepared; [8]: all chains done
   int64_t tokens = 0;
   // profiling: event pairs around launches, launch counters per stage kind
   cudaEvent_t* ev = nullptr;
@@ -198,16 +194,6 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
                        const kva_kv_cache* kv, void* debug_qkv, void* debug_gb, cudaStream_t s) {
   const kva_dims& d = h->d;
   int e = KVA_OK;
-  bool overlap = false;
-  // the caller's stream waits for the chains queued on the aux stream, on every exit
-  auto join = [&](int status) {
-    if (overlap) {
-      const int j = cuda_ok(cudaEventRecord(h->ov[8], h->aux));
-      const int w = j ? j : cuda_ok(cudaStreamWaitEvent(s, h->ov[8], 0));
-      if (!status) status = w;
-    }
-    return status;
-  };
   if (h->n_gdn) {
     GdnLaunch g;
     g.mix = mix;
@@ -237,26 +223,8 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     g.mix_dtype = d.compute_dtype;
     if ((e = staged(h, KVA_ST_GDN_PREPARE, s, [&] { return launch_gdn_prepare(g, s); }))) return e;
     if ((e = staged(h, KVA_ST_GDN_TAIL, s, [&] { return launch_gdn_tail(g, s); }))) return e;
-    // Without profiling, the 128-dimensional scan overlaps its two kernels across
-    // layer groups: the chain of group i (aux stream) runs while group i + 1 is
-    // prepared (and the KV rows are written) on the caller's stream.  Profiling keeps
-    // every launch on the caller's stream so that each one can be timed alone.
-    if (d.gdn_d_k == 128 && h->ev_cap == 0 && h->aux) {
-      const int G = h->n_gdn < 4 ? h->n_gdn : 4;
-      overlap = true;
-      for (int i = 0; i < G; ++i) {
-        const int l0 = h->n_gdn * i / G, l1 = h->n_gdn * (i + 1) / G;
-        if ((e = launch_gdn_chunk_prep(g, l0, l1 - l0, s))) break;
-        if ((e = cuda_ok(cudaEventRecord(h->ov[i], s)))) break;
-        if ((e = cuda_ok(cudaStreamWaitEvent(h->aux, h->ov[i], 0)))) break;
-        if ((e = launch_gdn_chain(g, l0, l1 - l0, h->aux))) break;
-        h->launches[KVA_ST_GDN_SCAN] += 2;
-      }
-      if (e) return join(e);
-    } else {
-      if ((e = staged(h, KVA_ST_GDN_SCAN, s, [&] { return launch_gdn_scan(g, s); }))) return e;
-      if (d.gdn_d_k == 128) ++h->launches[KVA_ST_GDN_SCAN];  // two kernels
-    }
+    if ((e = staged(h, KVA_ST_GDN_SCAN, s, [&] { return launch_gdn_scan(g, s); }))) return e;
+    if (d.gdn_d_k == 128) ++h->launches[KVA_ST_GDN_SCAN];  // two kernels
   }
   if (h->n_attn) {
     KvLaunch k;
@@ -277,9 +245,9 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     k.eps = d.norm_eps;
     k.err = h->status;
     k.mix_dtype = d.compute_dtype;
-    if ((e = staged(h, KVA_ST_KV_WRITE, s, [&] { return launch_kv_write(k, s); }))) return join(e);
+    if ((e = staged(h, KVA_ST_KV_WRITE, s, [&] { return launch_kv_write(k, s); }))) return e;
   }
-  return join(KVA_OK);
+  return KVA_OK;
 }
 
 }  // namespace
@@ -342,17 +310,8 @@ int kva_init(const kva_dims* dims, kva_handle** out) {
   h->gbuf = reinterpret_cast<float*>(b + L.off[8]);
   h->status = reinterpret_cast<int*>(b + L.off[9]);
   h->chunk = b + L.off[10];
-  bool ok = cudaMemset(h->status, 0, 256) == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
-  if (ok && h->n_gdn && dims->gdn_d_k == 128) {
-    ok = cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking) == cudaSuccess;
-    for (int i = 0; ok && i < 9; ++i)
-      ok = cudaEventCreateWithFlags(&h->ov[i], cudaEventDisableTiming) == cudaSuccess;
-  }
-  if (!ok) {
+  if (cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
-    for (int i = 0; i < 9; ++i)
-      if (h->ov[i]) cudaEventDestroy(h->ov[i]);
-    if (h->aux) cudaStreamDestroy(h->aux);
     cudaFree(h->ws);
     delete h;
     return KVA_ERR_CUDA;
@@ -440,9 +399,6 @@ void kva_free(kva_handle* h) {
     cudaGetDevice(&cur);
     cudaSetDevice(h->device);
     cudaDeviceSynchronize();
-    for (int i = 0; i < 9; ++i)
-      if (h->ov[i]) cudaEventDestroy(h->ov[i]);
-    if (h->aux) cudaStreamDestroy(h->aux);
     cudaFree(h->ws);
     cudaSetDevice(cur);
   }
