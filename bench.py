@@ -53,7 +53,7 @@ def parse():
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--kernel-case", choices=["heads", "gdn", "attention"], default=None,
+    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "gdn", "attention"], default=None,
                     help="run a small case of one hot kernel three times and exit (for ncu "
                          "captures; prints no JSON line)")
     return ap.parse_args()
@@ -414,6 +414,8 @@ def run_kernel_case(case):
     """Small cases of the hot kernels, each above L2 in size where the kernel streams HBM:
     heads   - the heads GEMM's CTA-pair kernel on M = 1024, K = 3072, N = 49 152 (302 MB of
               weights, 1/5.8 of the r3 head matrix)
+    heads_fused - kva_prefill_ubatch with the first 8 r3 late layers (6 gated-DeltaNet, 2
+              attention, no drafter): the heads GEMM with the state-update epilogue
     gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
               T = 1024, every launch on the caller's stream
     attention - one block-causal attention of the r3 trunk (T = 1024, 24 heads, window 1024)"""
@@ -426,6 +428,24 @@ def run_kernel_case(case):
         D = torch.empty(M, N, dtype=torch.half, device="cuda")
         for _ in range(3):
             K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512)
+    elif case == "heads_fused":
+        geom = KI.with_changes(KI.R3, layer_types=KI.R3.layer_types[:8], n_draft=0)
+        W = KI.make_projector_weights(geom, 1003, device="cuda")
+        W = {k: (v if k.startswith("g_") or k == "blocks" else v.half()) for k, v in W.items()}
+        W["blocks"] = [{k: (v if k.startswith("g_") else v.half()) for k, v in b.items()}
+                       for b in W["blocks"]]
+        P = {k: v.cuda() for k, v in KI.make_layer_params(geom, 2).items()}
+        st = KI.make_states(geom, 1, 3, std=0.1)
+        S, tail = st["state"][0].cuda(), st["conv_tail"][0].cuda().half()
+        res = KI.make_residual(geom, T_UB, 4, device="cuda")
+        kc = [torch.zeros(1, geom.attn_n_kv, 4096, geom.attn_d_h, dtype=torch.bfloat16, device="cuda")
+              for _ in range(geom.n_attn)]
+        kv = K.KvCache(kc, [torch.zeros_like(k) for k in kc], max_pos=4096)
+        h = K.kva_init(K.make_dims(geom, T_UB, 1, dtype=torch.float16))
+        for _ in range(3):
+            K.kva_prefill_ubatch(h, res, K.Weights(proj=W, layer=P), S, tail, kv, 0)
+        torch.cuda.synchronize()
+        K.kva_free(h)
     elif case == "gdn":
         geom = KI.with_changes(KI.R3, layer_types=KI.R3.layer_types[:8], n_draft=0)
         P = KI.make_layer_params(geom, 2)

@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "../../include/kva.h"
 #include "../../include/kva_ops.h"
@@ -39,6 +40,13 @@ struct kva_handle {
   float* gbuf = nullptr;          // [max_seq, n_gdn, 2, n_v, max_T]
   int* status = nullptr;          // device status word
   void* chunk = nullptr;          // per-chunk B1 and scalars of the 128-dimensional scan
+  // heads GEMM with the state-update epilogue (kva_prefill_ubatch), when the dims allow it
+  bool fused = false;
+  MixTile* tiles = nullptr;       // device table: [n_tiles], drafter tiles last
+  int n_tiles = 0, n_tiles_draft = 0;
+  void* halo = nullptr;           // raw rows around 128-token block edges
+  void* tail_new = nullptr;       // raw last 3 rows of the ubatch
+  int nblk = 0;
   cudaStream_t last_stream = nullptr;
   int64_t tokens = 0;
   // profiling: event pairs around launches, launch counters per stage kind
@@ -67,7 +75,7 @@ int staged(kva_handle* h, int kind, cudaStream_t s, F&& launch) {
 namespace {
 
 struct Layout {
-  size_t off[12];
+  size_t off[15];
   size_t total;
 };
 
@@ -116,11 +124,28 @@ int derive(const kva_dims* d, int* n_gdn, int* n_attn, int64_t* n_mix) {
   return KVA_OK;
 }
 
+// The fused heads epilogue needs 128-dim DeltaNet heads, key/value widths in whole
+// 256-column tiles, the gates in one tile, 256-dim attention heads with 64 rotary dims.
+bool fused_ok(const kva_dims* d, int ng, int na) {
+  if (ng) {
+    if (d->gdn_d_k != 128 || d->gdn_d_v != 128) return false;
+    if ((d->gdn_n_k * 128) % 256 || (d->gdn_n_v * 128) % 256 || 2 * d->gdn_n_v > 256) return false;
+  }
+  if (na && (d->attn_d_h != 256 || d->rope_dims != 64)) return false;
+  return d->n_draft_cols % 8 == 0;
+}
+
+int fused_tiles(const kva_dims* d, int ng, int na, int* n_draft_tiles) {
+  const int per_gdn = 2 * (d->gdn_n_k * 128 / 256) + d->gdn_n_v * 128 / 256 + 1;
+  *n_draft_tiles = (d->n_draft_cols + 255) / 256;
+  return ng * per_gdn + na * 2 * d->attn_n_kv + *n_draft_tiles;
+}
+
 Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
   const size_t T = d->max_T, S = d->max_seq;
   const size_t dm = d->d_model;
   const size_t C = 2ull * d->gdn_n_k * d->gdn_d_k + (size_t)d->gdn_n_v * d->gdn_d_v;
-  size_t sz[11];
+  size_t sz[14];
   sz[0] = T * d->hidden * 2;                                          // u_in
   sz[1] = T * dm * 2;                                                 // u
   sz[2] = T * dm * 4;                                                 // x
@@ -132,10 +157,17 @@ Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
   sz[8] = S * ng * 2 * (size_t)d->gdn_n_v * T * 4;                    // gbuf
   sz[9] = 256;                                                        // status
   sz[10] = d->gdn_d_k == 128 ? gdn_chunk_bytes((int)S, ng, d->gdn_n_v, (int)T) : 0;  // B1, scalars
-  (void)C;
+  int na = 0;
+  for (int i = 0; i < d->n_late; ++i) na += d->layer_type[i] == KVA_LAYER_ATTN;
+  const bool fz = fused_ok(d, ng, na);
+  int ndt = 0;
+  const size_t nblk = (T + 127) / 128;
+  sz[11] = fz ? ng * nblk * kMixHaloRows * C * 2 : 0;                      // halo rows
+  sz[12] = fz ? ng * 3 * C * 2 : 0;                                         // last rows
+  sz[13] = fz ? fused_tiles(d, ng, na, &ndt) * sizeof(MixTile) : 0;         // tile table
   Layout L;
   size_t o = 0;
-  for (int i = 0; i < 11; ++i) {
+  for (int i = 0; i < 14; ++i) {
     L.off[i] = o;
     o += align_up(sz[i]);
   }
@@ -189,14 +221,17 @@ int check_cache(const kva_handle* h, const kva_kv_cache* kv, int n_seq, const in
   return KVA_OK;
 }
 
+// fz: the heads GEMM already ran the fused epilogue (conv outputs except block edges,
+// gates, KV rows); only the edge fix-up, the conv tail and the scan remain.
 int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq, int T,
                        const int64_t* pos, const kva_weights* w, float* state, void* conv_state,
-                       const kva_kv_cache* kv, void* debug_qkv, void* debug_gb, cudaStream_t s) {
+                       const kva_kv_cache* kv, void* debug_qkv, void* debug_gb, cudaStream_t s,
+                       const MixParams* fz = nullptr) {
   const kva_dims& d = h->d;
   int e = KVA_OK;
   if (h->n_gdn) {
     GdnLaunch g;
-    g.mix = mix;
+    g.mix = fz ? static_cast<const void*>(h->kbuf) : mix;  // (unread when fused)
     g.mix_ld = mix_ld;
     g.mix_seq_stride = (int64_t)T * mix_ld;
     g.n_seq = n_seq;
@@ -221,12 +256,22 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     g.eps = d.norm_eps;
     g.err = h->status;
     g.mix_dtype = d.compute_dtype;
-    if ((e = staged(h, KVA_ST_GDN_PREPARE, s, [&] { return launch_gdn_prepare(g, s); }))) return e;
-    if ((e = staged(h, KVA_ST_GDN_TAIL, s, [&] { return launch_gdn_tail(g, s); }))) return e;
+    if (fz) {
+      if ((e = staged(h, KVA_ST_GDN_PREPARE, s, [&] {
+             return launch_gdn_halo_fix(*fz, h->n_gdn, s, d.compute_dtype, conv_state);
+           })))
+        return e;
+      if ((e = staged(h, KVA_ST_GDN_TAIL, s,
+                      [&] { return launch_gdn_tail_fused(*fz, h->n_gdn, conv_state, s); })))
+        return e;
+    } else {
+      if ((e = staged(h, KVA_ST_GDN_PREPARE, s, [&] { return launch_gdn_prepare(g, s); }))) return e;
+      if ((e = staged(h, KVA_ST_GDN_TAIL, s, [&] { return launch_gdn_tail(g, s); }))) return e;
+    }
     if ((e = staged(h, KVA_ST_GDN_SCAN, s, [&] { return launch_gdn_scan(g, s); }))) return e;
     if (d.gdn_d_k == 128) ++h->launches[KVA_ST_GDN_SCAN];  // two kernels
   }
-  if (h->n_attn) {
+  if (h->n_attn && !fz) {
     KvLaunch k;
     k.mix = mix;
     k.mix_ld = mix_ld;
@@ -310,6 +355,47 @@ int kva_init(const kva_dims* dims, kva_handle** out) {
   h->gbuf = reinterpret_cast<float*>(b + L.off[8]);
   h->status = reinterpret_cast<int*>(b + L.off[9]);
   h->chunk = b + L.off[10];
+  h->fused = fused_ok(dims, ng, na);
+  if (h->fused) {
+    h->halo = b + L.off[11];
+    h->tail_new = b + L.off[12];
+    h->tiles = reinterpret_cast<MixTile*>(b + L.off[13]);
+    h->nblk = (dims->max_T + 127) / 128;
+    // the tile table: every tile inside one layer segment, drafter tiles last
+    std::vector<MixTile> tab;
+    const int nkdk = dims->gdn_n_k * 128, nvdv = dims->gdn_n_v * 128;
+    int gi = 0, ai = 0;
+    for (int i = 0; i < dims->n_late; ++i) {
+      if (dims->layer_type[i] == KVA_LAYER_GDN) {
+        const int c = h->gdn_col[gi];
+        for (int j = 0; j < nkdk; j += 256) tab.push_back({c + j, 256, MIX_RAW, gi, j});
+        for (int j = 0; j < nkdk; j += 256) tab.push_back({c + nkdk + j, 256, MIX_GDN_K, gi, nkdk + j});
+        for (int j = 0; j < nvdv; j += 256)
+          tab.push_back({c + 2 * nkdk + j, 256, MIX_GDN_V, gi, 2 * nkdk + j});
+        tab.push_back({c + h->C, 2 * dims->gdn_n_v, MIX_GDN_AB, gi, 0});
+        ++gi;
+      } else {
+        const int c = h->attn_col[ai];
+        for (int j = 0; j < dims->attn_n_kv; ++j) tab.push_back({c + 256 * j, 256, MIX_ATT_K, ai, j});
+        for (int j = 0; j < dims->attn_n_kv; ++j)
+          tab.push_back({c + 256 * (dims->attn_n_kv + j), 256, MIX_ATT_V, ai, j});
+        ++ai;
+      }
+    }
+    h->n_tiles = static_cast<int>(tab.size());
+    for (int j = 0; j < dims->n_draft_cols; j += 256) {
+      const int w = dims->n_draft_cols - j < 256 ? dims->n_draft_cols - j : 256;
+      tab.push_back({static_cast<int>(nm) + j, w, MIX_DRAFT, 0, j});
+    }
+    h->n_tiles_draft = static_cast<int>(tab.size()) - h->n_tiles;
+    if (cudaMemcpy(h->tiles, tab.data(), tab.size() * sizeof(MixTile), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(h->ws);
+      delete h;
+      return KVA_ERR_CUDA;
+    }
+  }
   if (cudaMemset(h->status, 0, 256) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     cudaFree(h->ws);
@@ -426,7 +512,9 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   if ((e = check_cache(h, kv, 1, &pos, T))) return e;
   if (mixer_out && !a16(mixer_out)) return KVA_ERR_ALIGNMENT;
   if (draft_out && (!a16(draft_out) || d.n_draft_cols == 0)) return KVA_ERR_INVALID_ARG;
-  if (h->n_mix % 32 && draft_out) return KVA_ERR_UNSUPPORTED;
+  // the plain path splits the heads GEMM's output at n_mix (a multiple of its 32-column
+  // epilogue chunks); the fused path writes the drafter tiles on their own
+  if (!h->fused && h->n_mix % 32 && draft_out) return KVA_ERR_UNSUPPORTED;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int cur = 0;
@@ -545,7 +633,44 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
          return launch_rmsnorm(h->x, KVA_F32, dm, w->g_out, h->u, dm, T, dm, eps, s, cd);
        })))
     goto done;
-  {
+  if (h->fused) {
+    // the heads GEMM writes the state updates' inputs directly (no mixer round trip)
+    MixParams mp;
+    mp.tiles = h->tiles;
+    mp.T = T;
+    mp.pos = pos;
+    mp.n_k = d.gdn_n_k;
+    mp.n_v = d.gdn_n_v;
+    mp.C = h->C;
+    mp.conv_w = w->conv_w;
+    mp.A_log = w->A_log;
+    mp.dt_bias = w->dt_bias;
+    mp.kbuf = h->kbuf;
+    mp.vbuf = h->vbuf;
+    mp.gbuf = h->gbuf;
+    mp.halo = h->halo;
+    mp.tail_new = h->tail_new;
+    mp.nblk = h->nblk;
+    mp.eps = eps;
+    mp.n_kv = d.attn_n_kv;
+    mp.k_gain = w->k_norm_g;
+    mp.rope_dims = d.rope_dims;
+    mp.rope_theta = d.rope_theta;
+    if (h->n_attn) mp.cache = *kv;
+    mp.draft = draft_out;
+    mp.ld_draft = d.n_draft_cols;
+    mp.mixer_out = mixer_out;
+    mp.ld_mix = h->n_mix;
+    mp.err = h->status;
+    const int nt = h->n_tiles + (draft_out ? h->n_tiles_draft : 0);
+    if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] {
+           return launch_heads_fused(cd, h->u, dm, w->W_heads, h->n_mix + d.n_draft_cols, T, dm, nt,
+                                     mp, s);
+         })))
+      goto done;
+    e = update_states_impl(h, nullptr, 0, 1, T, &pos, w, deltanet_state, conv_state, kv, nullptr,
+                           nullptr, s, &mp);
+  } else {
     __nv_bfloat16* mix = mixer_out ? static_cast<__nv_bfloat16*>(mixer_out) : h->mixer;
     GemmArgs hd;
     hd.A = h->u;

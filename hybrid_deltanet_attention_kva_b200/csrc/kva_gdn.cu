@@ -612,6 +612,106 @@ int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s) {
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ after the fused heads GEMM
+// The heads GEMM's state-update epilogue (kva_gemm.cu) convolves every token whose 3
+// predecessors lie in the same 128-token block.  The first 3 tokens of each block are
+// done here from the raw rows it kept around block edges (and the old conv tail for
+// block 0): the same conv + SiLU + L2 norm as gdn_prepare_kernel.  Grid (block, layer,
+// 2048-channel group of the k | v channels), 8 channels per thread.
+template <typename TM>
+__global__ void __launch_bounds__(256) gdn_halo_fix_kernel(const MixParams mp, const void* conv_state) {
+  const int b = blockIdx.x, layer = blockIdx.y;
+  const int nkdk = mp.n_k * 128;
+  const int c0 = nkdk + blockIdx.z * 2048 + threadIdx.x * 8;  // conv channel (k or v)
+  const int C = mp.C;
+  const bool active = c0 < C;
+  const int cc = active ? c0 : nkdk;
+  const TM* halo = static_cast<const TM*>(mp.halo);
+  const TM* tail = static_cast<const TM*>(conv_state) + static_cast<int64_t>(layer) * 3 * C;
+  auto raw = [&](int u) {  // raw row u (>= -3) of [old tail; X] for these 8 channels
+    const TM* src;
+    if (u >= 128 * b) src = halo + ((static_cast<int64_t>(layer) * mp.nblk + b) * kMixHaloRows + (u - 128 * b)) * C;
+    else if (u >= 0) src = halo + ((static_cast<int64_t>(layer) * mp.nblk + b - 1) * kMixHaloRows + (u - 128 * b + 6)) * C;
+    else src = tail + static_cast<int64_t>(u + 3) * C;
+    return *reinterpret_cast<const uint4*>(src + cc);
+  };
+  float w[8][4];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float4 wv = *reinterpret_cast<const float4*>(mp.conv_w + (static_cast<int64_t>(layer) * C + cc + e) * 4);
+    w[e][0] = wv.x;
+    w[e][1] = wv.y;
+    w[e][2] = wv.z;
+    w[e][3] = wv.w;
+  }
+  const bool is_k = c0 < 2 * nkdk;
+#pragma unroll 1
+  for (int i = 0; i < 3; ++i) {
+    const int t = 128 * b + i;
+    if (t >= mp.T) break;  // uniform over the block
+    float x[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack8<TM>(raw(t - 3 + j), x[j]);
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      z[e] = silu_tanh(w[e][0] * x[0][e] + w[e][1] * x[1][e] + w[e][2] * x[2][e] + w[e][3] * x[3][e]);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss += z[e] * z[e];
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);  // 16 lanes = one head
+    if (is_k) {
+      const float sc = rsqrtf(ss + mp.eps);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] *= sc;
+    }
+    if (active) {
+      uint4 hv;
+      hv.x = pack_f16(z[0], z[1]);
+      hv.y = pack_f16(z[2], z[3]);
+      hv.z = pack_f16(z[4], z[5]);
+      hv.w = pack_f16(z[6], z[7]);
+      const int64_t row = static_cast<int64_t>(layer) * mp.T + t;
+      if (is_k)
+        *reinterpret_cast<uint4*>(static_cast<__half*>(mp.kbuf) + row * nkdk + (c0 - nkdk)) = hv;
+      else
+        *reinterpret_cast<uint4*>(static_cast<__half*>(mp.vbuf) + row * (C - 2 * nkdk) + (c0 - 2 * nkdk)) = hv;
+    }
+  }
+}
+
+// New conv tail from the last raw rows the fused epilogue kept (raw row T-3+i, or old
+// tail row T+i when T < 3); ascending i reads only rows not yet overwritten.
+__global__ void gdn_tail_fused_kernel(const MixParams mp, void* conv_state) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= mp.C) return;
+  const int layer = blockIdx.y;
+  const uint16_t* tn = static_cast<const uint16_t*>(mp.tail_new) + static_cast<int64_t>(layer) * 3 * mp.C + c;
+  uint16_t* tail = static_cast<uint16_t*>(conv_state) + static_cast<int64_t>(layer) * 3 * mp.C + c;
+  for (int i = 0; i < 3; ++i) {
+    const int u = mp.T - 3 + i;
+    tail[i * mp.C] = u >= 0 ? tn[i * mp.C] : tail[(mp.T + i) * mp.C];
+  }
+}
+
+int launch_gdn_halo_fix(const MixParams& mp, int n_gdn, cudaStream_t s, int dtype, const void* conv_state) {
+  if (mp.T == 0 || n_gdn == 0) return KVA_OK;
+  const int nkdk = mp.n_k * 128;
+  if ((mp.C - nkdk) % 8 || nkdk % 128) return KVA_ERR_UNSUPPORTED;
+  dim3 grid((mp.T + 127) / 128, n_gdn, (mp.C - nkdk + 2047) / 2048);
+  if (dtype == KVA_F16) gdn_halo_fix_kernel<__half><<<grid, 256, 0, s>>>(mp, conv_state);
+  else gdn_halo_fix_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(mp, conv_state);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+int launch_gdn_tail_fused(const MixParams& mp, int n_gdn, void* conv_state, cudaStream_t s) {
+  if (mp.T == 0 || n_gdn == 0) return KVA_OK;
+  dim3 grid((mp.C + 255) / 256, n_gdn);
+  gdn_tail_fused_kernel<<<grid, 256, 0, s>>>(mp, conv_state);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
 template <int D>
 static int launch_scan_d(const GdnLaunch& g, cudaStream_t s) {
   constexpr int bytes = ScanLayout<D>::BYTES;

@@ -64,7 +64,9 @@ __device__ __forceinline__ void store16x32(T* dst, const float* v, int valid) {
       reinterpret_cast<uint4*>(dst)[q] = pk;
     }
   } else {
-    for (int i = 0; i < valid; ++i) dst[i] = F16<T>::from(v[i]);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid) dst[i] = F16<T>::from(v[i]);
   }
 }
 
@@ -362,6 +364,322 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 
+// ------------------------------------------------------------------ state-update epilogue
+// The heads GEMM's accumulator tile (128 tokens x 256 columns of one layer segment per
+// CTA of the pair) goes straight to the state updates' inputs.  Every raw value is
+// first rounded to the mixer's 16-bit format, so the results equal those of the plain
+// path (mixer stored, then the conv / norm / gate / KV kernels).  Warp q of the
+// epilogue group owns TMEM lanes (tokens) [32q, 32q+32) of the block.
+constexpr int MIX_STAGE_LD = 36;                       // floats per staged row (16-byte rows)
+constexpr int MIX_STAGE_BYTES = 128 * MIX_STAGE_LD * 4;
+
+__device__ __forceinline__ void mix_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+template <typename T>
+__device__ __forceinline__ void mix_round32(const uint32_t (&r)[32], float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 f = F16<T>::unpack(F16<T>::pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])));
+    x[i] = f.x;
+    x[i + 1] = f.y;
+  }
+}
+
+// 32 values (already in the 16-bit grid) to a 16-bit row at dst (16-byte aligned)
+template <typename T>
+__device__ __forceinline__ void mix_store32(void* dst, const float (&x)[32], int valid) {
+  store16x32<T>(static_cast<T*>(dst), x, valid);
+}
+
+// conv over tokens t-3..t of 32 channels: this thread's row is staged, rows r-1..r-3 read back
+template <typename T>
+__device__ __forceinline__ void mix_conv32(const MixParams& mp, float* stage, int r, int gdn,
+                                           int ch0, const float (&x)[32], float (&z)[32]) {
+  float* my = stage + r * MIX_STAGE_LD;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    reinterpret_cast<float4*>(my)[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+  mix_sync();
+  if (r >= 3) {
+    const float* p1 = stage + (r - 1) * MIX_STAGE_LD;
+    const float* p2 = stage + (r - 2) * MIX_STAGE_LD;
+    const float* p3 = stage + (r - 3) * MIX_STAGE_LD;
+    const float4* w4 = reinterpret_cast<const float4*>(mp.conv_w + (static_cast<int64_t>(gdn) * mp.C + ch0) * 4);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 a1 = reinterpret_cast<const float4*>(p1)[j];
+      const float4 a2 = reinterpret_cast<const float4*>(p2)[j];
+      const float4 a3 = reinterpret_cast<const float4*>(p3)[j];
+      const float x1[4] = {a1.x, a1.y, a1.z, a1.w};
+      const float x2[4] = {a2.x, a2.y, a2.z, a2.w};
+      const float x3[4] = {a3.x, a3.y, a3.z, a3.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * j + e;
+        const float4 w = w4[i];
+        z[i] = silu_tanh(w.x * x3[e] + w.y * x2[e] + w.z * x1[e] + w.w * x[i]);
+      }
+    }
+  }
+  mix_sync();
+}
+
+// raw copies of gated-DeltaNet conv channels: the rows around 128-token block edges
+// (for the edge fix-up) and the ubatch's last 3 rows (the new conv tail)
+template <typename T>
+__device__ __forceinline__ void mix_gdn_raw(const MixParams& mp, int gdn, int t, int r, int ch0,
+                                            const float (&x)[32], int valid) {
+  if (t >= mp.T) return;
+  if (r < 3 || r >= 125) {
+    const int slot = r < 3 ? r : r - 122;
+    const int64_t row = (static_cast<int64_t>(gdn) * mp.nblk + (t >> 7)) * kMixHaloRows + slot;
+    mix_store32<T>(static_cast<T*>(mp.halo) + row * mp.C + ch0, x, valid);
+  }
+  if (t >= mp.T - 3) {
+    const int64_t row = static_cast<int64_t>(gdn) * 3 + (t - (mp.T - 3));
+    mix_store32<T>(static_cast<T*>(mp.tail_new) + row * mp.C + ch0, x, valid);
+  }
+}
+
+// row index of position `p` in a KV cache (sequence 0), or -1 when the page table is out of range
+__device__ __forceinline__ int64_t mix_cache_row(const kva_kv_cache& cc, int head, int n_kv, int64_t p,
+                                                 int* err) {
+  if (cc.layout == KVA_KV_PAGED) {
+    const int64_t pg_i = p / cc.page_size;
+    if (pg_i < 0 || pg_i >= cc.pages_per_seq) {
+      set_device_error(err, KVA_DEV_PAGE_OOB);
+      return -1;
+    }
+    const int page = cc.page_table[pg_i];
+    if (page < 0 || page >= cc.n_pages) {
+      set_device_error(err, KVA_DEV_PAGE_OOB);
+      return -1;
+    }
+    return (static_cast<int64_t>(page) * n_kv + head) * cc.page_size + p % cc.page_size;
+  }
+  return static_cast<int64_t>(head) * cc.max_pos + p;
+}
+
+template <typename C16>
+__device__ __forceinline__ void mix_cache_store32(void* base, int64_t row, int c0, const float (&v)[32]) {
+  C16* dst = static_cast<C16*>(base) + row * 256 + c0;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 pk;
+    pk.x = F16<C16>::pack(v[8 * q4 + 0], v[8 * q4 + 1]);
+    pk.y = F16<C16>::pack(v[8 * q4 + 2], v[8 * q4 + 3]);
+    pk.z = F16<C16>::pack(v[8 * q4 + 4], v[8 * q4 + 5]);
+    pk.w = F16<C16>::pack(v[8 * q4 + 6], v[8 * q4 + 7]);
+    reinterpret_cast<uint4*>(dst)[q4] = pk;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tmem_acc, int row0,
+                                               int n_blk, int q, int lane, float* stage) {
+  const MixTile tl = mp.tiles[n_blk];
+  const int r = q * 32 + lane;
+  const int t = row0 + r;
+  const bool row_ok = t < mp.T;
+  const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
+  const int n_chunks = (tl.ncols + 31) / 32;
+
+  // the raw 16-bit mixer (debug copy), for every kind
+  auto mixer_copy = [&](int c0, const float (&x)[32]) {
+    if (mp.mixer_out && row_ok)
+      mix_store32<T>(static_cast<T*>(mp.mixer_out) + t * mp.ld_mix + tl.col0 + c0, x,
+                     min(32, tl.ncols - c0));
+  };
+
+  if (tl.kind == MIX_GDN_K) {
+    // two 128-channel heads; the norm needs the whole head before any output, so the
+    // head's conv outputs wait as fp16 pairs (their sum of squares is taken in fp32)
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t zk[64];
+      float ss = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c0 = hh * 128 + ch * 32;
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(taddr + c0, rr);
+        tmem_ld_wait();
+        float x[32], z[32];
+        mix_round32<T>(rr, x);
+        mixer_copy(c0, x);
+        mix_gdn_raw<T>(mp, tl.layer, t, r, tl.sub + c0, x, 32);
+        mix_conv32<T>(mp, stage, r, tl.layer, tl.sub + c0, x, z);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          ss += z[i] * z[i] + z[i + 1] * z[i + 1];
+          zk[ch * 16 + i / 2] = pack_f16(z[i], z[i + 1]);
+        }
+      }
+      if (r >= 3 && row_ok) {
+        const float sc = rsqrtf(ss + mp.eps);
+        const int nkdk = mp.n_k * 128;
+        __half* dst = static_cast<__half*>(mp.kbuf) +
+                      (static_cast<int64_t>(tl.layer) * mp.T + t) * nkdk + (tl.sub - nkdk) + hh * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 16; ++q4) {
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = F16<__half>::unpack(zk[4 * q4 + e]);
+            o[e] = pack_f16(f.x * sc, f.y * sc);
+          }
+          reinterpret_cast<uint4*>(dst)[q4] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  } else if (tl.kind == MIX_GDN_V || tl.kind == MIX_RAW) {
+#pragma unroll 1
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const int c0 = ch * 32;
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + c0, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      mixer_copy(c0, x);
+      mix_gdn_raw<T>(mp, tl.layer, t, r, tl.sub + c0, x, min(32, tl.ncols - c0));
+      if (tl.kind == MIX_GDN_V) {
+        float z[32];
+        mix_conv32<T>(mp, stage, r, tl.layer, tl.sub + c0, x, z);
+        if (r >= 3 && row_ok) {
+          const int nkdk = mp.n_k * 128, nvdv = mp.n_v * 128;
+          __half* dst = static_cast<__half*>(mp.vbuf) +
+                        (static_cast<int64_t>(tl.layer) * mp.T + t) * nvdv + (tl.sub - 2 * nkdk) + c0;
+          store16x32<__half>(dst, z, 32);
+        }
+      }
+    }
+  } else if (tl.kind == MIX_GDN_AB) {
+    // columns [0, n_v) are a, [n_v, 2 n_v) are b: g = -exp(A_log) softplus(a + dt_bias),
+    // beta = sigmoid(b), written [layer][2][n_v][T]
+#pragma unroll 1
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const int c0 = ch * 32;
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + c0, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      mixer_copy(c0, x);
+      if (!row_ok) continue;
+      float* gb = mp.gbuf + static_cast<int64_t>(tl.layer) * 2 * mp.n_v * mp.T;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int j = c0 + i;
+        if (j >= tl.ncols) continue;
+        if (j < mp.n_v) {
+          const float xa = x[i] + mp.dt_bias[tl.layer * mp.n_v + j];
+          const float sp = xa > 20.f ? xa : log1pf(expf(xa));
+          gb[static_cast<int64_t>(j) * mp.T + t] = -expf(mp.A_log[tl.layer * mp.n_v + j]) * sp;
+        } else {
+          gb[static_cast<int64_t>(mp.n_v + (j - mp.n_v)) * mp.T + t] = 1.f / (1.f + expf(-x[i]));
+        }
+      }
+    }
+  } else if (tl.kind == MIX_ATT_K) {
+    // RMSNorm over the 256 dims x gain, then RoPE on dims [0, 64): pairs (d, d + 32),
+    // angle (pos + t) theta^(-2d/64) formed and range-reduced in fp64
+    float ss = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      mixer_copy(ch * 32, x);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss += x[i] * x[i];
+    }
+    const float sc = rsqrtf(ss / 256.f + mp.eps);
+    const float* gain = mp.k_gain + tl.layer * 256;
+    const int64_t p = mp.pos + t;
+    const int64_t crow = row_ok ? mix_cache_row(mp.cache, tl.sub, mp.n_kv, p, mp.err) : -1;
+    void* kbase = mp.cache.k[tl.layer];
+    const bool c_h = mp.cache.dtype == KVA_F16;
+    {
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(taddr, ra);
+      tmem_ld_32x32b_x32(taddr + 32, rb);
+      tmem_ld_wait();
+      float a[32], b[32];
+      mix_round32<T>(ra, a);
+      mix_round32<T>(rb, b);
+      if (crow >= 0) {
+        const double two_pi = 6.283185307179586476925286766559;
+        const double lt = log2(mp.rope_theta);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float k0 = a[i] * sc * gain[i], k1 = b[i] * sc * gain[32 + i];
+          const double inv = exp2(-(2.0 * i / mp.rope_dims) * lt);
+          const double ang = static_cast<double>(p) * inv;
+          const double qq = rint(ang / two_pi);
+          const float red = static_cast<float>(fma(-qq, two_pi, ang));
+          float sn, cs;
+          sincosf(red, &sn, &cs);
+          a[i] = k0 * cs - k1 * sn;
+          b[i] = k1 * cs + k0 * sn;
+        }
+        if (c_h) {
+          mix_cache_store32<__half>(kbase, crow, 0, a);
+          mix_cache_store32<__half>(kbase, crow, 32, b);
+        } else {
+          mix_cache_store32<__nv_bfloat16>(kbase, crow, 0, a);
+          mix_cache_store32<__nv_bfloat16>(kbase, crow, 32, b);
+        }
+      }
+    }
+#pragma unroll 1
+    for (int ch = 2; ch < 8; ++ch) {
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      if (crow < 0) continue;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] *= sc * gain[ch * 32 + i];
+      if (c_h) mix_cache_store32<__half>(kbase, crow, ch * 32, x);
+      else mix_cache_store32<__nv_bfloat16>(kbase, crow, ch * 32, x);
+    }
+  } else if (tl.kind == MIX_ATT_V) {
+    // the value head as stored in the mixer, in the cache's format
+    const int64_t crow = row_ok ? mix_cache_row(mp.cache, tl.sub, mp.n_kv, mp.pos + t, mp.err) : -1;
+    void* vbase = mp.cache.v[tl.layer];
+    const bool c_h = mp.cache.dtype == KVA_F16;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      mixer_copy(ch * 32, x);
+      if (crow < 0) continue;
+      if (c_h) mix_cache_store32<__half>(vbase, crow, ch * 32, x);
+      else mix_cache_store32<__nv_bfloat16>(vbase, crow, ch * 32, x);
+    }
+  } else {  // MIX_DRAFT
+#pragma unroll 1
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const int c0 = ch * 32;
+      uint32_t rr[32];
+      tmem_ld_32x32b_x32(taddr + c0, rr);
+      tmem_ld_wait();
+      float x[32];
+      mix_round32<T>(rr, x);
+      if (row_ok && mp.draft)
+        mix_store32<T>(static_cast<T*>(mp.draft) + t * mp.ld_draft + tl.sub + c0, x,
+                       min(32, tl.ncols - c0));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ CTA-pair variant
 // The same pipeline on a pair of CTAs (a cluster of 2) sharing one 256 x 256 tile
 // through tcgen05.mma.cta_group::2: each CTA loads its 128 rows of A and its 128 rows
@@ -381,13 +699,14 @@ struct PairCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SMEM_MIX = SMEM + MIX_STAGE_BYTES;  // + the conv staging tile
 };
 
 template <int EPI, typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                      const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
-                     const GemmParams p) {
+                     const GemmParams p, const __grid_constant__ MixParams mp) {
   using Cfg = PairCfg;
   constexpr int S = Cfg::STAGES;
   constexpr int BN = Cfg::BN;
@@ -403,6 +722,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* tempty = bars + 2 * S + 2;  // leader: both CTAs' epilogues released it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* mix_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  volatile int* mix_votes = reinterpret_cast<volatile int*>(reinterpret_cast<uint8_t*>(bars) + 160);
+  (void)mix_stage;
+  (void)mix_votes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -473,7 +796,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
           uint8_t* b = sB + stage * Cfg::B_BYTES;
-          if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
+          if constexpr (EPI == EPI_MIXER) {  // the tile's first weight row comes from the table
+            tma_load_2d_pair(b, &mB0, fb, kc, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2),
+                             pol_b);
+          } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
             tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
           } else if (p.b_mode == B_SEGMENTS) {
             const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
@@ -576,15 +902,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     for (int it = cid; it < items; it += ncl) {
       const int m_blk = it % num_m;
       const int n_blk = (it / num_m) / splits;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      if (!got) {
         *abort_flag = 1;
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      if constexpr (EPI == EPI_MIXER) {
+        // the four epilogue warps meet at named barriers inside the epilogue, so they
+        // leave together: every warp votes, all read the same four votes
+        if (lane == 0) mix_votes[q] = got ? 1 : 0;
+        mix_sync();
+        const bool all = mix_votes[0] && mix_votes[1] && mix_votes[2] && mix_votes[3];
+        mix_sync();
+        if (!all) break;
+      } else if (!got) {
         break;
       }
       tc_fence_after();
-      epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
-                                m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
-                                lane);
+      if constexpr (EPI == EPI_MIXER)
+        epilogue_mixer<T>(mp, tmem_base + static_cast<uint32_t>(acc * BN),
+                          m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q, lane,
+                          mix_stage);
+      else
+        epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
+                                  m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
+                                  lane);
       tc_fence_before();
       if (leader) mbar_arrive(&tempty[acc]);
       else mbar_arrive_remote(tempty_lead[acc]);
@@ -728,6 +1070,8 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
 }
 
 
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
 template <int EPI, typename T>
 static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   using Cfg = PairCfg;
@@ -771,11 +1115,56 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<2 * ncl, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p);
+  kern<<<2 * ncl, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p, MixParams());
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
-static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+template <typename T>
+static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64_t n_rows_w, int M,
+                                int K, int num_tiles, const MixParams& mp, cudaStream_t s) {
+  using Cfg = PairCfg;
+  const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap mA, mB;
+  if (!make_map(&mA, A, K, M, lda, Cfg::BM, dt)) return KVA_ERR_CUDA;
+  if (!make_map(&mB, W, K, n_rows_w, K, Cfg::BN / 2, dt)) return KVA_ERR_CUDA;
+  GemmParams p;
+  p.M = M;
+  p.N = num_tiles * Cfg::BN;  // one tile per table entry
+  p.K = K;
+  p.b_mode = B_SINGLE;
+  p.seg_rows = 0;
+  p.D = nullptr;
+  p.ldd = 0;
+  p.D1 = nullptr;
+  p.ldd1 = 0;
+  p.n_split = 0;
+  p.splits = 1;
+  p.err = mp.err;
+  const int num_m = (M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
+  const int max_cl = num_sms() / 2;
+  const int items = num_m * num_tiles;
+  int ncl = items < max_cl ? items : max_cl;
+  if (items > ncl && num_m > 1 && ncl >= num_m && num_m <= 16) ncl -= ncl % num_m;
+  auto kern = gemm_pair_kernel<EPI_MIXER, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_MIX) !=
+      cudaSuccess)
+    return KVA_ERR_CUDA;
+  kern<<<2 * ncl, 192, Cfg::SMEM_MIX, s>>>(mA, mB, mB, mB, p, mp);
+  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+int launch_heads_fused(int dtype, const void* A, int64_t lda, const void* W, int64_t n_rows_w,
+                       int M, int K, int num_tiles, const MixParams& mp, cudaStream_t s) {
+  if (M == 0 || num_tiles == 0) return KVA_OK;
+  if (!A || !W || !mp.tiles || M < 0 || K <= 0) return KVA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(W) || (lda % 8) || (K % 8)) return KVA_ERR_ALIGNMENT;
+  if (dtype == KVA_F16) return launch_heads_fused_t<__half>(A, lda, W, n_rows_w, M, K, num_tiles, mp, s);
+  if (dtype == KVA_BF16)
+    return launch_heads_fused_t<__nv_bfloat16>(A, lda, W, n_rows_w, M, K, num_tiles, mp, s);
+  return KVA_ERR_INVALID_ARG;
+}
+
 
 int launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return a.M == 0 ? KVA_OK : KVA_ERR_INVALID_ARG;

@@ -13,6 +13,7 @@ enum GemmEpilogue {
   EPI_STORE_F32 = 1,    // D = acc (fp32)
   EPI_ADD_F32 = 2,      // D += acc (fp32 residual stream)
   EPI_SWIGLU_BF16 = 3,  // D[:, j] = silu(gate_j) * up_j (16-bit), gate/up rows from B0/B1
+  EPI_MIXER = 4,        // heads GEMM with the state-update epilogue (internal: MixParams)
 };
 
 enum GemmBMode {
@@ -109,5 +110,65 @@ struct KvLaunch {
   int* err = nullptr;
 };
 int launch_kv_write(const KvLaunch& k, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Heads GEMM with the state-update epilogue (the wide head GEMM writes the scan's
+// inputs, the gates and the KV-cache rows directly instead of the mixer).
+// The N dimension is tiled per layer segment: every tile lies inside one segment.
+enum MixKind {
+  MIX_RAW = 0,      // q columns of a gated-DeltaNet layer: only conv-tail / halo / debug copies
+  MIX_GDN_K = 1,    // k columns: conv + SiLU + per-head L2 norm -> kbuf
+  MIX_GDN_V = 2,    // v columns: conv + SiLU -> vbuf
+  MIX_GDN_AB = 3,   // a | b columns: gates g, beta -> gbuf
+  MIX_ATT_K = 4,    // one attention key head: RMSNorm x gain, RoPE -> K cache
+  MIX_ATT_V = 5,    // one attention value head -> V cache
+  MIX_DRAFT = 6,    // drafter columns -> draft_out
+};
+struct MixTile {
+  int col0;    // first row of W_heads (column of the mixer) of the tile
+  int ncols;   // valid columns (<= 256)
+  int kind;    // MixKind
+  int layer;   // index among the gated-DeltaNet layers (GDN kinds) or the attention layers
+  int sub;     // offset inside the segment: conv channel of column 0 (GDN kinds), value
+               // channel (GDN V), key channel (GDN K), head (ATT kinds), drafter column
+};
+constexpr int kMixHaloRows = 6;  // rows 0, 1, 2, 125, 126, 127 of every 128-token block
+struct MixParams {
+  const MixTile* tiles = nullptr;
+  int T = 0;
+  int64_t pos = 0;
+  // gated-DeltaNet layers
+  int n_k = 0, n_v = 0, C = 0;    // C = conv channels (q | k | v)
+  const float* conv_w = nullptr;  // [n_gdn, C, 4]
+  const float* A_log = nullptr;   // [n_gdn, n_v]
+  const float* dt_bias = nullptr; // [n_gdn, n_v]
+  void* kbuf = nullptr;           // fp16 [n_gdn, T, n_k*128]
+  void* vbuf = nullptr;           // fp16 [n_gdn, T, n_v*128]
+  float* gbuf = nullptr;          // fp32 [n_gdn, 2, n_v, T]
+  void* halo = nullptr;           // 16-bit [n_gdn, nblk, 6, C] raw rows around block edges
+  void* tail_new = nullptr;       // 16-bit [n_gdn, 3, C] raw rows T-3 .. T-1
+  int nblk = 0;                   // 128-token blocks of the workspace (max_T / 128)
+  float eps = 1e-6f;
+  // attention layers
+  int n_kv = 0;                   // KV heads per attention layer (head dim 256)
+  const float* k_gain = nullptr;  // [n_attn, 256]
+  int rope_dims = 64;
+  double rope_theta = 1e7;
+  kva_kv_cache cache;
+  // outputs kept from the plain path
+  void* draft = nullptr;          // [T, n_draft_cols] or null
+  int64_t ld_draft = 0;
+  void* mixer_out = nullptr;      // [T, n_mix] debug copy of the raw mixer, or null
+  int64_t ld_mix = 0;
+  int* err = nullptr;
+};
+// The heads GEMM over `num_tiles` tiles of the table, A = z [M, K] (16-bit, lda), B = W_heads.
+int launch_heads_fused(int dtype, const void* A, int64_t lda, const void* W, int64_t n_rows_w,
+                       int M, int K, int num_tiles, const MixParams& mp, cudaStream_t s);
+// After the fused heads GEMM: the conv outputs of the first 3 rows of every 128-token block
+// (from the halo rows and the old conv tail), then the new conv tail.
+int launch_gdn_halo_fix(const MixParams& mp, int n_gdn, cudaStream_t s, int dtype,
+                        const void* conv_state);
+int launch_gdn_tail_fused(const MixParams& mp, int n_gdn, void* conv_state, cudaStream_t s);
 
 }  // namespace kva
