@@ -368,76 +368,136 @@ __global__ void __launch_bounds__(192, 1)
 // The heads GEMM's accumulator tile (128 tokens x 256 columns of one layer segment per
 // CTA of the pair) goes straight to the state updates' inputs.  Every raw value is
 // first rounded to the mixer's 16-bit format, so the results equal those of the plain
-// path (mixer stored, then the conv / norm / gate / KV kernels).  Warp q of the
-// epilogue group owns TMEM lanes (tokens) [32q, 32q+32) of the block.
-constexpr int MIX_STAGE_LD = 36;                       // floats per staged row (16-byte rows)
-constexpr int MIX_STAGE_BYTES = 128 * MIX_STAGE_LD * 4;
+// path (mixer stored, then the conv / norm / gate / KV kernels).  Eight epilogue warps
+// work in two groups of four: warp q of a group owns TMEM lanes (tokens) [32q, 32q+32),
+// and the groups split the tile's columns in 16-column chunks (a DeltaNet key tile: one
+// 128-channel head per group).  The groups meet only for the attention key's RMS over
+// its 256 dims and for the per-tile abort vote.
+constexpr int MIX_GROUPS = 2;
+constexpr int MIX_EPI_WARPS = 4 * MIX_GROUPS;
+constexpr int MIX_LD = 24;                          // 16-bit values per staged row (48-byte rows)
+constexpr int MIX_BUF_BYTES = 128 * MIX_LD * 2;     // one group's buffer of 16 channels
+constexpr int MIX_RMS_OFF = MIX_GROUPS * 2 * MIX_BUF_BYTES;         // [2][128] fp32 RMS partials
+constexpr int MIX_W_OFF = MIX_RMS_OFF + MIX_GROUPS * 128 * 4;        // [2][128] float4 conv weights
+constexpr int MIX_STAGE_BYTES = MIX_W_OFF + MIX_GROUPS * 128 * 16;
 
-__device__ __forceinline__ void mix_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// tcgen05.wait::ld that also orders the loaded registers: later reads of `r` cannot be
+// moved above the wait (used where the next chunk's load is in flight while the
+// current one is processed)
+__device__ __forceinline__ void tmem_wait_dep16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 
+// a group's 128 threads (named barriers 2 and 3)
+__device__ __forceinline__ void mix_sync_group(int g) {
+  asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory");
+}
+// all epilogue threads (named barrier 4), returning the AND of `v` over them
+__device__ __forceinline__ bool mix_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 4, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
+// 16 accumulator columns to the 16-bit grid: packed pairs and their float values
 template <typename T>
-__device__ __forceinline__ void mix_round32(const uint32_t (&r)[32], float (&x)[32]) {
+__device__ __forceinline__ void mix_round16(const uint32_t (&r)[16], uint32_t (&pk)[8], float (&x)[16]) {
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float2 f = F16<T>::unpack(F16<T>::pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])));
-    x[i] = f.x;
-    x[i + 1] = f.y;
+  for (int i = 0; i < 8; ++i) {
+    pk[i] = F16<T>::pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    const float2 f = F16<T>::unpack(pk[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
   }
 }
 
-// 32 values (already in the 16-bit grid) to a 16-bit row at dst (16-byte aligned)
-template <typename T>
-__device__ __forceinline__ void mix_store32(void* dst, const float (&x)[32], int valid) {
-  store16x32<T>(static_cast<T*>(dst), x, valid);
+// the first `valid` of 16 packed 16-bit values to dst (16-byte aligned)
+__device__ __forceinline__ void mix_put16(void* dst, const uint32_t (&pk)[8], int valid) {
+  if (valid >= 16) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    uint16_t* d = static_cast<uint16_t*>(dst);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < valid) d[i] = static_cast<uint16_t>((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xffffu));
+  }
 }
 
-// conv over tokens t-3..t of 32 channels: this thread's row is staged, rows r-1..r-3 read back
+// 16 floats packed in the 16-bit format C16
+template <typename C16>
+__device__ __forceinline__ void mix_pack16(const float (&x)[16], uint32_t (&pk)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = F16<C16>::pack(x[2 * i], x[2 * i + 1]);
+}
+
+// causal depthwise conv over tokens t-3..t of 16 channels (weights w4[i] = taps of channel
+// i, staged in shared memory), then SiLU: this thread's row
+// goes to the group's staging buffer (two buffers used in turn, so one barrier per chunk
+// suffices: a buffer is rewritten only after every thread has passed the barrier of the
+// chunk in between), rows r-1..r-3 come back from it.  Rows 0-2 of the block have no
+// predecessors here; the block-edge fix-up computes their outputs.
 template <typename T>
-__device__ __forceinline__ void mix_conv32(const MixParams& mp, float* stage, int r, int gdn,
-                                           int ch0, const float (&x)[32], float (&z)[32]) {
-  float* my = stage + r * MIX_STAGE_LD;
+__device__ __forceinline__ void mix_conv16(const float4* w4, uint8_t* gstage, int& turn,
+                                           int r, int g, const uint32_t (&pk)[8], const float (&x)[16],
+                                           float (&z)[16]) {
+  uint16_t* buf = reinterpret_cast<uint16_t*>(gstage + turn * MIX_BUF_BYTES);
+  turn ^= 1;
+  uint4* my = reinterpret_cast<uint4*>(buf + r * MIX_LD);
+  my[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  my[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  mix_sync_group(g);
+  if (r < 3) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    reinterpret_cast<float4*>(my)[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
-  mix_sync();
-  if (r >= 3) {
-    const float* p1 = stage + (r - 1) * MIX_STAGE_LD;
-    const float* p2 = stage + (r - 2) * MIX_STAGE_LD;
-    const float* p3 = stage + (r - 3) * MIX_STAGE_LD;
-    const float4* w4 = reinterpret_cast<const float4*>(mp.conv_w + (static_cast<int64_t>(gdn) * mp.C + ch0) * 4);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 a1 = reinterpret_cast<const float4*>(p1)[j];
-      const float4 a2 = reinterpret_cast<const float4*>(p2)[j];
-      const float4 a3 = reinterpret_cast<const float4*>(p3)[j];
-      const float x1[4] = {a1.x, a1.y, a1.z, a1.w};
-      const float x2[4] = {a2.x, a2.y, a2.z, a2.w};
-      const float x3[4] = {a3.x, a3.y, a3.z, a3.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * j + e;
-        const float4 w = w4[i];
-        z[i] = silu_tanh(w.x * x3[e] + w.y * x2[e] + w.z * x1[e] + w.w * x[i]);
-      }
-    }
+    for (int i = 0; i < 16; ++i) z[i] = 0.f;
+    return;
   }
-  mix_sync();
+  uint32_t p[3][8];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const uint4* src = reinterpret_cast<const uint4*>(buf + (r - 1 - k) * MIX_LD);
+    const uint4 u0 = src[0], u1 = src[1];
+    p[k][0] = u0.x; p[k][1] = u0.y; p[k][2] = u0.z; p[k][3] = u0.w;
+    p[k][4] = u1.x; p[k][5] = u1.y; p[k][6] = u1.z; p[k][7] = u1.w;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float4 wa = w4[i], wb = w4[i + 1];
+    const float2 x1 = F16<T>::unpack(p[0][i / 2]);
+    const float2 x2 = F16<T>::unpack(p[1][i / 2]);
+    const float2 x3 = F16<T>::unpack(p[2][i / 2]);
+    z[i] = silu_tanh(wa.x * x3.x + wa.y * x2.x + wa.z * x1.x + wa.w * x[i]);
+    z[i + 1] = silu_tanh(wb.x * x3.y + wb.y * x2.y + wb.z * x1.y + wb.w * x[i + 1]);
+  }
 }
 
 // raw copies of gated-DeltaNet conv channels: the rows around 128-token block edges
-// (for the edge fix-up) and the ubatch's last 3 rows (the new conv tail)
+// (key and value channels, for the edge fix-up) and the ubatch's last 3 rows (every
+// channel: the new conv tail)
 template <typename T>
-__device__ __forceinline__ void mix_gdn_raw(const MixParams& mp, int gdn, int t, int r, int ch0,
-                                            const float (&x)[32], int valid) {
+__device__ __forceinline__ void mix_gdn_raw(const MixParams& mp, bool halo, int gdn, int t, int r,
+                                            int ch0, const uint32_t (&pk)[8]) {
   if (t >= mp.T) return;
-  if (r < 3 || r >= 125) {
+  if (halo && (r < 3 || r >= 125)) {
     const int slot = r < 3 ? r : r - 122;
     const int64_t row = (static_cast<int64_t>(gdn) * mp.nblk + (t >> 7)) * kMixHaloRows + slot;
-    mix_store32<T>(static_cast<T*>(mp.halo) + row * mp.C + ch0, x, valid);
+    mix_put16(static_cast<T*>(mp.halo) + row * mp.C + ch0, pk, 16);
   }
   if (t >= mp.T - 3) {
     const int64_t row = static_cast<int64_t>(gdn) * 3 + (t - (mp.T - 3));
-    mix_store32<T>(static_cast<T*>(mp.tail_new) + row * mp.C + ch0, x, valid);
+    mix_put16(static_cast<T*>(mp.tail_new) + row * mp.C + ch0, pk, 16);
   }
 }
 
@@ -460,163 +520,176 @@ __device__ __forceinline__ int64_t mix_cache_row(const kva_kv_cache& cc, int hea
   return static_cast<int64_t>(head) * cc.max_pos + p;
 }
 
-template <typename C16>
-__device__ __forceinline__ void mix_cache_store32(void* base, int64_t row, int c0, const float (&v)[32]) {
-  C16* dst = static_cast<C16*>(base) + row * 256 + c0;
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    uint4 pk;
-    pk.x = F16<C16>::pack(v[8 * q4 + 0], v[8 * q4 + 1]);
-    pk.y = F16<C16>::pack(v[8 * q4 + 2], v[8 * q4 + 3]);
-    pk.z = F16<C16>::pack(v[8 * q4 + 4], v[8 * q4 + 5]);
-    pk.w = F16<C16>::pack(v[8 * q4 + 6], v[8 * q4 + 7]);
-    reinterpret_cast<uint4*>(dst)[q4] = pk;
-  }
+// 16 values of one cache row (256 dims per head) from column c0, in the cache's format
+__device__ __forceinline__ void mix_cache_put16(const kva_kv_cache& cc, void* base, int64_t row, int c0,
+                                                const float (&v)[16]) {
+  uint32_t pk[8];
+  if (cc.dtype == KVA_F16) mix_pack16<__half>(v, pk);
+  else mix_pack16<__nv_bfloat16>(v, pk);
+  mix_put16(static_cast<uint16_t*>(base) + row * 256 + c0, pk, 16);
 }
+
+__device__ __forceinline__ void mix_sync_all() { asm volatile("bar.sync 4, 256;" ::: "memory"); }
 
 template <typename T>
 __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tmem_acc, int row0,
-                                               int n_blk, int q, int lane, float* stage) {
+                                               int n_blk, int q, int g, int lane, uint8_t* stage,
+                                               int& turn) {
   const MixTile tl = mp.tiles[n_blk];
   const int r = q * 32 + lane;
   const int t = row0 + r;
   const bool row_ok = t < mp.T;
   const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
-  const int n_chunks = (tl.ncols + 31) / 32;
+  const int n16 = (tl.ncols + 15) / 16;
+  uint8_t* gstage = stage + g * 2 * MIX_BUF_BYTES;
+  float* rms_part = reinterpret_cast<float*>(stage + MIX_GROUPS * 2 * MIX_BUF_BYTES);
 
-  // the raw 16-bit mixer (debug copy), for every kind
-  auto mixer_copy = [&](int c0, const float (&x)[32]) {
+  // one 16-column chunk from TMEM in the 16-bit grid, with the raw mixer's debug copy
+  auto load16 = [&](int c0, uint32_t(&pk)[8], float(&x)[16]) {
+    uint32_t rr[16];
+    tmem_ld_32x32b_x16(taddr + c0, rr);
+    tmem_ld_wait();
+    mix_round16<T>(rr, pk, x);
     if (mp.mixer_out && row_ok)
-      mix_store32<T>(static_cast<T*>(mp.mixer_out) + t * mp.ld_mix + tl.col0 + c0, x,
-                     min(32, tl.ncols - c0));
+      mix_put16(static_cast<T*>(mp.mixer_out) + t * mp.ld_mix + tl.col0 + c0, pk, min(16, tl.ncols - c0));
   };
 
-  if (tl.kind == MIX_GDN_K) {
-    // two 128-channel heads; the norm needs the whole head before any output, so the
-    // head's conv outputs wait as fp16 pairs (their sum of squares is taken in fp32)
-#pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
-      uint32_t zk[64];
-      float ss = 0.f;
+  if (tl.kind == MIX_GDN_K || tl.kind == MIX_GDN_V) {
+    // conv tiles.  A key tile: one 128-channel head per group (chunks 8g..8g+7), whose
+    // norm needs the whole head before any output, so the conv outputs wait as fp16
+    // pairs (their sum of squares is taken in fp32).  A value tile: chunks g, g+2, ...
+    // Each thread stages one channel's taps for its group; the next chunk's TMEM load
+    // is in flight while the current one is processed.
+    const bool is_k = tl.kind == MIX_GDN_K;
+    auto chunk_col = [&](int k) { return is_k ? (g * 8 + k) * 16 : (g + 2 * k) * 16; };
+    float4* wsm = reinterpret_cast<float4*>(stage + MIX_W_OFF) + g * 128;
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(mp.conv_w) +
+                            static_cast<int64_t>(tl.layer) * mp.C + tl.sub + chunk_col(r >> 4) + (r & 15));
+    const int nkdk = mp.n_k * 128, nvdv = mp.n_v * 128;
+    uint32_t nx[16];
+    tmem_ld_32x32b_x16(taddr + chunk_col(0), nx);
+    uint32_t zk[64];
+    float ss = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c0 = hh * 128 + ch * 32;
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(taddr + c0, rr);
-        tmem_ld_wait();
-        float x[32], z[32];
-        mix_round32<T>(rr, x);
-        mixer_copy(c0, x);
-        mix_gdn_raw<T>(mp, tl.layer, t, r, tl.sub + c0, x, 32);
-        mix_conv32<T>(mp, stage, r, tl.layer, tl.sub + c0, x, z);
+    for (int k = 0; k < 8; ++k) {
+      const int c0 = chunk_col(k);
+      tmem_wait_dep16(nx);
+      uint32_t pk[8];
+      float x[16], z[16];
+      mix_round16<T>(nx, pk, x);
+      if (k < 7) tmem_ld_32x32b_x16(taddr + chunk_col(k + 1), nx);
+      if (k == 0) wsm[r] = wv;  // read after the first conv barrier
+      if (mp.mixer_out && row_ok)
+        mix_put16(static_cast<T*>(mp.mixer_out) + t * mp.ld_mix + tl.col0 + c0, pk, 16);
+      mix_gdn_raw<T>(mp, true, tl.layer, t, r, tl.sub + c0, pk);
+      mix_conv16<T>(wsm + k * 16, gstage, turn, r, g, pk, x, z);
+      if (is_k) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 16; i += 2) {
           ss += z[i] * z[i] + z[i + 1] * z[i + 1];
-          zk[ch * 16 + i / 2] = pack_f16(z[i], z[i + 1]);
+          zk[k * 8 + i / 2] = pack_f16(z[i], z[i + 1]);
         }
-      }
-      if (r >= 3 && row_ok) {
-        const float sc = rsqrtf(ss + mp.eps);
-        const int nkdk = mp.n_k * 128;
-        __half* dst = static_cast<__half*>(mp.kbuf) +
-                      (static_cast<int64_t>(tl.layer) * mp.T + t) * nkdk + (tl.sub - nkdk) + hh * 128;
-#pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = F16<__half>::unpack(zk[4 * q4 + e]);
-            o[e] = pack_f16(f.x * sc, f.y * sc);
-          }
-          reinterpret_cast<uint4*>(dst)[q4] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
+      } else if (r >= 3 && row_ok) {
+        uint32_t o[8];
+        mix_pack16<__half>(z, o);
+        mix_put16(static_cast<__half*>(mp.vbuf) + (static_cast<int64_t>(tl.layer) * mp.T + t) * nvdv +
+                      (tl.sub - 2 * nkdk) + c0,
+                  o, 16);
       }
     }
-  } else if (tl.kind == MIX_GDN_V || tl.kind == MIX_RAW) {
-#pragma unroll 1
-    for (int ch = 0; ch < n_chunks; ++ch) {
-      const int c0 = ch * 32;
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + c0, rr);
-      tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
-      mixer_copy(c0, x);
-      mix_gdn_raw<T>(mp, tl.layer, t, r, tl.sub + c0, x, min(32, tl.ncols - c0));
-      if (tl.kind == MIX_GDN_V) {
-        float z[32];
-        mix_conv32<T>(mp, stage, r, tl.layer, tl.sub + c0, x, z);
-        if (r >= 3 && row_ok) {
-          const int nkdk = mp.n_k * 128, nvdv = mp.n_v * 128;
-          __half* dst = static_cast<__half*>(mp.vbuf) +
-                        (static_cast<int64_t>(tl.layer) * mp.T + t) * nvdv + (tl.sub - 2 * nkdk) + c0;
-          store16x32<__half>(dst, z, 32);
+    if (is_k && r >= 3 && row_ok) {
+      const float sc = rsqrtf(ss + mp.eps);
+      __half* dst = static_cast<__half*>(mp.kbuf) +
+                    (static_cast<int64_t>(tl.layer) * mp.T + t) * nkdk + (tl.sub - nkdk) + g * 128;
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = F16<__half>::unpack(zk[4 * q4 + e]);
+          o[e] = pack_f16(f.x * sc, f.y * sc);
         }
+        reinterpret_cast<uint4*>(dst)[q4] = make_uint4(o[0], o[1], o[2], o[3]);
       }
+    }
+  } else if (tl.kind == MIX_RAW) {
+    // query channels feed only the new conv tail (and the debug copy): other warps skip them
+    if (!mp.mixer_out && !__any_sync(0xffffffffu, row_ok && t >= mp.T - 3)) return;
+#pragma unroll 1
+    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+      const int c0 = ch * 16;
+      uint32_t pk[8];
+      float x[16];
+      load16(c0, pk, x);
+      mix_gdn_raw<T>(mp, false, tl.layer, t, r, tl.sub + c0, pk);
     }
   } else if (tl.kind == MIX_GDN_AB) {
     // columns [0, n_v) are a, [n_v, 2 n_v) are b: g = -exp(A_log) softplus(a + dt_bias),
     // beta = sigmoid(b), written [layer][2][n_v][T]
+    float* gb = mp.gbuf + static_cast<int64_t>(tl.layer) * 2 * mp.n_v * mp.T;
 #pragma unroll 1
-    for (int ch = 0; ch < n_chunks; ++ch) {
-      const int c0 = ch * 32;
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + c0, rr);
-      tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
-      mixer_copy(c0, x);
+    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+      const int c0 = ch * 16;
+      uint32_t pk[8];
+      float x[16];
+      load16(c0, pk, x);
       if (!row_ok) continue;
-      float* gb = mp.gbuf + static_cast<int64_t>(tl.layer) * 2 * mp.n_v * mp.T;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const int j = c0 + i;
         if (j >= tl.ncols) continue;
+        float o;
         if (j < mp.n_v) {
           const float xa = x[i] + mp.dt_bias[tl.layer * mp.n_v + j];
           const float sp = xa > 20.f ? xa : log1pf(expf(xa));
-          gb[static_cast<int64_t>(j) * mp.T + t] = -expf(mp.A_log[tl.layer * mp.n_v + j]) * sp;
+          o = -expf(mp.A_log[tl.layer * mp.n_v + j]) * sp;
         } else {
-          gb[static_cast<int64_t>(mp.n_v + (j - mp.n_v)) * mp.T + t] = 1.f / (1.f + expf(-x[i]));
+          o = 1.f / (1.f + expf(-x[i]));
         }
+        gb[static_cast<int64_t>(j) * mp.T + t] = o;
       }
     }
   } else if (tl.kind == MIX_ATT_K) {
-    // RMSNorm over the 256 dims x gain, then RoPE on dims [0, 64): pairs (d, d + 32),
-    // angle (pos + t) theta^(-2d/64) formed and range-reduced in fp64
+    // RMSNorm over the 256 dims x gain (each group sums its 128), then RoPE on dims
+    // [0, 64): pairs (d, d + 32), angle (pos + t) theta^(-2d/64) formed and range-reduced
+    // in fp64
+    const int cb = g * 128;
     float ss = 0.f;
 #pragma unroll 1
     for (int ch = 0; ch < 8; ++ch) {
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
-      tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
-      mixer_copy(ch * 32, x);
+      uint32_t pk[8];
+      float x[16];
+      load16(cb + ch * 16, pk, x);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ss += x[i] * x[i];
+      for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
     }
-    const float sc = rsqrtf(ss / 256.f + mp.eps);
+    rms_part[g * 128 + r] = ss;
+    mix_sync_all();
+    const float sc = rsqrtf((rms_part[r] + rms_part[128 + r]) / 256.f + mp.eps);
     const float* gain = mp.k_gain + tl.layer * 256;
     const int64_t p = mp.pos + t;
     const int64_t crow = row_ok ? mix_cache_row(mp.cache, tl.sub, mp.n_kv, p, mp.err) : -1;
     void* kbase = mp.cache.k[tl.layer];
-    const bool c_h = mp.cache.dtype == KVA_F16;
-    {
-      uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(taddr, ra);
-      tmem_ld_32x32b_x32(taddr + 32, rb);
-      tmem_ld_wait();
-      float a[32], b[32];
-      mix_round32<T>(ra, a);
-      mix_round32<T>(rb, b);
-      if (crow >= 0) {
-        const double two_pi = 6.283185307179586476925286766559;
-        const double lt = log2(mp.rope_theta);
+    int ch0 = 0;
+    if (g == 0) {
+      const double two_pi = 6.283185307179586476925286766559;
+      const double lt = log2(mp.rope_theta);
+#pragma unroll 1
+      for (int d0 = 0; d0 < 32; d0 += 16) {
+        uint32_t ra[16], rb[16];
+        tmem_ld_32x32b_x16(taddr + d0, ra);
+        tmem_ld_32x32b_x16(taddr + 32 + d0, rb);
+        tmem_ld_wait();
+        uint32_t pa[8], pb[8];
+        float a[16], b[16];
+        mix_round16<T>(ra, pa, a);
+        mix_round16<T>(rb, pb, b);
+        if (crow < 0) continue;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float k0 = a[i] * sc * gain[i], k1 = b[i] * sc * gain[32 + i];
-          const double inv = exp2(-(2.0 * i / mp.rope_dims) * lt);
+        for (int i = 0; i < 16; ++i) {
+          const int d = d0 + i;
+          const float k0 = a[i] * sc * gain[d], k1 = b[i] * sc * gain[32 + d];
+          const double inv = exp2(-(2.0 * d / mp.rope_dims) * lt);
           const double ang = static_cast<double>(p) * inv;
           const double qq = rint(ang / two_pi);
           const float red = static_cast<float>(fma(-qq, two_pi, ang));
@@ -625,57 +698,48 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
           a[i] = k0 * cs - k1 * sn;
           b[i] = k1 * cs + k0 * sn;
         }
-        if (c_h) {
-          mix_cache_store32<__half>(kbase, crow, 0, a);
-          mix_cache_store32<__half>(kbase, crow, 32, b);
-        } else {
-          mix_cache_store32<__nv_bfloat16>(kbase, crow, 0, a);
-          mix_cache_store32<__nv_bfloat16>(kbase, crow, 32, b);
-        }
+        mix_cache_put16(mp.cache, kbase, crow, d0, a);
+        mix_cache_put16(mp.cache, kbase, crow, 32 + d0, b);
       }
+      ch0 = 4;  // dims 64..127 follow
     }
 #pragma unroll 1
-    for (int ch = 2; ch < 8; ++ch) {
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
+    for (int ch = ch0; ch < 8; ++ch) {
+      const int c0 = cb + ch * 16;
+      uint32_t rr[16];
+      tmem_ld_32x32b_x16(taddr + c0, rr);
       tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
+      uint32_t pk[8];
+      float x[16];
+      mix_round16<T>(rr, pk, x);
       if (crow < 0) continue;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] *= sc * gain[ch * 32 + i];
-      if (c_h) mix_cache_store32<__half>(kbase, crow, ch * 32, x);
-      else mix_cache_store32<__nv_bfloat16>(kbase, crow, ch * 32, x);
+      for (int i = 0; i < 16; ++i) x[i] *= sc * gain[c0 + i];
+      mix_cache_put16(mp.cache, kbase, crow, c0, x);
     }
   } else if (tl.kind == MIX_ATT_V) {
     // the value head as stored in the mixer, in the cache's format
     const int64_t crow = row_ok ? mix_cache_row(mp.cache, tl.sub, mp.n_kv, mp.pos + t, mp.err) : -1;
     void* vbase = mp.cache.v[tl.layer];
-    const bool c_h = mp.cache.dtype == KVA_F16;
 #pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + ch * 32, rr);
-      tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
-      mixer_copy(ch * 32, x);
-      if (crow < 0) continue;
-      if (c_h) mix_cache_store32<__half>(vbase, crow, ch * 32, x);
-      else mix_cache_store32<__nv_bfloat16>(vbase, crow, ch * 32, x);
+    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+      uint32_t pk[8];
+      float x[16];
+      load16(ch * 16, pk, x);
+      if (crow >= 0) mix_cache_put16(mp.cache, vbase, crow, ch * 16, x);
     }
   } else {  // MIX_DRAFT
 #pragma unroll 1
-    for (int ch = 0; ch < n_chunks; ++ch) {
-      const int c0 = ch * 32;
-      uint32_t rr[32];
-      tmem_ld_32x32b_x32(taddr + c0, rr);
+    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+      const int c0 = ch * 16;
+      uint32_t rr[16];
+      tmem_ld_32x32b_x16(taddr + c0, rr);
       tmem_ld_wait();
-      float x[32];
-      mix_round32<T>(rr, x);
+      uint32_t pk[8];
+      float x[16];
+      mix_round16<T>(rr, pk, x);
       if (row_ok && mp.draft)
-        mix_store32<T>(static_cast<T*>(mp.draft) + t * mp.ld_draft + tl.sub + c0, x,
-                       min(32, tl.ncols - c0));
+        mix_put16(static_cast<T*>(mp.draft) + t * mp.ld_draft + tl.sub + c0, pk, min(16, tl.ncols - c0));
     }
   }
 }
@@ -699,11 +763,14 @@ struct PairCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
-  static constexpr int SMEM_MIX = SMEM + MIX_STAGE_BYTES;  // + the conv staging tile
+  static constexpr int SMEM_MIX = SMEM + MIX_STAGE_BYTES;  // + the conv staging buffers
+  // producer warp, MMA warp, then the epilogue warps (eight for the state-update epilogue)
+  static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
+  static constexpr int threads(int epi) { return 64 + 32 * epi_warps(epi); }
 };
 
 template <int EPI, typename T>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI), 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                      const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
                      const GemmParams p, const __grid_constant__ MixParams mp) {
@@ -722,10 +789,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* tempty = bars + 2 * S + 2;  // leader: both CTAs' epilogues released it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* mix_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
-  volatile int* mix_votes = reinterpret_cast<volatile int*>(reinterpret_cast<uint8_t*>(bars) + 160);
+  uint8_t* mix_stage = reinterpret_cast<uint8_t*>(bars) + 256;
   (void)mix_stage;
-  (void)mix_votes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -739,7 +804,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 256);
+      mbar_init(&tempty[i], 2 * 32 * Cfg::epi_warps(EPI));  // every epilogue thread of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -893,8 +958,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ------------------------------------------------ epilogue warps 2..5 (both CTAs)
-    const int q = warp & 3;
+    // ------------------------------------------------ epilogue warps 2.. (both CTAs)
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int grp = (warp - 2) >> 2;        // column group (state-update epilogue)
+    (void)grp;
+    int turn = 0;                           // the group's next conv staging buffer
+    (void)turn;
     const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                      mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
@@ -908,21 +977,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
       }
       if constexpr (EPI == EPI_MIXER) {
-        // the four epilogue warps meet at named barriers inside the epilogue, so they
-        // leave together: every warp votes, all read the same four votes
-        if (lane == 0) mix_votes[q] = got ? 1 : 0;
-        mix_sync();
-        const bool all = mix_votes[0] && mix_votes[1] && mix_votes[2] && mix_votes[3];
-        mix_sync();
-        if (!all) break;
+        // the epilogue warps meet at named barriers inside the epilogue, so they leave
+        // together: a barrier-reduction vote over all of them
+        if (!mix_all(got)) break;
       } else if (!got) {
         break;
       }
       tc_fence_after();
       if constexpr (EPI == EPI_MIXER)
         epilogue_mixer<T>(mp, tmem_base + static_cast<uint32_t>(acc * BN),
-                          m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q, lane,
-                          mix_stage);
+                          m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q, grp, lane,
+                          mix_stage, turn);
       else
         epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
                                   m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
@@ -1115,7 +1180,7 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<2 * ncl, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p, MixParams());
+  kern<<<2 * ncl, Cfg::threads(EPI), Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p, MixParams());
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
@@ -1150,7 +1215,7 @@ static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_MIX) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<2 * ncl, 192, Cfg::SMEM_MIX, s>>>(mA, mB, mB, mB, p, mp);
+  kern<<<2 * ncl, Cfg::threads(EPI_MIXER), Cfg::SMEM_MIX, s>>>(mA, mB, mB, mB, p, mp);
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
