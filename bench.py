@@ -92,10 +92,12 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def heads_traffic(geom_name):
-    """dram bytes per launch of the heads GEMM from the committed ncu summary, or None
-    when the summary is missing or the GEMM source changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"gemm_heads_{geom_name}_T1024.md")
+def heads_traffic(geom_name, fused):
+    """dram bytes per launch of the heads GEMM (with the state-update epilogue when `fused`)
+    from the committed ncu summary, or None when the summary is missing or the GEMM source
+    changed since it was taken."""
+    kind = "gemm_heads_fused" if fused else "gemm_heads"
+    path = os.path.join(ROOT, "profiles", f"{kind}_{geom_name}_T1024.md")
     src = os.path.join(ROOT, "hybrid_deltanet_attention_kva_b200", "csrc", "kva_gemm.cu")
     if not os.path.exists(path):
         return None
@@ -198,6 +200,7 @@ def run_ours(args, rank, world, local_rank):
     draft = (torch.empty(T_UB, geom.n_draft_cols, dtype=dt, device=dev)
              if geom.n_draft else None)
     h = K.kva_init(K.make_dims(geom, T_UB, 1, dtype=dt))
+    fused = K.kva_heads_fused(h)
     stream = torch.cuda.current_stream()
     n_ub = CACHE_POS // T_UB
 
@@ -318,12 +321,14 @@ def run_ours(args, rank, world, local_rank):
                   else "weights exceed L2 and stream from HBM every step",
         },
         "roofline": {
-            "bound": "tensor", "kernel": "gemm_heads (one wide GEMM over all per-layer and drafter heads)",
+            "bound": "tensor",
+            "kernel": "gemm_heads (one wide GEMM over all per-layer and drafter heads"
+                      + (", state-update epilogue)" if fused else ")"),
             "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
             "peak_kind": f"{src} bf16 sustained (kernel timed inside a long step loop)",
             "frac_of_burst": achieved / peaks["bf16_tflops"],
             "flops_per_launch": heads_flops, "avg_launch_ms": heads_ms,
-            "traffic": heads_traffic(geom.name),
+            "traffic": heads_traffic(geom.name, fused),
         },
         "path_roofline": {
             "flops_alg": flops, "bytes_alg": bytes_, "t_roof_ms": t_roof * 1e3,

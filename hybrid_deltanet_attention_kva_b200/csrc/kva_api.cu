@@ -751,6 +751,12 @@ int kva_stats(kva_handle* h, int64_t* tokens_approximated) {
   return KVA_OK;
 }
 
+int kva_heads_fused(kva_handle* h, int32_t* fused) {
+  if (!h || !fused) return KVA_ERR_INVALID_ARG;
+  *fused = h->fused ? 1 : 0;
+  return KVA_OK;
+}
+
 const char* kva_strerror(int32_t status) {
   switch (status) {
     case KVA_OK: return "ok";

@@ -102,6 +102,7 @@ def _load() -> C.CDLL:
                                     P, P, C.POINTER(KvaKvCache), P, P, P]),
         "kva_get_device_status": (I32, [P, C.POINTER(I32)]),
         "kva_stats": (I32, [P, C.POINTER(I64)]),
+        "kva_heads_fused": (I32, [P, C.POINTER(I32)]),
         "kva_free": (None, [P]),
         "kva_profile_enable": (I32, [P, I32]),
         "kva_profile_read": (I32, [P, C.POINTER(KvaProfile)]),
@@ -122,7 +123,7 @@ def _load() -> C.CDLL:
 
 _lib = _load()
 EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update_states",
-            "kva_get_device_status", "kva_stats", "kva_free", "kva_strerror",
+            "kva_get_device_status", "kva_stats", "kva_heads_fused", "kva_free", "kva_strerror",
             "kva_profile_enable", "kva_profile_read",
             "kva_op_rmsnorm", "kva_op_gemm", "kva_op_attention", "kva_op_gdn_scan",
             "kva_gdn_layer_update_noalloc")
@@ -278,6 +279,13 @@ def kva_stats(handle: int) -> int:
     n = C.c_int64()
     _check(_lib.kva_stats(handle, C.byref(n)), "kva_stats")
     return n.value
+
+
+def kva_heads_fused(handle: int) -> bool:
+    """True when kva_prefill_ubatch runs the state updates in the heads GEMM's epilogue."""
+    f = C.c_int32()
+    _check(_lib.kva_heads_fused(handle, C.byref(f)), "kva_heads_fused")
+    return bool(f.value)
 
 
 def kva_profile_enable(handle: int, capacity: int) -> None:

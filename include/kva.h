@@ -191,6 +191,14 @@ int kva_get_device_status(kva_handle* h, int32_t* status);
 /* Tokens sent through the approximated path since kva_init (host counter). */
 int kva_stats(kva_handle* h, int64_t* tokens_approximated);
 
+/* *fused = 1 when kva_prefill_ubatch runs the state updates' inputs (conv + SiLU, L2 norms,
+ * gates, k RMSNorm + RoPE + KV cache rows) in the epilogue of the heads GEMM, so the mixer
+ * inputs never reach HBM; 0 when it writes the mixer and runs them as separate kernels.
+ * The dims decide (128-dim DeltaNet heads, key/value widths in whole 256-column tiles,
+ * 256-dim attention heads with 64 rotary dims); both give the same results.
+ * KVA_ERR_INVALID_ARG for a null argument. */
+int kva_heads_fused(kva_handle* h, int32_t* fused);
+
 /* Stage kinds of the launch plan (for profiling and launch counts). */
 typedef enum kva_stage {
   KVA_ST_RMSNORM = 0,     /* every RMSNorm */

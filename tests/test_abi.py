@@ -106,6 +106,8 @@ def test_host_validation_rejects_before_any_launch():
                                None) == K.KVA_ERR_INVALID_ARG
     n = C.c_int64()
     assert L.kva_stats(None, C.byref(n)) == K.KVA_ERR_INVALID_ARG
+    f = C.c_int32()
+    assert L.kva_heads_fused(None, C.byref(f)) == K.KVA_ERR_INVALID_ARG
     s = C.c_int32()
     assert L.kva_get_device_status(None, C.byref(s)) == K.KVA_ERR_INVALID_ARG
     # per-step ops: misaligned / invalid shapes are refused on the host

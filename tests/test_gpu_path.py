@@ -283,6 +283,16 @@ TINY128 = KI.with_changes(KI.TINY, name="tiny128", gdn_d_k=128, gdn_d_v=128, att
                           rope_dims=64, n_draft=1)
 
 
+def test_heads_fused_flag_follows_the_dims(K):
+    # 64-dim DeltaNet heads take the plain path; 128-dim heads (and r3) the fused epilogue
+    for geom, want in ((KI.TINY, False), (TINY128, True), (KI.R3, True)):
+        h = K.kva_init(K.make_dims(geom, 256, 1, dtype=torch.float16))
+        try:
+            assert K.kva_heads_fused(h) is want, geom.name
+        finally:
+            K.kva_free(h)
+
+
 @pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
 def test_prefill_fused_heads_ragged_and_carry(K, dt):
     geom = TINY128
