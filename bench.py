@@ -53,7 +53,7 @@ def parse():
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "gdn", "attention"], default=None,
+    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "resid", "gdn", "attention"], default=None,
                     help="run a small case of one hot kernel three times and exit (for ncu "
                          "captures; prints no JSON line)")
     return ap.parse_args()
@@ -419,6 +419,8 @@ def run_kernel_case(case):
     """Small cases of the hot kernels, each above L2 in size where the kernel streams HBM:
     heads   - the heads GEMM's CTA-pair kernel on M = 1024, K = 3072, N = 49 152 (302 MB of
               weights, 1/5.8 of the r3 head matrix)
+    resid   - the r3 FFN down projection with the residual-add epilogue: M = 1024, N = 3072,
+              K = 8448, fp32 partial sums added into the residual stream (split K)
     heads_fused - kva_prefill_ubatch with the first 8 r3 late layers (6 gated-DeltaNet, 2
               attention, no drafter): the heads GEMM with the state-update epilogue
     gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
@@ -433,6 +435,13 @@ def run_kernel_case(case):
         D = torch.empty(M, N, dtype=torch.half, device="cuda")
         for _ in range(3):
             K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512)
+    elif case == "resid":
+        M, Kd, N = 1024, 8448, 3072
+        A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+        B = (torch.randn(N, Kd, device="cuda") * 0.02).half()
+        D = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_ADD_F32, block_n=512)
     elif case == "heads_fused":
         geom = KI.with_changes(KI.R3, layer_types=KI.R3.layer_types[:8], n_draft=0)
         W = KI.make_projector_weights(geom, 1003, device="cuda")

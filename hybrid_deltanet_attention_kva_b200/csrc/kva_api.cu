@@ -525,13 +525,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   const int H = d.hidden, dm = d.d_model, F = d.ffn;
   const int cd = d.compute_dtype;
   const float eps = d.norm_eps;
-  // 1. RMSNorm(residual) -> Linear{H -> d} into the fp32 residual stream x
-  if (cudaMemsetAsync(h->x, 0, static_cast<size_t>(T) * dm * sizeof(float), s) != cudaSuccess) {
-    e = KVA_ERR_CUDA;
-    goto done;
-  }
+  // 1. RMSNorm(residual) (which also clears x) -> Linear{H -> d} into the fp32 residual stream x
   if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
-         return launch_rmsnorm(residual, residual_dtype, H, w->g_in, h->u_in, H, T, H, eps, s, cd);
+         return launch_rmsnorm(residual, residual_dtype, H, w->g_in, h->u_in, H, T, H, eps, s, cd,
+                               h->x, dm, dm);
        })))
     goto done;
   {

@@ -44,6 +44,7 @@ template <typename E>
 __global__ void __launch_bounds__(ATT_THREADS)
     attention_kernel(const E* __restrict__ qkv, int64_t ldq, E* __restrict__ out, int64_t ldo,
                      int T, int d_model, int window, float scale_log2) {
+  griddep_wait_and_release();
   extern __shared__ __align__(128) uint8_t att_smem[];
   const uint32_t sQ = smem_u32(att_smem);
   const uint32_t sK0 = sQ + ATT_BQ * 256;
@@ -235,16 +236,18 @@ int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T
     if (cudaFuncSetAttribute(attention_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ATT_SMEM) != cudaSuccess)
       return KVA_ERR_CUDA;
-    attention_kernel<__half><<<grid, ATT_THREADS, ATT_SMEM, s>>>(
-        static_cast<const __half*>(qkv), ldq, static_cast<__half*>(out), ldo, T, d_model, window,
-        scale_log2);
+    if (launch_pdl(attention_kernel<__half>, grid, dim3(ATT_THREADS), ATT_SMEM, s,
+                   static_cast<const __half*>(qkv), ldq, static_cast<__half*>(out), ldo, T, d_model,
+                   window, scale_log2) != cudaSuccess)
+      return KVA_ERR_CUDA;
   } else {
     if (cudaFuncSetAttribute(attention_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) != cudaSuccess)
       return KVA_ERR_CUDA;
-    attention_kernel<__nv_bfloat16><<<grid, ATT_THREADS, ATT_SMEM, s>>>(
-        static_cast<const __nv_bfloat16*>(qkv), ldq, static_cast<__nv_bfloat16*>(out), ldo, T,
-        d_model, window, scale_log2);
+    if (launch_pdl(attention_kernel<__nv_bfloat16>, grid, dim3(ATT_THREADS), ATT_SMEM, s,
+                   static_cast<const __nv_bfloat16*>(qkv), ldq, static_cast<__nv_bfloat16*>(out), ldo,
+                   T, d_model, window, scale_log2) != cudaSuccess)
+      return KVA_ERR_CUDA;
   }
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }

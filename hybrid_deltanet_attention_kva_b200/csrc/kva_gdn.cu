@@ -50,6 +50,7 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
 
 template <typename TM>
 __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnLaunch p) {
+  griddep_wait_and_release();
   const int slot = blockIdx.z;  // seq * n_gdn + layer
   const int seq = slot / p.n_gdn, layer = slot % p.n_gdn;
   const int T = p.T;
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prepare_kernel(const GdnL
 
 // The tail holds raw 16-bit values: a bit copy, whatever their format.
 __global__ void gdn_tail_kernel(const GdnLaunch p) {
+  griddep_wait_and_release();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= p.C) return;
   const int slot = blockIdx.y;
@@ -253,6 +255,7 @@ __device__ __forceinline__ uint32_t ld_smem_u32(const uint8_t* p) {
 // time-bounded waits.
 template <int D>
 __global__ void __launch_bounds__(ScanLayout<D>::NT, 1) gdn_scan_kernel(const GdnLaunch p) {
+  griddep_wait_and_release();
   using L = ScanLayout<D>;
   constexpr int NSW = L::NSW;
   constexpr int RB = 2 * D;
@@ -594,13 +597,14 @@ int launch_gdn_prepare(const GdnLaunch& g, cudaStream_t s) {
   if (e) return e;
   // channel blocks vary fastest, so the blocks in flight read whole row segments
   dim3 grid((g.C + PREP_CH - 1) / PREP_CH + 1, (g.T + PREP_TT - 1) / PREP_TT, g.n_seq * g.n_gdn);
+  cudaError_t r;
   if (g.mix_dtype == KVA_F16)
-    gdn_prepare_kernel<__half><<<grid, PREP_THREADS, 0, s>>>(g);
+    r = launch_pdl(gdn_prepare_kernel<__half>, grid, dim3(PREP_THREADS), 0, s, g);
   else if (g.mix_dtype == KVA_BF16)
-    gdn_prepare_kernel<__nv_bfloat16><<<grid, PREP_THREADS, 0, s>>>(g);
+    r = launch_pdl(gdn_prepare_kernel<__nv_bfloat16>, grid, dim3(PREP_THREADS), 0, s, g);
   else
     return KVA_ERR_INVALID_ARG;
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s) {
@@ -608,8 +612,7 @@ int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s) {
   int e = check_gdn(g);
   if (e) return e;
   dim3 grid((g.C + 255) / 256, g.n_seq * g.n_gdn);
-  gdn_tail_kernel<<<grid, 256, 0, s>>>(g);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return launch_pdl(gdn_tail_kernel, grid, dim3(256), 0, s, g) == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ after the fused heads GEMM
@@ -620,6 +623,7 @@ int launch_gdn_tail(const GdnLaunch& g, cudaStream_t s) {
 // 2048-channel group of the k | v channels), 8 channels per thread.
 template <typename TM>
 __global__ void __launch_bounds__(256) gdn_halo_fix_kernel(const MixParams mp, const void* conv_state) {
+  griddep_wait_and_release();
   const int b = blockIdx.x, layer = blockIdx.y;
   const int nkdk = mp.n_k * 128;
   const int c0 = nkdk + blockIdx.z * 2048 + threadIdx.x * 8;  // conv channel (k or v)
@@ -684,6 +688,7 @@ __global__ void __launch_bounds__(256) gdn_halo_fix_kernel(const MixParams mp, c
 // New conv tail from the last raw rows the fused epilogue kept (raw row T-3+i, or old
 // tail row T+i when T < 3); ascending i reads only rows not yet overwritten.
 __global__ void gdn_tail_fused_kernel(const MixParams mp, void* conv_state) {
+  griddep_wait_and_release();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= mp.C) return;
   const int layer = blockIdx.y;
@@ -700,16 +705,18 @@ int launch_gdn_halo_fix(const MixParams& mp, int n_gdn, cudaStream_t s, int dtyp
   const int nkdk = mp.n_k * 128;
   if ((mp.C - nkdk) % 8 || nkdk % 128) return KVA_ERR_UNSUPPORTED;
   dim3 grid((mp.T + 127) / 128, n_gdn, (mp.C - nkdk + 2047) / 2048);
-  if (dtype == KVA_F16) gdn_halo_fix_kernel<__half><<<grid, 256, 0, s>>>(mp, conv_state);
-  else gdn_halo_fix_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(mp, conv_state);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  const cudaError_t r =
+      dtype == KVA_F16 ? launch_pdl(gdn_halo_fix_kernel<__half>, grid, dim3(256), 0, s, mp, conv_state)
+                       : launch_pdl(gdn_halo_fix_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, mp, conv_state);
+  return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 int launch_gdn_tail_fused(const MixParams& mp, int n_gdn, void* conv_state, cudaStream_t s) {
   if (mp.T == 0 || n_gdn == 0) return KVA_OK;
   dim3 grid((mp.C + 255) / 256, n_gdn);
-  gdn_tail_fused_kernel<<<grid, 256, 0, s>>>(mp, conv_state);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return launch_pdl(gdn_tail_fused_kernel, grid, dim3(256), 0, s, mp, conv_state) == cudaSuccess
+             ? KVA_OK
+             : KVA_ERR_CUDA;
 }
 
 template <int D>
@@ -719,8 +726,9 @@ static int launch_scan_d(const GdnLaunch& g, cudaStream_t s) {
                            bytes) != cudaSuccess)
     return KVA_ERR_CUDA;
   dim3 grid(g.n_v, g.n_gdn, g.n_seq);
-  gdn_scan_kernel<D><<<grid, ScanLayout<D>::NT, bytes, s>>>(g);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return launch_pdl(gdn_scan_kernel<D>, grid, dim3(ScanLayout<D>::NT), bytes, s, g) == cudaSuccess
+             ? KVA_OK
+             : KVA_ERR_CUDA;
 }
 
 int launch_gdn_scan(const GdnLaunch& g, cudaStream_t s) {

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
   uint8_t* B1 = sm + Cp::B1;
   const uint32_t sL = smem_u32(sm + Cp::L);
   const uint32_t kb = smem_u32(sm + Cp::K);
+  griddep_wait_and_release();  // K, g and beta come from the kernels before
 
   // K rows of the chunk, raw g and beta (zero past T: identity steps); the B1
   // staging tile starts from zero (its blocks above the diagonal stay zero)
@@ -381,6 +382,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = *tslot;
+  griddep_wait_and_release();  // state, K, V and B1 come from the kernels before
   const uint32_t lrow = static_cast<uint32_t>(32 * qd) << 16;
   const uint32_t tS = tb + lrow + COL_S + 64 * hc;  // this thread's 64 state columns
   const uint32_t tA = tb + lrow + COL_A;
@@ -612,8 +614,9 @@ int launch_gdn_chunk_prep(const GdnLaunch& g, int l0, int nl, cudaStream_t s) {
                            Cp::ALLOC) != cudaSuccess)
     return KVA_ERR_CUDA;
   dim3 gp(g.n_v, n_chunks, static_cast<unsigned>(g.n_seq * nl));
-  gdn_chunk_prep_kernel<<<gp, Cp::THREADS, Cp::ALLOC, s>>>(mK, g, l0, nl);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return launch_pdl(gdn_chunk_prep_kernel, gp, dim3(Cp::THREADS), Cp::ALLOC, s, mK, g, l0, nl) == cudaSuccess
+             ? KVA_OK
+             : KVA_ERR_CUDA;
 }
 
 int launch_gdn_chain(const GdnLaunch& g, int l0, int nl, cudaStream_t s) {
@@ -633,8 +636,9 @@ int launch_gdn_chain(const GdnLaunch& g, int l0, int nl, cudaStream_t s) {
                            Sc::ALLOC) != cudaSuccess)
     return KVA_ERR_CUDA;
   dim3 grid(g.n_v, nl, g.n_seq);
-  gdn_scan_tc_kernel<<<grid, NTHREADS, Sc::ALLOC, s>>>(mK, mV, mB, g, l0);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return launch_pdl(gdn_scan_tc_kernel, grid, dim3(NTHREADS), Sc::ALLOC, s, mK, mV, mB, g, l0) == cudaSuccess
+             ? KVA_OK
+             : KVA_ERR_CUDA;
 }
 
 int launch_gdn_scan_tc(const GdnLaunch& g, cudaStream_t s) {

@@ -48,6 +48,7 @@ struct GemmParams {
   int64_t ldd1;
   int64_t n_split;
   int splits;  // K ranges per tile (ADD_F32 only; partial sums added atomically)
+  int d_tma;   // ADD_F32 on CTA pairs: tiles added to D by TMA reductions (tensor map mD)
   int* err;
 };
 
@@ -202,6 +203,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();  // operands and outputs belong to earlier kernels
 
   const int num_m = (p.M + Cfg::BM - 1) / Cfg::BM;
   const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
@@ -753,6 +755,57 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
 // bytes that the tensor core reads from shared memory per MMA, the limit of the
 // one-CTA 128 x 256 tile.  TMA loads of both CTAs complete on the leader's barrier
 // (no multicast loads); MMA completion is committed to both CTAs' barriers.
+// ADD_F32 on CTA pairs: the fp32 accumulator tile goes to the residual stream by TMA
+// reduce-add.  Each 32-column chunk (128 rows x 128 bytes, 128-byte swizzle: 16-byte
+// piece j of row r at piece j ^ (r & 7), so the row-per-thread writes are conflict-free)
+// is staged in one of two shared buffers and added to D by one bulk tensor reduction,
+// coalesced and done at L2.  A buffer is refilled only after the reduction issued from
+// it two chunks earlier has finished reading it.
+constexpr int RED_BUF_BYTES = 128 * 128;
+
+__device__ __forceinline__ void red_sync() { asm volatile("bar.sync 5, 128;" ::: "memory"); }
+// the AND of `v` over the four epilogue warps (same barrier)
+__device__ __forceinline__ bool red_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 5, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void epilogue_add_tma(const CUtensorMap* mD, uint32_t tmem_acc, int row0,
+                                                 int col0, int q, int lane, uint8_t* stage, int& turn,
+                                                 bool issuer) {
+  const int r = q * 32 + lane;
+  const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+  for (int c = 0; c < 256; c += 32) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr + c, v);
+    tmem_ld_wait();
+    uint8_t* buf = stage + turn * RED_BUF_BYTES;
+    turn ^= 1;
+    if (issuer) bulk_wait_read<1>();
+    red_sync();  // the buffer is free
+    uint8_t* row = buf + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) =
+          make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    fence_proxy_async_smem();
+    red_sync();  // the chunk is staged
+    if (issuer) {
+      tma_reduce_add_2d(mD, buf, col0 + c, row0);
+      bulk_commit();
+    }
+  }
+}
+
 struct PairCfg {
   static constexpr int BM = 128;  // rows per CTA (256 per pair)
   static constexpr int BN = 256;  // tile columns (128 B rows held by each CTA)
@@ -764,6 +817,8 @@ struct PairCfg {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
   static constexpr int SMEM_MIX = SMEM + MIX_STAGE_BYTES;  // + the conv staging buffers
+  // ADD_F32 by TMA reduction: the two staging buffers start 1024 bytes after the barriers
+  static constexpr int SMEM_RED = STAGES * STAGE_BYTES + 1024 + 1024 + 2 * RED_BUF_BYTES;
   // producer warp, MMA warp, then the epilogue warps (eight for the state-update epilogue)
   static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
   static constexpr int threads(int epi) { return 64 + 32 * epi_warps(epi); }
@@ -773,7 +828,8 @@ template <int EPI, typename T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI), 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                      const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
-                     const GemmParams p, const __grid_constant__ MixParams mp) {
+                     const __grid_constant__ CUtensorMap mD, const GemmParams p,
+                     const __grid_constant__ MixParams mp) {
   using Cfg = PairCfg;
   constexpr int S = Cfg::STAGES;
   constexpr int BN = Cfg::BN;
@@ -791,6 +847,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* mix_stage = reinterpret_cast<uint8_t*>(bars) + 256;
   (void)mix_stage;
+  uint8_t* red_stage = reinterpret_cast<uint8_t*>(bars) + 1024;  // 1024-byte aligned
+  (void)red_stage;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -824,6 +882,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   cluster_sync();  // the peer's barriers exist before anything arrives on them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();  // operands and outputs belong to earlier kernels
 
   const int num_m = (p.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
   const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
@@ -962,8 +1021,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int grp = (warp - 2) >> 2;        // column group (state-update epilogue)
     (void)grp;
-    int turn = 0;                           // the group's next conv staging buffer
+    int turn = 0;                           // the next staging buffer (conv rows / reductions)
     (void)turn;
+    const bool issuer = warp == 2 && lane == 0;  // issues the TMA reductions
+    (void)issuer;
     const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                      mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
@@ -980,6 +1041,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         // the epilogue warps meet at named barriers inside the epilogue, so they leave
         // together: a barrier-reduction vote over all of them
         if (!mix_all(got)) break;
+      } else if (EPI == EPI_ADD_F32 && p.d_tma) {
+        if (!red_all(got)) break;  // the reduction epilogue has named barriers too
       } else if (!got) {
         break;
       }
@@ -988,6 +1051,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         epilogue_mixer<T>(mp, tmem_base + static_cast<uint32_t>(acc * BN),
                           m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q, grp, lane,
                           mix_stage, turn);
+      else if (EPI == EPI_ADD_F32 && p.d_tma)
+        epilogue_add_tma(&mD, tmem_base + static_cast<uint32_t>(acc * BN),
+                         m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk * BN, q, lane,
+                         red_stage, turn, issuer);
       else
         epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
                                   m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
@@ -998,6 +1065,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    // the reductions have read their buffers and written D before the CTA exits
+    if (EPI == EPI_ADD_F32 && p.d_tma && issuer) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -1038,6 +1107,21 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t ro
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp32 row-major [rows, inner] (row stride ld elements) as a reduction target: box
+// [128 rows, 32 columns] = 128 bytes per row, 128-byte swizzle.
+static bool make_map_f32_red(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -1100,7 +1184,7 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
     const void* src = a.B[i < nb ? i : 0];
     if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, box_b, dt)) return KVA_ERR_CUDA;
   }
-  GemmParams p;
+  GemmParams p = {};
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
@@ -1130,7 +1214,8 @@ static int launch_instance(const GemmArgs& a, cudaStream_t s) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<grid, 192, Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p);
+  if (launch_pdl(kern, dim3(grid), dim3(192), Cfg::SMEM, s, mA, mB[0], mB[1], mB[2], p) != cudaSuccess)
+    return KVA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
@@ -1151,7 +1236,7 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
     const void* src = a.B[i < nb ? i : 0];
     if (!make_map(&mB[i], src, a.K, b_rows, a.ldb, Cfg::BN / 2, dt)) return KVA_ERR_CUDA;
   }
-  GemmParams p;
+  GemmParams p = {};
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
@@ -1163,6 +1248,15 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   p.ldd1 = a.ldd1;
   p.n_split = a.n_split;
   p.err = a.err;
+  // residual adds by TMA reduction when D is a plain fp32 matrix the tensor map can describe
+  CUtensorMap mD = mA;
+  p.d_tma = 0;
+  if (EPI == EPI_ADD_F32 && a.n_split == 0 && (reinterpret_cast<uintptr_t>(a.D) & 15u) == 0 &&
+      a.ldd % 4 == 0 && a.N % 4 == 0) {
+    if (!make_map_f32_red(&mD, a.D, a.N, a.M, a.ldd)) return KVA_ERR_CUDA;
+    p.d_tma = 1;
+  }
+  const int smem = p.d_tma ? Cfg::SMEM_RED : Cfg::SMEM;
   const int n_per_tile = paired ? Cfg::BN / 2 : Cfg::BN;
   const int num_m = (a.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
   const int num_k = (a.K + Cfg::BK - 1) / Cfg::BK;
@@ -1177,10 +1271,11 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   int ncl = items < max_cl ? items : max_cl;
   if (items > ncl && num_m > 1 && ncl >= num_m && num_m <= 16) ncl -= ncl % num_m;
   auto kern = gemm_pair_kernel<EPI, T>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<2 * ncl, Cfg::threads(EPI), Cfg::SMEM, s>>>(mA, mB[0], mB[1], mB[2], p, MixParams());
+  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI)), smem, s, mA, mB[0], mB[1], mB[2], mD, p,
+                 MixParams()) != cudaSuccess)
+    return KVA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
@@ -1193,7 +1288,7 @@ static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64
   CUtensorMap mA, mB;
   if (!make_map(&mA, A, K, M, lda, Cfg::BM, dt)) return KVA_ERR_CUDA;
   if (!make_map(&mB, W, K, n_rows_w, K, Cfg::BN / 2, dt)) return KVA_ERR_CUDA;
-  GemmParams p;
+  GemmParams p = {};
   p.M = M;
   p.N = num_tiles * Cfg::BN;  // one tile per table entry
   p.K = K;
@@ -1215,7 +1310,9 @@ static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_MIX) !=
       cudaSuccess)
     return KVA_ERR_CUDA;
-  kern<<<2 * ncl, Cfg::threads(EPI_MIXER), Cfg::SMEM_MIX, s>>>(mA, mB, mB, mB, p, mp);
+  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI_MIXER)), Cfg::SMEM_MIX, s, mA, mB, mB, mB, mA,
+                 p, mp) != cudaSuccess)
+    return KVA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 

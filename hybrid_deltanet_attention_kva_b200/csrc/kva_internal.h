@@ -8,6 +8,28 @@
 
 namespace kva {
 
+// Every kernel of the library is launched with programmatic stream serialization: it may
+// be scheduled while the kernel before it on the stream is finishing.  Each kernel runs
+// only set-up work that touches no global memory (barrier init, TMEM allocation, tensor
+// map prefetch) before griddepcontrol.wait, which returns once the previous grid has
+// completed and its writes are visible; right after it, the kernel lets the next one be
+// scheduled.  So at most two grids are in flight and each one sees all earlier results.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 enum GemmEpilogue {
   EPI_STORE_BF16 = 0,   // D = acc (in the 16-bit operand format)
   EPI_STORE_F32 = 1,    // D = acc (fp32)
@@ -50,9 +72,10 @@ int num_sms();
 bool make_map_3d_16bit(void* map, const void* base, bool fp16, int64_t d0, int64_t d1,
                        int64_t d2, int box0, int box1);
 int launch_gemm(const GemmArgs& a, cudaStream_t s);
+// `zero` (optional): also clear the first nz fp32 values of each row of zero (row stride ldz)
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
                    int64_t ldo, int rows, int n, float eps, cudaStream_t s,
-                   int out_dtype = KVA_BF16);
+                   int out_dtype = KVA_BF16, float* zero = nullptr, int64_t ldz = 0, int nz = 0);
 int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
                      int window, cudaStream_t s, int dtype = KVA_BF16);
 

@@ -30,6 +30,7 @@ struct VecT<4> {
 
 template <int EPL, typename TM, typename TC>
 __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
+  griddep_wait_and_release();
   using V = typename VecT<EPL>::T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -139,7 +140,8 @@ int launch_kv_write(const KvLaunch& k, cudaStream_t s) {
     return KVA_ERR_INVALID_ARG;
   dim3 grid((k.T + 7) / 8, k.n_kv * k.n_attn, k.n_seq);
   const bool mh = k.mix_dtype == KVA_F16, ch = k.cache.dtype == KVA_F16;
-#define KVA_KV_LAUNCH(EPL, TM, TC) kv_write_kernel<EPL, TM, TC><<<grid, 256, 0, s>>>(k)
+  cudaError_t r;
+#define KVA_KV_LAUNCH(EPL, TM, TC) r = launch_pdl(kv_write_kernel<EPL, TM, TC>, grid, dim3(256), 0, s, k)
   if (epl == 8) {
     if (mh && ch) KVA_KV_LAUNCH(8, __half, __half);
     else if (mh) KVA_KV_LAUNCH(8, __half, __nv_bfloat16);
@@ -152,7 +154,7 @@ int launch_kv_write(const KvLaunch& k, cudaStream_t s) {
     else KVA_KV_LAUNCH(4, __nv_bfloat16, __nv_bfloat16);
   }
 #undef KVA_KV_LAUNCH
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 }  // namespace kva

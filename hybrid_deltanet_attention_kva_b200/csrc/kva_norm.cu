@@ -30,8 +30,15 @@ template <typename T, typename TO>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, int64_t ldx,
                                                       const float* __restrict__ g,
                                                       TO* __restrict__ out, int64_t ldo, int n,
-                                                      float eps) {
+                                                      float eps, float* __restrict__ zero,
+                                                      int64_t ldz, int nz) {
+  griddep_wait_and_release();
   const int row = blockIdx.x;
+  if (zero) {  // clear this row of another buffer (the next GEMM accumulates into it)
+    float* zr = zero + row * ldz;
+    for (int i = threadIdx.x * 4; i < nz; i += blockDim.x * 4)
+      *reinterpret_cast<float4*>(zr + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const T* xr = x + row * ldx;
   TO* orow = out + row * ldo;
   float ss = 0.f;
@@ -61,34 +68,36 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, i
 }
 
 template <typename TO>
-static void rms_dispatch(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
-                         int64_t ldo, int rows, int n, float eps, cudaStream_t s) {
+static cudaError_t rms_dispatch(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
+                                int64_t ldo, int rows, int n, float eps, cudaStream_t s, float* zero,
+                                int64_t ldz, int nz) {
   TO* o = static_cast<TO*>(out);
   if (x_dtype == KVA_F32)
-    rmsnorm_kernel<float, TO><<<rows, 256, 0, s>>>(static_cast<const float*>(x), ldx, g, o, ldo, n, eps);
-  else if (x_dtype == KVA_BF16)
-    rmsnorm_kernel<__nv_bfloat16, TO><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                            ldx, g, o, ldo, n, eps);
-  else
-    rmsnorm_kernel<__half, TO><<<rows, 256, 0, s>>>(static_cast<const __half*>(x), ldx, g, o, ldo,
-                                                     n, eps);
+    return launch_pdl(rmsnorm_kernel<float, TO>, dim3(rows), dim3(256), 0, s,
+                      static_cast<const float*>(x), ldx, g, o, ldo, n, eps, zero, ldz, nz);
+  if (x_dtype == KVA_BF16)
+    return launch_pdl(rmsnorm_kernel<__nv_bfloat16, TO>, dim3(rows), dim3(256), 0, s,
+                      static_cast<const __nv_bfloat16*>(x), ldx, g, o, ldo, n, eps, zero, ldz, nz);
+  return launch_pdl(rmsnorm_kernel<__half, TO>, dim3(rows), dim3(256), 0, s,
+                    static_cast<const __half*>(x), ldx, g, o, ldo, n, eps, zero, ldz, nz);
 }
 
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
-                   int64_t ldo, int rows, int n, float eps, cudaStream_t s, int out_dtype) {
+                   int64_t ldo, int rows, int n, float eps, cudaStream_t s, int out_dtype,
+                   float* zero, int64_t ldz, int nz) {
   if (rows == 0) return KVA_OK;
   if (!x || !g || !out || rows < 0 || n <= 0) return KVA_ERR_INVALID_ARG;
   if (x_dtype != KVA_F32 && x_dtype != KVA_BF16 && x_dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   if (out_dtype != KVA_BF16 && out_dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
-  if (n % 4 || ldx % 4 || ldo % 4) return KVA_ERR_ALIGNMENT;
+  if (n % 4 || ldx % 4 || ldo % 4 || nz % 4 || ldz % 4) return KVA_ERR_ALIGNMENT;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(g) |
-       reinterpret_cast<uintptr_t>(out)) & 15u)
+       reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(zero)) & 15u)
     return KVA_ERR_ALIGNMENT;
-  if (out_dtype == KVA_F16)
-    rms_dispatch<__half>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s);
-  else
-    rms_dispatch<__nv_bfloat16>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s);
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  const cudaError_t r =
+      out_dtype == KVA_F16
+          ? rms_dispatch<__half>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s, zero, ldz, nz)
+          : rms_dispatch<__nv_bfloat16>(x, x_dtype, ldx, g, out, ldo, rows, n, eps, s, zero, ldz, nz);
+  return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 }  // namespace kva

@@ -45,7 +45,8 @@ def test_rmsnorm(K, dtype, rows, n, odt):
 # ------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("M,N,K_,bn", [(128, 256, 64, 256), (200, 1296, 520, 0), (1024, 3072, 3072, 128),
                                        (77, 512, 256, 256), (1024, 2560, 5120, 0), (600, 1040, 704, 512),
-                                       (1024, 3072, 3072, 256)])
+                                       (1024, 3072, 3072, 256), (1024, 3072, 8448, 512),
+                                       (1000, 3072, 5120, 512)])
 @pytest.mark.parametrize("epi", [0, 1, 2])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 def test_gemm_epilogues(K, M, N, K_, bn, epi, dt):
