@@ -533,6 +533,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     goto done;
   {
     GemmArgs a;
+    a.b_const = true;  // weights
     a.A = h->u_in;
     a.lda = H;
     a.B[0] = w->W_in;
@@ -555,6 +556,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
          })))
       goto done;
     GemmArgs q;
+    q.b_const = true;  // weights
     q.A = h->u;
     q.lda = dm;
     q.B[0] = B.Wq;
@@ -573,10 +575,12 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     q.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(q, s); }))) goto done;
     if ((e = staged(h, KVA_ST_ATTENTION, s, [&] {
-           return launch_attention(h->qkv, 3 * dm, h->o, dm, T, d.n_heads, d.attn_window, s, cd);
+           return launch_attention(h->qkv, 3 * dm, h->o, dm, T, d.n_heads, d.attn_window, s, cd,
+                                   h->status);
          })))
       goto done;
     GemmArgs o;
+    o.b_const = true;  // weights
     o.A = h->o;
     o.lda = dm;
     o.B[0] = B.Wo;
@@ -595,6 +599,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
          })))
       goto done;
     GemmArgs gu;
+    gu.b_const = true;  // weights
     gu.A = h->u;
     gu.lda = dm;
     gu.B[0] = B.Wg;
@@ -611,6 +616,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     gu.dtype = cd;
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(gu, s); }))) goto done;
     GemmArgs dn;
+    dn.b_const = true;  // weights
     dn.A = h->qkv;
     dn.lda = F;
     dn.B[0] = B.Wd;
@@ -670,6 +676,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   } else {
     __nv_bfloat16* mix = mixer_out ? static_cast<__nv_bfloat16*>(mixer_out) : h->mixer;
     GemmArgs hd;
+    hd.b_const = true;  // weights
     hd.A = h->u;
     hd.lda = dm;
     hd.B[0] = w->W_heads;

@@ -3,224 +3,351 @@
 // 1024-token blocks for r3, full causal within the ubatch for r2).
 //
 // Key j is visible to query i iff j <= i and floor(i/W) == floor(j/W), indices
-// local to the ubatch (W = window, or the whole ubatch when window = 0).
-// Flash-style: 64-query tiles, 4 warps x 16 query rows; a CTA takes the query tiles
-// b and n-1-b of one head so every CTA does the same causal work (two CTAs per SM),
-// 64-key tiles double-buffered in shared memory with cp.async, S = Q K^T and
-// O += P V on mma.sync (16-bit in, fp32 accumulate), online softmax in fp32 with
-// exp2.  qkv is [T, 3d] 16-bit (q | k | v, head h at columns h*128 of each
-// part), output [T, d] in the same format (bf16 or fp16).
+// local to the ubatch (W = window, or the whole ubatch when window = 0).  qkv is
+// [T, 3d] 16-bit (q | k | v, head h at columns h*128 of each part), the output [T, d]
+// in the same format (bf16 or fp16).
+//
+// Flash attention on the tcgen05 tensor cores.  One CTA per (head, 128-query tile),
+// the tiles with the most causal work first.
+//   warp 8   TMA producer: Q once, then 128-key K and V tiles into two stages each
+//            (128-byte swizzle; K and V have their own full / empty barriers, so the
+//            next K tile is loaded as soon as its S product has read the stage)
+//   warp 9   one thread issues the MMAs: S_j = Q K_j^T (both operands K-major in
+//            shared memory) into TMEM buffer j % 2, and O += P_j V_j with P_j read
+//            from TMEM and V_j as an MN-major shared-memory operand
+//   warps 0-7  two threads per query row (TMEM lane = row; warps w and w + 4 take
+//            columns 0-63 and 64-127): read their half of the row of S_j, mask it,
+//            trade half-row maxima through shared memory, keep a running reference
+//            max (O and the row sum are rescaled only when the tile's max exceeds the
+//            reference by more than 8 in log2 units, so P stays below 2^8), write
+//            P_j = 2^(s - ref) in the operand format to TMEM buffer j % 2; at the end
+//            divide O by the row sum and store it.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512).
+// S_{j+1} is issued before P_j is ready, so the tensor cores compute the next scores
+// while the softmax warps work.  Every barrier wait has a time limit.
 #include <cmath>
 
 #include "kva_common.cuh"
 
 namespace kva {
 
-constexpr int ATT_BQ = 64;
-constexpr int ATT_BKV = 64;
+constexpr int ATT_BQ = 128;
+constexpr int ATT_BKV = 128;
 constexpr int ATT_D = 128;
-constexpr int ATT_THREADS = 128;
-constexpr int ATT_SMEM = (ATT_BQ + 4 * ATT_BKV) * ATT_D * 2;  // Q + 2 x (K, V)
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_HALF = 128 * 64 * 2;  // one 64-dim half of a 128-row tile (16 KB)
+constexpr int ATT_TILE = 2 * ATT_HALF;  // a 128 x 128 16-bit tile
+constexpr int ATT_OFF_K = ATT_TILE;     // K stages
+constexpr int ATT_OFF_V = 3 * ATT_TILE; // V stages
+constexpr int ATT_OFF_BAR = 5 * ATT_TILE;
+// after the barriers: half-row maxima [parity 2][half 2][128] and row-sum halves [half 2][128]
+constexpr int ATT_OFF_X = ATT_OFF_BAR + 256;
+constexpr int ATT_X_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
+constexpr int ATT_SMEM = ATT_OFF_X + ATT_X_BYTES + 1024;  // + alignment slack
 
-// byte offset of (row, 16-byte chunk) in a [rows][128] 16-bit tile, XOR swizzled
-__device__ __forceinline__ uint32_t att_off(int row, int chunk) {
-  return static_cast<uint32_t>(row * 256 + ((chunk ^ (row & 7)) << 4));
+// the 256 softmax threads (named barrier 1), returning the AND of `v` over them
+__device__ __forceinline__ bool att_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+constexpr uint32_t ATT_COL_S = 0, ATT_COL_O = 256, ATT_COL_P = 384;
+constexpr float ATT_RESCALE = 8.f;  // log2 of the largest P value allowed before a rescale
+
+__device__ __forceinline__ float att_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <typename E>
-__device__ __forceinline__ void att_load_tile(uint32_t dst, const E* src, int64_t ld,
-                                              int row0, int rows, int T, int tid) {
-  // rows x 16 chunks of 16 bytes; rows at or beyond T are zero-filled
-  for (int i = tid; i < rows * 16; i += ATT_THREADS) {
-    const int r = i >> 4, c = i & 15;
-    const int gr = row0 + r;
-    const bool ok = gr < T;
-    const E* g = src + static_cast<int64_t>(ok ? gr : 0) * ld + c * 8;
-    cp_async16(dst + att_off(r, c), g, ok ? 16u : 0u);
-  }
-}
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attention_kernel(const __grid_constant__ CUtensorMap mQKV, E* __restrict__ out, int64_t ldo,
+                     int T, int d_model, int n_heads, int window, float scale_log2, int* err) {
+  extern __shared__ uint8_t att_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(att_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + ATT_OFF_BAR);
+  uint64_t* bar_q = bars;        // Q landed
+  uint64_t* fullK = bars + 1;    // [2] K tile landed
+  uint64_t* emptyK = bars + 3;   // [2] S product done with the K stage
+  uint64_t* fullV = bars + 5;    // [2] V tile landed
+  uint64_t* emptyV = bars + 7;   // [2] P V product done with the V stage
+  uint64_t* barS = bars + 9;     // [2] S_j in TMEM
+  uint64_t* barP = bars + 11;    // [2] P_j in TMEM (256 softmax threads)
+  uint64_t* barO = bars + 13;    // O += P_j V_j done
+  uint64_t* bar_drain = bars + 14;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
-template <typename E>
-__global__ void __launch_bounds__(ATT_THREADS)
-    attention_kernel(const E* __restrict__ qkv, int64_t ldq, E* __restrict__ out, int64_t ldo,
-                     int T, int d_model, int window, float scale_log2) {
-  griddep_wait_and_release();
-  extern __shared__ __align__(128) uint8_t att_smem[];
-  const uint32_t sQ = smem_u32(att_smem);
-  const uint32_t sK0 = sQ + ATT_BQ * 256;
-  const uint32_t sV0 = sK0 + 2 * ATT_BKV * 256;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
-  // causal balance: CTA b takes query tiles b and n_qt - 1 - b (equal total key tiles)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (T + ATT_BQ - 1) / ATT_BQ;
-  const int h = blockIdx.y;
-  for (int pass = 0; pass < 2; ++pass) {
-    const int qt = pass == 0 ? static_cast<int>(blockIdx.x) : n_qt - 1 - static_cast<int>(blockIdx.x);
-    if (pass == 1 && qt <= static_cast<int>(blockIdx.x)) break;
-    const int q0 = qt * ATT_BQ;
-    __syncthreads();  // the previous pass finished reading shared memory
-    const int W = window > 0 ? window : 0x3fffffff;
+  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / n_heads;  // most causal work first
+  const int h = static_cast<int>(blockIdx.x) % n_heads;
+  const int q0 = qt * ATT_BQ;
+  const int W = window > 0 ? window : 0x3fffffff;
+  const int q_last = min(T, q0 + ATT_BQ) - 1;
+  const int t_lo = ((q0 / W) * W) / ATT_BKV;  // first key tile any row of the tile may see
+  const int n_kv = q_last / ATT_BKV - t_lo + 1;
 
-    const E* Qg = qkv + h * ATT_D;
-    const E* Kg = qkv + d_model + h * ATT_D;
-    const E* Vg = qkv + 2 * d_model + h * ATT_D;
-
-    const int q_last = min(T, q0 + ATT_BQ) - 1;
-    const int kv_lo = (q0 / W) * W;             // first key any row of the tile may see
-    const int kv_hi = q_last + 1;               // one past the last visible key
-    const int t_lo = (kv_lo / ATT_BKV) * ATT_BKV;
-    const int n_tiles = (kv_hi - t_lo + ATT_BKV - 1) / ATT_BKV;
-
-    att_load_tile(sQ, Qg, ldq, q0, ATT_BQ, T, tid);
-    att_load_tile(sK0, Kg, ldq, t_lo, ATT_BKV, T, tid);
-    att_load_tile(sV0, Vg, ldq, t_lo, ATT_BKV, T, tid);
-    cp_async_commit();
-
-    // rows of this thread
-    const int r0 = q0 + warp * 16 + g;
-    const int r1 = r0 + 8;
-    const int lo0 = (r0 / W) * W, lo1 = (r1 / W) * W;
-
-    float o[16][4];
-  #pragma unroll
-    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    uint32_t qf[8][4];
-
-    for (int it = 0; it < n_tiles; ++it) {
-      const int buf = it & 1;
-      if (it + 1 < n_tiles) {
-        const int nb = (it + 1) & 1;
-        att_load_tile(sK0 + nb * ATT_BKV * 256, Kg, ldq, t_lo + (it + 1) * ATT_BKV, ATT_BKV, T, tid);
-        att_load_tile(sV0 + nb * ATT_BKV * 256, Vg, ldq, t_lo + (it + 1) * ATT_BKV, ATT_BKV, T, tid);
-        cp_async_commit();
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncthreads();
-      if (it == 0) {
-        // Q fragments for this warp's 16 rows, all 8 k-steps
-  #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const int mi = lane >> 3;
-          const int row = warp * 16 + (mi & 1) * 8 + (lane & 7);
-          const int ch = ks * 2 + (mi >> 1);
-          ldmatrix_x4(qf[ks], sQ + att_off(row, ch));
-        }
-      }
-      const uint32_t sK = sK0 + buf * ATT_BKV * 256;
-      const uint32_t sV = sV0 + buf * ATT_BKV * 256;
-      const int j0 = t_lo + it * ATT_BKV;
-
-      float s[8][4];
-  #pragma unroll
-      for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-  #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-  #pragma unroll
-        for (int nt = 0; nt < 8; nt += 2) {
-          uint32_t kb[4];
-          const int mi = lane >> 3;
-          const int row = nt * 8 + (mi >> 1) * 8 + (lane & 7);
-          const int ch = ks * 2 + (mi & 1);
-          ldmatrix_x4(kb, sK + att_off(row, ch));
-          uint32_t b0[2] = {kb[0], kb[1]}, b1[2] = {kb[2], kb[3]};
-          F16<E>::mma(s[nt], qf[ks], b0);
-          F16<E>::mma(s[nt + 1], qf[ks], b1);
-        }
-      }
-      // mask + row max
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-  #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-  #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + nt * 8 + 2 * c + e;
-          const bool v0 = j <= r0 && j >= lo0 && j < T;
-          const bool v1 = j <= r1 && j >= lo1 && j < T;
-          s[nt][e] = v0 ? s[nt][e] : -INFINITY;
-          s[nt][2 + e] = v1 ? s[nt][2 + e] : -INFINITY;
-          mx0 = fmaxf(mx0, s[nt][e]);
-          mx1 = fmaxf(mx1, s[nt][2 + e]);
-        }
-      }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float ref0 = mn0 == -INFINITY ? 0.f : mn0 * scale_log2;
-      const float ref1 = mn1 == -INFINITY ? 0.f : mn1 * scale_log2;
-      const float al0 = exp2f(m0 == -INFINITY ? -INFINITY : m0 * scale_log2 - ref0);
-      const float al1 = exp2f(m1 == -INFINITY ? -INFINITY : m1 * scale_log2 - ref1);
-      m0 = mn0;
-      m1 = mn1;
-      float rs0 = 0.f, rs1 = 0.f;
-  #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-  #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          s[nt][e] = exp2f(s[nt][e] * scale_log2 - ref0);
-          s[nt][2 + e] = exp2f(s[nt][2 + e] * scale_log2 - ref1);
-          rs0 += s[nt][e];
-          rs1 += s[nt][2 + e];
-        }
-      }
-      rs0 += __shfl_xor_sync(0xffffffffu, rs0, 1);
-      rs0 += __shfl_xor_sync(0xffffffffu, rs0, 2);
-      rs1 += __shfl_xor_sync(0xffffffffu, rs1, 1);
-      rs1 += __shfl_xor_sync(0xffffffffu, rs1, 2);
-      l0 = l0 * al0 + rs0;
-      l1 = l1 * al1 + rs1;
-  #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        o[i][0] *= al0;
-        o[i][1] *= al0;
-        o[i][2] *= al1;
-        o[i][3] *= al1;
-      }
-      // O += P V
-  #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4];
-        a[0] = F16<E>::pack(s[2 * kk][0], s[2 * kk][1]);
-        a[1] = F16<E>::pack(s[2 * kk][2], s[2 * kk][3]);
-        a[2] = F16<E>::pack(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        a[3] = F16<E>::pack(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-  #pragma unroll
-        for (int dt = 0; dt < 16; dt += 2) {
-          uint32_t vb[4];
-          const int mi = lane >> 3;
-          const int row = kk * 16 + (mi & 1) * 8 + (lane & 7);
-          const int ch = dt + (mi >> 1);
-          ldmatrix_x4_trans(vb, sV + att_off(row, ch));
-          uint32_t b0[2] = {vb[0], vb[1]}, b1[2] = {vb[2], vb[3]};
-          F16<E>::mma(o[dt], a, b0);
-          F16<E>::mma(o[dt + 1], a, b1);
-        }
-      }
-      __syncthreads();  // buffer `buf` is refilled two iterations later
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&fullK[i], 1);
+      mbar_init(&emptyK[i], 1);
+      mbar_init(&fullV[i], 1);
+      mbar_init(&emptyV[i], 1);
+      mbar_init(&barS[i], 1);
+      mbar_init(&barP[i], 256);
     }
+    mbar_init(barO, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mQKV);
+  }
+  if (warp == 9) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = *tslot;
+  griddep_wait_and_release();  // q, k, v come from the GEMM before
 
-    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
-    const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-  #pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-      const int col = h * ATT_D + dt * 8 + 2 * c;
-      if (r0 < T)
-        *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(r0) * ldo + col) =
-            F16<E>::pack(o[dt][0] * inv0, o[dt][1] * inv0);
-      if (r1 < T)
-        *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(r1) * ldo + col) =
-            F16<E>::pack(o[dt][2] * inv1, o[dt][3] * inv1);
+  if (warp == 8) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol = l2_policy_evict_normal();
+      const int cq = h * ATT_D, ck = d_model + h * ATT_D, cv = 2 * d_model + h * ATT_D;
+      mbar_arrive_expect_tx(bar_q, ATT_TILE);
+      tma_load_2d(sm, &mQKV, bar_q, cq, q0, pol);
+      tma_load_2d(sm + ATT_HALF, &mQKV, bar_q, cq + 64, q0, pol);
+      bool ok = true;
+      int issued = 0;  // tiles whose K and V were both requested
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1u;  // the release of tile j - 2
+        const int k0 = (t_lo + j) * ATT_BKV;
+        if (j >= 2 && !mbar_wait(&emptyK[s], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* kd = sm + ATT_OFF_K + s * ATT_TILE;
+        mbar_arrive_expect_tx(&fullK[s], ATT_TILE);
+        tma_load_2d(kd, &mQKV, &fullK[s], ck, k0, pol);
+        tma_load_2d(kd + ATT_HALF, &mQKV, &fullK[s], ck + 64, k0, pol);
+        if (j >= 2 && !mbar_wait(&emptyV[s], ph, abort_flag)) {
+          ok = false;
+          mbar_wait_limit(&fullK[s], (j >> 1) & 1);  // this K tile lands before exit
+          break;
+        }
+        uint8_t* vd = sm + ATT_OFF_V + s * ATT_TILE;
+        mbar_arrive_expect_tx(&fullV[s], ATT_TILE);
+        tma_load_2d(vd, &mQKV, &fullV[s], cv, k0, pol);
+        tma_load_2d(vd + ATT_HALF, &mQKV, &fullV[s], cv + 64, k0, pol);
+        issued = j + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      // every copy requested has landed before the CTA exits
+      mbar_wait_limit(bar_q, 0);
+      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
+        mbar_wait_limit(&fullK[j & 1], (j >> 1) & 1);
+        mbar_wait_limit(&fullV[j & 1], (j >> 1) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idS = idesc_f16kind_f32(ATT_BQ, ATT_BKV, F16<E>::umma_fmt);
+      constexpr uint32_t idO = idesc_f16kind_f32_major(ATT_BQ, ATT_D, F16<E>::umma_fmt, false, true);
+      const uint32_t sQ = smem_u32(sm);
+      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&fullK[s], (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + ATT_OFF_K + s * ATT_TILE);
+#pragma unroll
+        for (int k = 0; k < ATT_D / 16; ++k) {  // 16 dims per MMA: half k / 4, 32 bytes each
+          const uint32_t off = (k >> 2) * ATT_HALF + (k & 3) * 32;
+          umma_f16_ss(tb + ATT_COL_S + s * 128, sdesc_k_sw128(sQ + off), sdesc_k_sw128(sK + off), idS,
+                      k > 0 ? 1u : 0u);
+        }
+        umma_commit(&barS[s]);
+        umma_commit(&emptyK[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j & 1;
+        if (j + 1 < n_kv && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&barP[s], (j >> 1) & 1, abort_flag) ||
+            !mbar_wait(&fullV[s], (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sV = smem_u32(sm + ATT_OFF_V + s * ATT_TILE);
+#pragma unroll
+        for (int k = 0; k < ATT_BKV / 16; ++k)  // 16 keys per MMA: 8 columns of P, 16 rows of V
+          umma_f16_ts(tb + ATT_COL_O, tb + ATT_COL_P + s * 64 + k * 8,
+                      sdesc_mn_sw128(sV + k * 2048, ATT_HALF), idO, (j > 0 || k > 0) ? 1u : 0u);
+        umma_commit(barO);
+        umma_commit(&emptyV[s]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_device_error(err, KVA_DEV_WAIT_TIMEOUT);
+      }
+      // every MMA issued completes before TMEM is released
+      umma_commit(bar_drain);
+      mbar_wait_limit(bar_drain, 0);
+    }
+  } else {
+    // ------------------------------------------------ softmax and output (warps 0-7)
+    const int qd = warp & 3, hc = warp >> 2;  // TMEM lane quarter, column half
+    const int r = qd * 32 + lane;
+    const int i = q0 + r;                     // query row
+    const int kb = (i / W) * W;               // its first visible key
+    const uint32_t lrow = static_cast<uint32_t>(qd * 32) << 16;
+    float* xch = reinterpret_cast<float*>(sm + ATT_OFF_X);  // [parity][half][row]
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;  // every wait so far succeeded; a failure stops all of them at the next vote
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&barS[s], (j >> 1) & 1, abort_flag));
+      float x[64];
+      float mh = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        uint32_t ra[32], rb[32];
+        const uint32_t ts = tb + lrow + ATT_COL_S + s * 128 + hc * 64;
+        tmem_ld_32x32b_x32(ts, ra);
+        tmem_ld_32x32b_x32(ts + 32, rb);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          x[e] = __uint_as_float(ra[e]);
+          x[32 + e] = __uint_as_float(rb[e]);
+        }
+        const int k0 = (t_lo + j) * ATT_BKV + hc * 64;
+        if (k0 + 63 > i || k0 < kb) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (k0 + e > i || k0 + e < kb) x[e] = -INFINITY;
+        }
+        float mx[16];  // a tree of maxima instead of one 64-long dependent chain
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mx[e] = fmaxf(fmaxf(x[e], x[16 + e]), fmaxf(x[32 + e], x[48 + e]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) mx[e] = fmaxf(mx[e], mx[e + w]);
+        mh = mx[0];
+        xch[(s * 2 + hc) * 128 + r] = mh;
+      }
+      if (!att_all(ok)) {  // also: both halves' maxima are in shared memory
+        ok = false;
+        break;
+      }
+      // the tile max in log2 units (the scale is positive); a slot is rewritten two tiles
+      // later, after the partner has passed the next vote
+      const float mt = fmaxf(mh, xch[(s * 2 + (hc ^ 1)) * 128 + r]) * scale_log2;
+      float factor = 1.f;
+      bool resc = false;
+      if (mt > m_ref + ATT_RESCALE) {  // also the first visible key (m_ref = -inf)
+        factor = att_ex2(m_ref - mt);
+        l *= factor;
+        m_ref = mt;
+        resc = j > 0;
+      }
+      const float ref = m_ref == -INFINITY ? 0.f : m_ref;  // nothing visible yet: P = 0
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = att_ex2(fmaf(x[2 * e], scale_log2, -ref));
+        const float p1 = att_ex2(fmaf(x[2 * e + 1], scale_log2, -ref));
+        l += p0 + p1;
+        pk[e] = F16<E>::pack(p0, p1);
+      }
+      tmem_st_32x32b_x32(tb + lrow + ATT_COL_P + s * 64 + hc * 32, pk);
+      if (__any_sync(0xffffffffu, resc)) {
+        // the reference moved: O (complete up to P_{j-1} V_{j-1}) scales with it
+        ok = __all_sync(0xffffffffu, mbar_wait(barO, (j - 1) & 1, abort_flag));
+        if (ok) {
+          tc_fence_after();
+          const float f = resc ? factor : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            const uint32_t to = tb + lrow + ATT_COL_O + hc * 64 + c * 32;
+            tmem_ld_32x32b_x32(to, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st_32x32b_x32(to, o);
+          }
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&barP[s]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(barO, (n_kv - 1) & 1, abort_flag));
+    float* lx = xch + 4 * 128;  // [half][row] row-sum halves
+    lx[hc * 128 + r] = l;
+    if (att_all(ok)) {
+      tc_fence_after();
+      const float lt = l + lx[(hc ^ 1) * 128 + r];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      E* orow = out + static_cast<int64_t>(i) * ldo + h * ATT_D + hc * 64;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tb + lrow + ATT_COL_O + hc * 64 + c * 32, o);
+        tmem_ld_wait();
+        if (i < T) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = F16<E>::pack(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+            v.y = F16<E>::pack(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+            v.z = F16<E>::pack(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+            v.w = F16<E>::pack(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 32)[q4] = v;
+          }
+        }
+      }
+    } else {
+      *abort_flag = 1;
+      set_device_error(err, KVA_DEV_WAIT_TIMEOUT);
     }
   }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tb, 512);
 }
 
+// ------------------------------------------------------------------ host side
 int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
-                     int window, cudaStream_t s, int dtype) {
+                     int window, cudaStream_t s, int dtype, int* err) {
   if (T == 0) return KVA_OK;
   if (!qkv || !out || T < 0 || n_heads <= 0 || window < 0) return KVA_ERR_INVALID_ARG;
   if (dtype != KVA_BF16 && dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
@@ -230,26 +357,27 @@ int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T
   const int d_model = n_heads * ATT_D;
   if (ldq < 3 * d_model || ldo < d_model) return KVA_ERR_INVALID_ARG;
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ATT_D));
+  CUtensorMap m;
+  if (!make_map_2d_16bit(&m, qkv, dtype == KVA_F16, 3 * static_cast<int64_t>(d_model), T, ldq, 64,
+                         ATT_BQ))
+    return KVA_ERR_CUDA;
   const int n_qt = (T + ATT_BQ - 1) / ATT_BQ;
-  dim3 grid((n_qt + 1) / 2, n_heads);
+  const dim3 grid(n_qt * n_heads);
+  cudaError_t r;
   if (dtype == KVA_F16) {
     if (cudaFuncSetAttribute(attention_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ATT_SMEM) != cudaSuccess)
       return KVA_ERR_CUDA;
-    if (launch_pdl(attention_kernel<__half>, grid, dim3(ATT_THREADS), ATT_SMEM, s,
-                   static_cast<const __half*>(qkv), ldq, static_cast<__half*>(out), ldo, T, d_model,
-                   window, scale_log2) != cudaSuccess)
-      return KVA_ERR_CUDA;
+    r = launch_pdl(attention_kernel<__half>, grid, dim3(ATT_THREADS), ATT_SMEM, s, m,
+                   static_cast<__half*>(out), ldo, T, d_model, n_heads, window, scale_log2, err);
   } else {
     if (cudaFuncSetAttribute(attention_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) != cudaSuccess)
       return KVA_ERR_CUDA;
-    if (launch_pdl(attention_kernel<__nv_bfloat16>, grid, dim3(ATT_THREADS), ATT_SMEM, s,
-                   static_cast<const __nv_bfloat16*>(qkv), ldq, static_cast<__nv_bfloat16*>(out), ldo,
-                   T, d_model, window, scale_log2) != cudaSuccess)
-      return KVA_ERR_CUDA;
+    r = launch_pdl(attention_kernel<__nv_bfloat16>, grid, dim3(ATT_THREADS), ATT_SMEM, s, m,
+                   static_cast<__nv_bfloat16*>(out), ldo, T, d_model, n_heads, window, scale_log2, err);
   }
-  return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+  return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 }  // namespace kva

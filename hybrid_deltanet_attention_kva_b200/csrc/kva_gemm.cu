@@ -49,6 +49,7 @@ struct GemmParams {
   int64_t n_split;
   int splits;  // K ranges per tile (ADD_F32 only; partial sums added atomically)
   int d_tma;   // ADD_F32 on CTA pairs: tiles added to D by TMA reductions (tensor map mD)
+  int b_const; // CTA pairs: the first stages' B tiles are loaded before griddepcontrol.wait
   int* err;
 };
 
@@ -756,51 +757,35 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
 // one-CTA 128 x 256 tile.  TMA loads of both CTAs complete on the leader's barrier
 // (no multicast loads); MMA completion is committed to both CTAs' barriers.
 // ADD_F32 on CTA pairs: the fp32 accumulator tile goes to the residual stream by TMA
-// reduce-add.  Each 32-column chunk (128 rows x 128 bytes, 128-byte swizzle: 16-byte
-// piece j of row r at piece j ^ (r & 7), so the row-per-thread writes are conflict-free)
-// is staged in one of two shared buffers and added to D by one bulk tensor reduction,
-// coalesced and done at L2.  A buffer is refilled only after the reduction issued from
-// it two chunks earlier has finished reading it.
-constexpr int RED_BUF_BYTES = 128 * 128;
-
-__device__ __forceinline__ void red_sync() { asm volatile("bar.sync 5, 128;" ::: "memory"); }
-// the AND of `v` over the four epilogue warps (same barrier)
-__device__ __forceinline__ bool red_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 5, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return r != 0;
-}
+// reduce-add.  Each epilogue warp owns 32 rows; it stages every 32-column chunk of them
+// (32 rows x 128 bytes, 128-byte swizzle: 16-byte piece j of row r at piece j ^ (r & 7),
+// so the row-per-lane writes are conflict-free) in one of its two shared buffers, and
+// its lane 0 adds the block to D with one bulk tensor reduction, coalesced and done at
+// L2.  A buffer is refilled only after the reduction issued from it two chunks earlier
+// has finished reading it.  No barrier is shared between warps.
+constexpr int RED_BUF_BYTES = 32 * 128;
 
 __device__ __forceinline__ void epilogue_add_tma(const CUtensorMap* mD, uint32_t tmem_acc, int row0,
-                                                 int col0, int q, int lane, uint8_t* stage, int& turn,
-                                                 bool issuer) {
-  const int r = q * 32 + lane;
+                                                 int col0, int q, int lane, uint8_t* wstage, int& turn) {
   const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
   for (int c = 0; c < 256; c += 32) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(taddr + c, v);
     tmem_ld_wait();
-    uint8_t* buf = stage + turn * RED_BUF_BYTES;
+    uint8_t* buf = wstage + turn * RED_BUF_BYTES;
     turn ^= 1;
-    if (issuer) bulk_wait_read<1>();
-    red_sync();  // the buffer is free
-    uint8_t* row = buf + r * 128;
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();  // the buffer is free
+    uint8_t* row = buf + lane * 128;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) =
           make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     fence_proxy_async_smem();
-    red_sync();  // the chunk is staged
-    if (issuer) {
-      tma_reduce_add_2d(mD, buf, col0 + c, row0);
+    __syncwarp();  // the block is staged
+    if (lane == 0) {
+      tma_reduce_add_2d(mD, buf, col0 + c, row0 + q * 32);
       bulk_commit();
     }
   }
@@ -817,8 +802,9 @@ struct PairCfg {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
   static constexpr int SMEM_MIX = SMEM + MIX_STAGE_BYTES;  // + the conv staging buffers
-  // ADD_F32 by TMA reduction: the two staging buffers start 1024 bytes after the barriers
-  static constexpr int SMEM_RED = STAGES * STAGE_BYTES + 1024 + 1024 + 2 * RED_BUF_BYTES;
+  // ADD_F32 by TMA reduction: each epilogue warp's two staging buffers, 1024 bytes after
+  // the barriers
+  static constexpr int SMEM_RED = STAGES * STAGE_BYTES + 1024 + 1024 + 4 * 2 * RED_BUF_BYTES;
   // producer warp, MMA warp, then the epilogue warps (eight for the state-update epilogue)
   static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
   static constexpr int threads(int epi) { return 64 + 32 * epi_warps(epi); }
@@ -882,7 +868,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   cluster_sync();  // the peer's barriers exist before anything arrives on them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  griddep_wait_and_release();  // operands and outputs belong to earlier kernels
 
   const int num_m = (p.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
   const int n_per_tile = (EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN;
@@ -892,26 +877,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   const int items = num_m * num_n * splits;
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
+  // producer state (warp 0, lane 0)
+  const uint64_t pol_a = l2_policy_evict_last();
+  const uint64_t pol_b = l2_policy_evict_normal();
+  uint32_t armed = 0;
+  auto load_b = [&](int stage, int n_blk, int kc, uint32_t fb) {
+    uint8_t* b = sB + stage * Cfg::B_BYTES;
+    if constexpr (EPI == EPI_MIXER) {  // the tile's first weight row comes from the table
+      tma_load_2d_pair(b, &mB0, fb, kc, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2), pol_b);
+    } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
+      tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
+    } else if (p.b_mode == B_SEGMENTS) {
+      const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
+      const int seg = n0 / p.seg_rows;
+      const int r = n0 - seg * p.seg_rows;
+      const CUtensorMap* m = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
+      tma_load_2d_pair(b, m, fb, kc, r, pol_b);
+    } else {
+      tma_load_2d_pair(b, &mB0, fb, kc, n_blk * BN + static_cast<int>(rank) * (BN / 2), pol_b);
+    }
+  };
+  // Weights are never written by the kernels on the stream: the first item's first stages
+  // of B are requested before waiting for the previous kernel (their stages are fresh, so
+  // no empty-barrier wait is needed); only A waits.
+  int npre = 0;
+  if (warp == 0 && lane == 0 && p.b_const && cid < items) {
+    const int n_blk = (cid / num_m) / splits, sp = (cid / num_m) % splits;
+    const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+    npre = kb1 - kb0 < S ? kb1 - kb0 : S;
+    for (int q = 0; q < npre; ++q) {
+      if (leader) {
+        mbar_arrive_expect_tx(&full[q], 2 * Cfg::STAGE_BYTES);
+        armed |= 1u << q;
+      }
+      load_b(q, n_blk, (kb0 + q) * Cfg::BK, mapa_shared(smem_u32(&full[q]), 0));
+    }
+  }
+  griddep_wait_and_release();  // activations and outputs belong to earlier kernels
+
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
-      const uint64_t pol_a = l2_policy_evict_last();
-      const uint64_t pol_b = l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed = 0;
+      int cnt = 0;  // k-blocks issued
       bool ok = true;
       for (int it = cid; it < items && ok; it += ncl) {
         const int m_blk = it % num_m;
         const int ns = it / num_m;
         const int n_blk = ns / splits, sp = ns % splits;
         const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+        for (int kb = kb0; kb < kb1; ++kb, ++cnt) {
+          const bool pre = cnt < npre;  // B already requested, stage armed
+          if (!pre && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          if (leader) {
+          if (leader && !pre) {
             mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
             armed |= 1u << stage;
           }
@@ -919,21 +941,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           const int kc = kb * Cfg::BK;
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
-          uint8_t* b = sB + stage * Cfg::B_BYTES;
-          if constexpr (EPI == EPI_MIXER) {  // the tile's first weight row comes from the table
-            tma_load_2d_pair(b, &mB0, fb, kc, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2),
-                             pol_b);
-          } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
-            tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
-          } else if (p.b_mode == B_SEGMENTS) {
-            const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
-            const int seg = n0 / p.seg_rows;
-            const int r = n0 - seg * p.seg_rows;
-            const CUtensorMap* m = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
-            tma_load_2d_pair(b, m, fb, kc, r, pol_b);
-          } else {
-            tma_load_2d_pair(b, &mB0, fb, kc, n_blk * BN + static_cast<int>(rank) * (BN / 2), pol_b);
-          }
+          if (!pre) load_b(stage, n_blk, kc, fb);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -1023,8 +1031,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
     (void)grp;
     int turn = 0;                           // the next staging buffer (conv rows / reductions)
     (void)turn;
-    const bool issuer = warp == 2 && lane == 0;  // issues the TMA reductions
-    (void)issuer;
+
     const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                      mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
@@ -1041,8 +1048,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         // the epilogue warps meet at named barriers inside the epilogue, so they leave
         // together: a barrier-reduction vote over all of them
         if (!mix_all(got)) break;
-      } else if (EPI == EPI_ADD_F32 && p.d_tma) {
-        if (!red_all(got)) break;  // the reduction epilogue has named barriers too
       } else if (!got) {
         break;
       }
@@ -1054,7 +1059,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       else if (EPI == EPI_ADD_F32 && p.d_tma)
         epilogue_add_tma(&mD, tmem_base + static_cast<uint32_t>(acc * BN),
                          m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk * BN, q, lane,
-                         red_stage, turn, issuer);
+                         red_stage + q * 2 * RED_BUF_BYTES, turn);
       else
         epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
                                   m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
@@ -1066,7 +1071,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       if (acc == 0) acc_phase ^= 1u;
     }
     // the reductions have read their buffers and written D before the CTA exits
-    if (EPI == EPI_ADD_F32 && p.d_tma && issuer) bulk_wait_all();
+    if (EPI == EPI_ADD_F32 && p.d_tma && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -1112,17 +1117,33 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t ro
 }
 
 // fp32 row-major [rows, inner] (row stride ld elements) as a reduction target: box
-// [128 rows, 32 columns] = 128 bytes per row, 128-byte swizzle.
+// [32 rows, 32 columns] = 128 bytes per row, 128-byte swizzle.
 static bool make_map_f32_red(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
-  cuuint32_t box[2] = {32, 128};
+  cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_map_2d_16bit(void* map, const void* base, bool fp16, int64_t inner, int64_t rows,
+                       int64_t ld, int box_inner, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(static_cast<CUtensorMap*>(map),
+                   fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -1248,6 +1269,7 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   p.ldd1 = a.ldd1;
   p.n_split = a.n_split;
   p.err = a.err;
+  p.b_const = a.b_const ? 1 : 0;
   // residual adds by TMA reduction when D is a plain fp32 matrix the tensor map can describe
   CUtensorMap mD = mA;
   p.d_tma = 0;
@@ -1301,6 +1323,7 @@ static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64
   p.n_split = 0;
   p.splits = 1;
   p.err = mp.err;
+  p.b_const = 1;  // the heads matrix and the tile table are fixed
   const int num_m = (M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
   const int max_cl = num_sms() / 2;
   const int items = num_m * num_tiles;

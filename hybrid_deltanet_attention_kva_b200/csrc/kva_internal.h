@@ -62,6 +62,8 @@ struct GemmArgs {
   int dtype = KVA_BF16;     // 16-bit format of A, B and 16-bit outputs: KVA_BF16 or KVA_F16
   int splits = 0;           // ADD_F32 only: K ranges per tile (0: choose)
   int* err = nullptr;       // device status word
+  bool b_const = false;     // B is never written by kernels on the stream (weights): the
+                            // first stages' B tiles may be loaded before the previous kernel ends
 };
 
 int num_sms();
@@ -76,8 +78,13 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s);
 int launch_rmsnorm(const void* x, int x_dtype, int64_t ldx, const float* g, void* out,
                    int64_t ldo, int rows, int n, float eps, cudaStream_t s,
                    int out_dtype = KVA_BF16, float* zero = nullptr, int64_t ldz = 0, int nz = 0);
+// err (optional): device status word for a wait that timed out
 int launch_attention(const void* qkv, int64_t ldq, void* out, int64_t ldo, int T, int n_heads,
-                     int window, cudaStream_t s, int dtype = KVA_BF16);
+                     int window, cudaStream_t s, int dtype = KVA_BF16, int* err = nullptr);
+// 16-bit row-major [rows, inner] (row stride ld elements) for TMA, box [box_rows, box_inner],
+// 128-byte swizzle (box_inner x 2 bytes must be 128)
+bool make_map_2d_16bit(void* map, const void* base, bool fp16, int64_t inner, int64_t rows,
+                       int64_t ld, int box_inner, int box_rows);
 
 struct GdnLaunch {
   int mix_dtype = KVA_BF16;     // format of the mixer inputs and of the conv tail

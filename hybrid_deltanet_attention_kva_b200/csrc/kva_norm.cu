@@ -1,8 +1,8 @@
 // RMSNorm rows -> bf16 or fp16 ("Qwen3.8-27B-KVA" model card, architecture:
 // RMSNorm before the input Linear, before each attention and FFN sub-block, and
 // once before all heads).  out = x / sqrt(mean(x^2) + eps) * g, stats in fp32.
-// HBM-bound: one read of x (fp32 or bf16), one bf16 write; the second pass over
-// the row hits L1.
+// Bandwidth-bound: one read of x (fp32 or 16-bit), one 16-bit write; the second
+// pass over the row hits L1.
 #include "kva_common.cuh"
 
 namespace kva {
@@ -26,6 +26,8 @@ __device__ __forceinline__ float4 load4<__half>(const __half* p) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// One block of 256 threads per row (many rows' loads in flight across the GPU), the
+// sum of squares reduced through shared memory, the second pass over the row from L1.
 template <typename T, typename TO>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, int64_t ldx,
                                                       const float* __restrict__ g,

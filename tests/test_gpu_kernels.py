@@ -147,6 +147,31 @@ def test_attention(K, T, heads, window, dt):
     assert_rms_close(out, want, what="attention", elem=BF16_ELEM, scale=scale)
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_attention_rising_scores(K, dt):
+    # scores grow along the keys (a shared direction u in q and, with a ramp, in k), so the
+    # running row max moves by far more than 2^8 from one 128-key tile to the next and the
+    # accumulated output is rescaled on most tiles
+    T, heads = 700, 2
+    d = heads * 128
+    g = _gen(9701)
+    u = torch.randn(128, generator=g, dtype=torch.float64)
+    u = u / u.norm()
+    q = torch.randn(T, heads, 128, generator=g, dtype=torch.float64) + 4.0 * u
+    k = torch.randn(T, heads, 128, generator=g, dtype=torch.float64) + \
+        (torch.arange(T, dtype=torch.float64) / 8.0)[:, None, None] * u
+    v = torch.randn(T, heads, 128, generator=g, dtype=torch.float64)
+    qkv = torch.cat([q.reshape(T, d), k.reshape(T, d), v.reshape(T, d)], 1).to(dt)
+    out = torch.full((T, d), float("nan"), dtype=dt, device="cuda")
+    K.kva_op_attention(qkv.cuda(), out, heads, 0)
+    torch.cuda.synchronize()
+    x = f64(qkv)
+    Q, Kk, V = (x[:, i * d:(i + 1) * d].reshape(T, heads, 128) for i in range(3))
+    want = R.block_causal_attention(Q, Kk, V, 0).reshape(T, d)
+    scale = R.block_causal_attention(Q, Kk, np.abs(V), 0).reshape(T, d)
+    assert_rms_close(out, want, what="attention, rising scores", elem=BF16_ELEM, scale=scale)
+
+
 # ------------------------------------------------------------------ scan
 def _scan_inputs(seed, n_layers, T, n_k, n_v, d, g_scale=1.0, beta=None, gzero=False):
     g = _gen(seed)
