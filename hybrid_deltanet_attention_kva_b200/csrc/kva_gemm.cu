@@ -881,10 +881,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   const uint64_t pol_a = l2_policy_evict_last();
   const uint64_t pol_b = l2_policy_evict_normal();
   uint32_t armed = 0;
+  // B tile of N block n_blk (for EPI_MIXER: `n_blk` is the tile's first weight row from the
+  // table, read once per item so no global load sits between the stages' TMA issues)
   auto load_b = [&](int stage, int n_blk, int kc, uint32_t fb) {
     uint8_t* b = sB + stage * Cfg::B_BYTES;
-    if constexpr (EPI == EPI_MIXER) {  // the tile's first weight row comes from the table
-      tma_load_2d_pair(b, &mB0, fb, kc, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2), pol_b);
+    if constexpr (EPI == EPI_MIXER) {
+      tma_load_2d_pair(b, &mB0, fb, kc, n_blk + static_cast<int>(rank) * (BN / 2), pol_b);
     } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
       tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
     } else if (p.b_mode == B_SEGMENTS) {
@@ -910,7 +912,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         mbar_arrive_expect_tx(&full[q], 2 * Cfg::STAGE_BYTES);
         armed |= 1u << q;
       }
-      load_b(q, n_blk, (kb0 + q) * Cfg::BK, mapa_shared(smem_u32(&full[q]), 0));
+      load_b(q, EPI == EPI_MIXER ? mp.tiles[n_blk].col0 : n_blk, (kb0 + q) * Cfg::BK,
+             mapa_shared(smem_u32(&full[q]), 0));
     }
   }
   griddep_wait_and_release();  // activations and outputs belong to earlier kernels
@@ -927,6 +930,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         const int ns = it / num_m;
         const int n_blk = ns / splits, sp = ns % splits;
         const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+        const int bsel = EPI == EPI_MIXER ? mp.tiles[n_blk].col0 : n_blk;
         for (int kb = kb0; kb < kb1; ++kb, ++cnt) {
           const bool pre = cnt < npre;  // B already requested, stage armed
           if (!pre && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -941,7 +945,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           const int kc = kb * Cfg::BK;
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
-          if (!pre) load_b(stage, n_blk, kc, fb);
+          if (!pre) load_b(stage, bsel, kc, fb);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
