@@ -881,39 +881,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   const uint64_t pol_a = l2_policy_evict_last();
   const uint64_t pol_b = l2_policy_evict_normal();
   uint32_t armed = 0;
-  // B tile of N block n_blk (for EPI_MIXER: `n_blk` is the tile's first weight row from the
-  // table, read once per item so no global load sits between the stages' TMA issues)
-  auto load_b = [&](int stage, int n_blk, int kc, uint32_t fb) {
-    uint8_t* b = sB + stage * Cfg::B_BYTES;
+  // This CTA's half of the B tile of an item: tensor map and first row.  For EPI_MIXER
+  // the row comes from the tile table; it is read once per item, so no global load sits
+  // between the stages' TMA issues.
+  struct BSrc {
+    const CUtensorMap* m;
+    int row;
+  };
+  auto b_src = [&](int it) -> BSrc {
+    const int n_blk = (it / num_m) / splits;
     if constexpr (EPI == EPI_MIXER) {
-      tma_load_2d_pair(b, &mB0, fb, kc, n_blk + static_cast<int>(rank) * (BN / 2), pol_b);
+      return {&mB0, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2)};
     } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
-      tma_load_2d_pair(b, rank ? &mB1 : &mB0, fb, kc, n_blk * (BN / 2), pol_b);
+      return {rank ? &mB1 : &mB0, n_blk * (BN / 2)};
     } else if (p.b_mode == B_SEGMENTS) {
       const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
       const int seg = n0 / p.seg_rows;
-      const int r = n0 - seg * p.seg_rows;
-      const CUtensorMap* m = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
-      tma_load_2d_pair(b, m, fb, kc, r, pol_b);
+      return {seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2), n0 - seg * p.seg_rows};
     } else {
-      tma_load_2d_pair(b, &mB0, fb, kc, n_blk * BN + static_cast<int>(rank) * (BN / 2), pol_b);
+      return {&mB0, n_blk * BN + static_cast<int>(rank) * (BN / 2)};
     }
+  };
+  auto k_range = [&](int it, int& kb0, int& kb1) {
+    const int sp = (it / num_m) % splits;
+    kb0 = sp * num_k / splits;
+    kb1 = (sp + 1) * num_k / splits;
   };
   // Weights are never written by the kernels on the stream: the first item's first stages
   // of B are requested before waiting for the previous kernel (their stages are fresh, so
   // no empty-barrier wait is needed); only A waits.
   int npre = 0;
   if (warp == 0 && lane == 0 && p.b_const && cid < items) {
-    const int n_blk = (cid / num_m) / splits, sp = (cid / num_m) % splits;
-    const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
+    int kb0, kb1;
+    k_range(cid, kb0, kb1);
+    const BSrc bs = b_src(cid);
     npre = kb1 - kb0 < S ? kb1 - kb0 : S;
     for (int q = 0; q < npre; ++q) {
       if (leader) {
         mbar_arrive_expect_tx(&full[q], 2 * Cfg::STAGE_BYTES);
         armed |= 1u << q;
       }
-      load_b(q, EPI == EPI_MIXER ? mp.tiles[n_blk].col0 : n_blk, (kb0 + q) * Cfg::BK,
-             mapa_shared(smem_u32(&full[q]), 0));
+      tma_load_2d_pair(sB + q * Cfg::B_BYTES, bs.m, mapa_shared(smem_u32(&full[q]), 0),
+                       (kb0 + q) * Cfg::BK, bs.row, pol_b);
     }
   }
   griddep_wait_and_release();  // activations and outputs belong to earlier kernels
@@ -925,12 +934,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       uint32_t phase = 0;
       int cnt = 0;  // k-blocks issued
       bool ok = true;
+      int kb0, kb1;
+      if (cid < items) k_range(cid, kb0, kb1);
+      BSrc bs = cid < items ? b_src(cid) : BSrc{&mB0, 0};
       for (int it = cid; it < items && ok; it += ncl) {
         const int m_blk = it % num_m;
-        const int ns = it / num_m;
-        const int n_blk = ns / splits, sp = ns % splits;
-        const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
-        const int bsel = EPI == EPI_MIXER ? mp.tiles[n_blk].col0 : n_blk;
+        const int nit = it + ncl;  // this CTA's next item
+        int nkb0 = 0, nkb1 = 0;
+        BSrc nbs = bs;
+        if (nit < items) {
+          k_range(nit, nkb0, nkb1);
+          nbs = b_src(nit);
+        }
         for (int kb = kb0; kb < kb1; ++kb, ++cnt) {
           const bool pre = cnt < npre;  // B already requested, stage armed
           if (!pre && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -945,12 +960,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           const int kc = kb * Cfg::BK;
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
-          if (!pre) load_b(stage, bsel, kc, fb);
+          if (!pre) tma_load_2d_pair(sB + stage * Cfg::B_BYTES, bs.m, fb, kc, bs.row, pol_b);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
+        kb0 = nkb0;
+        kb1 = nkb1;
+        bs = nbs;
       }
       if (!ok) {
         *abort_flag = 1;
