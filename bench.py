@@ -296,6 +296,9 @@ def run_ours(args, rank, world, local_rank):
     heads_ms = gh["ms"] / max(gh["timed"], 1)
     achieved = heads_flops / (heads_ms / 1e3) / 1e12
     peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # the step runs in a long loop under the power cap: the sustained tensor peak is the
+    # matching denominator; the burst figure (stricter) stays the headline fraction
+    t_roof_s = max(flops / (peak_s * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
     line = {
         "metric": METRIC,
         "value": world * args.steps * T_UB / (ms / 1e3),
@@ -334,6 +337,8 @@ def run_ours(args, rank, world, local_rank):
             "flops_alg": flops, "bytes_alg": bytes_, "t_roof_ms": t_roof * 1e3,
             "frac": t_roof / (ms_step / 1e3), "peaks": f"{src}: {peaks['bf16_tflops']} TFLOP/s bf16, "
                                                      f"{peaks['hbm_gbs']} GB/s",
+            "t_roof_sustained_ms": t_roof_s * 1e3, "frac_of_sustained": t_roof_s / (ms_step / 1e3),
+            "sustained_peak": f"{src}: {peak_s} TFLOP/s bf16 sustained",
         },
         "stages_ms_per_step": {k: v["ms"] / n_prof for k, v in prof.items()},
         "gpu_launches": launches,
