@@ -38,6 +38,13 @@ Readings where the pages are silent (each also stated where it is used):
       pair (i, i + rope_dims/2) rotated by (pos + t) * theta^(-2i/rope_dims).
   R10 attention-layer V is stored as predicted (no norm, no rotation).
   R11 the scan covers every token of the ubatch.
+  R15 quantized KV cache ([KVA] "Other notes": q8_0 caches, with the same Hadamard
+      rotation applied to the approximated K/V as the exact path applies): every
+      d_h-dim K row (after k RMSNorm + RoPE) and V row is multiplied by the
+      orthonormal Walsh-Hadamard matrix H_{d_h} / sqrt(d_h) (Sylvester order:
+      H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]), then stored as q8_0 blocks of 32
+      consecutive values: scale d = max|x| / 127 kept in fp16, codes round(x / d)
+      (half away from zero) as int8; a value reads back as fp16(d) * code.
 """
 from __future__ import annotations
 
@@ -294,6 +301,46 @@ def attn_kv(Yl: np.ndarray, k_gain: np.ndarray, pos0: int, geom):
     return k, v
 
 
+def hadamard_rotate(x: np.ndarray) -> np.ndarray:
+    """x [..., n] times the orthonormal Walsh-Hadamard matrix H_n / sqrt(n), n a power
+    of two, Sylvester order (R15).  Written as the recursion that defines H_n: the
+    transform of the two halves, then their sum and difference."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    assert n >= 1 and n & (n - 1) == 0
+
+    def h(v):
+        m = v.shape[-1]
+        if m == 1:
+            return v
+        a, b = h(v[..., :m // 2]), h(v[..., m // 2:])
+        return np.concatenate([a + b, a - b], axis=-1)
+
+    return h(x) / math.sqrt(n)
+
+
+def q8_0_quantize(x: np.ndarray):
+    """q8_0 blocks of the last axis (a multiple of 32), decided in float32 (R15).
+
+    Returns (d float16 [..., n/32], codes int8 [..., n]).  The rounding decision is
+    taken in float32 on float32 inputs, the precision the cache writer computes in."""
+    x = np.asarray(x, dtype=np.float32)
+    blk = x.reshape(*x.shape[:-1], x.shape[-1] // 32, 32)
+    amax = np.max(np.abs(blk), axis=-1)
+    d = (amax / np.float32(127.0)).astype(np.float32)
+    inv = np.where(d > 0, np.float32(1.0) / np.where(d > 0, d, np.float32(1.0)), np.float32(0.0))
+    y = (blk * inv[..., None]).astype(np.float32)
+    codes = np.sign(y) * np.floor(np.abs(y) + np.float32(0.5))  # half away from zero
+    return d.astype(np.float16), codes.astype(np.int8).reshape(x.shape)
+
+
+def q8_0_dequantize(d: np.ndarray, codes: np.ndarray) -> np.ndarray:
+    """fp16(d) * code per block of 32, in float64 (R15)."""
+    c = np.asarray(codes, dtype=np.float64)
+    blk = c.reshape(*c.shape[:-1], c.shape[-1] // 32, 32)
+    return (blk * np.asarray(d, dtype=np.float64)[..., None]).reshape(c.shape)
+
+
 def kv_slots(pos0: int, T: int, page_table: Optional[np.ndarray] = None,
              page_size: int = 0) -> np.ndarray:
     """Cache row of each token: pos itself (contiguous) or page*page_size + offset."""
@@ -310,13 +357,16 @@ def update_states(Y: np.ndarray, geom, params: Dict[str, np.ndarray],
                   state: np.ndarray, tail: np.ndarray, kcache: List[np.ndarray],
                   vcache: List[np.ndarray], pos0: int,
                   page_table: Optional[np.ndarray] = None, page_size: int = 0,
-                  scan: str = "sequential", debug: Optional[Dict] = None):
+                  scan: str = "sequential", debug: Optional[Dict] = None,
+                  kv_rotate: bool = False):
     """Cheap state updates for one ubatch of one sequence ([KVA] 'Afterwards ...').
 
     Y [T, >= n_mix] mixer inputs.  state [n_gdn, n_v, d_v, d_k], tail
     [n_gdn, K-1, C] are returned updated (new arrays).  Caches are written in
     place: contiguous kcache[l] [n_kv, max_pos, d_h]; paged kcache[l]
     [n_pages, n_kv, page_size, d_h] addressed through page_table[pages].
+    kv_rotate: the caches hold the Hadamard-rotated rows of a q8_0 cache (R15),
+    before quantization (q8_0_quantize gives the stored form).
     """
     T = Y.shape[0]
     offs = geom.layer_offsets
@@ -335,6 +385,8 @@ def update_states(Y: np.ndarray, geom, params: Dict[str, np.ndarray],
     for ai, li in enumerate(geom.attn_layers()):
         Yl = Y[:, offs[li]:offs[li] + geom.attn_width]
         K, V = attn_kv(Yl, params["k_norm_g"][ai], pos0, geom)
+        if kv_rotate:
+            K, V = hadamard_rotate(K), hadamard_rotate(V)
         if page_table is None:
             kcache[ai][:, slots, :] = K.transpose(1, 0, 2)
             vcache[ai][:, slots, :] = V.transpose(1, 0, 2)
@@ -349,14 +401,14 @@ def update_states(Y: np.ndarray, geom, params: Dict[str, np.ndarray],
 
 def prefill_ubatch(residual: np.ndarray, W: Dict, geom, params: Dict, state, tail,
                    kcache, vcache, pos0: int, scan: str = "sequential",
-                   debug: Optional[Dict] = None):
+                   debug: Optional[Dict] = None, kv_rotate: bool = False):
     """Projector + state updates for one ubatch ([KVA] 'What the hell?').
 
     Returns (Y [T, n_total] mixer + drafter outputs, new state, new tail).
     """
     Y = projector(residual, W, geom)
     state, tail = update_states(Y, geom, params, state, tail, kcache, vcache, pos0,
-                                scan=scan, debug=debug)
+                                scan=scan, debug=debug, kv_rotate=kv_rotate)
     return Y, state, tail
 
 

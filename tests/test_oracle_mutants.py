@@ -117,7 +117,23 @@ def _chunked_no_decay_mask(S0, k, v, g, beta, chunk=64):
 
 R_orig = {name: getattr(R, name) for name in (
     "rope_apply", "rope_inv_freq", "causal_conv_silu", "delta_scan_sequential",
-    "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked")}
+    "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked", "hadamard_rotate",
+    "q8_0_quantize")}
+
+def _hadamard_unnormalised(x):
+    # the +-1 Walsh-Hadamard matrix without the 1/sqrt(n) that makes it orthonormal
+    return R_orig["hadamard_rotate"](x) * math.sqrt(np.asarray(x).shape[-1])
+
+
+def _q8_0_truncating(x):
+    # codes truncated toward zero instead of rounded
+    d, _ = R_orig["q8_0_quantize"](x)
+    x = np.asarray(x, dtype=np.float32)
+    blk = x.reshape(*x.shape[:-1], x.shape[-1] // 32, 32)
+    dd = d.astype(np.float32)[..., None]
+    c = np.trunc(np.where(dd > 0, blk / np.where(dd > 0, dd, 1), 0)).astype(np.int8)
+    return d, c.reshape(x.shape)
+
 
 MUTANTS = [
     ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
@@ -132,6 +148,9 @@ MUTANTS = [
     ("rmsnorm", _rms_eps_outside, [P.test_rmsnorm_closed_forms]),
     ("gdn_gates", _gates_exp_not_softplus, [P.test_gates_special_values]),
     ("delta_scan_chunked", _chunked_no_decay_mask, [lambda: P.test_scan_chunked_equals_sequential(150, 64)]),
+    ("hadamard_rotate", _hadamard_unnormalised,
+     [P.test_hadamard_rotation_keeps_dot_products_and_undoes_itself]),
+    ("q8_0_quantize", _q8_0_truncating, [P.test_q8_0_closed_form_block]),
 ]
 
 

@@ -372,3 +372,52 @@ def test_update_states_two_ubatches_equal_one():
     kn = R.rmsnorm(Yk.reshape(T, geom.attn_n_kv, geom.attn_d_h), P["k_norm_g"][0])
     np.testing.assert_allclose(np.linalg.norm(K, axis=-1), np.linalg.norm(kn, axis=-1), rtol=1e-12)
     np.testing.assert_array_equal(K[:, :, geom.rope_dims:], kn[:, :, geom.rope_dims:])
+
+
+# ------------------------------------------------------------------ q8_0 cache with rotation
+@pytest.mark.parametrize("n", [1, 2, 8, 128, 256])
+def test_hadamard_rotation_is_the_normalised_sylvester_matrix(n):
+    # scipy's hadamard(n) is the Sylvester-ordered matrix of +-1 entries
+    from scipy.linalg import hadamard
+    x = RNG.standard_normal((5, n))
+    np.testing.assert_allclose(R.hadamard_rotate(x), x @ hadamard(n).T / math.sqrt(n), rtol=0,
+                               atol=1e-12)
+
+
+def test_hadamard_rotation_keeps_dot_products_and_undoes_itself():
+    # attention scores are unchanged when both q and k are rotated; H / sqrt(n) is its own inverse
+    q, k = RNG.standard_normal((7, 256)), RNG.standard_normal((7, 256))
+    Hq, Hk = R.hadamard_rotate(q), R.hadamard_rotate(k)
+    np.testing.assert_allclose((Hq * Hk).sum(-1), (q * k).sum(-1), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(R.hadamard_rotate(Hq), q, rtol=0, atol=1e-12)
+
+
+def test_q8_0_closed_form_block():
+    # amax 127 -> d = 1 exactly, codes are the nearest integers (x_j = j - 16 + 1/4 -> j - 16)
+    x = np.arange(32, dtype=np.float64) - 16 + 0.25
+    x[31] = 127.0
+    want = np.concatenate([np.arange(31) - 16, [127]]).astype(np.int8)
+    d, c = R.q8_0_quantize(x[None])
+    assert d.dtype == np.float16 and float(d[0, 0]) == 1.0
+    np.testing.assert_array_equal(c[0], want)
+    # a power-of-two scale moves d only
+    d2, c2 = R.q8_0_quantize(x[None] * 2.0 ** -5)
+    assert float(d2[0, 0]) == 2.0 ** -5
+    np.testing.assert_array_equal(c2, c)
+    np.testing.assert_array_equal(R.q8_0_dequantize(d2, c2)[0], want * 2.0 ** -5)
+    # an all-zero block: zero scale, zero codes
+    dz, cz = R.q8_0_quantize(np.zeros((1, 64)))
+    assert np.all(dz == 0) and np.all(cz == 0)
+
+
+def test_q8_0_error_bound_and_full_scale_code():
+    x = RNG.standard_normal((50, 256)) * np.exp(RNG.standard_normal((50, 1)))
+    d, c = R.q8_0_quantize(x)
+    xf = x.astype(np.float32).astype(np.float64).reshape(50, 8, 32)
+    d32 = np.max(np.abs(xf), axis=-1) / 127.0
+    back = R.q8_0_dequantize(d, c).reshape(50, 8, 32)
+    # half a step of the float32 scale plus the fp16 storage of the scale for the largest code
+    bound = d32 / 2 * (1 + 1e-6) + 127 * np.abs(d32 - d.astype(np.float64))
+    assert np.all(np.abs(back - xf) <= bound[..., None])
+    # every non-zero block uses the full code range at its largest element
+    assert np.all(np.max(np.abs(c.reshape(50, 8, 32).astype(np.int32)), axis=-1) == 127)
