@@ -222,7 +222,8 @@ int check_cache(const kva_handle* h, const kva_kv_cache* kv, int n_seq, const in
 }
 
 // fz: the heads GEMM already ran the fused epilogue (conv outputs except block edges,
-// gates, KV rows); only the edge fix-up, the conv tail and the scan remain.
+// gates, KV rows); only the edge fix-up, the conv tail and the scan remain, and the KV
+// writer when the epilogue left the attention k/v raw (fz->att_raw, a q8_0 cache).
 int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq, int T,
                        const int64_t* pos, const kva_weights* w, float* state, void* conv_state,
                        const kva_kv_cache* kv, void* debug_qkv, void* debug_gb, cudaStream_t s,
@@ -271,11 +272,11 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     if ((e = staged(h, KVA_ST_GDN_SCAN, s, [&] { return launch_gdn_scan(g, s); }))) return e;
     if (d.gdn_d_k == 128) ++h->launches[KVA_ST_GDN_SCAN];  // two kernels
   }
-  if (h->n_attn && !fz) {
+  if (h->n_attn && (!fz || fz->att_raw)) {
     KvLaunch k;
-    k.mix = mix;
-    k.mix_ld = mix_ld;
-    k.mix_seq_stride = (int64_t)T * mix_ld;
+    k.mix = fz ? fz->att_raw : mix;
+    k.mix_ld = fz ? fz->ld_att_raw : mix_ld;
+    k.mix_seq_stride = (int64_t)T * k.mix_ld;
     k.n_seq = n_seq;
     k.T = T;
     k.n_attn = h->n_attn;
@@ -664,6 +665,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     mp.ld_draft = d.n_draft_cols;
     mp.mixer_out = mixer_out;
     mp.ld_mix = h->n_mix;
+    if (h->n_attn && kv->dtype == KVA_Q8_0) {  // the rotated q8_0 rows come from the KV writer
+      mp.att_raw = h->mixer;
+      mp.ld_att_raw = h->n_mix;
+    }
     mp.err = h->status;
     const int nt = h->n_tiles + (draft_out ? h->n_tiles_draft : 0);
     if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] {

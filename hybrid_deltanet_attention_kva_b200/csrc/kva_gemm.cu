@@ -652,6 +652,15 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
         gb[static_cast<int64_t>(j) * mp.T + t] = o;
       }
     }
+  } else if ((tl.kind == MIX_ATT_K || tl.kind == MIX_ATT_V) && mp.att_raw) {
+    // a q8_0 cache: the attention k / v stay raw (the KV writer rotates and quantizes them)
+#pragma unroll 1
+    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+      uint32_t pk[8];
+      float x[16];
+      load16(ch * 16, pk, x);
+      if (row_ok) mix_put16(static_cast<T*>(mp.att_raw) + t * mp.ld_att_raw + tl.col0 + ch * 16, pk, 16);
+    }
   } else if (tl.kind == MIX_ATT_K) {
     // RMSNorm over the 256 dims x gain (each group sums its 128), then RoPE on dims
     // [0, 64): pairs (d, d + 32), angle (pos + t) theta^(-2d/64) formed and range-reduced

@@ -190,6 +190,8 @@ struct MixParams {
   int64_t ld_draft = 0;
   void* mixer_out = nullptr;      // [T, n_mix] debug copy of the raw mixer, or null
   int64_t ld_mix = 0;
+  void* att_raw = nullptr;        // [T, ld_att_raw] at mixer columns: attention k/v stay raw here
+  int64_t ld_att_raw = 0;         //   (a q8_0 cache is written by the plain KV writer after)
   int* err = nullptr;
 };
 // The heads GEMM over `num_tiles` tiles of the table, A = z [M, K] (16-bit, lda), B = W_heads.

@@ -30,7 +30,7 @@ KVA_DEV_PAGE_OOB = 0x1
 KVA_DEV_WAIT_TIMEOUT = 0x2
 
 KVA_LAYER_GDN, KVA_LAYER_ATTN = 0, 1
-KVA_BF16, KVA_F32, KVA_F16 = 0, 1, 2
+KVA_BF16, KVA_F32, KVA_F16, KVA_Q8_0 = 0, 1, 2, 3
 _DT = {torch.bfloat16: KVA_BF16, torch.float32: KVA_F32, torch.float16: KVA_F16}
 KVA_KV_CONTIGUOUS, KVA_KV_PAGED = 0, 1
 EPI_STORE_BF16, EPI_STORE_F32, EPI_ADD_F32, EPI_SWIGLU_BF16 = 0, 1, 2, 3
@@ -205,14 +205,18 @@ class Weights:
 
 
 class KvCache:
-    """kva_kv_cache over lists of per-layer K and V tensors."""
+    """kva_kv_cache over lists of per-layer K and V tensors: bf16 / fp16 rows of d_h values,
+    or uint8 rows of d_h * 34 / 32 bytes for the Hadamard-rotated q8_0 format."""
 
     def __init__(self, k: Sequence[torch.Tensor], v: Sequence[torch.Tensor], *,
                  max_pos: int = 0, page_table: Optional[torch.Tensor] = None,
                  page_size: int = 0, n_pages: int = 0):
         self._keep = list(k) + list(v)
         self.c = KvaKvCache()
-        self.c.dtype = _DT[k[0].dtype] if len(k) else KVA_BF16
+        if len(k) and k[0].dtype == torch.uint8:
+            self.c.dtype = KVA_Q8_0
+        else:
+            self.c.dtype = _DT[k[0].dtype] if len(k) else KVA_BF16
         self.c.n_layers = len(k)
         for i, (kk, vv) in enumerate(zip(k, v)):
             self.c.k[i] = _ptr(kk)

@@ -62,7 +62,8 @@ typedef enum kva_status {
 #define KVA_DEV_WAIT_TIMEOUT 0x2  /* a pipeline wait inside a kernel gave up */
 
 typedef enum kva_layer_type { KVA_LAYER_GDN = 0, KVA_LAYER_ATTN = 1 } kva_layer_type;
-typedef enum kva_dtype { KVA_BF16 = 0, KVA_F32 = 1, KVA_F16 = 2 } kva_dtype;
+/* KVA_Q8_0 is a KV-cache format only: see kva_kv_cache. */
+typedef enum kva_dtype { KVA_BF16 = 0, KVA_F32 = 1, KVA_F16 = 2, KVA_Q8_0 = 3 } kva_dtype;
 typedef enum kva_kv_layout { KVA_KV_CONTIGUOUS = 0, KVA_KV_PAGED = 1 } kva_kv_layout;
 
 /* Geometry.  The r3 projector of the model card is
@@ -127,12 +128,19 @@ typedef struct kva_weights {
   const float* k_norm_g;/* [n_attn, d_h] k RMSNorm gain */
 } kva_weights;
 
-/* KV caches of the attention layers (device pointers, bf16, written in place).
- * CONTIGUOUS: k[l], v[l] are [n_seq, n_kv, max_pos, d_h]; token p of sequence s
+/* KV caches of the attention layers (device pointers, written in place).
+ * CONTIGUOUS: k[l], v[l] are [n_seq, n_kv, max_pos, row]; token p of sequence s
  *             goes to row p.
- * PAGED:      k[l], v[l] are [n_pages, n_kv, page_size, d_h]; token p of sequence s
+ * PAGED:      k[l], v[l] are [n_pages, n_kv, page_size, row]; token p of sequence s
  *             goes to page page_table[s * pages_per_seq + p / page_size], row
- *             p % page_size.  page_table is int32 on the device. */
+ *             p % page_size.  page_table is int32 on the device.
+ * A row is d_h values in bf16 or fp16 (dtype KVA_BF16 / KVA_F16), or, for KVA_Q8_0,
+ * the quantized-cache form of the model card's other notes (q8_0 caches get the same
+ * Hadamard rotation for the approximated K/V as the exact path): the row (K after k
+ * RMSNorm + RoPE, V as predicted) times the orthonormal Walsh-Hadamard matrix
+ * H_{d_h} / sqrt(d_h) in Sylvester order, stored as d_h / 32 blocks of 34 bytes, each
+ * an fp16 scale d = max|x| / 127 followed by 32 int8 codes round(x / d) (half away
+ * from zero); a value reads back as d * code.  Row size d_h * 34 / 32 bytes. */
 typedef struct kva_kv_cache {
   int32_t layout;            /* kva_kv_layout */
   int32_t n_layers;          /* must equal the number of attention layers */
@@ -143,7 +151,7 @@ typedef struct kva_kv_cache {
   int32_t n_pages;           /* PAGED: pages in each layer's pool */
   int32_t pages_per_seq;     /* PAGED: columns of page_table */
   const int32_t* page_table; /* PAGED: [n_seq, pages_per_seq] */
-  int32_t dtype;             /* element format of the caches: KVA_BF16 or KVA_F16 */
+  int32_t dtype;             /* row format of the caches: KVA_BF16, KVA_F16 or KVA_Q8_0 */
 } kva_kv_cache;
 
 typedef struct kva_handle kva_handle;

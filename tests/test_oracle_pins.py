@@ -421,3 +421,13 @@ def test_q8_0_error_bound_and_full_scale_code():
     assert np.all(np.abs(back - xf) <= bound[..., None])
     # every non-zero block uses the full code range at its largest element
     assert np.all(np.max(np.abs(c.reshape(50, 8, 32).astype(np.int32)), axis=-1) == 127)
+
+
+def test_q8_0_rounds_half_away_from_zero_exactly():
+    # d = 1: codes of values just below / at / above a half (float32 ties and near-ties)
+    below = np.nextafter(np.float32(0.5), np.float32(0))
+    x = np.zeros(32, dtype=np.float32)
+    x[:6] = [below, 0.5, 1.5, -0.5, -below, 2.5]
+    x[31] = 127.0
+    _, c = R.q8_0_quantize(x[None])
+    np.testing.assert_array_equal(c[0, :6], [0, 1, 2, -1, 0, 3])
