@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16",
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
+    ap.add_argument("--kv-cache", choices=["bf16", "q8_0"], default="bf16",
+                    help="KV cache rows: bf16, or Hadamard-rotated q8_0 blocks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "resid", "gdn", "attention"], default=None,
@@ -190,8 +192,12 @@ def run_ours(args, rank, world, local_rank):
     n_pool = 4
     res = [KI.make_residual(geom, T_UB, multi.rank_seed(seed + 100 + i, rank), device="cuda")
            for i in range(n_pool)]
-    kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h, dtype=torch.bfloat16, device=dev)
-          for _ in range(geom.n_attn)]
+    if args.kv_cache == "q8_0":  # rows of d_h / 32 blocks of 34 bytes
+        kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h * 34 // 32, dtype=torch.uint8,
+                          device=dev) for _ in range(geom.n_attn)]
+    else:
+        kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h, dtype=torch.bfloat16, device=dev)
+              for _ in range(geom.n_attn)]
     vc = [torch.zeros_like(k) for k in kc]
     kv = K.KvCache(kc, vc, max_pos=CACHE_POS)
     Wt = K.Weights(proj=W, layer=P)
@@ -318,6 +324,7 @@ def run_ours(args, rank, world, local_rank):
             "workload": f"{geom.name} projector + state updates, 1024-token ubatch, state / conv "
                         f"tail / KV cache carried, positions 0..{CACHE_POS - 1}",
             "geometry": geom.name, "tokens_per_step": T_UB, "d_model": geom.d_model,
+            "kv_cache": args.kv_cache if args.kv_cache == "bf16" else "q8_0 (Hadamard-rotated)",
             "heads": geom.n_heads, "ffn": geom.ffn, "late_layers": f"{geom.n_gdn} gdn + {geom.n_attn} attn",
             "drafter_cols": geom.n_draft_cols, "parallelism": f"independent sequence per GPU x{world}",
             "l2": "weights (2.48 GB) exceed L2 and stream from HBM every step" if geom.name == "r3"

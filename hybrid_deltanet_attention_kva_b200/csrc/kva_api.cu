@@ -285,6 +285,8 @@ int update_states_impl(kva_handle* h, const void* mix, int64_t mix_ld, int n_seq
     k.d_h = d.attn_d_h;
     k.rope_dims = d.rope_dims;
     k.rope_theta = d.rope_theta;
+    for (int i = 0; i < d.rope_dims / 2 && i < 128; ++i)
+      k.inv_freq[i] = std::pow(d.rope_theta, -2.0 * i / d.rope_dims);
     k.k_gain = w->k_norm_g;
     for (int i = 0; i < n_seq; ++i) k.pos[i] = pos[i];
     k.cache = *kv;
@@ -660,6 +662,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     mp.k_gain = w->k_norm_g;
     mp.rope_dims = d.rope_dims;
     mp.rope_theta = d.rope_theta;
+    for (int i = 0; i < 32; ++i) mp.inv_freq[i] = std::pow(d.rope_theta, -2.0 * i / 64);
     if (h->n_attn) mp.cache = *kv;
     mp.draft = draft_out;
     mp.ld_draft = d.n_draft_cols;

@@ -663,8 +663,8 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
     }
   } else if (tl.kind == MIX_ATT_K) {
     // RMSNorm over the 256 dims x gain (each group sums its 128), then RoPE on dims
-    // [0, 64): pairs (d, d + 32), angle (pos + t) theta^(-2d/64) formed and range-reduced
-    // in fp64
+    // [0, 64): pairs (d, d + 32), angle (pos + t) theta^(-2d/64) (frequencies from the
+    // host's fp64 table) formed and range-reduced in fp64
     const int cb = g * 128;
     float ss = 0.f;
 #pragma unroll 1
@@ -685,7 +685,7 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
     int ch0 = 0;
     if (g == 0) {
       const double two_pi = 6.283185307179586476925286766559;
-      const double lt = log2(mp.rope_theta);
+      const double inv_two_pi = 0.15915494309189533576888376337251;
 #pragma unroll 1
       for (int d0 = 0; d0 < 32; d0 += 16) {
         uint32_t ra[16], rb[16];
@@ -701,9 +701,8 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
         for (int i = 0; i < 16; ++i) {
           const int d = d0 + i;
           const float k0 = a[i] * sc * gain[d], k1 = b[i] * sc * gain[32 + d];
-          const double inv = exp2(-(2.0 * d / mp.rope_dims) * lt);
-          const double ang = static_cast<double>(p) * inv;
-          const double qq = rint(ang / two_pi);
+          const double ang = static_cast<double>(p) * mp.inv_freq[d];
+          const double qq = rint(ang * inv_two_pi);
           const float red = static_cast<float>(fma(-qq, two_pi, ang));
           float sn, cs;
           sincosf(red, &sn, &cs);

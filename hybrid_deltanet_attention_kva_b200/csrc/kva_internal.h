@@ -133,6 +133,7 @@ struct KvLaunch {
   int layer_col[KVA_MAX_LATE] = {0};
   int n_kv = 0, d_h = 0, rope_dims = 0;
   double rope_theta = 1e7;
+  double inv_freq[128] = {0};     // theta^(-2i / rope_dims), i < rope_dims / 2 (fp64, host)
   const float* k_gain = nullptr;  // [n_attn, d_h]
   int64_t pos[kMaxSeqPos] = {0};
   kva_kv_cache cache;
@@ -184,6 +185,7 @@ struct MixParams {
   const float* k_gain = nullptr;  // [n_attn, 256]
   int rope_dims = 64;
   double rope_theta = 1e7;
+  double inv_freq[32] = {0};      // theta^(-2i / 64), i < 32 (fp64, host)
   kva_kv_cache cache;
   // outputs kept from the plain path
   void* draft = nullptr;          // [T, n_draft_cols] or null

@@ -6,8 +6,9 @@
 //
 // One warp per (token, KV head): each lane holds d_h/32 consecutive dims as one
 // 16- (or 8-) byte vector; the RMS is a warp reduction; RoPE pairs (i, i+r/2)
-// meet through one xor shuffle; the angle (pos * theta^(-2i/r)) is formed and
-// range-reduced in fp64 before sincosf, so it stays exact at 32k+ positions.
+// meet through one xor shuffle; the angle (pos * theta^(-2i/r), the frequencies from a
+// table the host fills in fp64) is formed and range-reduced in fp64 before sincosf, so
+// it stays exact at 32k+ positions.
 // K and V rows are written with one vector store per lane (coalesced rows of
 // 512 bytes); V is copied bit for bit.  Paged caches go through the page table,
 // an out-of-range entry skips the write and sets the device status word.
@@ -86,14 +87,13 @@ __device__ __forceinline__ void kv_k_rope(const KvLaunch& p, int t, int seq, int
   for (int i = 0; i < EPL; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, k[i], off);
   if (dim0 < p.rope_dims) {
     const double two_pi = 6.283185307179586476925286766559;
-    const double lt = log2(p.rope_theta);
+    const double inv_two_pi = 0.15915494309189533576888376337251;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int d = dim0 + i;
       const int pi = d < half ? d : d - half;
-      const double inv = exp2(-(2.0 * pi / p.rope_dims) * lt);
-      const double ang = static_cast<double>(pos) * inv;
-      const double q = rint(ang / two_pi);
+      const double ang = static_cast<double>(pos) * p.inv_freq[pi];
+      const double q = rint(ang * inv_two_pi);
       const float red = static_cast<float>(fma(-q, two_pi, ang));
       float sn, cs;
       sincosf(red, &sn, &cs);
