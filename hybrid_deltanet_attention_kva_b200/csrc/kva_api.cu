@@ -125,20 +125,21 @@ int derive(const kva_dims* d, int* n_gdn, int* n_attn, int64_t* n_mix) {
 }
 
 // The fused heads epilogue needs 128-dim DeltaNet heads, key/value widths in whole
-// 256-column tiles, the gates in one tile, 256-dim attention heads with 64 rotary dims.
+// 256-column tiles, a layer's gates in half a tile, 256-dim attention heads with 64
+// rotary dims.
 bool fused_ok(const kva_dims* d, int ng, int na) {
   if (ng) {
     if (d->gdn_d_k != 128 || d->gdn_d_v != 128) return false;
-    if ((d->gdn_n_k * 128) % 256 || (d->gdn_n_v * 128) % 256 || 2 * d->gdn_n_v > 256) return false;
+    if ((d->gdn_n_k * 128) % 256 || (d->gdn_n_v * 128) % 256 || 2 * d->gdn_n_v > 128) return false;
   }
   if (na && (d->attn_d_h != 256 || d->rope_dims != 64)) return false;
   return d->n_draft_cols % 8 == 0;
 }
 
 int fused_tiles(const kva_dims* d, int ng, int na, int* n_draft_tiles) {
-  const int per_gdn = 2 * (d->gdn_n_k * 128 / 256) + d->gdn_n_v * 128 / 256 + 1;
+  const int per_gdn = 2 * (d->gdn_n_k * 128 / 256) + d->gdn_n_v * 128 / 256;
   *n_draft_tiles = (d->n_draft_cols + 255) / 256;
-  return ng * per_gdn + na * 2 * d->attn_n_kv + *n_draft_tiles;
+  return ng * per_gdn + (ng + 1) / 2 + na * 2 * d->attn_n_kv + *n_draft_tiles;  // gates: 2 layers a tile
 }
 
 Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
@@ -368,27 +369,34 @@ int kva_init(const kva_dims* dims, kva_handle** out) {
     std::vector<MixTile> tab;
     const int nkdk = dims->gdn_n_k * 128, nvdv = dims->gdn_n_v * 128;
     int gi = 0, ai = 0;
+    auto tile = [](int col0, int ncols, int kind, int layer, int sub) {
+      return MixTile{col0, col0 + 128, ncols, kind, layer, sub};
+    };
     for (int i = 0; i < dims->n_late; ++i) {
       if (dims->layer_type[i] == KVA_LAYER_GDN) {
         const int c = h->gdn_col[gi];
-        for (int j = 0; j < nkdk; j += 256) tab.push_back({c + j, 256, MIX_RAW, gi, j});
-        for (int j = 0; j < nkdk; j += 256) tab.push_back({c + nkdk + j, 256, MIX_GDN_K, gi, nkdk + j});
+        for (int j = 0; j < nkdk; j += 256) tab.push_back(tile(c + j, 256, MIX_RAW, gi, j));
+        for (int j = 0; j < nkdk; j += 256) tab.push_back(tile(c + nkdk + j, 256, MIX_GDN_K, gi, nkdk + j));
         for (int j = 0; j < nvdv; j += 256)
-          tab.push_back({c + 2 * nkdk + j, 256, MIX_GDN_V, gi, 2 * nkdk + j});
-        tab.push_back({c + h->C, 2 * dims->gdn_n_v, MIX_GDN_AB, gi, 0});
+          tab.push_back(tile(c + 2 * nkdk + j, 256, MIX_GDN_V, gi, 2 * nkdk + j));
+        // the gates of layers 2m and 2m + 1 share one tile, one layer per half
+        if (gi % 2 == 1)
+          tab.push_back({h->gdn_col[gi - 1] + h->C, c + h->C, 2 * dims->gdn_n_v, MIX_GDN_AB, gi - 1, gi});
+        else if (gi == h->n_gdn - 1)
+          tab.push_back({c + h->C, c + h->C, 2 * dims->gdn_n_v, MIX_GDN_AB, gi, -1});
         ++gi;
       } else {
         const int c = h->attn_col[ai];
-        for (int j = 0; j < dims->attn_n_kv; ++j) tab.push_back({c + 256 * j, 256, MIX_ATT_K, ai, j});
+        for (int j = 0; j < dims->attn_n_kv; ++j) tab.push_back(tile(c + 256 * j, 256, MIX_ATT_K, ai, j));
         for (int j = 0; j < dims->attn_n_kv; ++j)
-          tab.push_back({c + 256 * (dims->attn_n_kv + j), 256, MIX_ATT_V, ai, j});
+          tab.push_back(tile(c + 256 * (dims->attn_n_kv + j), 256, MIX_ATT_V, ai, j));
         ++ai;
       }
     }
     h->n_tiles = static_cast<int>(tab.size());
     for (int j = 0; j < dims->n_draft_cols; j += 256) {
       const int w = dims->n_draft_cols - j < 256 ? dims->n_draft_cols - j : 256;
-      tab.push_back({static_cast<int>(nm) + j, w, MIX_DRAFT, 0, j});
+      tab.push_back(tile(static_cast<int>(nm) + j, w, MIX_DRAFT, 0, j));
     }
     h->n_tiles_draft = static_cast<int>(tab.size()) - h->n_tiles;
     if (cudaMemcpy(h->tiles, tab.data(), tab.size() * sizeof(MixTile), cudaMemcpyHostToDevice) !=

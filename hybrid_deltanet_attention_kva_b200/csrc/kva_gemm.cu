@@ -627,25 +627,35 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
       mix_gdn_raw<T>(mp, false, tl.layer, t, r, tl.sub + c0, pk);
     }
   } else if (tl.kind == MIX_GDN_AB) {
-    // columns [0, n_v) are a, [n_v, 2 n_v) are b: g = -exp(A_log) softplus(a + dt_bias),
+    // the gates of two layers, one per tile half (group g: columns [128 g, 128 g + 128)
+    // from weight row g ? col1 : col0, layer g ? sub : layer; sub < 0: no second layer).
+    // Columns [0, n_v) are a, [n_v, 2 n_v) are b: g = -exp(A_log) softplus(a + dt_bias),
     // beta = sigmoid(b), written [layer][2][n_v][T]
-    float* gb = mp.gbuf + static_cast<int64_t>(tl.layer) * 2 * mp.n_v * mp.T;
+    const int lay = g ? tl.sub : tl.layer;
+    if (lay < 0) return;  // no named barrier in this branch
+    const int colbase = g ? tl.col1 : tl.col0;
+    float* gb = mp.gbuf + static_cast<int64_t>(lay) * 2 * mp.n_v * mp.T;
 #pragma unroll 1
-    for (int ch = g; ch < n16; ch += MIX_GROUPS) {
+    for (int ch = 0; ch < n16; ++ch) {
       const int c0 = ch * 16;
+      uint32_t rr[16];
+      tmem_ld_32x32b_x16(taddr + 128 * g + c0, rr);
+      tmem_ld_wait();
       uint32_t pk[8];
       float x[16];
-      load16(c0, pk, x);
+      mix_round16<T>(rr, pk, x);
       if (!row_ok) continue;
+      if (mp.mixer_out)
+        mix_put16(static_cast<T*>(mp.mixer_out) + t * mp.ld_mix + colbase + c0, pk, min(16, tl.ncols - c0));
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int j = c0 + i;
         if (j >= tl.ncols) continue;
         float o;
         if (j < mp.n_v) {
-          const float xa = x[i] + mp.dt_bias[tl.layer * mp.n_v + j];
+          const float xa = x[i] + mp.dt_bias[lay * mp.n_v + j];
           const float sp = xa > 20.f ? xa : log1pf(expf(xa));
-          o = -expf(mp.A_log[tl.layer * mp.n_v + j]) * sp;
+          o = -expf(mp.A_log[lay * mp.n_v + j]) * sp;
         } else {
           o = 1.f / (1.f + expf(-x[i]));
         }
@@ -898,8 +908,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   };
   auto b_src = [&](int it) -> BSrc {
     const int n_blk = (it / num_m) / splits;
-    if constexpr (EPI == EPI_MIXER) {
-      return {&mB0, mp.tiles[n_blk].col0 + static_cast<int>(rank) * (BN / 2)};
+    if constexpr (EPI == EPI_MIXER) {  // the table gives each half's first weight row
+      return {&mB0, rank ? mp.tiles[n_blk].col1 : mp.tiles[n_blk].col0};
     } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
       return {rank ? &mB1 : &mB0, n_blk * (BN / 2)};
     } else if (p.b_mode == B_SEGMENTS) {

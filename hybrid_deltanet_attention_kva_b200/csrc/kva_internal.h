@@ -150,18 +150,20 @@ enum MixKind {
   MIX_RAW = 0,      // q columns of a gated-DeltaNet layer: only conv-tail / halo / debug copies
   MIX_GDN_K = 1,    // k columns: conv + SiLU + per-head L2 norm -> kbuf
   MIX_GDN_V = 2,    // v columns: conv + SiLU -> vbuf
-  MIX_GDN_AB = 3,   // a | b columns: gates g, beta -> gbuf
+  MIX_GDN_AB = 3,   // a | b columns of two layers (one per tile half): gates g, beta -> gbuf
   MIX_ATT_K = 4,    // one attention key head: RMSNorm x gain, RoPE -> K cache
   MIX_ATT_V = 5,    // one attention value head -> V cache
   MIX_DRAFT = 6,    // drafter columns -> draft_out
 };
 struct MixTile {
-  int col0;    // first row of W_heads (column of the mixer) of the tile
-  int ncols;   // valid columns (<= 256)
+  int col0;    // first row of W_heads (column of the mixer) of the tile's columns 0-127
+  int col1;    // first row of its columns 128-255 (col0 + 128, except for gate tiles)
+  int ncols;   // valid columns (<= 256; per half for gate tiles)
   int kind;    // MixKind
   int layer;   // index among the gated-DeltaNet layers (GDN kinds) or the attention layers
   int sub;     // offset inside the segment: conv channel of column 0 (GDN kinds), value
-               // channel (GDN V), key channel (GDN K), head (ATT kinds), drafter column
+               // channel (GDN V), key channel (GDN K), head (ATT kinds), drafter column;
+               // for a gate tile the layer of its second half (-1: none)
 };
 constexpr int kMixHaloRows = 6;  // rows 0, 1, 2, 125, 126, 127 of every 128-token block
 struct MixParams {

@@ -293,9 +293,14 @@ def test_heads_fused_flag_follows_the_dims(K):
             K.kva_free(h)
 
 
-@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
-def test_prefill_fused_heads_ragged_and_carry(K, dt):
-    geom = TINY128
+# three gated-DeltaNet layers: the gates of layers 0 and 1 share a tile, layer 2's tile
+# has its second half empty
+TINY128_3 = KI.with_changes(TINY128, name="tiny128_3", layer_types=(KI.GDN, KI.ATTN, KI.GDN, KI.GDN))
+
+
+@pytest.mark.parametrize("dt,geom", [(torch.float16, TINY128), (torch.bfloat16, TINY128),
+                                     (torch.float16, TINY128_3)])
+def test_prefill_fused_heads_ragged_and_carry(K, dt, geom):
     splits = [300, 2, 130]
     r = _run_prefill(K, geom, splits, torch.float32, 3100, draft=True, n_outliers=0, dt=dt)
     Wn = R.weights_to_f64(r["W"])
