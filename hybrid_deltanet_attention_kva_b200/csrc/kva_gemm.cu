@@ -48,7 +48,7 @@ struct GemmParams {
   int64_t ldd1;
   int64_t n_split;
   int splits;  // K ranges per tile (ADD_F32 only; partial sums added atomically)
-  int d_tma;   // ADD_F32 on CTA pairs: tiles added to D by TMA reductions (tensor map mD)
+  int d_tma;   // CTA pairs: D written (ADD_F32: added) by TMA from staged chunks (tensor map mD)
   int b_const; // CTA pairs: the first stages' B tiles are loaded before griddepcontrol.wait
   int* err;
 };
@@ -809,6 +809,57 @@ __device__ __forceinline__ void epilogue_add_tma(const CUtensorMap* mD, uint32_t
   }
 }
 
+// 16-bit outputs (STORE, SWIGLU) on CTA pairs: the same per-warp staging, chunks of 64
+// output columns (32 rows x 128 bytes, 128-byte swizzle) written by TMA bulk stores.
+template <int EPI, typename T>
+__device__ __forceinline__ void epilogue_store_tma(const CUtensorMap* mD, uint32_t tmem_acc, int row0,
+                                                   int col0, int ncols_tile, int q, int lane,
+                                                   uint8_t* wstage, int& turn) {
+  const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+  for (int c = 0; c < ncols_tile; c += 64) {
+    uint32_t pk[32];
+    if constexpr (EPI == EPI_SWIGLU_BF16) {  // gate columns c.., up columns 128 + c..
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t gr[32], ur[32];
+        tmem_ld_32x32b_x32(taddr + c + 32 * h, gr);
+        tmem_ld_32x32b_x32(taddr + 128 + c + 32 * h, ur);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[16 * h + i] = F16<T>::pack(silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]),
+                                        silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]));
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + c + 32 * h, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[16 * h + i] = F16<T>::pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      }
+    }
+    uint8_t* buf = wstage + turn * RED_BUF_BYTES;
+    turn ^= 1;
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();  // the buffer is free
+    uint8_t* row = buf + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) =
+          make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();  // the block is staged
+    if (lane == 0) {
+      tma_store_2d(mD, buf, col0 + c, row0 + q * 32);
+      bulk_commit();
+    }
+  }
+}
+
 struct PairCfg {
   static constexpr int BM = 128;  // rows per CTA (256 per pair)
   static constexpr int BN = 256;  // tile columns (128 B rows held by each CTA)
@@ -1100,6 +1151,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         epilogue_add_tma(&mD, tmem_base + static_cast<uint32_t>(acc * BN),
                          m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk * BN, q, lane,
                          red_stage + q * 2 * RED_BUF_BYTES, turn);
+      else if ((EPI == EPI_STORE_BF16 || EPI == EPI_SWIGLU_BF16) && p.d_tma)
+        epilogue_store_tma<EPI, T>(&mD, tmem_base + static_cast<uint32_t>(acc * BN),
+                                   m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM,
+                                   n_blk * n_per_tile, n_per_tile, q, lane,
+                                   red_stage + q * 2 * RED_BUF_BYTES, turn);
       else
         epilogue_tile<BN, EPI, T>(p, tmem_base + static_cast<uint32_t>(acc * BN),
                                   m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, n_blk, q,
@@ -1111,7 +1167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       if (acc == 0) acc_phase ^= 1u;
     }
     // the reductions have read their buffers and written D before the CTA exits
-    if (EPI == EPI_ADD_F32 && p.d_tma && lane == 0) bulk_wait_all();
+    if (EPI != EPI_MIXER && p.d_tma && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -1316,6 +1372,13 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   if (EPI == EPI_ADD_F32 && a.n_split == 0 && (reinterpret_cast<uintptr_t>(a.D) & 15u) == 0 &&
       a.ldd % 4 == 0 && a.N % 4 == 0) {
     if (!make_map_f32_red(&mD, a.D, a.N, a.M, a.ldd)) return KVA_ERR_CUDA;
+    p.d_tma = 1;
+  }
+  // 16-bit outputs by TMA stores (box 32 rows x 64 columns)
+  if ((EPI == EPI_STORE_BF16 || EPI == EPI_SWIGLU_BF16) && a.n_split == 0 &&
+      (reinterpret_cast<uintptr_t>(a.D) & 15u) == 0 && a.ldd % 8 == 0 && a.N % 8 == 0) {
+    if (!make_map_2d_16bit(&mD, a.D, std::is_same<T, __half>::value, a.N, a.M, a.ldd, 64, 32))
+      return KVA_ERR_CUDA;
     p.d_tma = 1;
   }
   const int smem = p.d_tma ? Cfg::SMEM_RED : Cfg::SMEM;
