@@ -4,17 +4,21 @@
 // the q/k/v/o and SwiGLU projections of the 3 causal blocks, and the one wide
 // GEMM over all per-layer heads concatenated).
 //
-// Design (one CTA per SM, 192 threads):
-//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per stage,
-//               128-byte swizzle, into a STAGES-deep shared-memory ring.
-//   warp 1      TMEM allocator + single-thread MMA issuer: 4 x tcgen05.mma
-//               (M=128, N=BN, K=16) per stage into one of two TMEM accumulators
-//               (2 x BN fp32 columns), tcgen05.commit frees the stage.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, fused store /
-//               residual add / SwiGLU, while the MMA warp already accumulates
-//               the next tile in the other TMEM buffer.
-// Tiles are visited M-fastest so the 8 M tiles of a 1024-token ubatch that
-// share one weight tile run together and read it from HBM once.
+// Two kernels share one design.  gemm_tc_kernel: one CTA per SM, 128 x BN tiles.
+// gemm_pair_kernel (the path's default): a cluster of two CTAs on one 256 x 256
+// tile through tcgen05.mma.cta_group::2.
+//   warp 0      TMA producer: A tile [128 x 64] and this CTA's B tile per stage,
+//               128-byte swizzle, into a STAGES-deep shared-memory ring (the
+//               weights' first stages are requested before the PDL wait).
+//   warp 1      TMEM allocator + single-thread MMA issuer: 4 tcgen05.mma (K = 16)
+//               per stage into one of two TMEM accumulators, tcgen05.commit frees
+//               the stage.
+//   warps 2..   epilogue, while the MMA warp accumulates the next tile in the other
+//               TMEM buffer: 16-bit stores and residual adds through per-warp
+//               shared staging and TMA (bulk stores / reduce-adds), SwiGLU, or the
+//               heads GEMM's state-update epilogue (eight warps, see below).
+// Tiles are visited M-fastest so the M tiles of a 1024-token ubatch that share
+// one weight tile run together and read it from HBM once.
 #include <cuda.h>
 
 #include <cstdio>
