@@ -195,6 +195,19 @@ int check_weights(const kva_handle* h, const kva_weights* w, bool projector) {
       if (!a16(p)) return KVA_ERR_ALIGNMENT;
     }
   }
+  if (w->weight_format == KVA_W_Q8_0) {
+    const kva_dims& d = h->d;
+    if (d.hidden % 64 || d.d_model % 64 || d.ffn % 64) return KVA_ERR_UNSUPPORTED;
+    if (!w->W_in_scale || !w->W_heads_scale) return KVA_ERR_INVALID_ARG;
+    if (!a16(w->W_in_scale) || !a16(w->W_heads_scale)) return KVA_ERR_ALIGNMENT;
+    for (int b = 0; b < d.n_blocks; ++b)
+      for (int i = 0; i < 7; ++i) {
+        if (!w->block_scale[b][i]) return KVA_ERR_INVALID_ARG;
+        if (!a16(w->block_scale[b][i])) return KVA_ERR_ALIGNMENT;
+      }
+  } else if (w->weight_format != KVA_W_16) {
+    return KVA_ERR_INVALID_ARG;
+  }
   return KVA_OK;
 }
 
@@ -534,6 +547,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   h->last_stream = s;
 
   const int H = d.hidden, dm = d.d_model, F = d.ffn;
+  const bool q8w = w->weight_format == KVA_W_Q8_0;  // q8_0 projector weights (codes + scales)
   const int cd = d.compute_dtype;
   const float eps = d.norm_eps;
   // 1. RMSNorm(residual) (which also clears x) -> Linear{H -> d} into the fp32 residual stream x
@@ -557,6 +571,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     a.epilogue = EPI_ADD_F32;  // into a zeroed x, so the K range can be split
     a.err = h->status;
     a.dtype = cd;
+    if (q8w) {
+      a.q8 = true;
+      a.Bs[0] = w->W_in_scale;
+    }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(a, s); }))) goto done;
   }
   // 2. the causal transformer blocks (pre-norm, residual adds fused in the GEMM epilogues)
@@ -584,6 +602,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     q.epilogue = EPI_STORE_BF16;
     q.err = h->status;
     q.dtype = cd;
+    if (q8w) {
+      q.q8 = true;
+      for (int i = 0; i < 3; ++i) q.Bs[i] = w->block_scale[b][i];
+    }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(q, s); }))) goto done;
     if ((e = staged(h, KVA_ST_ATTENTION, s, [&] {
            return launch_attention(h->qkv, 3 * dm, h->o, dm, T, d.n_heads, d.attn_window, s, cd,
@@ -604,6 +626,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     o.epilogue = EPI_ADD_F32;
     o.err = h->status;
     o.dtype = cd;
+    if (q8w) {
+      o.q8 = true;
+      o.Bs[0] = w->block_scale[b][3];
+    }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(o, s); }))) goto done;
     if ((e = staged(h, KVA_ST_RMSNORM, s, [&] {
            return launch_rmsnorm(h->x, KVA_F32, dm, B.g_ffn, h->u, dm, T, dm, eps, s, cd);
@@ -625,6 +651,11 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     gu.epilogue = EPI_SWIGLU_BF16;
     gu.err = h->status;
     gu.dtype = cd;
+    if (q8w) {
+      gu.q8 = true;
+      gu.Bs[0] = w->block_scale[b][4];
+      gu.Bs[1] = w->block_scale[b][5];
+    }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(gu, s); }))) goto done;
     GemmArgs dn;
     dn.b_const = true;  // weights
@@ -640,6 +671,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     dn.epilogue = EPI_ADD_F32;
     dn.err = h->status;
     dn.dtype = cd;
+    if (q8w) {
+      dn.q8 = true;
+      dn.Bs[0] = w->block_scale[b][6];
+    }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(dn, s); }))) goto done;
   }
   // 3. RMSNorm -> all per-layer heads (+ drafter heads) in one wide GEMM
@@ -647,7 +682,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
          return launch_rmsnorm(h->x, KVA_F32, dm, w->g_out, h->u, dm, T, dm, eps, s, cd);
        })))
     goto done;
-  if (h->fused) {
+  if (h->fused && !q8w) {
     // the heads GEMM writes the state updates' inputs directly (no mixer round trip)
     MixParams mp;
     mp.tiles = h->tiles;
@@ -710,7 +745,24 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     }
     hd.err = h->status;
     hd.dtype = cd;
+    if (q8w) {  // the mixer rows; the drafter rows follow as a GEMM of their own
+      hd.q8 = true;
+      hd.Bs[0] = w->W_heads_scale;
+      hd.lds = h->n_mix + d.n_draft_cols;
+      hd.N = static_cast<int>(h->n_mix);
+      hd.D1 = nullptr;
+      hd.n_split = 0;
+    }
     if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] { return launch_gemm(hd, s); }))) goto done;
+    if (q8w && draft_out) {
+      GemmArgs dr = hd;
+      dr.B[0] = static_cast<const int8_t*>(w->W_heads) + h->n_mix * static_cast<int64_t>(dm);
+      dr.Bs[0] = static_cast<const __half*>(w->W_heads_scale) + h->n_mix;
+      dr.D = draft_out;
+      dr.ldd = d.n_draft_cols;
+      dr.N = d.n_draft_cols;
+      if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] { return launch_gemm(dr, s); }))) goto done;
+    }
     // 4. state updates on the mixer inputs
     e = update_states_impl(h, mix, h->n_mix, 1, T, &pos, w, deltanet_state, conv_state, kv,
                            nullptr, nullptr, s);
@@ -823,6 +875,36 @@ int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B,
   a.K = K;
   a.epilogue = epilogue;
   a.block_n = block_n;
+  a.err = err;
+  a.dtype = dtype;
+  if (M < 0 || N < 0 || K < 0) return KVA_ERR_INVALID_ARG;
+  return launch_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {
+  if (!Bq || !Bs) return KVA_ERR_INVALID_ARG;
+  if (b_mode < KVA_B_SINGLE || b_mode > KVA_B_PAIRED) return KVA_ERR_INVALID_ARG;
+  GemmArgs a;
+  a.A = A;
+  a.lda = lda;
+  const int nb = b_mode == KVA_B_SINGLE ? 1 : (b_mode == KVA_B_PAIRED ? 2 : 3);
+  for (int i = 0; i < nb; ++i) {
+    a.B[i] = Bq[i];
+    a.Bs[i] = Bs[i];
+  }
+  a.q8 = true;
+  a.b_mode = b_mode;
+  a.ldb = K;
+  a.seg_rows = seg_rows;
+  a.D = D;
+  a.ldd = ldd;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.epilogue = epilogue;
+  a.block_n = 512;
   a.err = err;
   a.dtype = dtype;
   if (M < 0 || N < 0 || K < 0) return KVA_ERR_INVALID_ARG;

@@ -878,26 +878,67 @@ struct PairCfg {
   // ADD_F32 by TMA reduction: each epilogue warp's two staging buffers, 1024 bytes after
   // the barriers
   static constexpr int SMEM_RED = STAGES * STAGE_BYTES + 1024 + 1024 + 4 * 2 * RED_BUF_BYTES;
-  // producer warp, MMA warp, then the epilogue warps (eight for the state-update epilogue)
+  // q8_0 weights: five stages, each with the raw codes (128 rows x 64 int8, 64-byte
+  // swizzle) and scales ([2 blocks][128 rows] fp16) of this CTA's B half
+  static constexpr int STAGES_Q8 = 5;
+  static constexpr int RAW_CODES = 128 * 64;
+  static constexpr int RAW_BYTES = RAW_CODES + 2 * 128 * 2;
+  static constexpr int SMEM_Q8 = STAGES_Q8 * (STAGE_BYTES + RAW_BYTES) + 1024 + 256;
+  // producer warp, MMA warp, the epilogue warps (eight for the state-update epilogue), then
+  // for q8_0 weights four converter warps
   static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
-  static constexpr int threads(int epi) { return 64 + 32 * epi_warps(epi); }
+  static constexpr int threads(int epi, int wq = 0) { return 64 + 32 * (epi_warps(epi) + (wq ? 4 : 0)); }
 };
 
-template <int EPI, typename T>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI), 1)
+// q8_0 weights: row r of this CTA's B half, one stage (64 k values): the codes (64-byte
+// swizzle: 16-byte piece j at j ^ ((r >> 1) & 3)) times the scale of their 32-value block,
+// rounded once to the operand format, written in the 128-byte-swizzled K-major layout the
+// MMA reads (16-byte piece c of 8 values at c ^ (r & 7)).
+template <typename T>
+__device__ __forceinline__ void q8_0_dequant_row(const uint8_t* raw, uint8_t* b_stage, int r) {
+  const uint8_t* crow = raw + r * 64;
+  const __half* sc = reinterpret_cast<const __half*>(raw + PairCfg::RAW_CODES);
+  const float s0 = __half2float(sc[r]), s1 = __half2float(sc[128 + r]);
+  uint8_t* brow = b_stage + r * 128;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {  // values 16 j .. 16 j + 15 (block j / 2)
+    const uint4 w = *reinterpret_cast<const uint4*>(crow + ((j ^ ((r >> 1) & 3)) << 4));
+    const float d = j < 2 ? s0 : s1;
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t pk[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t v = ws[q];
+      pk[2 * q] = F16<T>::pack(static_cast<float>(static_cast<int8_t>(v & 0xffu)) * d,
+                               static_cast<float>(static_cast<int8_t>((v >> 8) & 0xffu)) * d);
+      pk[2 * q + 1] = F16<T>::pack(static_cast<float>(static_cast<int8_t>((v >> 16) & 0xffu)) * d,
+                                   static_cast<float>(static_cast<int8_t>(v >> 24)) * d);
+    }
+    *reinterpret_cast<uint4*>(brow + (((2 * j) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(brow + (((2 * j + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  }
+}
+
+// WQ = 1: B is q8_0 (mB* map the int8 codes, mS* the fp16 scales); converter warps
+// dequantize each stage into the 16-bit B buffer the MMA reads.
+template <int EPI, typename T, int WQ = 0>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI, WQ), 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                      const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mB2,
-                     const __grid_constant__ CUtensorMap mD, const GemmParams p,
-                     const __grid_constant__ MixParams mp) {
+                     const __grid_constant__ CUtensorMap mS0, const __grid_constant__ CUtensorMap mS1,
+                     const __grid_constant__ CUtensorMap mS2, const __grid_constant__ CUtensorMap mD,
+                     const GemmParams p, const __grid_constant__ MixParams mp) {
   using Cfg = PairCfg;
-  constexpr int S = Cfg::STAGES;
+  constexpr int S = WQ ? Cfg::STAGES_Q8 : Cfg::STAGES;
   constexpr int BN = Cfg::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * Cfg::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::B_BYTES);
+  uint8_t* sR = sB + S * Cfg::B_BYTES;  // q8_0 raw stages (WQ)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + (WQ ? S * Cfg::RAW_BYTES : 0));
+  uint64_t* rawfull = bars + 16;        // WQ: this CTA's raw codes and scales of a stage landed
   uint64_t* full = bars;            // leader: both CTAs' bytes of a stage
   uint64_t* empty = bars + S;       // both: the pair's MMAs on a stage completed
   uint64_t* tfull = bars + 2 * S;   // both: the pair's accumulator is ready
@@ -916,8 +957,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], WQ ? 1 + 2 * 4 : 1);  // WQ: + the converter warps of both CTAs
       mbar_init(&empty[i], 1);
+      if (WQ) mbar_init(&rawfull[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -958,21 +1000,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   // the row comes from the tile table; it is read once per item, so no global load sits
   // between the stages' TMA issues.
   struct BSrc {
-    const CUtensorMap* m;
+    const CUtensorMap* m;  // the B matrix (WQ: its codes)
+    const CUtensorMap* s;  // WQ: its scales
     int row;
   };
   auto b_src = [&](int it) -> BSrc {
     const int n_blk = (it / num_m) / splits;
     if constexpr (EPI == EPI_MIXER) {  // the table gives each half's first weight row
-      return {&mB0, rank ? mp.tiles[n_blk].col1 : mp.tiles[n_blk].col0};
+      return {&mB0, &mS0, rank ? mp.tiles[n_blk].col1 : mp.tiles[n_blk].col0};
     } else if (p.b_mode == B_PAIRED) {  // gate rows in the leader, up rows in the peer
-      return {rank ? &mB1 : &mB0, n_blk * (BN / 2)};
+      return {rank ? &mB1 : &mB0, rank ? &mS1 : &mS0, n_blk * (BN / 2)};
     } else if (p.b_mode == B_SEGMENTS) {
       const int n0 = n_blk * BN + static_cast<int>(rank) * (BN / 2);
       const int seg = n0 / p.seg_rows;
-      return {seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2), n0 - seg * p.seg_rows};
+      return {seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2), seg == 0 ? &mS0 : (seg == 1 ? &mS1 : &mS2),
+              n0 - seg * p.seg_rows};
     } else {
-      return {&mB0, n_blk * BN + static_cast<int>(rank) * (BN / 2)};
+      return {&mB0, &mS0, n_blk * BN + static_cast<int>(rank) * (BN / 2)};
     }
   };
   auto k_range = [&](int it, int& kb0, int& kb1) {
@@ -984,7 +1028,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   // of B are requested before waiting for the previous kernel (their stages are fresh, so
   // no empty-barrier wait is needed); only A waits.
   int npre = 0;
-  if (warp == 0 && lane == 0 && p.b_const && cid < items) {
+  if (!WQ && warp == 0 && lane == 0 && p.b_const && cid < items) {
     int kb0, kb1;
     k_range(cid, kb0, kb1);
     const BSrc bs = b_src(cid);
@@ -1009,7 +1053,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       bool ok = true;
       int kb0, kb1;
       if (cid < items) k_range(cid, kb0, kb1);
-      BSrc bs = cid < items ? b_src(cid) : BSrc{&mB0, 0};
+      BSrc bs = cid < items ? b_src(cid) : BSrc{&mB0, &mS0, 0};
+      uint32_t rarmed = 0;  // WQ: raw stages armed
       for (int it = cid; it < items && ok; it += ncl) {
         const int m_blk = it % num_m;
         const int nit = it + ncl;  // this CTA's next item
@@ -1025,15 +1070,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
             ok = false;
             break;
           }
-          if (leader && !pre) {
-            mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+          if (leader && !pre) {  // WQ: the B bytes come from the converters' arrivals
+            mbar_arrive_expect_tx(&full[stage], 2 * (WQ ? Cfg::A_BYTES : Cfg::STAGE_BYTES));
             armed |= 1u << stage;
           }
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           const int kc = kb * Cfg::BK;
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
-          if (!pre) tma_load_2d_pair(sB + stage * Cfg::B_BYTES, bs.m, fb, kc, bs.row, pol_b);
+          if constexpr (WQ) {  // this CTA's codes (64 k x 128 rows) and scales (2 blocks x 128 rows)
+            uint8_t* raw = sR + stage * Cfg::RAW_BYTES;
+            mbar_arrive_expect_tx(&rawfull[stage], Cfg::RAW_BYTES);
+            rarmed |= 1u << stage;
+            tma_load_2d(raw, bs.m, &rawfull[stage], kc, bs.row, pol_b);
+            tma_load_2d(raw + Cfg::RAW_CODES, bs.s, &rawfull[stage], bs.row, kc / 32, pol_b);
+          } else if (!pre) {
+            tma_load_2d_pair(sB + stage * Cfg::B_BYTES, bs.m, fb, kc, bs.row, pol_b);
+          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -1065,6 +1118,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           }
         }
       }
+      if (WQ) {  // and every raw stage this CTA requested
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < S; ++i) {
+          if (st == 0) {
+            st = S - 1;
+            ph ^= 1u;
+          } else {
+            --st;
+          }
+          if (rarmed & (1u << st)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&rawfull[st], ph)) {
+              if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+            }
+          }
+        }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -1085,7 +1156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         const int sp = (it / num_m) % splits;
         const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait<WQ != 0>(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
@@ -1118,6 +1189,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       while (!mbar_try_wait(&tfull[acc], acc_phase)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) break;
       }
+    }
+  } else if (WQ && warp >= 2 + Cfg::epi_warps(EPI)) {
+    // ------------------------------------------------ q8_0 converters (both CTAs)
+    // thread r of the four warps owns row r of this CTA's B half: once a stage's raw codes
+    // and scales have landed it writes the stage's 16-bit B rows; each warp then arrives
+    // on the leader's full barrier (its stores made visible to the tensor cores first)
+    const int r = (warp - 2 - Cfg::epi_warps(EPI)) * 32 + lane;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int it = cid; it < items && ok; it += ncl) {
+      int kb0, kb1;
+      k_range(it, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&rawfull[stage], phase, abort_flag));
+        if (!ok) break;
+        q8_0_dequant_row<T>(sR + stage * Cfg::RAW_BYTES, sB + stage * Cfg::B_BYTES, r);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive(&full[stage]);
+          else mbar_arrive_remote(mapa_shared(smem_u32(&full[stage]), 0));
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
     }
   } else {
     // ------------------------------------------------ epilogue warps 2.. (both CTAs)
@@ -1245,6 +1348,31 @@ bool make_map_2d_16bit(void* map, const void* base, bool fp16, int64_t inner, in
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// q8_0 weights: codes int8 [rows, K] (box 128 rows x 64 bytes, 64-byte swizzle) and scales
+// fp16 [K / 32, rows] (box 2 blocks x 128 rows).
+static bool make_map_q8_codes(CUtensorMap* m, const void* base, int64_t K, int64_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+static bool make_map_q8_scales(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t ld) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 32)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {128, 2};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_map_3d_16bit(void* map, const void* base, bool fp16, int64_t d0, int64_t d1,
@@ -1402,10 +1530,58 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   auto kern = gemm_pair_kernel<EPI, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return KVA_ERR_CUDA;
-  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI)), smem, s, mA, mB[0], mB[1], mB[2], mD, p,
-                 MixParams()) != cudaSuccess)
+  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI)), smem, s, mA, mB[0], mB[1], mB[2], mA, mA,
+                 mA, mD, p, MixParams()) != cudaSuccess)
     return KVA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
+}
+
+// q8_0 weights on CTA pairs: B[i] are the int8 codes, Bs[i] the fp16 scales of matrix i.
+template <int EPI, typename T>
+static int launch_pair_q8(const GemmArgs& a, cudaStream_t s) {
+  using Cfg = PairCfg;
+  const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool paired = a.b_mode == B_PAIRED;
+  CUtensorMap mA, mB[3], mS[3];
+  if (!make_map(&mA, a.A, a.K, a.M, a.lda, Cfg::BM, dt)) return KVA_ERR_CUDA;
+  const int nb = a.b_mode == B_SINGLE ? 1 : (paired ? 2 : 3);
+  const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
+  for (int i = 0; i < 3; ++i) {
+    const int j = i < nb ? i : 0;
+    if (!make_map_q8_codes(&mB[i], a.B[j], a.K, b_rows) ||
+        !make_map_q8_scales(&mS[i], a.Bs[j], a.K, b_rows, a.lds > 0 ? a.lds : b_rows))
+      return KVA_ERR_CUDA;
+  }
+  GemmParams p = {};
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.b_mode = a.b_mode;
+  p.seg_rows = static_cast<int>(a.seg_rows);
+  p.D = a.D;
+  p.ldd = a.ldd;
+  p.err = a.err;
+  const int n_per_tile = paired ? Cfg::BN / 2 : Cfg::BN;
+  const int num_m = (a.M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
+  const int num_k = (a.K + Cfg::BK - 1) / Cfg::BK;
+  const int max_cl = num_sms() / 2;
+  int splits = 1;
+  if (EPI == EPI_ADD_F32) {
+    const int t = num_m * ((a.N + n_per_tile - 1) / n_per_tile);
+    splits = a.splits > 0 ? a.splits : choose_splits(t, max_cl, num_k);
+  }
+  p.splits = splits;
+  const int items = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
+  int ncl = items < max_cl ? items : max_cl;
+  if (items > ncl && num_m > 1 && ncl >= num_m && num_m <= 16) ncl -= ncl % num_m;
+  auto kern = gemm_pair_kernel<EPI, T, 1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_Q8) != cudaSuccess)
+    return KVA_ERR_CUDA;
+  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI, 1)), Cfg::SMEM_Q8, s, mA, mB[0], mB[1], mB[2],
+                 mS[0], mS[1], mS[2], mA, p, MixParams()) != cudaSuccess)
+    return KVA_ERR_CUDA;
+  return KVA_OK;
 }
 
 template <typename T>
@@ -1441,7 +1617,7 @@ static int launch_heads_fused_t(const void* A, int64_t lda, const void* W, int64
       cudaSuccess)
     return KVA_ERR_CUDA;
   if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI_MIXER)), Cfg::SMEM_MIX, s, mA, mB, mB, mB, mA,
-                 p, mp) != cudaSuccess)
+                 mA, mA, mA, p, mp) != cudaSuccess)
     return KVA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
@@ -1484,6 +1660,24 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (bn != 128 && bn != 256 && bn != 512) return KVA_ERR_UNSUPPORTED;
   if (a.dtype != KVA_BF16 && a.dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   const bool h = a.dtype == KVA_F16;
+  if (a.q8) {  // q8_0 weights: CTA pairs, plain epilogues (STORE, ADD_F32, SWIGLU)
+    if (a.K % 64 || a.n_split || bn != 512) return KVA_ERR_UNSUPPORTED;
+    const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
+    if (b_rows % 8 || a.lds % 8) return KVA_ERR_ALIGNMENT;  // scale rows of 16-byte multiples
+    for (int i = 0; i < (a.b_mode == B_SINGLE ? 1 : (a.b_mode == B_PAIRED ? 2 : 3)); ++i)
+      if (!a.Bs[i] || !aligned16(a.Bs[i]) || !a.B[i] || !aligned16(a.B[i])) return KVA_ERR_INVALID_ARG;
+    switch (a.epilogue) {
+      case EPI_STORE_BF16:
+        return h ? launch_pair_q8<EPI_STORE_BF16, __half>(a, s) : launch_pair_q8<EPI_STORE_BF16, __nv_bfloat16>(a, s);
+      case EPI_ADD_F32:
+        return h ? launch_pair_q8<EPI_ADD_F32, __half>(a, s) : launch_pair_q8<EPI_ADD_F32, __nv_bfloat16>(a, s);
+      case EPI_SWIGLU_BF16:
+        return h ? launch_pair_q8<EPI_SWIGLU_BF16, __half>(a, s)
+                 : launch_pair_q8<EPI_SWIGLU_BF16, __nv_bfloat16>(a, s);
+      default:
+        return KVA_ERR_UNSUPPORTED;
+    }
+  }
 #define KVA_GEMM_CASE(E)                                                                   \
   case E:                                                                                  \
     if (bn == 512) return h ? launch_pair<E, __half>(a, s) : launch_pair<E, __nv_bfloat16>(a, s); \

@@ -32,6 +32,18 @@ typedef enum kva_b_mode {
   KVA_B_PAIRED = 2    /* B[0] gate, B[1] up, each [N, K]; only with KVA_EPI_SWIGLU_BF16 */
 } kva_b_mode;
 
+/* The same with q8_0 weights ("Qwen3.8-27B-KVA" model card, projector quantization: q8_0
+ * projector weights at about the quality of 16-bit ones).  Each B matrix [rows, K] is given
+ * as int8 codes Bq[i] [rows, K] (row stride K) and fp16 scales Bs[i] [K / 32, rows] (the
+ * scales of one 32-wide K block for all rows contiguous); its weight (r, k) is
+ * Bs[i][k / 32][r] * Bq[i][r][k], rounded once to dtype for the tensor cores.
+ * CTA pairs only; epilogue KVA_EPI_STORE_BF16, KVA_EPI_ADD_F32 or KVA_EPI_SWIGLU_BF16; no
+ * output split.  K a multiple of 64, rows (N, or seg_rows) a multiple of 8, seg_rows a
+ * multiple of 256; pointers 16-byte aligned. */
+int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream);
+
 /* RMSNorm of `rows` rows of width n ("Qwen3.8-27B-KVA" model card, architecture):
  * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out [rows, ldo] in out_dtype (bf16 / fp16).
  * x is [rows, ldx] in x_dtype.  n, ldx, ldo multiples of 4; pointers 16-byte aligned. */

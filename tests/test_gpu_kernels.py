@@ -229,3 +229,64 @@ def test_scan_strong_decay_no_overflow(K):
     torch.cuda.synchronize()
     want = R.delta_scan_sequential(f64(S0[0]), f64(k[0]), f64(v[0]), f64(gb[0, 0].T), f64(gb[0, 1].T))
     assert_state_close(st[0], want)
+
+
+# ------------------------------------------------------------------ GEMM with q8_0 weights
+# The kernel rounds every dequantized weight once to the operand format: harmless for fp16
+# (2^-11), but bf16 keeps 8 significant bits, the same input rounding that puts the bf16 path
+# under its stated 4e-2 x RMS bar instead of 2e-2.
+Q8_TOL = {torch.float16: 2e-2, torch.bfloat16: 4e-2}
+
+
+def _q8_weights(g, rows, K, scale=0.05):
+    """Random weights as q8_0 (codes int8 [rows, K], scales fp16 [K/32, rows]) and their
+    dequantized float64 values (the oracle's quantizer and dequantizer)."""
+    W = (torch.randn(rows, K, generator=g, dtype=torch.float64) * scale).numpy()
+    d, codes = R.q8_0_quantize(W)
+    Wd = R.q8_0_dequantize(d, codes)
+    return torch.from_numpy(codes), torch.from_numpy(np.ascontiguousarray(d.T)), Wd
+
+
+@pytest.mark.parametrize("M,N,K_,epi", [(1024, 3072, 3072, 0), (600, 1040, 704, 0), (77, 256, 128, 0),
+                                        (1024, 3072, 8448, 2), (1000, 2048, 1024, 2)])
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_gemm_q8_0_weights(K, M, N, K_, epi, dt):
+    g = _gen(M * 3 + N + K_ + epi)
+    A = torch.randn(M, K_, generator=g).to(dt)
+    Bq, Bs, Wd = _q8_weights(g, N, K_)
+    want = R.projector_heads(f64(A), Wd)
+    if epi == K.EPI_STORE_BF16:
+        D = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    else:
+        D0 = torch.randn(M, N, generator=g)
+        D = D0.cuda()
+        want = want + f64(D0)
+    K.kva_op_gemm_q8_0(A.cuda(), [Bq.cuda()], [Bs.cuda()], D, N=N, epilogue=epi)
+    torch.cuda.synchronize()
+    # the GPU rounds every dequantized weight once to the operand format
+    assert_rms_close(D, want, tol=Q8_TOL[dt], what=f"q8_0 gemm epi={epi}",
+                     elem=BF16_ELEM if epi == 0 else 0.0)
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_gemm_q8_0_swiglu_and_segments(K, dt):
+    g = _gen(4242)
+    M, F, Kd = 1000, 1024, 512
+    A = torch.randn(M, Kd, generator=g).to(dt)
+    Gq, Gs, Gd = _q8_weights(g, F, Kd)
+    Uq, Us, Ud = _q8_weights(g, F, Kd)
+    D = torch.empty(M, F, dtype=dt, device="cuda")
+    K.kva_op_gemm_q8_0(A.cuda(), [Gq.cuda(), Uq.cuda()], [Gs.cuda(), Us.cuda()], D, N=F,
+                       epilogue=K.EPI_SWIGLU_BF16, b_mode=K.B_PAIRED)
+    a = f64(A)
+    gate, up = a @ Gd.T, a @ Ud.T
+    want = gate / (1.0 + np.exp(-gate)) * up
+    assert_rms_close(D, want, tol=Q8_TOL[dt], what="q8_0 swiglu", elem=BF16_ELEM)
+    # q | k | v from three q8_0 matrices of 512 rows each
+    seg = 512
+    parts = [_q8_weights(g, seg, Kd) for _ in range(3)]
+    D2 = torch.empty(M, 3 * seg, dtype=dt, device="cuda")
+    K.kva_op_gemm_q8_0(A.cuda(), [p[0].cuda() for p in parts], [p[1].cuda() for p in parts], D2,
+                       N=3 * seg, b_mode=K.B_SEGMENTS, seg_rows=seg)
+    want2 = a @ np.concatenate([p[2] for p in parts]).T
+    assert_rms_close(D2, want2, tol=Q8_TOL[dt], what="q8_0 segments", elem=BF16_ELEM)

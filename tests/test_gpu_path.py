@@ -412,3 +412,74 @@ def test_prefill_full_size_sampled(K, cfg, dt):
     for name, m in metrics.items():
         if "max_over_rms" in m:
             assert m.get("max_excess_over_rms", m["max_over_rms"]) <= tol_out, (name, m)
+
+
+# ------------------------------------------------------------------ q8_0 projector weights
+def _q8_projector(W):
+    """Every projector matrix as q8_0 (the oracle's quantizer): (GPU weight dict with int8
+    codes and fp16 scales [K/32, N], float64 dequantized weights for the oracle)."""
+    def q(t):
+        d, c = R.q8_0_quantize(f64(t))
+        return (torch.from_numpy(c).cuda(), torch.from_numpy(np.ascontiguousarray(d.T)).cuda(),
+                R.q8_0_dequantize(d, c))
+    gpu = {"g_in": W["g_in"].cuda(), "g_out": W["g_out"].cuda(), "blocks": []}
+    ref = {"g_in": f64(W["g_in"]), "g_out": f64(W["g_out"]), "blocks": []}
+    for name in ("W_in", "W_heads"):
+        c, s, deq = q(W[name])
+        gpu[name], gpu[name + "_scale"], ref[name] = c, s, deq
+    for b in W["blocks"]:
+        gb = {"g_attn": b["g_attn"].cuda(), "g_ffn": b["g_ffn"].cuda()}
+        rb = {"g_attn": f64(b["g_attn"]), "g_ffn": f64(b["g_ffn"])}
+        for name in ("Wq", "Wk", "Wv", "Wo", "Wg", "Wu", "Wd"):
+            c, s, deq = q(b[name])
+            gb[name], gb[name + "_scale"], rb[name] = c, s, deq
+        gpu["blocks"].append(gb)
+        ref["blocks"].append(rb)
+    return gpu, ref
+
+
+@pytest.mark.parametrize("geom,draft", [(KI.TINY, False), (TINY128, True)])
+def test_prefill_q8_0_projector_weights(K, geom, draft):
+    """q8_0 projector weights (TINY128 would take the fused heads epilogue with 16-bit
+    weights; q8_0 weights run the heads GEMM plain and the drafter rows as a GEMM of their
+    own)."""
+    dt = torch.float16
+    splits = [300, 2, 130]
+    W = KI.make_projector_weights(geom, 5200)
+    Wg, Wn = _q8_projector(W)
+    P = KI.make_layer_params(geom, 5201)
+    st = KI.make_states(geom, 1, 5202)
+    res = KI.make_residual(geom, sum(splits), 5203, dtype=torch.float32, n_outliers=0)
+    caches = Caches(K, geom, 1, sum(splits) + 16)
+    h = K.kva_init(K.make_dims(geom, max(splits), 1, dtype=dt))
+    S = st["state"][0].cuda()
+    tail = st["conv_tail"][0].to(dt).cuda()
+    mixers, drafts = [], []
+    try:
+        Wt = K.Weights(proj=Wg, layer={k: v.cuda() for k, v in P.items()})
+        pos = 0
+        for T in splits:
+            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda")
+            do = torch.empty(T, geom.n_draft_cols, dtype=dt, device="cuda") if draft else None
+            K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wt, S, tail, caches.c, pos, draft_out=do,
+                                 mixer_out=mo)
+            mixers.append(mo)
+            drafts.append(do)
+            pos += T
+        torch.cuda.synchronize()
+        assert K.kva_get_device_status(h) == 0
+    finally:
+        K.kva_free(h)
+    Pn = {k: f64(v) for k, v in P.items()}
+    kc, vc, _, _ = caches.oracle_views(0)
+    S_o, tail_o = f64(st["state"][0]), f64(st["conv_tail"][0].to(dt))
+    pos = 0
+    for i, T in enumerate(splits):
+        Y, S_o, tail_o = R.prefill_ubatch(f64(res[pos:pos + T]), Wn, geom, Pn, S_o, tail_o, kc, vc, pos)
+        assert_rms_close(mixers[i], Y[:, :geom.n_mix], what=f"mixer ubatch {i}")
+        if draft:
+            assert_rms_close(drafts[i], Y[:, geom.n_mix:], what=f"drafter ubatch {i}")
+        pos += T
+    assert_state_close(S, S_o)
+    assert_rms_close(tail, tail_o, what="conv tail")
+    caches.compare(v_exact=False)
