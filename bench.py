@@ -51,11 +51,13 @@ def parse():
     ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16",
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
+    ap.add_argument("--weights", choices=["f16", "q8_0"], default="f16",
+                    help="projector matrices: 16-bit, or q8_0 codes with fp16 scales per 32")
     ap.add_argument("--kv-cache", choices=["bf16", "q8_0"], default="bf16",
                     help="KV cache rows: bf16, or Hadamard-rotated q8_0 blocks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "resid", "gdn", "attention"], default=None,
+    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "heads_q8", "resid", "gdn", "attention"], default=None,
                     help="run a small case of one hot kernel three times and exit (for ncu "
                          "captures; prints no JSON line)")
     return ap.parse_args()
@@ -186,6 +188,24 @@ def run_ours(args, rank, world, local_rank):
         W = {k: (v if k.startswith("g_") or k == "blocks" else v.to(dt)) for k, v in W.items()}
         W["blocks"] = [{k: (v if k.startswith("g_") else v.to(dt)) for k, v in b.items()}
                        for b in W["blocks"]]
+    if args.weights == "q8_0":
+        # synthetic q8_0 matrices of the same shapes: random int8 codes and fp16 scales (the
+        # values are as arbitrary as the 16-bit weights'; the format is what is timed)
+        gq = torch.Generator(device="cuda")
+        gq.manual_seed(seed + 7)
+
+        def q8(t):
+            n, k = t.shape
+            codes = torch.randint(-127, 128, (n, k), generator=gq, device="cuda", dtype=torch.int8)
+            scales = (torch.rand(k // 32, n, generator=gq, device="cuda") * 2e-4 + 1e-4).half()
+            return codes, scales
+
+        for name in ("W_in", "W_heads"):
+            W[name], W[name + "_scale"] = q8(W[name])
+        for b in W["blocks"]:
+            for name in ("Wq", "Wk", "Wv", "Wo", "Wg", "Wu", "Wd"):
+                b[name], b[name + "_scale"] = q8(b[name])
+        torch.cuda.empty_cache()
     P = KI.make_layer_params(geom, seed + 1, device="cuda")
     st = KI.make_states(geom, 1, seed + 2, device="cuda")
     st["conv_tail"] = st["conv_tail"].to(dt)
@@ -318,7 +338,8 @@ def run_ours(args, rank, world, local_rank):
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
     gh = prof["gemm_heads"]
     heads_flops = 2.0 * T_UB * geom.n_total * geom.d_model
-    heads_ms = gh["ms"] / max(gh["timed"], 1)
+    # per step (one launch; with q8_0 weights the drafter rows are a second launch)
+    heads_ms = gh["ms"] / n_prof
     achieved = heads_flops / (heads_ms / 1e3) / 1e12
     peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     # the step runs in a long loop under the power cap: the sustained tensor peak is the
@@ -344,6 +365,7 @@ def run_ours(args, rank, world, local_rank):
                         f"tail / KV cache carried, positions 0..{CACHE_POS - 1}",
             "geometry": geom.name, "tokens_per_step": T_UB, "d_model": geom.d_model,
             "kv_cache": args.kv_cache if args.kv_cache == "bf16" else "q8_0 (Hadamard-rotated)",
+            "projector_weights": args.dtype if args.weights == "f16" else "q8_0 (int8 codes, fp16 scale per 32)",
             "heads": geom.n_heads, "ffn": geom.ffn, "late_layers": f"{geom.n_gdn} gdn + {geom.n_attn} attn",
             "drafter_cols": geom.n_draft_cols, "parallelism": f"independent sequence per GPU x{world}",
             "l2": "weights (2.48 GB) exceed L2 and stream from HBM every step" if geom.name == "r3"
@@ -352,12 +374,14 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {
             "bound": "tensor",
             "kernel": "gemm_heads (one wide GEMM over all per-layer and drafter heads"
-                      + (", state-update epilogue)" if fused else ")"),
+                      + (", state-update epilogue)" if fused and args.weights == "f16" else
+                         (", q8_0 weights dequantized by converter warps)" if args.weights == "q8_0"
+                          else ")")),
             "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
             "peak_kind": f"{src} bf16 sustained (kernel timed inside a long step loop)",
             "frac_of_burst": achieved / peaks["bf16_tflops"],
             "flops_per_launch": heads_flops, "avg_launch_ms": heads_ms,
-            "traffic": heads_traffic(geom.name, fused),
+            "traffic": heads_traffic(geom.name, fused) if args.weights == "f16" else None,
         },
         "path_roofline": {
             "flops_alg": flops, "bytes_alg": bytes_, "t_roof_ms": t_roof * 1e3,
@@ -446,12 +470,28 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def _time_case(case, fn, flops, reps=20):
+    """CUDA-event time of `reps` back-to-back launches (the weights, above L2 in size, stream
+    from HBM each time); prints one JSON line."""
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    print(json.dumps({"case": case, "us_per_launch": round(us, 2), "tflops": round(flops / us * 1e-6, 1)}))
+
+
 def run_kernel_case(case):
     """Small cases of the hot kernels, each above L2 in size where the kernel streams HBM:
     heads   - the heads GEMM's CTA-pair kernel on M = 1024, K = 3072, N = 49 152 (302 MB of
               weights, 1/5.8 of the r3 head matrix)
     resid   - the r3 FFN down projection with the residual-add epilogue: M = 1024, N = 3072,
               K = 8448, fp32 partial sums added into the residual stream (split K)
+    heads_q8 - the heads case with q8_0 weights (int8 codes, fp16 scales per 32; 151 MB of
+              codes), dequantized by the converter warps
     heads_fused - kva_prefill_ubatch with the first 8 r3 late layers (6 gated-DeltaNet, 2
               attention, no drafter): the heads GEMM with the state-update epilogue
     gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
@@ -466,6 +506,18 @@ def run_kernel_case(case):
         D = torch.empty(M, N, dtype=torch.half, device="cuda")
         for _ in range(3):
             K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512)
+        _time_case(case, lambda: K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512),
+                   2.0 * M * N * Kd)
+    elif case == "heads_q8":
+        M, Kd, N = 1024, 3072, 49152
+        A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+        Bq = torch.randint(-127, 128, (N, Kd), device="cuda", dtype=torch.int8)
+        Bs = (torch.rand(Kd // 32, N, device="cuda") * 2e-4 + 1e-4).half()
+        D = torch.empty(M, N, dtype=torch.half, device="cuda")
+        for _ in range(3):
+            K.kva_op_gemm_q8_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16)
+        _time_case(case, lambda: K.kva_op_gemm_q8_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16),
+                   2.0 * M * N * Kd)
     elif case == "resid":
         M, Kd, N = 1024, 8448, 3072
         A = (torch.randn(M, Kd, device="cuda") * 0.5).half()

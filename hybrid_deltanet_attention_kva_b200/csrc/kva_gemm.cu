@@ -885,34 +885,54 @@ struct PairCfg {
   static constexpr int RAW_BYTES = RAW_CODES + 2 * 128 * 2;
   static constexpr int SMEM_Q8 = STAGES_Q8 * (STAGE_BYTES + RAW_BYTES) + 1024 + 256;
   // producer warp, MMA warp, the epilogue warps (eight for the state-update epilogue), then
-  // for q8_0 weights four converter warps
+  // for q8_0 weights eight converter warps (two per 32-row quarter, one per 32-value block)
+  static constexpr int CONV_WARPS = 8;
   static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
-  static constexpr int threads(int epi, int wq = 0) { return 64 + 32 * (epi_warps(epi) + (wq ? 4 : 0)); }
+  static constexpr int threads(int epi, int wq = 0) {
+    return 64 + 32 * (epi_warps(epi) + (wq ? CONV_WARPS : 0));
+  }
 };
 
-// q8_0 weights: row r of this CTA's B half, one stage (64 k values): the codes (64-byte
-// swizzle: 16-byte piece j at j ^ ((r >> 1) & 3)) times the scale of their 32-value block,
-// rounded once to the operand format, written in the 128-byte-swizzled K-major layout the
-// MMA reads (16-byte piece c of 8 values at c ^ (r & 7)).
+// q8_0 weights: row r of this CTA's B half, values 32 h .. 32 h + 31 of one stage (one
+// 32-value block): the codes (64-byte swizzle: 16-byte piece j at j ^ ((r >> 1) & 3)) times
+// the block's scale, rounded once to the operand format, written in the 128-byte-swizzled
+// K-major layout the MMA reads (16-byte piece c of 8 values at c ^ (r & 7)).  fp16: a code
+// c sits in the mantissa of the half 1024 + 128 + c (one byte permute of c ^ 0x80 under the
+// exponent byte 0x64), so subtracting 1152 gives c exactly and one half2 multiply by the
+// scale rounds the exact product once, as an fp32 product rounded to fp16 would.
 template <typename T>
-__device__ __forceinline__ void q8_0_dequant_row(const uint8_t* raw, uint8_t* b_stage, int r) {
+__device__ __forceinline__ void q8_0_dequant_block(const uint8_t* raw, uint8_t* b_stage, int r, int h) {
   const uint8_t* crow = raw + r * 64;
-  const __half* sc = reinterpret_cast<const __half*>(raw + PairCfg::RAW_CODES);
-  const float s0 = __half2float(sc[r]), s1 = __half2float(sc[128 + r]);
+  const __half sc = reinterpret_cast<const __half*>(raw + PairCfg::RAW_CODES)[h * 128 + r];
   uint8_t* brow = b_stage + r * 128;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {  // values 16 j .. 16 j + 15 (block j / 2)
+  for (int jj = 0; jj < 2; ++jj) {  // 16 values per piece
+    const int j = 2 * h + jj;
     const uint4 w = *reinterpret_cast<const uint4*>(crow + ((j ^ ((r >> 1) & 3)) << 4));
-    const float d = j < 2 ? s0 : s1;
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     uint32_t pk[8];
+    if constexpr (std::is_same<T, __half>::value) {
+      const __half2 s2 = __half2half2(sc);
+      const __half2 bias = __float2half2_rn(1152.f);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t v = ws[q];
-      pk[2 * q] = F16<T>::pack(static_cast<float>(static_cast<int8_t>(v & 0xffu)) * d,
-                               static_cast<float>(static_cast<int8_t>((v >> 8) & 0xffu)) * d);
-      pk[2 * q + 1] = F16<T>::pack(static_cast<float>(static_cast<int8_t>((v >> 16) & 0xffu)) * d,
-                                   static_cast<float>(static_cast<int8_t>(v >> 24)) * d);
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t x = ws[q] ^ 0x80808080u;
+        const uint32_t lo = __byte_perm(x, 0x64646464u, 0x4140), hi = __byte_perm(x, 0x64646464u, 0x4342);
+        const __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&lo), bias), s2);
+        const __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&hi), bias), s2);
+        pk[2 * q] = *reinterpret_cast<const uint32_t*>(&a);
+        pk[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+    } else {
+      const float d = __half2float(sc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t v = ws[q];
+        pk[2 * q] = F16<T>::pack(static_cast<float>(static_cast<int8_t>(v & 0xffu)) * d,
+                                 static_cast<float>(static_cast<int8_t>((v >> 8) & 0xffu)) * d);
+        pk[2 * q + 1] = F16<T>::pack(static_cast<float>(static_cast<int8_t>((v >> 16) & 0xffu)) * d,
+                                     static_cast<float>(static_cast<int8_t>(v >> 24)) * d);
+      }
     }
     *reinterpret_cast<uint4*>(brow + (((2 * j) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     *reinterpret_cast<uint4*>(brow + (((2 * j + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -957,7 +977,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], WQ ? 1 + 2 * 4 : 1);  // WQ: + the converter warps of both CTAs
+      mbar_init(&full[i], WQ ? 1 + 2 * Cfg::CONV_WARPS : 1);  // WQ: + both CTAs' converter warps
       mbar_init(&empty[i], 1);
       if (WQ) mbar_init(&rawfull[i], 1);
     }
@@ -1192,10 +1212,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
     }
   } else if (WQ && warp >= 2 + Cfg::epi_warps(EPI)) {
     // ------------------------------------------------ q8_0 converters (both CTAs)
-    // thread r of the four warps owns row r of this CTA's B half: once a stage's raw codes
-    // and scales have landed it writes the stage's 16-bit B rows; each warp then arrives
-    // on the leader's full barrier (its stores made visible to the tensor cores first)
-    const int r = (warp - 2 - Cfg::epi_warps(EPI)) * 32 + lane;
+    // converter warp c owns rows 32 (c & 3) .. + 31 of this CTA's B half and the stage's
+    // 32-value block c >> 2: once a stage's raw codes and scales have landed it writes its
+    // part of the 16-bit B tile; each warp then arrives on the leader's full barrier (its
+    // stores made visible to the tensor cores first)
+    const int cw = warp - 2 - Cfg::epi_warps(EPI);
+    const int r = (cw & 3) * 32 + lane, hb = cw >> 2;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -1205,7 +1227,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       for (int kb = kb0; kb < kb1; ++kb) {
         ok = __all_sync(0xffffffffu, mbar_wait(&rawfull[stage], phase, abort_flag));
         if (!ok) break;
-        q8_0_dequant_row<T>(sR + stage * Cfg::RAW_BYTES, sB + stage * Cfg::B_BYTES, r);
+        q8_0_dequant_block<T>(sR + stage * Cfg::RAW_BYTES, sB + stage * Cfg::B_BYTES, r, hb);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -330,7 +330,9 @@ def q8_0_quantize(x: np.ndarray):
     d = (amax / np.float32(127.0)).astype(np.float32)
     inv = np.where(d > 0, np.float32(1.0) / np.where(d > 0, d, np.float32(1.0)), np.float32(0.0))
     y = (blk * inv[..., None]).astype(np.float32)
-    codes = np.sign(y) * np.floor(np.abs(y) + np.float32(0.5))  # half away from zero
+    # half away from zero, decided exactly: y - trunc(y) has no rounding error in float32
+    t = np.trunc(y)
+    codes = t + np.sign(y) * (np.abs(y - t) >= np.float32(0.5))
     return d.astype(np.float16), codes.astype(np.int8).reshape(x.shape)
 
 
