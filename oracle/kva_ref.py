@@ -45,6 +45,15 @@ Readings where the pages are silent (each also stated where it is used):
       H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]), then stored as q8_0 blocks of 32
       consecutive values: scale d = max|x| / 127 kept in fp16, codes round(x / d)
       (half away from zero) as int8; a value reads back as fp16(d) * code.
+  R16 q8_0 projector weights ([KVA] "Projector quantization"): each projector matrix
+      W [N, K] as q8_0 blocks (R15's block rule) of 32 consecutive input values of a
+      row; a weight is fp16(d) * code.
+  R17 q4_0 projector weights (the same section's q4_0 row): blocks of 32 consecutive
+      input values of a row; m = the block's value of largest magnitude (the first one
+      on a tie), d = m / -8 (so m itself is code 0), code q = min(15, floor(x / d + 8.5))
+      decided in float32 (8 when d = 0); a weight is fp16(d) * (q - 8).  Stored as the
+      fp16 scale and 16 bytes per block, byte j holding the code of value j in its low
+      nibble and that of value j + 16 in its high nibble.
 """
 from __future__ import annotations
 
@@ -341,6 +350,44 @@ def q8_0_dequantize(d: np.ndarray, codes: np.ndarray) -> np.ndarray:
     c = np.asarray(codes, dtype=np.float64)
     blk = c.reshape(*c.shape[:-1], c.shape[-1] // 32, 32)
     return (blk * np.asarray(d, dtype=np.float64)[..., None]).reshape(c.shape)
+
+
+def q4_0_quantize(x: np.ndarray):
+    """q4_0 blocks of the last axis (a multiple of 32), decided in float32 (R17).
+
+    Returns (d float16 [..., n/32], codes uint8 [..., n] in 0..15, one per value)."""
+    x = np.asarray(x, dtype=np.float32)
+    blk = x.reshape(*x.shape[:-1], x.shape[-1] // 32, 32)
+    first = np.argmax(np.abs(blk), axis=-1)[..., None]  # argmax keeps the first maximum
+    m = np.take_along_axis(blk, first, axis=-1)[..., 0]
+    d = (m / np.float32(-8.0)).astype(np.float32)
+    inv = np.where(d != 0, np.float32(1.0) / np.where(d != 0, d, np.float32(1.0)), np.float32(0.0))
+    y = (blk * inv[..., None] + np.float32(8.5)).astype(np.float32)
+    codes = np.minimum(np.floor(y), 15.0)
+    return d.astype(np.float16), codes.astype(np.uint8).reshape(x.shape)
+
+
+def q4_0_dequantize(d: np.ndarray, codes: np.ndarray) -> np.ndarray:
+    """fp16(d) * (code - 8) per block of 32, in float64 (R17); codes one per value."""
+    c = np.asarray(codes, dtype=np.float64) - 8.0
+    blk = c.reshape(*c.shape[:-1], c.shape[-1] // 32, 32)
+    return (blk * np.asarray(d, dtype=np.float64)[..., None]).reshape(c.shape)
+
+
+def q4_0_pack(codes: np.ndarray) -> np.ndarray:
+    """Codes [..., n] (0..15) -> bytes [..., n/2]: per block of 32, byte j = code j in the
+    low nibble, code j + 16 in the high nibble (R17)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    blk = c.reshape(*c.shape[:-1], c.shape[-1] // 32, 2, 16)
+    return (blk[..., 0, :] | (blk[..., 1, :] << 4)).reshape(*c.shape[:-1], c.shape[-1] // 2)
+
+
+def q4_0_unpack(packed: np.ndarray) -> np.ndarray:
+    """Bytes [..., n/2] -> codes [..., n], the inverse of q4_0_pack."""
+    b = np.asarray(packed, dtype=np.uint8)
+    blk = b.reshape(*b.shape[:-1], b.shape[-1] // 16, 16)
+    out = np.stack([blk & 0x0F, blk >> 4], axis=-2)
+    return out.reshape(*b.shape[:-1], b.shape[-1] * 2)
 
 
 def kv_slots(pos0: int, T: int, page_table: Optional[np.ndarray] = None,

@@ -135,6 +135,23 @@ def _q8_0_truncating(x):
     return d, c.reshape(x.shape)
 
 
+def _q4_0_pack_halves_swapped(codes):
+    # value j in the high nibble and value j + 16 in the low one
+    c = np.asarray(codes, dtype=np.uint8)
+    blk = c.reshape(*c.shape[:-1], c.shape[-1] // 32, 2, 16)
+    return ((blk[..., 0, :] << 4) | blk[..., 1, :]).reshape(*c.shape[:-1], c.shape[-1] // 2)
+
+
+def _q4_0_positive_scale(x):
+    # d = max|x| / 8 with the sign dropped: the codes of negative blocks flip
+    x = np.asarray(x, dtype=np.float32)
+    blk = x.reshape(*x.shape[:-1], x.shape[-1] // 32, 32)
+    d = (np.max(np.abs(blk), axis=-1) / np.float32(8.0)).astype(np.float32)
+    inv = np.where(d != 0, np.float32(1.0) / np.where(d != 0, d, np.float32(1.0)), np.float32(0.0))
+    c = np.minimum(np.floor(blk * inv[..., None] + np.float32(8.5)), 15.0)
+    return d.astype(np.float16), c.astype(np.uint8).reshape(x.shape)
+
+
 MUTANTS = [
     ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
     ("rope_apply", _rope_interleaved, [P.test_rope_equals_complex_rotation]),
@@ -151,6 +168,8 @@ MUTANTS = [
     ("hadamard_rotate", _hadamard_unnormalised,
      [P.test_hadamard_rotation_keeps_dot_products_and_undoes_itself]),
     ("q8_0_quantize", _q8_0_truncating, [P.test_q8_0_closed_form_block]),
+    ("q4_0_pack", _q4_0_pack_halves_swapped, [P.test_q4_0_closed_form_blocks]),
+    ("q4_0_quantize", _q4_0_positive_scale, [P.test_q4_0_closed_form_blocks]),
 ]
 
 

@@ -431,3 +431,61 @@ def test_q8_0_rounds_half_away_from_zero_exactly():
     x[31] = 127.0
     _, c = R.q8_0_quantize(x[None])
     np.testing.assert_array_equal(c[0, :6], [0, 1, 2, -1, 0, 3])
+
+
+# ------------------------------------------------------------------ q4_0 projector weights
+def test_q4_0_closed_form_blocks():
+    # values j - 8 then 7 - j: the first value of largest magnitude is -8, so d = -8 / -8 = 1
+    # and every value is its own code minus 8; byte j packs code j (low) and 15 - j (high)
+    x = np.concatenate([np.arange(16) - 8.0, 7.0 - np.arange(16)])
+    d, c = R.q4_0_quantize(x[None])
+    assert d.dtype == np.float16 and float(d[0, 0]) == 1.0
+    np.testing.assert_array_equal(c[0], np.concatenate([np.arange(16), 15 - np.arange(16)]))
+    packed = R.q4_0_pack(c)
+    np.testing.assert_array_equal(packed[0], 240 - 15 * np.arange(16))
+    np.testing.assert_array_equal(R.q4_0_unpack(packed), c)
+    np.testing.assert_array_equal(R.q4_0_dequantize(d, c)[0], x)
+    # times -1/4: the first largest value is now +2, so d = -1/4 and the codes stay
+    d2, c2 = R.q4_0_quantize(x[None] * -0.25)
+    assert float(d2[0, 0]) == -0.25
+    np.testing.assert_array_equal(c2, c)
+    np.testing.assert_array_equal(R.q4_0_dequantize(d2, c2)[0], x * -0.25)
+    # the opposite extreme is clamped to code 15 (7 d), halves round up (x / d + 8.5, floor)
+    y = np.zeros(32)
+    y[:7] = [-8.0, 8.0, 0.5, -0.5, 1.5, -1.5, 2.25]
+    y[7] = -2.75
+    d3, c3 = R.q4_0_quantize(y[None])
+    assert float(d3[0, 0]) == 1.0
+    np.testing.assert_array_equal(c3[0, :9], [0, 15, 9, 8, 10, 7, 10, 5, 8])
+    np.testing.assert_array_equal(R.q4_0_dequantize(d3, c3)[0, :3], [-8.0, 7.0, 1.0])
+    np.testing.assert_array_equal(R.q4_0_pack(c3)[0, :3], [0x80, 0x8F, 0x89])
+    # a tie in magnitude: the first one (+4) sets d = -1/2; the later -4 clamps to 7 d
+    z = np.zeros(32)
+    z[3], z[10], z[20] = 4.0, -4.0, 1.0
+    d4, c4 = R.q4_0_quantize(z[None])
+    assert float(d4[0, 0]) == -0.5
+    np.testing.assert_array_equal(R.q4_0_dequantize(d4, c4)[0, [3, 10, 20]], [4.0, -3.5, 1.0])
+    # an all-zero block: zero scale, code 8 (value 0)
+    dz, cz = R.q4_0_quantize(np.zeros((1, 64)))
+    assert np.all(dz == 0) and np.all(cz == 8)
+
+
+def test_q4_0_error_bound_and_range():
+    x = RNG.standard_normal((40, 256)) * np.exp(RNG.standard_normal((40, 1)))
+    d, c = R.q4_0_quantize(x)
+    assert c.dtype == np.uint8 and c.max() <= 15
+    xf = x.astype(np.float32).astype(np.float64).reshape(40, 8, 32)
+    first = np.argmax(np.abs(xf), axis=-1)[..., None]
+    m = np.take_along_axis(xf, first, axis=-1)[..., 0]
+    d32 = m / -8.0
+    back = R.q4_0_dequantize(d, c).reshape(40, 8, 32)
+    ratio = xf / d32[..., None]                      # in [-8, 8]
+    store = 8 * np.abs(d32 - d.astype(np.float64))   # the fp16 scale, at most 8 steps away
+    step = np.abs(d32)[..., None]
+    # half a step inside the code range, up to a full step where code 15 is clamped
+    bound = np.where(ratio <= 7.5, step / 2, step) * (1 + 1e-5) + store[..., None]
+    assert np.all(np.abs(back - xf) <= bound)
+    # the value that sets the scale comes back up to the scale's fp16 rounding
+    mb = np.take_along_axis(back, first, axis=-1)[..., 0]
+    assert np.all(np.abs(mb - m) <= store * (1 + 1e-9))
+    np.testing.assert_array_equal(R.q4_0_unpack(R.q4_0_pack(c)), c)
