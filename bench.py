@@ -51,15 +51,16 @@ def parse():
     ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16",
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
-    ap.add_argument("--weights", choices=["f16", "q8_0"], default="f16",
-                    help="projector matrices: 16-bit, or q8_0 codes with fp16 scales per 32")
+    ap.add_argument("--weights", choices=["f16", "q8_0", "q4_0"], default="f16",
+                    help="projector matrices: 16-bit, or q8_0 / q4_0 codes with fp16 scales per 32")
     ap.add_argument("--kv-cache", choices=["bf16", "q8_0"], default="bf16",
                     help="KV cache rows: bf16, or Hadamard-rotated q8_0 blocks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--kernel-case", choices=["heads", "heads_fused", "heads_q8", "resid", "gdn", "attention"], default=None,
+    ap.add_argument("--kernel-case", default=None,
+                    choices=["heads", "heads_fused", "heads_q8", "heads_q4", "resid", "gdn", "attention"],
                     help="run a small case of one hot kernel three times and exit (for ncu "
-                         "captures; prints no JSON line)")
+                         "captures; the GEMM cases then print their CUDA-event time)")
     return ap.parse_args()
 
 
@@ -188,15 +189,19 @@ def run_ours(args, rank, world, local_rank):
         W = {k: (v if k.startswith("g_") or k == "blocks" else v.to(dt)) for k, v in W.items()}
         W["blocks"] = [{k: (v if k.startswith("g_") else v.to(dt)) for k, v in b.items()}
                        for b in W["blocks"]]
-    if args.weights == "q8_0":
-        # synthetic q8_0 matrices of the same shapes: random int8 codes and fp16 scales (the
-        # values are as arbitrary as the 16-bit weights'; the format is what is timed)
+    if args.weights != "f16":
+        # synthetic q8_0 / q4_0 matrices of the same shapes: random codes (int8, or two 4-bit
+        # codes per byte) and fp16 scales (the values are as arbitrary as the 16-bit weights';
+        # the format is what is timed)
         gq = torch.Generator(device="cuda")
         gq.manual_seed(seed + 7)
 
         def q8(t):
             n, k = t.shape
-            codes = torch.randint(-127, 128, (n, k), generator=gq, device="cuda", dtype=torch.int8)
+            if args.weights == "q4_0":
+                codes = torch.randint(0, 256, (n, k // 2), generator=gq, device="cuda", dtype=torch.uint8)
+            else:
+                codes = torch.randint(-127, 128, (n, k), generator=gq, device="cuda", dtype=torch.int8)
             scales = (torch.rand(k // 32, n, generator=gq, device="cuda") * 2e-4 + 1e-4).half()
             return codes, scales
 
@@ -338,7 +343,7 @@ def run_ours(args, rank, world, local_rank):
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
     gh = prof["gemm_heads"]
     heads_flops = 2.0 * T_UB * geom.n_total * geom.d_model
-    # per step (one launch; with q8_0 weights the drafter rows are a second launch)
+    # per step (one launch; with quantized weights the drafter rows are a second launch)
     heads_ms = gh["ms"] / n_prof
     achieved = heads_flops / (heads_ms / 1e3) / 1e12
     peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -365,7 +370,9 @@ def run_ours(args, rank, world, local_rank):
                         f"tail / KV cache carried, positions 0..{CACHE_POS - 1}",
             "geometry": geom.name, "tokens_per_step": T_UB, "d_model": geom.d_model,
             "kv_cache": args.kv_cache if args.kv_cache == "bf16" else "q8_0 (Hadamard-rotated)",
-            "projector_weights": args.dtype if args.weights == "f16" else "q8_0 (int8 codes, fp16 scale per 32)",
+            "projector_weights": args.dtype if args.weights == "f16" else
+                                 {"q8_0": "q8_0 (int8 codes, fp16 scale per 32)",
+                                  "q4_0": "q4_0 (4-bit codes, fp16 scale per 32)"}[args.weights],
             "heads": geom.n_heads, "ffn": geom.ffn, "late_layers": f"{geom.n_gdn} gdn + {geom.n_attn} attn",
             "drafter_cols": geom.n_draft_cols, "parallelism": f"independent sequence per GPU x{world}",
             "l2": "weights (2.48 GB) exceed L2 and stream from HBM every step" if geom.name == "r3"
@@ -375,8 +382,8 @@ def run_ours(args, rank, world, local_rank):
             "bound": "tensor",
             "kernel": "gemm_heads (one wide GEMM over all per-layer and drafter heads"
                       + (", state-update epilogue)" if fused and args.weights == "f16" else
-                         (", q8_0 weights dequantized by converter warps)" if args.weights == "q8_0"
-                          else ")")),
+                         (f", {args.weights} weights dequantized by converter warps)"
+                          if args.weights != "f16" else ")")),
             "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
             "peak_kind": f"{src} bf16 sustained (kernel timed inside a long step loop)",
             "frac_of_burst": achieved / peaks["bf16_tflops"],
@@ -492,6 +499,7 @@ def run_kernel_case(case):
               K = 8448, fp32 partial sums added into the residual stream (split K)
     heads_q8 - the heads case with q8_0 weights (int8 codes, fp16 scales per 32; 151 MB of
               codes), dequantized by the converter warps
+    heads_q4 - the same with q4_0 weights (75 MB of packed 4-bit codes)
     heads_fused - kva_prefill_ubatch with the first 8 r3 late layers (6 gated-DeltaNet, 2
               attention, no drafter): the heads GEMM with the state-update epilogue
     gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
@@ -517,6 +525,16 @@ def run_kernel_case(case):
         for _ in range(3):
             K.kva_op_gemm_q8_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16)
         _time_case(case, lambda: K.kva_op_gemm_q8_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16),
+                   2.0 * M * N * Kd)
+    elif case == "heads_q4":
+        M, Kd, N = 1024, 3072, 49152
+        A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+        Bq = torch.randint(0, 256, (N, Kd // 2), device="cuda", dtype=torch.uint8)
+        Bs = (torch.rand(Kd // 32, N, device="cuda") * 2e-4 + 1e-4).half()
+        D = torch.empty(M, N, dtype=torch.half, device="cuda")
+        for _ in range(3):
+            K.kva_op_gemm_q4_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16)
+        _time_case(case, lambda: K.kva_op_gemm_q4_0(A, [Bq], [Bs], D, N=N, epilogue=K.EPI_STORE_BF16),
                    2.0 * M * N * Kd)
     elif case == "resid":
         M, Kd, N = 1024, 8448, 3072

@@ -195,7 +195,7 @@ int check_weights(const kva_handle* h, const kva_weights* w, bool projector) {
       if (!a16(p)) return KVA_ERR_ALIGNMENT;
     }
   }
-  if (w->weight_format == KVA_W_Q8_0) {
+  if (w->weight_format == KVA_W_Q8_0 || w->weight_format == KVA_W_Q4_0) {
     const kva_dims& d = h->d;
     if (d.hidden % 64 || d.d_model % 64 || d.ffn % 64) return KVA_ERR_UNSUPPORTED;
     if (!w->W_in_scale || !w->W_heads_scale) return KVA_ERR_INVALID_ARG;
@@ -547,7 +547,9 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
   h->last_stream = s;
 
   const int H = d.hidden, dm = d.d_model, F = d.ffn;
-  const bool q8w = w->weight_format == KVA_W_Q8_0;  // q8_0 projector weights (codes + scales)
+  // quantized projector weights (codes + scales): GemmArgs::wq is the weight format
+  const int wq = w->weight_format;
+  const bool qw = wq != KVA_W_16;
   const int cd = d.compute_dtype;
   const float eps = d.norm_eps;
   // 1. RMSNorm(residual) (which also clears x) -> Linear{H -> d} into the fp32 residual stream x
@@ -571,8 +573,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     a.epilogue = EPI_ADD_F32;  // into a zeroed x, so the K range can be split
     a.err = h->status;
     a.dtype = cd;
-    if (q8w) {
-      a.q8 = true;
+    if (qw) {
+      a.wq = wq;
       a.Bs[0] = w->W_in_scale;
     }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(a, s); }))) goto done;
@@ -602,8 +604,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     q.epilogue = EPI_STORE_BF16;
     q.err = h->status;
     q.dtype = cd;
-    if (q8w) {
-      q.q8 = true;
+    if (qw) {
+      q.wq = wq;
       for (int i = 0; i < 3; ++i) q.Bs[i] = w->block_scale[b][i];
     }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(q, s); }))) goto done;
@@ -626,8 +628,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     o.epilogue = EPI_ADD_F32;
     o.err = h->status;
     o.dtype = cd;
-    if (q8w) {
-      o.q8 = true;
+    if (qw) {
+      o.wq = wq;
       o.Bs[0] = w->block_scale[b][3];
     }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(o, s); }))) goto done;
@@ -651,8 +653,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     gu.epilogue = EPI_SWIGLU_BF16;
     gu.err = h->status;
     gu.dtype = cd;
-    if (q8w) {
-      gu.q8 = true;
+    if (qw) {
+      gu.wq = wq;
       gu.Bs[0] = w->block_scale[b][4];
       gu.Bs[1] = w->block_scale[b][5];
     }
@@ -671,8 +673,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     dn.epilogue = EPI_ADD_F32;
     dn.err = h->status;
     dn.dtype = cd;
-    if (q8w) {
-      dn.q8 = true;
+    if (qw) {
+      dn.wq = wq;
       dn.Bs[0] = w->block_scale[b][6];
     }
     if ((e = staged(h, KVA_ST_GEMM_TRUNK, s, [&] { return launch_gemm(dn, s); }))) goto done;
@@ -682,7 +684,7 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
          return launch_rmsnorm(h->x, KVA_F32, dm, w->g_out, h->u, dm, T, dm, eps, s, cd);
        })))
     goto done;
-  if (h->fused && !q8w) {
+  if (h->fused && !qw) {
     // the heads GEMM writes the state updates' inputs directly (no mixer round trip)
     MixParams mp;
     mp.tiles = h->tiles;
@@ -745,8 +747,8 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
     }
     hd.err = h->status;
     hd.dtype = cd;
-    if (q8w) {  // the mixer rows; the drafter rows follow as a GEMM of their own
-      hd.q8 = true;
+    if (qw) {  // the mixer rows; the drafter rows follow as a GEMM of their own
+      hd.wq = wq;
       hd.Bs[0] = w->W_heads_scale;
       hd.lds = h->n_mix + d.n_draft_cols;
       hd.N = static_cast<int>(h->n_mix);
@@ -754,9 +756,10 @@ int kva_prefill_ubatch(kva_handle* h, const void* residual, int32_t residual_dty
       hd.n_split = 0;
     }
     if ((e = staged(h, KVA_ST_GEMM_HEADS, s, [&] { return launch_gemm(hd, s); }))) goto done;
-    if (q8w && draft_out) {
+    if (qw && draft_out) {
       GemmArgs dr = hd;
-      dr.B[0] = static_cast<const int8_t*>(w->W_heads) + h->n_mix * static_cast<int64_t>(dm);
+      dr.B[0] = static_cast<const uint8_t*>(w->W_heads) +
+                h->n_mix * static_cast<int64_t>(wq == KVA_W_Q4_0 ? dm / 2 : dm);
       dr.Bs[0] = static_cast<const __half*>(w->W_heads_scale) + h->n_mix;
       dr.D = draft_out;
       dr.ldd = d.n_draft_cols;
@@ -881,9 +884,9 @@ int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B,
   return launch_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
-int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
-                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
-                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {
+static int op_gemm_quant(int wq, int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                         const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                         int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {
   if (!Bq || !Bs) return KVA_ERR_INVALID_ARG;
   if (b_mode < KVA_B_SINGLE || b_mode > KVA_B_PAIRED) return KVA_ERR_INVALID_ARG;
   GemmArgs a;
@@ -894,7 +897,7 @@ int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* cons
     a.B[i] = Bq[i];
     a.Bs[i] = Bs[i];
   }
-  a.q8 = true;
+  a.wq = wq;
   a.b_mode = b_mode;
   a.ldb = K;
   a.seg_rows = seg_rows;
@@ -909,6 +912,20 @@ int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* cons
   a.dtype = dtype;
   if (M < 0 || N < 0 || K < 0) return KVA_ERR_INVALID_ARG;
   return launch_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {
+  return op_gemm_quant(KVA_W_Q8_0, dtype, A, lda, Bq, Bs, b_mode, seg_rows, D, ldd, M, N, K, epilogue,
+                       err, stream);
+}
+
+int kva_op_gemm_q4_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {
+  return op_gemm_quant(KVA_W_Q4_0, dtype, A, lda, Bq, Bs, b_mode, seg_rows, D, ldd, M, N, K, epilogue,
+                       err, stream);
 }
 
 int kva_op_attention(int32_t dtype, const void* qkv, int64_t ldq, void* out, int64_t ldo,

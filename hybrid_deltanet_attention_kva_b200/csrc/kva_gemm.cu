@@ -884,6 +884,15 @@ struct PairCfg {
   static constexpr int RAW_CODES = 128 * 64;
   static constexpr int RAW_BYTES = RAW_CODES + 2 * 128 * 2;
   static constexpr int SMEM_Q8 = STAGES_Q8 * (STAGE_BYTES + RAW_BYTES) + 1024 + 256;
+  // q4_0 weights: six stages, each with the packed codes (128 rows x 32 bytes, 32-byte
+  // swizzle) and the same scales
+  static constexpr int STAGES_Q4 = 6;
+  static constexpr int RAW_CODES_Q4 = 128 * 32;
+  static constexpr int RAW_BYTES_Q4 = RAW_CODES_Q4 + 2 * 128 * 2;
+  static constexpr int SMEM_Q4 = STAGES_Q4 * (STAGE_BYTES + RAW_BYTES_Q4) + 1024 + 256;
+  static constexpr int stages(int wq) { return wq == 1 ? STAGES_Q8 : (wq == 2 ? STAGES_Q4 : STAGES); }
+  static constexpr int raw_bytes(int wq) { return wq == 1 ? RAW_BYTES : (wq == 2 ? RAW_BYTES_Q4 : 0); }
+  static constexpr int raw_codes(int wq) { return wq == 1 ? RAW_CODES : RAW_CODES_Q4; }
   // producer warp, MMA warp, the epilogue warps (eight for the state-update epilogue), then
   // for q8_0 weights eight converter warps (two per 32-row quarter, one per 32-value block)
   static constexpr int CONV_WARPS = 8;
@@ -939,8 +948,47 @@ __device__ __forceinline__ void q8_0_dequant_block(const uint8_t* raw, uint8_t* 
   }
 }
 
-// WQ = 1: B is q8_0 (mB* map the int8 codes, mS* the fp16 scales); converter warps
-// dequantize each stage into the 16-bit B buffer the MMA reads.
+// q4_0 weights: row r of this CTA's B half, values 32 h .. 32 h + 31 of one stage (one
+// 32-value block): 16 bytes of codes (32-byte swizzle: 16-byte piece h at h ^ ((r >> 2) & 1)),
+// byte j holding value j in its low nibble and value j + 16 in its high nibble; each value
+// is fp16(d) (code - 8), rounded once to the operand format and written as in the q8_0
+// case.  fp16: a code c under the exponent byte 0x64 is the half 1024 + c, so subtracting
+// 1032 gives c - 8 exactly.
+template <typename T>
+__device__ __forceinline__ void q4_0_dequant_block(const uint8_t* raw, uint8_t* b_stage, int r, int h) {
+  const __half sc = reinterpret_cast<const __half*>(raw + PairCfg::RAW_CODES_Q4)[h * 128 + r];
+  const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 32 + ((h ^ ((r >> 2) & 1)) << 4));
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint8_t* brow = b_stage + r * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {  // values 8 c .. 8 c + 7 of the block
+    uint32_t pk[4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t word = ws[(c & 1) * 2 + t];
+      const uint32_t nib = (c >> 1) ? (word >> 4) & 0x0F0F0F0Fu : word & 0x0F0F0F0Fu;
+      if constexpr (std::is_same<T, __half>::value) {
+        const __half2 s2 = __half2half2(sc);
+        const __half2 bias = __float2half2_rn(1032.f);
+        const uint32_t lo = __byte_perm(nib, 0x64646464u, 0x4140), hi = __byte_perm(nib, 0x64646464u, 0x4342);
+        const __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&lo), bias), s2);
+        const __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&hi), bias), s2);
+        pk[2 * t] = *reinterpret_cast<const uint32_t*>(&a);
+        pk[2 * t + 1] = *reinterpret_cast<const uint32_t*>(&b);
+      } else {
+        const float d = __half2float(sc);
+        pk[2 * t] = F16<T>::pack(static_cast<float>(static_cast<int>(nib & 0xffu) - 8) * d,
+                                 static_cast<float>(static_cast<int>((nib >> 8) & 0xffu) - 8) * d);
+        pk[2 * t + 1] = F16<T>::pack(static_cast<float>(static_cast<int>((nib >> 16) & 0xffu) - 8) * d,
+                                     static_cast<float>(static_cast<int>(nib >> 24) - 8) * d);
+      }
+    }
+    *reinterpret_cast<uint4*>(brow + (((4 * h + c) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// WQ = 1: B is q8_0, WQ = 2: B is q4_0 (mB* map the codes, mS* the fp16 scales); converter
+// warps dequantize each stage into the 16-bit B buffer the MMA reads.
 template <int EPI, typename T, int WQ = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI, WQ), 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
@@ -949,16 +997,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
                      const __grid_constant__ CUtensorMap mS2, const __grid_constant__ CUtensorMap mD,
                      const GemmParams p, const __grid_constant__ MixParams mp) {
   using Cfg = PairCfg;
-  constexpr int S = WQ ? Cfg::STAGES_Q8 : Cfg::STAGES;
+  constexpr int S = Cfg::stages(WQ);
+  constexpr int RAWB = Cfg::raw_bytes(WQ);
   constexpr int BN = Cfg::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * Cfg::A_BYTES;
-  uint8_t* sR = sB + S * Cfg::B_BYTES;  // q8_0 raw stages (WQ)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + (WQ ? S * Cfg::RAW_BYTES : 0));
-  uint64_t* rawfull = bars + 16;        // WQ: this CTA's raw codes and scales of a stage landed
+  uint8_t* sR = sB + S * Cfg::B_BYTES;  // raw stages of quantized weights (WQ)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + S * RAWB);
+  uint64_t* rawfull = bars + 20;        // WQ: this CTA's raw codes and scales of a stage landed
+  static_assert(!WQ || (2 * S + 5 <= 20 && 20 + S <= 32), "barrier block");
   uint64_t* full = bars;            // leader: both CTAs' bytes of a stage
   uint64_t* empty = bars + S;       // both: the pair's MMAs on a stage completed
   uint64_t* tfull = bars + 2 * S;   // both: the pair's accumulator is ready
@@ -1099,11 +1149,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &mA, fb, kc,
                            m_blk * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM, pol_a);
           if constexpr (WQ) {  // this CTA's codes (64 k x 128 rows) and scales (2 blocks x 128 rows)
-            uint8_t* raw = sR + stage * Cfg::RAW_BYTES;
-            mbar_arrive_expect_tx(&rawfull[stage], Cfg::RAW_BYTES);
+            uint8_t* raw = sR + stage * RAWB;
+            mbar_arrive_expect_tx(&rawfull[stage], RAWB);
             rarmed |= 1u << stage;
-            tma_load_2d(raw, bs.m, &rawfull[stage], kc, bs.row, pol_b);
-            tma_load_2d(raw + Cfg::RAW_CODES, bs.s, &rawfull[stage], bs.row, kc / 32, pol_b);
+            tma_load_2d(raw, bs.m, &rawfull[stage], WQ == 2 ? kc / 2 : kc, bs.row, pol_b);
+            tma_load_2d(raw + Cfg::raw_codes(WQ), bs.s, &rawfull[stage], bs.row, kc / 32, pol_b);
           } else if (!pre) {
             tma_load_2d_pair(sB + stage * Cfg::B_BYTES, bs.m, fb, kc, bs.row, pol_b);
           }
@@ -1227,7 +1277,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       for (int kb = kb0; kb < kb1; ++kb) {
         ok = __all_sync(0xffffffffu, mbar_wait(&rawfull[stage], phase, abort_flag));
         if (!ok) break;
-        q8_0_dequant_block<T>(sR + stage * Cfg::RAW_BYTES, sB + stage * Cfg::B_BYTES, r, hb);
+        if constexpr (WQ == 2)
+          q4_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
+        else
+          q8_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -1383,6 +1436,18 @@ static bool make_map_q8_codes(CUtensorMap* m, const void* base, int64_t K, int64
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// q4_0 weights: packed codes uint8 [rows, K / 2] (box 128 rows x 32 bytes, 32-byte swizzle)
+static bool make_map_q4_codes(CUtensorMap* m, const void* base, int64_t K, int64_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 static bool make_map_q8_scales(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t ld) {
@@ -1558,9 +1623,10 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   return cudaPeekAtLastError() == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
-// q8_0 weights on CTA pairs: B[i] are the int8 codes, Bs[i] the fp16 scales of matrix i.
-template <int EPI, typename T>
-static int launch_pair_q8(const GemmArgs& a, cudaStream_t s) {
+// Quantized weights on CTA pairs (WQ 1: q8_0, 2: q4_0): B[i] are the codes, Bs[i] the fp16
+// scales of matrix i.
+template <int EPI, typename T, int WQ>
+static int launch_pair_wq(const GemmArgs& a, cudaStream_t s) {
   using Cfg = PairCfg;
   const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -1571,7 +1637,9 @@ static int launch_pair_q8(const GemmArgs& a, cudaStream_t s) {
   const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
   for (int i = 0; i < 3; ++i) {
     const int j = i < nb ? i : 0;
-    if (!make_map_q8_codes(&mB[i], a.B[j], a.K, b_rows) ||
+    const bool codes_ok = WQ == 2 ? make_map_q4_codes(&mB[i], a.B[j], a.K, b_rows)
+                                  : make_map_q8_codes(&mB[i], a.B[j], a.K, b_rows);
+    if (!codes_ok ||
         !make_map_q8_scales(&mS[i], a.Bs[j], a.K, b_rows, a.lds > 0 ? a.lds : b_rows))
       return KVA_ERR_CUDA;
   }
@@ -1597,10 +1665,11 @@ static int launch_pair_q8(const GemmArgs& a, cudaStream_t s) {
   const int items = num_m * ((a.N + n_per_tile - 1) / n_per_tile) * splits;
   int ncl = items < max_cl ? items : max_cl;
   if (items > ncl && num_m > 1 && ncl >= num_m && num_m <= 16) ncl -= ncl % num_m;
-  auto kern = gemm_pair_kernel<EPI, T, 1>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_Q8) != cudaSuccess)
+  auto kern = gemm_pair_kernel<EPI, T, WQ>;
+  constexpr int smem = WQ == 2 ? Cfg::SMEM_Q4 : Cfg::SMEM_Q8;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return KVA_ERR_CUDA;
-  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI, 1)), Cfg::SMEM_Q8, s, mA, mB[0], mB[1], mB[2],
+  if (launch_pdl(kern, dim3(2 * ncl), dim3(Cfg::threads(EPI, WQ)), smem, s, mA, mB[0], mB[1], mB[2],
                  mS[0], mS[1], mS[2], mA, p, MixParams()) != cudaSuccess)
     return KVA_ERR_CUDA;
   return KVA_OK;
@@ -1682,23 +1751,25 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (bn != 128 && bn != 256 && bn != 512) return KVA_ERR_UNSUPPORTED;
   if (a.dtype != KVA_BF16 && a.dtype != KVA_F16) return KVA_ERR_INVALID_ARG;
   const bool h = a.dtype == KVA_F16;
-  if (a.q8) {  // q8_0 weights: CTA pairs, plain epilogues (STORE, ADD_F32, SWIGLU)
+  if (a.wq) {  // q8_0 / q4_0 weights: CTA pairs, plain epilogues (STORE, ADD_F32, SWIGLU)
     if (a.K % 64 || a.n_split || bn != 512) return KVA_ERR_UNSUPPORTED;
     const int64_t b_rows = a.b_mode == B_SEGMENTS ? a.seg_rows : a.N;
     if (b_rows % 8 || a.lds % 8) return KVA_ERR_ALIGNMENT;  // scale rows of 16-byte multiples
     for (int i = 0; i < (a.b_mode == B_SINGLE ? 1 : (a.b_mode == B_PAIRED ? 2 : 3)); ++i)
       if (!a.Bs[i] || !aligned16(a.Bs[i]) || !a.B[i] || !aligned16(a.B[i])) return KVA_ERR_INVALID_ARG;
+    if (a.wq != 1 && a.wq != 2) return KVA_ERR_INVALID_ARG;
+#define KVA_WQ_CASE(E)                                                                          \
+  case E:                                                                                       \
+    if (a.wq == 1) return h ? launch_pair_wq<E, __half, 1>(a, s) : launch_pair_wq<E, __nv_bfloat16, 1>(a, s); \
+    return h ? launch_pair_wq<E, __half, 2>(a, s) : launch_pair_wq<E, __nv_bfloat16, 2>(a, s);
     switch (a.epilogue) {
-      case EPI_STORE_BF16:
-        return h ? launch_pair_q8<EPI_STORE_BF16, __half>(a, s) : launch_pair_q8<EPI_STORE_BF16, __nv_bfloat16>(a, s);
-      case EPI_ADD_F32:
-        return h ? launch_pair_q8<EPI_ADD_F32, __half>(a, s) : launch_pair_q8<EPI_ADD_F32, __nv_bfloat16>(a, s);
-      case EPI_SWIGLU_BF16:
-        return h ? launch_pair_q8<EPI_SWIGLU_BF16, __half>(a, s)
-                 : launch_pair_q8<EPI_SWIGLU_BF16, __nv_bfloat16>(a, s);
+      KVA_WQ_CASE(EPI_STORE_BF16)
+      KVA_WQ_CASE(EPI_ADD_F32)
+      KVA_WQ_CASE(EPI_SWIGLU_BF16)
       default:
         return KVA_ERR_UNSUPPORTED;
     }
+#undef KVA_WQ_CASE
   }
 #define KVA_GEMM_CASE(E)                                                                   \
   case E:                                                                                  \

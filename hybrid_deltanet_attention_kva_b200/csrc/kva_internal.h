@@ -64,9 +64,10 @@ struct GemmArgs {
   int* err = nullptr;       // device status word
   bool b_const = false;     // B is never written by kernels on the stream (weights): the
                             // first stages' B tiles may be loaded before the previous kernel ends
-  bool q8 = false;          // B[i] are q8_0 codes (int8 [rows, K]) with fp16 scales Bs[i]
-  const void* Bs[3] = {nullptr, nullptr, nullptr};  //   [K / 32, rows]; weight = scale * code
-  int64_t lds = 0;          // q8: row stride of Bs in scales (0: the matrix's rows)
+  int wq = 0;               // 0: 16-bit B; 1: B[i] are q8_0 codes (int8 [rows, K]); 2: q4_0
+                            //   codes (uint8 [rows, K / 2], two per byte); fp16 scales Bs[i]
+  const void* Bs[3] = {nullptr, nullptr, nullptr};  //   [K / 32, rows]
+  int64_t lds = 0;          // wq: row stride of Bs in scales (0: the matrix's rows)
 };
 
 int num_sms();

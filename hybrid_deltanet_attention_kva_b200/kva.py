@@ -65,7 +65,7 @@ class KvaWeights(C.Structure):
                 ("block_scale", (C.c_void_p * 7) * MAX_BLOCKS)]
 
 
-KVA_W_16, KVA_W_Q8_0 = 0, 1
+KVA_W_16, KVA_W_Q8_0, KVA_W_Q4_0 = 0, 1, 2
 Q8_MATRICES = ("Wq", "Wk", "Wv", "Wo", "Wg", "Wu", "Wd")
 
 
@@ -118,6 +118,8 @@ def _load() -> C.CDLL:
                               I32, I32, I32, I32, P, P]),
         "kva_op_gemm_q8_0": (I32, [I32, P, I64, C.POINTER(P), C.POINTER(P), I32, I64, P, I64, I32, I32,
                                    I32, I32, P, P]),
+        "kva_op_gemm_q4_0": (I32, [I32, P, I64, C.POINTER(P), C.POINTER(P), I32, I64, P, I64, I32, I32,
+                                   I32, I32, P, P]),
         "kva_op_attention": (I32, [I32, P, I64, P, I64, I32, I32, I32, P]),
         "kva_op_gdn_scan": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "kva_gdn_layer_update_noalloc": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, F32, P]),
@@ -133,7 +135,8 @@ _lib = _load()
 EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update_states",
             "kva_get_device_status", "kva_stats", "kva_heads_fused", "kva_free", "kva_strerror",
             "kva_profile_enable", "kva_profile_read",
-            "kva_op_rmsnorm", "kva_op_gemm", "kva_op_gemm_q8_0", "kva_op_attention", "kva_op_gdn_scan",
+            "kva_op_rmsnorm", "kva_op_gemm", "kva_op_gemm_q8_0", "kva_op_gemm_q4_0", "kva_op_attention",
+            "kva_op_gdn_scan",
             "kva_gdn_layer_update_noalloc")
 
 
@@ -203,8 +206,9 @@ class Weights:
                     setattr(cb, name, self._p(b[name]))
             self.c.g_out = self._p(proj["g_out"])
             self.c.W_heads = self._p(proj["W_heads"])
-            if "W_heads_scale" in proj:  # q8_0: int8 codes above, fp16 scales [K/32, N] here
-                self.c.weight_format = KVA_W_Q8_0
+            if "W_heads_scale" in proj:  # codes above (int8: q8_0, packed uint8: q4_0), fp16
+                # scales [K/32, N] here
+                self.c.weight_format = KVA_W_Q4_0 if proj["W_heads"].dtype == torch.uint8 else KVA_W_Q8_0
                 self.c.W_in_scale = self._p(proj["W_in_scale"])
                 self.c.W_heads_scale = self._p(proj["W_heads_scale"])
                 for i, b in enumerate(proj["blocks"]):
@@ -349,6 +353,18 @@ def kva_op_gemm_q8_0(A: torch.Tensor, Bq: Sequence[torch.Tensor], Bs: Sequence[t
     sc = (C.c_void_p * 3)(*([_ptr(b) for b in Bs] + [None] * (3 - len(Bs))))
     _check(_lib.kva_op_gemm_q8_0(_DT[A.dtype], _ptr(A), K, q, sc, b_mode, seg_rows, _ptr(D), D.shape[1],
                                  M, N, K, epilogue, _ptr(err), _stream(stream)), "kva_op_gemm_q8_0")
+
+
+def kva_op_gemm_q4_0(A: torch.Tensor, Bq: Sequence[torch.Tensor], Bs: Sequence[torch.Tensor],
+                     D: torch.Tensor, *, N: int, epilogue: int = EPI_STORE_BF16, b_mode: int = B_SINGLE,
+                     seg_rows: int = 0, err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """D = A dequant(B)^T with q4_0 weights: Bq[i] uint8 [rows, K/2] packed codes, Bs[i] fp16
+    [K/32, rows] scales (see include/kva_ops.h)."""
+    M, K = A.shape
+    q = (C.c_void_p * 3)(*([_ptr(b) for b in Bq] + [None] * (3 - len(Bq))))
+    sc = (C.c_void_p * 3)(*([_ptr(b) for b in Bs] + [None] * (3 - len(Bs))))
+    _check(_lib.kva_op_gemm_q4_0(_DT[A.dtype], _ptr(A), K, q, sc, b_mode, seg_rows, _ptr(D), D.shape[1],
+                                 M, N, K, epilogue, _ptr(err), _stream(stream)), "kva_op_gemm_q4_0")
 
 
 def kva_op_attention(qkv: torch.Tensor, out: torch.Tensor, n_heads: int, window: int,

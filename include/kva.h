@@ -131,15 +131,19 @@ typedef struct kva_weights {
    * KVA_W_Q8_0: every projector matrix pointer above (W_in, each block's Wq..Wd, W_heads)
    * holds int8 codes [N, K] row-major instead, and the matching *_scale pointer below
    * fp16 scales [K / 32, N] (one 32-wide K block of all N rows contiguous); the weight
-   * (n, k) is scale[k / 32][n] * code[n][k].  Every K (H, d, ffn) must be a multiple of
-   * 64.  The prefill then runs the heads GEMM without the fused state-update epilogue. */
+   * (n, k) is scale[k / 32][n] * code[n][k].  KVA_W_Q4_0: the same with packed 4-bit
+   * codes, uint8 [N, K / 2]: per 32-wide K block of a row 16 bytes, byte j holding the code
+   * c (0..15) of element j in its low nibble and that of element j + 16 in its high
+   * nibble; the weight is scale[k / 32][n] * (c - 8).  Every K (H, d, ffn) must be a
+   * multiple of 64.  The prefill then runs the heads GEMM without the fused state-update
+   * epilogue. */
   int32_t weight_format;
   const void* W_in_scale;
   const void* W_heads_scale;
   const void* block_scale[KVA_MAX_BLOCKS][7]; /* Wq, Wk, Wv, Wo, Wg, Wu, Wd */
 } kva_weights;
 
-typedef enum kva_weight_format { KVA_W_16 = 0, KVA_W_Q8_0 = 1 } kva_weight_format;
+typedef enum kva_weight_format { KVA_W_16 = 0, KVA_W_Q8_0 = 1, KVA_W_Q4_0 = 2 } kva_weight_format;
 
 /* KV caches of the attention layers (device pointers, written in place).
  * CONTIGUOUS: k[l], v[l] are [n_seq, n_kv, max_pos, row]; token p of sequence s

@@ -44,6 +44,16 @@ int kva_op_gemm_q8_0(int32_t dtype, const void* A, int64_t lda, const void* cons
                      const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
                      int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream);
 
+/* The same with q4_0 weights (the same section's q4_0 projector, about half the bytes of
+ * q8_0).  Each B matrix [rows, K] is given as packed codes Bq[i], uint8 [rows, K / 2] (row
+ * stride K / 2): per 32-wide K block of a row 16 bytes, byte j holding the code c (0..15)
+ * of element j in its low nibble and that of element j + 16 in its high nibble; scales
+ * Bs[i] as above.  Its weight (r, k) is Bs[i][k / 32][r] * (c(r, k) - 8), rounded once to
+ * dtype for the tensor cores.  Same modes, sizes and errors as kva_op_gemm_q8_0. */
+int kva_op_gemm_q4_0(int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
+                     const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
+                     int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream);
+
 /* RMSNorm of `rows` rows of width n ("Qwen3.8-27B-KVA" model card, architecture):
  * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out [rows, ldo] in out_dtype (bf16 / fp16).
  * x is [rows, ldx] in x_dtype.  n, ldx, ldo multiples of 4; pointers 16-byte aligned. */

@@ -268,6 +268,59 @@ def test_gemm_q8_0_weights(K, M, N, K_, epi, dt):
                      elem=BF16_ELEM if epi == 0 else 0.0)
 
 
+def _q4_weights(g, rows, K, scale=0.05):
+    """Random weights as q4_0 (packed codes uint8 [rows, K/2], scales fp16 [K/32, rows]) and
+    their dequantized float64 values (the oracle's quantizer, packer and dequantizer)."""
+    W = (torch.randn(rows, K, generator=g, dtype=torch.float64) * scale).numpy()
+    d, codes = R.q4_0_quantize(W)
+    Wd = R.q4_0_dequantize(d, codes)
+    return (torch.from_numpy(R.q4_0_pack(codes)), torch.from_numpy(np.ascontiguousarray(d.T)), Wd)
+
+
+@pytest.mark.parametrize("M,N,K_,epi", [(1024, 3072, 3072, 0), (600, 1040, 704, 0), (77, 256, 128, 0),
+                                        (1000, 2048, 1024, 2)])
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_gemm_q4_0_weights(K, M, N, K_, epi, dt):
+    g = _gen(M * 5 + N + K_ + epi)
+    A = torch.randn(M, K_, generator=g).to(dt)
+    Bq, Bs, Wd = _q4_weights(g, N, K_)
+    want = R.projector_heads(f64(A), Wd)
+    if epi == K.EPI_STORE_BF16:
+        D = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    else:
+        D0 = torch.randn(M, N, generator=g)
+        D = D0.cuda()
+        want = want + f64(D0)
+    K.kva_op_gemm_q4_0(A.cuda(), [Bq.cuda()], [Bs.cuda()], D, N=N, epilogue=epi)
+    torch.cuda.synchronize()
+    # d (c - 8) has at most 15 significant bits: one rounding to the operand format
+    assert_rms_close(D, want, tol=Q8_TOL[dt], what=f"q4_0 gemm epi={epi}",
+                     elem=BF16_ELEM if epi == 0 else 0.0)
+
+
+def test_gemm_q4_0_swiglu_and_segments(K):
+    g = _gen(4343)
+    dt = torch.float16
+    M, F, Kd = 1000, 1024, 512
+    A = torch.randn(M, Kd, generator=g).to(dt)
+    Gq, Gs, Gd = _q4_weights(g, F, Kd)
+    Uq, Us, Ud = _q4_weights(g, F, Kd)
+    D = torch.empty(M, F, dtype=dt, device="cuda")
+    K.kva_op_gemm_q4_0(A.cuda(), [Gq.cuda(), Uq.cuda()], [Gs.cuda(), Us.cuda()], D, N=F,
+                       epilogue=K.EPI_SWIGLU_BF16, b_mode=K.B_PAIRED)
+    a = f64(A)
+    gate, up = a @ Gd.T, a @ Ud.T
+    assert_rms_close(D, gate / (1.0 + np.exp(-gate)) * up, tol=Q8_TOL[dt], what="q4_0 swiglu",
+                     elem=BF16_ELEM)
+    seg = 512
+    parts = [_q4_weights(g, seg, Kd) for _ in range(3)]
+    D2 = torch.empty(M, 3 * seg, dtype=dt, device="cuda")
+    K.kva_op_gemm_q4_0(A.cuda(), [p[0].cuda() for p in parts], [p[1].cuda() for p in parts], D2,
+                       N=3 * seg, b_mode=K.B_SEGMENTS, seg_rows=seg)
+    want2 = a @ np.concatenate([p[2] for p in parts]).T
+    assert_rms_close(D2, want2, tol=Q8_TOL[dt], what="q4_0 segments", elem=BF16_ELEM)
+
+
 @pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
 def test_gemm_q8_0_swiglu_and_segments(K, dt):
     g = _gen(4242)

@@ -414,11 +414,16 @@ def test_prefill_full_size_sampled(K, cfg, dt):
             assert m.get("max_excess_over_rms", m["max_over_rms"]) <= tol_out, (name, m)
 
 
-# ------------------------------------------------------------------ q8_0 projector weights
-def _q8_projector(W):
-    """Every projector matrix as q8_0 (the oracle's quantizer): (GPU weight dict with int8
-    codes and fp16 scales [K/32, N], float64 dequantized weights for the oracle)."""
+# ------------------------------------------------------------------ quantized projector weights
+def _q8_projector(W, fmt="q8_0"):
+    """Every projector matrix as q8_0 or q4_0 (the oracle's quantizer): (GPU weight dict with
+    the codes (int8 [N, K], or packed uint8 [N, K/2]) and fp16 scales [K/32, N], float64
+    dequantized weights for the oracle)."""
     def q(t):
+        if fmt == "q4_0":
+            d, c = R.q4_0_quantize(f64(t))
+            return (torch.from_numpy(R.q4_0_pack(c)).cuda(),
+                    torch.from_numpy(np.ascontiguousarray(d.T)).cuda(), R.q4_0_dequantize(d, c))
         d, c = R.q8_0_quantize(f64(t))
         return (torch.from_numpy(c).cuda(), torch.from_numpy(np.ascontiguousarray(d.T)).cuda(),
                 R.q8_0_dequantize(d, c))
@@ -438,15 +443,16 @@ def _q8_projector(W):
     return gpu, ref
 
 
-@pytest.mark.parametrize("geom,draft", [(KI.TINY, False), (TINY128, True)])
-def test_prefill_q8_0_projector_weights(K, geom, draft):
-    """q8_0 projector weights (TINY128 would take the fused heads epilogue with 16-bit
-    weights; q8_0 weights run the heads GEMM plain and the drafter rows as a GEMM of their
-    own)."""
+@pytest.mark.parametrize("geom,draft,fmt", [(KI.TINY, False, "q8_0"), (TINY128, True, "q8_0"),
+                                            (TINY128, True, "q4_0"), (KI.TINY, False, "q4_0")])
+def test_prefill_q8_0_projector_weights(K, geom, draft, fmt):
+    """q8_0 / q4_0 projector weights (TINY128 would take the fused heads epilogue with 16-bit
+    weights; quantized weights run the heads GEMM plain and the drafter rows as a GEMM of
+    their own)."""
     dt = torch.float16
     splits = [300, 2, 130]
     W = KI.make_projector_weights(geom, 5200)
-    Wg, Wn = _q8_projector(W)
+    Wg, Wn = _q8_projector(W, fmt)
     P = KI.make_layer_params(geom, 5201)
     st = KI.make_states(geom, 1, 5202)
     res = KI.make_residual(geom, sum(splits), 5203, dtype=torch.float32, n_outliers=0)
