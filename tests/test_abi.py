@@ -49,7 +49,8 @@ def test_struct_layouts_match_the_c_compiler(tmp_path):
     """sizeof / offsetof of every ABI struct, from gcc compiling the header, equal ctypes'."""
     import hybrid_deltanet_attention_kva_b200 as K
     fields = {"kva_dims": (K.KvaDims, ["rope_theta", "norm_eps", "max_seq", "layer_type"]),
-              "kva_weights": (K.KvaWeights, ["blocks", "W_heads", "k_norm_g"]),
+              "kva_weights": (K.KvaWeights, ["blocks", "W_heads", "k_norm_g", "weight_format",
+                                             "W_in_scale", "W_heads_scale", "block_scale"]),
               "kva_block_weights": (K.KvaBlockWeights, ["Wd"]),
               "kva_kv_cache": (K.KvaKvCache, ["v", "max_pos", "page_table"])}
     src = ["#include <stdio.h>", "#include <stddef.h>", '#include "kva.h"', "int main(void){"]
@@ -122,7 +123,56 @@ def test_host_validation_rejects_before_any_launch():
                          64, 64, 64, 0, 0, None, None) == K.KVA_ERR_INVALID_ARG
     assert L.kva_op_gemm(1, C.c_void_p(16), 64, arr, 0, 64, 0, C.c_void_p(16), 64, None, 0, 0,
                          64, 64, 64, 0, 0, None, None) == K.KVA_ERR_INVALID_ARG  # fp32 operands
+    # quantized-weight GEMMs: K a multiple of 64, scales present and aligned, rows of 8
+    one = (C.c_void_p * 3)(16, None, None)
+    no_scale = (C.c_void_p * 3)(None, None, None)
+    odd_scale = (C.c_void_p * 3)(8, None, None)
+    for op in (L.kva_op_gemm_q8_0, L.kva_op_gemm_q4_0):
+        assert op(0, C.c_void_p(16), 96, one, one, 0, 0, C.c_void_p(16), 64, 64, 64, 96, 0, None,
+                  None) == K.KVA_ERR_UNSUPPORTED                        # K = 96
+        assert op(0, C.c_void_p(16), 128, one, no_scale, 0, 0, C.c_void_p(16), 64, 64, 64, 128, 0,
+                  None, None) == K.KVA_ERR_INVALID_ARG                  # no scales
+        assert op(0, C.c_void_p(16), 128, one, odd_scale, 0, 0, C.c_void_p(16), 64, 64, 64, 128, 0,
+                  None, None) == K.KVA_ERR_INVALID_ARG                  # misaligned scales
+        assert op(0, C.c_void_p(16), 128, one, one, 0, 0, C.c_void_p(16), 64, 64, 60, 128, 0, None,
+                  None) == K.KVA_ERR_ALIGNMENT                          # 60 scale rows
+        assert op(0, C.c_void_p(16), 128, one, one, 3, 0, C.c_void_p(16), 64, 64, 64, 128, 0, None,
+                  None) == K.KVA_ERR_INVALID_ARG                        # b_mode
+        assert op(0, C.c_void_p(16), 128, None, one, 0, 0, C.c_void_p(16), 64, 64, 64, 128, 0, None,
+                  None) == K.KVA_ERR_INVALID_ARG                        # no codes
+        assert op(1, C.c_void_p(16), 128, one, one, 0, 0, C.c_void_p(16), 64, 64, 64, 128, 0, None,
+                  None) == K.KVA_ERR_INVALID_ARG                        # fp32 operands
     assert L.kva_op_attention(0, C.c_void_p(16), 384, C.c_void_p(16), 128, 16, 1, -1, None) \
         == K.KVA_ERR_INVALID_ARG
     assert L.kva_op_gdn_scan(C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), 1,
                              1, 8, 1, 1, 96, None) == K.KVA_ERR_UNSUPPORTED
+
+
+def test_binding_constants_match_the_headers(tmp_path):
+    """Every enumerator and status bit of the headers has the binding's value (compiled by gcc)."""
+    import hybrid_deltanet_attention_kva_b200 as K
+    names = set()
+    for h in ("kva.h", "kva_ops.h"):
+        with open(os.path.join(ROOT, "include", h)) as f:
+            txt = f.read()
+        for body in re.findall(r"typedef enum \w+ \{(.*?)\}", txt, re.S):
+            names |= set(re.findall(r"\b(KVA_\w+)\s*=", body))
+        names |= set(re.findall(r"^#define (KVA_DEV_\w+)", txt, re.M))
+    assert {"KVA_W_Q4_0", "KVA_Q8_0", "KVA_EPI_SWIGLU_BF16", "KVA_DEV_WAIT_TIMEOUT"} <= names
+    src = ["#include <stdio.h>", '#include "kva.h"', '#include "kva_ops.h"', "int main(void){"]
+    src += [f'printf("{n} %d\\n", (int)({n}));' for n in sorted(names)]
+    src.append("return 0;}")
+    c = tmp_path / "consts.c"
+    c.write_text("\n".join(src))
+    exe = tmp_path / "consts"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    got = {a: int(b) for a, b in (line.split() for line in subprocess.run(
+        [str(exe)], capture_output=True, text=True, check=True).stdout.splitlines())}
+    for n, v in got.items():
+        if n.startswith("KVA_ST_") and n != "KVA_ST_COUNT":  # stages: by name, in order
+            assert K.ST_NAMES[v] == n[len("KVA_ST_"):].lower(), n
+            continue
+        # the binding drops the KVA_ prefix of the epilogue, B-mode and stage enumerators
+        short = n[4:] if n.startswith(("KVA_EPI_", "KVA_B_", "KVA_ST_")) else n
+        assert hasattr(K, short), n
+        assert getattr(K, short) == v, (n, getattr(K, short), v)
