@@ -192,7 +192,12 @@ def make_dims(geom, max_T: int, max_seq: int = 1, dtype=torch.float16) -> KvaDim
 
 
 class Weights:
-    """kva_weights over torch tensors (kept alive by this object)."""
+    """kva_weights over torch tensors (kept alive by this object).
+
+    proj: g_in, W_in, blocks (g_attn, Wq, Wk, Wv, Wo, g_ffn, Wg, Wu, Wd each), g_out, W_heads.
+    16-bit matrices give KVA_W_16.  Quantized matrices come with a "<name>_scale" tensor
+    each (fp16 [K/32, N]): int8 codes [N, K] are q8_0, uint8 packed codes [N, K/2] q4_0.
+    layer: conv_w, A_log, dt_bias, k_norm_g of the late layers."""
 
     def __init__(self, proj: Optional[Dict] = None, layer: Optional[Dict] = None):
         self._keep = []
@@ -208,7 +213,10 @@ class Weights:
             self.c.W_heads = self._p(proj["W_heads"])
             if "W_heads_scale" in proj:  # codes above (int8: q8_0, packed uint8: q4_0), fp16
                 # scales [K/32, N] here
-                self.c.weight_format = KVA_W_Q4_0 if proj["W_heads"].dtype == torch.uint8 else KVA_W_Q8_0
+                fmt = {torch.uint8: KVA_W_Q4_0, torch.int8: KVA_W_Q8_0}.get(proj["W_heads"].dtype)
+                if fmt is None:
+                    raise ValueError("quantized W_heads must be int8 (q8_0) or uint8 (q4_0) codes")
+                self.c.weight_format = fmt
                 self.c.W_in_scale = self._p(proj["W_in_scale"])
                 self.c.W_heads_scale = self._p(proj["W_heads_scale"])
                 for i, b in enumerate(proj["blocks"]):
