@@ -176,3 +176,30 @@ def test_binding_constants_match_the_headers(tmp_path):
         short = n[4:] if n.startswith(("KVA_EPI_", "KVA_B_", "KVA_ST_")) else n
         assert hasattr(K, short), n
         assert getattr(K, short) == v, (n, getattr(K, short), v)
+
+
+def test_weight_format_follows_the_code_dtype(monkeypatch):
+    """q8_0 for int8 codes, q4_0 for packed uint8 codes, an error for anything else (pointers
+    faked: no device memory is touched)."""
+    import torch
+    import hybrid_deltanet_attention_kva_b200 as K
+    from hybrid_deltanet_attention_kva_b200 import kva as kmod
+    monkeypatch.setattr(kmod, "_ptr", lambda t: None if t is None else 16)
+    names = ("Wq", "Wk", "Wv", "Wo", "Wg", "Wu", "Wd")
+
+    def proj(codes_dtype, quant=True):
+        z = torch.zeros(2, dtype=codes_dtype)
+        blk = {"g_attn": z, "g_ffn": z, **{n: z for n in names}}
+        p = {"g_in": z, "W_in": z, "g_out": z, "W_heads": z, "blocks": [blk]}
+        if quant:
+            p["W_in_scale"] = p["W_heads_scale"] = z
+            blk.update({n + "_scale": z for n in names})
+        return p
+
+    assert K.Weights(proj=proj(torch.float16, quant=False)).c.weight_format == K.KVA_W_16
+    assert K.Weights(proj=proj(torch.int8)).c.weight_format == K.KVA_W_Q8_0
+    w4 = K.Weights(proj=proj(torch.uint8))
+    assert w4.c.weight_format == K.KVA_W_Q4_0
+    assert w4.c.W_heads_scale == 16 and w4.c.block_scale[0][6] == 16
+    with pytest.raises(ValueError):
+        K.Weights(proj=proj(torch.int16))
