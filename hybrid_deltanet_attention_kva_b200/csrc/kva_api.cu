@@ -1,7 +1,7 @@
 // C ABI of libkva: argument validation, workspace ownership and the launch plan
-// of one KVA ubatch ("Qwen3.8-27B-KVA" model card, "What the hell?": the
-// projector maps the layer-31 residual to the token-mixer inputs of every late
-// layer, then the cheap state updates run on them).
+// of one KVA ubatch ("Qwen3.8-27B-KVA" model card, "What the hell?": from each
+// token's layer-31 residual the projector predicts what every late layer's token
+// mixer takes as input, and the cheap state updates then consume those predictions).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

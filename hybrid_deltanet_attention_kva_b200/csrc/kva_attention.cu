@@ -1,6 +1,6 @@
 // Block-causal multi-head attention of the projector blocks ("Qwen3.8-27B-KVA"
-// model card, architecture table row "attention": heads @ 128, causal within
-// 1024-token blocks for r3, full causal within the ubatch for r2).
+// model card, architecture table, attention row: 128-dim heads; r3 cuts the causal
+// mask into 1024-token blocks, r2 keeps it causal over the whole ubatch).
 //
 // Key j is visible to query i iff j <= i and floor(i/W) == floor(j/W), indices
 // local to the ubatch (W = window, or the whole ubatch when window = 0).  qkv is

@@ -1,6 +1,7 @@
 // Full-attention late layers: k RMSNorm per KV head, partial RoPE and the KV
-// cache write ("Qwen3.8-27B-KVA" model card, table "late layer type": k_proj /
-// v_proj outputs before k_norm / rope; "Qwen3.8-27B-MLA" model card, "What this
+// cache write ("Qwen3.8-27B-KVA" model card, late-layer table: the projector
+// predicts the k and v projections, and the k norm and RoPE come after it;
+// "Qwen3.8-27B-MLA" model card, "What this
 // is": 4 KV heads of dim 256 with 64 rotary dims, whose lowest pairs turn
 // 3.4 / 2.1 / 1.2 degrees across 131k tokens, i.e. theta = 1e7).
 //
@@ -139,8 +140,8 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const KvLaunch p) {
 }
 
 // ------------------------------------------------------------------ q8_0 cache rows
-// Quantized KV cache ("Qwen3.8-27B-KVA" model card, other notes: q8_0 caches, with the
-// same Hadamard rotation applied to the approximated K/V as the exact path applies).
+// Quantized KV cache ("Qwen3.8-27B-KVA" model card, other notes: with q8_0 caches the
+// approximated K/V rows are rotated by the same Hadamard transform the exact layers use).
 // Each d_h-dim row (k after RMSNorm and RoPE, v as predicted) is multiplied by the
 // orthonormal Walsh-Hadamard matrix H / sqrt(d_h), Sylvester order, then stored as q8_0
 // blocks of 32 values: fp16 scale d = max|x| / 127, int8 codes round(x / d), half away

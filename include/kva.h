@@ -3,11 +3,11 @@
  *
  * What the path computes ("Qwen3.8-27B-KVA: late-layer KV approximation" model
  * card, sections "What the hell?" and the architecture table):
- *   for one ubatch of T tokens, a projector maps the layer-31 residual
- *   (H = 5120 per token) to the token-mixer inputs of every late layer:
- *       RMSNorm -> Linear{H -> d} -> n_blocks x causal transformer block
+ *   for one ubatch of T tokens, a projector predicts from the layer-31
+ *   residual (H = 5120 per token) the input of every late layer's token mixer:
+ *       RMSNorm, Linear{H -> d}, n_blocks causal transformer blocks
  *       (MHA at head dim 128, causal within the ubatch / within `attn_window`
- *       blocks, SwiGLU FFN) -> RMSNorm -> one Linear head per late layer
+ *       blocks, SwiGLU FFN), RMSNorm, then a linear head for each late layer
  *       (+ optional drafter heads);
  *   then the cheap state updates run on those mixer inputs:
  *       gated-DeltaNet layers: causal depthwise conv1d (kernel 4) + SiLU,
@@ -152,8 +152,8 @@ typedef enum kva_weight_format { KVA_W_16 = 0, KVA_W_Q8_0 = 1, KVA_W_Q4_0 = 2 } 
  *             goes to page page_table[s * pages_per_seq + p / page_size], row
  *             p % page_size.  page_table is int32 on the device.
  * A row is d_h values in bf16 or fp16 (dtype KVA_BF16 / KVA_F16), or, for KVA_Q8_0,
- * the quantized-cache form of the model card's other notes (q8_0 caches get the same
- * Hadamard rotation for the approximated K/V as the exact path): the row (K after k
+ * the quantized-cache form of the model card's other notes (with q8_0 caches the
+ * approximated rows are rotated by the exact layers' Hadamard transform): the row (K after k
  * RMSNorm + RoPE, V as predicted) times the orthonormal Walsh-Hadamard matrix
  * H_{d_h} / sqrt(d_h) in Sylvester order, stored as d_h / 32 blocks of 34 bytes, each
  * an fp16 scale d = max|x| / 127 followed by 32 int8 codes round(x / d) (half away

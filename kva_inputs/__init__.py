@@ -10,8 +10,8 @@ Geometry facts, each from the pages:
   * projector widths and FFN sizes r2 / r3 -- "Qwen3.8-27B-KVA" model card,
     architecture table (width d, heads @ 128, SwiGLU FFN, trunk/heads/total).
   * per-late-layer mixer widths (10240 + 48 + 48 per gated-DeltaNet layer,
-    1024 + 1024 per full-attention layer) -- same card, table "late layer type /
-    predicted per token / dims".
+    1024 + 1024 per full-attention layer) -- same card, the late-layer table of
+    "What the hell?".
   * 48 gated-DeltaNet + 16 full-attention layers in 64, late half 32..63 --
     same card, "What the hell?" section.
   * 4 KV heads of dim 256 and 64 rotary dims per KV head -- "Qwen3.8-27B-MLA"

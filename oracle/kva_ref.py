@@ -38,8 +38,8 @@ Readings where the pages are silent (each also stated where it is used):
       pair (i, i + rope_dims/2) rotated by (pos + t) * theta^(-2i/rope_dims).
   R10 attention-layer V is stored as predicted (no norm, no rotation).
   R11 the scan covers every token of the ubatch.
-  R15 quantized KV cache ([KVA] "Other notes": q8_0 caches, with the same Hadamard
-      rotation applied to the approximated K/V as the exact path applies): every
+  R15 quantized KV cache ([KVA] "Other notes": with q8_0 caches the approximated
+      K/V rows are rotated by the Hadamard transform the exact layers use): every
       d_h-dim K row (after k RMSNorm + RoPE) and V row is multiplied by the
       orthonormal Walsh-Hadamard matrix H_{d_h} / sqrt(d_h) (Sylvester order:
       H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]), then stored as q8_0 blocks of 32
@@ -111,8 +111,9 @@ def block_causal_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray,
                            window: int) -> np.ndarray:
     """Softmax attention per head with the block-causal mask.
 
-    [KVA] table row 'attention': 24 heads @ 128, causal within 1024-token
-    blocks (r3) / 20 heads @ 128, full causal (r2).  Q, K, V: [T, n_h, dh].
+    [KVA] architecture table, attention row: r3 has 24 heads of 128 dims with
+    the causal mask cut into 1024-token blocks, r2 20 heads of 128 dims with a
+    plain causal mask.  Q, K, V: [T, n_h, dh].
     """
     T, n_h, dh = Q.shape
     mask = attention_mask(T, window)
@@ -152,7 +153,8 @@ def projector_trunk(residual: np.ndarray, W: Dict, geom) -> np.ndarray:
 
 def projector_heads(z: np.ndarray, W_heads: np.ndarray,
                     rows: Optional[slice] = None) -> np.ndarray:
-    """'one Linear head per late layer' ([KVA]); rows selects a head block."""
+    """A linear head for each late layer ([KVA] architecture), all concatenated
+    along the output rows; rows selects a head block."""
     Wh = W_heads if rows is None else W_heads[rows]
     return z @ Wh.T
 
