@@ -54,6 +54,12 @@ Readings where the pages are silent (each also stated where it is used):
       decided in float32 (8 when d = 0); a weight is fp16(d) * (q - 8).  Stored as the
       fp16 scale and 16 bytes per block, byte j holding the code of value j in its low
       nibble and that of value j + 16 in its high nibble.
+
+Pins: every function here is checked in tests/test_oracle_pins.py against printed
+values, closed forms, brute force or invariants, and tests/test_oracle_mutants.py plants
+plausible mistakes that those pins catch.  projector_trunk, projector and prefill_ubatch
+as wholes are parity unpinned: the pages print no activations and no trained weights,
+so only their parts are pinned.
 """
 from __future__ import annotations
 

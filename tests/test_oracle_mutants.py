@@ -118,7 +118,7 @@ def _chunked_no_decay_mask(S0, k, v, g, beta, chunk=64):
 R_orig = {name: getattr(R, name) for name in (
     "rope_apply", "rope_inv_freq", "causal_conv_silu", "delta_scan_sequential",
     "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked", "hadamard_rotate",
-    "q8_0_quantize")}
+    "q8_0_quantize", "projector_block")}
 
 def _hadamard_unnormalised(x):
     # the +-1 Walsh-Hadamard matrix without the 1/sqrt(n) that makes it orthonormal
@@ -152,6 +152,17 @@ def _q4_0_positive_scale(x):
     return d.astype(np.float16), c.astype(np.uint8).reshape(x.shape)
 
 
+def _block_gate_up_swapped(x, blk, n_heads, head_dim, window):
+    # the SiLU applied to the up projection instead of the gate
+    sw = dict(blk, Wg=blk["Wu"], Wu=blk["Wg"])
+    return R_orig["projector_block"](x, sw, n_heads, head_dim, window)
+
+
+def _block_values_from_keys(x, blk, n_heads, head_dim, window):
+    # attention values taken from the key projection
+    return R_orig["projector_block"](x, dict(blk, Wv=blk["Wk"]), n_heads, head_dim, window)
+
+
 MUTANTS = [
     ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
     ("rope_apply", _rope_interleaved, [P.test_rope_equals_complex_rotation]),
@@ -169,6 +180,8 @@ MUTANTS = [
      [P.test_hadamard_rotation_keeps_dot_products_and_undoes_itself]),
     ("q8_0_quantize", _q8_0_truncating, [P.test_q8_0_closed_form_block]),
     ("q4_0_pack", _q4_0_pack_halves_swapped, [P.test_q4_0_closed_form_blocks]),
+    ("projector_block", _block_gate_up_swapped, [P.test_projector_block_single_token_attends_to_itself]),
+    ("projector_block", _block_values_from_keys, [P.test_projector_block_single_token_attends_to_itself]),
     ("q4_0_quantize", _q4_0_positive_scale, [P.test_q4_0_closed_form_blocks]),
 ]
 

@@ -312,6 +312,24 @@ def test_projector_with_zero_output_projections_is_linear_chain():
     np.testing.assert_allclose(Y, R.rmsnorm(h, W["g_out"]) @ W["W_heads"].T, rtol=1e-10)
 
 
+def test_projector_block_single_token_attends_to_itself():
+    # one token: the softmax over a single key is 1, so attention returns V whatever Q and K
+    # are, and the block is x + Wo Wv u + Wd (silu(Wg u') * Wu u') written per vector
+    geom, W = _tiny_f64()
+    blk = W["blocks"][1]
+    x = RNG.standard_normal(geom.d_model) * 3
+    u = x / math.sqrt(np.mean(x * x) + R.EPS) * blk["g_attn"]
+    x1 = x + blk["Wo"] @ (blk["Wv"] @ u)
+    u2 = x1 / math.sqrt(np.mean(x1 * x1) + R.EPS) * blk["g_ffn"]
+    gate, up = blk["Wg"] @ u2, blk["Wu"] @ u2
+    want = x1 + blk["Wd"] @ (gate / (1.0 + np.exp(-gate)) * up)
+    got = R.projector_block(x[None], blk, geom.n_heads, geom.head_dim, geom.window)[0]
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+    other = dict(blk, Wq=blk["Wq"] * -7.0, Wk=RNG.standard_normal(blk["Wk"].shape))
+    got2 = R.projector_block(x[None], other, geom.n_heads, geom.head_dim, geom.window)[0]
+    np.testing.assert_allclose(got2, want, rtol=1e-10, atol=1e-12)
+
+
 def test_projector_is_causal_and_position_free():
     geom, W = _tiny_f64()
     res = RNG.standard_normal((20, geom.hidden))
