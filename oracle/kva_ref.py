@@ -55,11 +55,12 @@ Readings where the pages are silent (each also stated where it is used):
       fp16 scale and 16 bytes per block, byte j holding the code of value j in its low
       nibble and that of value j + 16 in its high nibble.
 
-Pins: every function here is checked in tests/test_oracle_pins.py against printed
-values, closed forms, brute force or invariants, and tests/test_oracle_mutants.py plants
-plausible mistakes that those pins catch.  projector_trunk, projector and prefill_ubatch
-as wholes are parity unpinned: the pages print no activations and no trained weights,
-so only their parts are pinned.
+Pins: the building blocks here are checked in tests/test_oracle_pins.py against printed
+values, closed forms, brute force or invariants; composed steps (gdn_prepare,
+update_states) through their parts and the two-ubatches-equal-one invariant; and
+tests/test_oracle_mutants.py plants plausible mistakes that those pins catch.
+projector_trunk, projector and prefill_ubatch as wholes are parity unpinned: the pages
+print no activations and no trained weights, so only their parts are pinned.
 """
 from __future__ import annotations
 
