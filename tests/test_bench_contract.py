@@ -36,3 +36,30 @@ def test_reference_arm_is_silent_on_other_ranks(capsys):
     import bench
     bench.run_reference(argparse.Namespace(workload="r3", steps=1, warmup=0), 1, 2)
     assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_work_from_the_parameter_counts():
+    """The roofline's FLOPs and bytes per 1024-token ubatch, recomputed from the printed
+    parameter counts: 2 T per linear parameter, causal attention over the unmasked pairs of
+    every projector block, 4 d_k d_v per token and value head for the recurrence; bytes are
+    the 16-bit weights once, the residual in, the states read and written, the KV rows and
+    the drafter outputs written."""
+    sys.path.insert(0, ROOT)
+    import bench
+    T = 1024
+    for g in (KI.R3, KI.R2):
+        params = g.param_counts()["total"]
+        w = g.window or T
+        pairs = sum(min(i % w, i) + 1 for i in range(T))          # unmasked (query, key) pairs
+        attn = g.n_blocks * g.n_heads * pairs * 4 * g.head_dim
+        scan = g.n_gdn * g.gdn_n_v * T * 4 * g.gdn_d_k * g.gdn_d_v
+        flops = 2 * T * params + attn + scan
+        state = g.n_gdn * g.gdn_n_v * g.gdn_d_k * g.gdn_d_v * 4
+        kv = 2 * g.n_attn * T * g.attn_n_kv * g.attn_d_h * 2
+        approx_bytes = 2 * params + T * g.hidden * 2 + 2 * state + kv + T * g.n_draft * g.hidden * 2
+        got_f, got_b = bench.algorithmic(g)
+        assert abs(got_f - flops) / flops < 1e-3, (g.name, got_f, flops)
+        # the conv tails and the fp32 gains are the only terms left out here (< 0.5 %)
+        assert 0 <= got_b - approx_bytes < 5e-3 * approx_bytes, (g.name, got_b, approx_bytes)
+    f3, b3 = bench.algorithmic(KI.R3)
+    assert round(f3 / 1e12, 3) == 2.632 and round(b3 / 1e9, 2) == 2.72
