@@ -57,10 +57,14 @@ Readings where the pages are silent (each also stated where it is used):
 
 Pins: the building blocks here are checked in tests/test_oracle_pins.py against printed
 values, closed forms, brute force or invariants; composed steps (gdn_prepare,
-update_states) through their parts and the two-ubatches-equal-one invariant; and
-tests/test_oracle_mutants.py plants plausible mistakes that those pins catch.
-projector_trunk, projector and prefill_ubatch as wholes are parity unpinned: the pages
-print no activations and no trained weights, so only their parts are pinned.
+update_states) through their parts and the two-ubatches-equal-one invariant; the
+projector as a whole (projector_trunk, projector) on one token, where every block has a
+per-vector closed form, chained over three independently drawn blocks in order, and by
+causality and ubatch locality at longer T; prefill_ubatch is projector followed by
+update_states.  tests/test_oracle_mutants.py plants plausible mistakes that those pins
+catch (among them a trunk that repeats its first block or runs the blocks in reverse).
+The pages print no activations and no trained weights, so no pin compares against a
+value of a trained projector.
 """
 from __future__ import annotations
 

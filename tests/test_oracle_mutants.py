@@ -118,7 +118,7 @@ def _chunked_no_decay_mask(S0, k, v, g, beta, chunk=64):
 R_orig = {name: getattr(R, name) for name in (
     "rope_apply", "rope_inv_freq", "causal_conv_silu", "delta_scan_sequential",
     "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked", "hadamard_rotate",
-    "q8_0_quantize", "projector_block")}
+    "q8_0_quantize", "projector_block", "projector_trunk")}
 
 def _hadamard_unnormalised(x):
     # the +-1 Walsh-Hadamard matrix without the 1/sqrt(n) that makes it orthonormal
@@ -163,6 +163,17 @@ def _block_values_from_keys(x, blk, n_heads, head_dim, window):
     return R_orig["projector_block"](x, dict(blk, Wv=blk["Wk"]), n_heads, head_dim, window)
 
 
+def _trunk_block0_repeated(residual, W, geom):
+    # runs the first block as often as there are blocks
+    return R_orig["projector_trunk"](residual, dict(W, blocks=[W["blocks"][0]] * len(W["blocks"])),
+                                     geom)
+
+
+def _trunk_blocks_reversed(residual, W, geom):
+    # runs the blocks last to first
+    return R_orig["projector_trunk"](residual, dict(W, blocks=list(W["blocks"])[::-1]), geom)
+
+
 MUTANTS = [
     ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
     ("rope_apply", _rope_interleaved, [P.test_rope_equals_complex_rotation]),
@@ -183,6 +194,10 @@ MUTANTS = [
     ("projector_block", _block_gate_up_swapped, [P.test_projector_block_single_token_attends_to_itself]),
     ("projector_block", _block_values_from_keys, [P.test_projector_block_single_token_attends_to_itself]),
     ("q4_0_quantize", _q4_0_positive_scale, [P.test_q4_0_closed_form_blocks]),
+    ("projector_trunk", _trunk_block0_repeated,
+     [P.test_projector_chains_its_distinct_blocks_in_order_on_one_token]),
+    ("projector_trunk", _trunk_blocks_reversed,
+     [P.test_projector_chains_its_distinct_blocks_in_order_on_one_token]),
 ]
 
 

@@ -330,6 +330,42 @@ def test_projector_block_single_token_attends_to_itself():
     np.testing.assert_allclose(got2, want, rtol=1e-10, atol=1e-12)
 
 
+def _block_on_one_token(x, blk):
+    # a block on a single token, written per vector: the lone key gets softmax weight 1,
+    # so attention returns Wv u; then the SwiGLU FFN on the renormalised stream
+    u = x / math.sqrt(np.mean(x * x) + R.EPS) * blk["g_attn"]
+    x1 = x + blk["Wo"] @ (blk["Wv"] @ u)
+    u2 = x1 / math.sqrt(np.mean(x1 * x1) + R.EPS) * blk["g_ffn"]
+    gate, up = blk["Wg"] @ u2, blk["Wu"] @ u2
+    return x1 + blk["Wd"] @ (gate / (1.0 + np.exp(-gate)) * up)
+
+
+def test_projector_chains_its_distinct_blocks_in_order_on_one_token():
+    # [KVA] architecture: RMSNorm -> Linear{H -> d} -> block 0 -> block 1 -> block 2 -> RMSNorm
+    # -> heads.  On one token every block has the closed form above; the blocks are drawn
+    # independently, so repeating one block or running them in another order changes z.
+    geom, W = _tiny_f64()
+    assert len(W["blocks"]) == 3
+    for i in range(3):
+        for j in range(i + 1, 3):
+            assert np.abs(W["blocks"][i]["Wd"] - W["blocks"][j]["Wd"]).max() > 1e-3
+    r = RNG.standard_normal(geom.hidden) * 2
+    x = W["W_in"] @ (r / math.sqrt(np.mean(r * r) + R.EPS) * W["g_in"])
+    for blk in W["blocks"]:
+        x = _block_on_one_token(x, blk)
+    z = x / math.sqrt(np.mean(x * x) + R.EPS) * W["g_out"]
+    got_z = R.projector_trunk(r[None], W, geom)[0]
+    np.testing.assert_allclose(got_z, z, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(R.projector(r[None], W, geom)[0], W["W_heads"] @ z,
+                               rtol=1e-10, atol=1e-12)
+    # the order matters at this scale: reversed blocks give a different z
+    xr = W["W_in"] @ (r / math.sqrt(np.mean(r * r) + R.EPS) * W["g_in"])
+    for blk in W["blocks"][::-1]:
+        xr = _block_on_one_token(xr, blk)
+    zr = xr / math.sqrt(np.mean(xr * xr) + R.EPS) * W["g_out"]
+    assert np.abs(zr - z).max() > 1e-6
+
+
 def test_projector_is_causal_and_position_free():
     geom, W = _tiny_f64()
     res = RNG.standard_normal((20, geom.hidden))
