@@ -40,6 +40,7 @@ T_UB = 1024
 CACHE_POS = 32768
 METRIC = "KVA prefill tokens/s on 1 B200 (1024-tok ubatch) and % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LONG_LOOP_S = 2.0  # a loop at least this long reaches the power-capped steady state
 
 
 def parse():
@@ -48,7 +49,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["r3", "r2"], default="r3")
+    ap.add_argument("--workload", choices=["r3", "r2", "state"], default="r3",
+                    help="r3 / r2: kva_prefill_ubatch on 1024-token ubatches; state: "
+                         "kva_update_states alone on 8 sequences x 1024 tokens per call (paged "
+                         "cache, the state-update stress workload)")
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16",
                     help="16-bit operand format of the projector GEMMs (fp32 accumulate)")
     ap.add_argument("--weights", choices=["f16", "q8_0", "q4_0"], default="f16",
@@ -65,6 +69,8 @@ def parse():
 
 
 def geometry(name):
+    if name == "state":
+        return KI.workload(5).geom
     return KI.R3 if name == "r3" else KI.R2
 
 
@@ -272,9 +278,16 @@ def run_ours(args, rank, world, local_rank):
     # launch (all launches then stay on the caller's stream, each timed alone)
     n_prof = max(1, min(args.steps, 50))
     K.kva_profile_enable(h, n_prof * 40 + 64)
+    pclocks = Clocks(local_rank)
+    time.sleep(0.3)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
     for i in range(n_prof):
         step(args.warmup + args.steps + i)
+    p1.record(stream)
     torch.cuda.synchronize()
+    prof_s = p0.elapsed_time(p1) / 1e3
+    pclk = pclocks.stop()
     prof = K.kva_profile_read(h)
     K.kva_profile_enable(h, 0)
     status |= K.kva_get_device_status(h)
@@ -347,9 +360,13 @@ def run_ours(args, rank, world, local_rank):
     heads_ms = gh["ms"] / n_prof
     achieved = heads_flops / (heads_ms / 1e3) / 1e12
     peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    # the step runs in a long loop under the power cap: the sustained tensor peak is the
-    # matching denominator; the burst figure (stricter) stays the headline fraction
+    # The sustained peak is the matching denominator only for a kernel timed inside a loop
+    # that runs for seconds (the power-capped steady state); the profiled pass is shorter,
+    # so its kernel is held to the burst peak.
+    long_prof = prof_s >= LONG_LOOP_S
+    peak_k = peak_s if long_prof else peaks["bf16_tflops"]
     t_roof_s = max(flops / (peak_s * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    long_timed = ms / 1e3 >= LONG_LOOP_S
     line = {
         "metric": METRIC,
         "value": world * args.steps * T_UB / (ms / 1e3),
@@ -384,17 +401,22 @@ def run_ours(args, rank, world, local_rank):
                       + (", state-update epilogue)" if fused and args.weights == "f16" else
                          (f", {args.weights} weights dequantized by converter warps)"
                           if args.weights != "f16" else ")")),
-            "achieved": achieved, "peak": peak_s, "unit": "TFLOP/s", "frac": achieved / peak_s,
-            "peak_kind": f"{src} bf16 sustained (kernel timed inside a long step loop)",
-            "frac_of_burst": achieved / peaks["bf16_tflops"],
+            "achieved": achieved, "peak": peak_k, "unit": "TFLOP/s", "frac": achieved / peak_k,
+            "peak_kind": (f"{src} bf16 sustained (the profiled pass ran {prof_s:.2f} s)" if long_prof
+                          else f"{src} bf16 burst (the profiled pass ran {prof_s:.2f} s, shorter "
+                               f"than the {LONG_LOOP_S:.0f} s a power-capped steady state needs)"),
             "flops_per_launch": heads_flops, "avg_launch_ms": heads_ms,
+            "profiled_steps": n_prof, "profiled_pass_s": prof_s, "profiled_pass_clocks": pclk,
             "traffic": heads_traffic(geom.name, fused) if args.weights == "f16" else None,
         },
         "path_roofline": {
             "flops_alg": flops, "bytes_alg": bytes_, "t_roof_ms": t_roof * 1e3,
             "frac": t_roof / (ms_step / 1e3), "peaks": f"{src}: {peaks['bf16_tflops']} TFLOP/s bf16, "
                                                      f"{peaks['hbm_gbs']} GB/s",
-            "t_roof_sustained_ms": t_roof_s * 1e3, "frac_of_sustained": t_roof_s / (ms_step / 1e3),
+            "timed_region_s": ms / 1e3,
+            # beside a timed region of seconds only (the power-capped steady state)
+            "t_roof_sustained_ms": t_roof_s * 1e3 if long_timed else None,
+            "frac_of_sustained": t_roof_s / (ms_step / 1e3) if long_timed else None,
             "sustained_peak": f"{src}: {peak_s} TFLOP/s bf16 sustained",
         },
         "stages_ms_per_step": {k: v["ms"] / n_prof for k, v in prof.items()},
@@ -405,6 +427,161 @@ def run_ours(args, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(geom, seed, tokens=512)
+    print(json.dumps(line), flush=True)
+    multi.finish()
+
+
+# ----------------------------------------------------------------------------- state updates alone
+STATE_SEQ = 8
+
+
+def state_algorithmic(geom, n_seq, T):
+    """Bytes one kva_update_states call must move (HBM-bound; see the design notes): the
+    mixer inputs read once, every DeltaNet state read and written, the conv tails read and
+    written, the K/V rows written; FLOPs of the recurrence 4*d_k*d_v per token per v head."""
+    mix = n_seq * T * geom.n_mix * 2
+    state = n_seq * geom.n_gdn * geom.gdn_n_v * geom.gdn_d_k * geom.gdn_d_v * 4
+    tail = n_seq * geom.n_gdn * (geom.conv_k - 1) * geom.gdn_conv_ch * 2
+    kv = n_seq * T * geom.n_attn * 2 * geom.attn_n_kv * geom.attn_d_h * 2
+    flops = n_seq * T * geom.n_gdn * geom.gdn_n_v * 4 * geom.gdn_d_k * geom.gdn_d_v
+    return flops, mix + 2 * state + 2 * tail + kv, {"mixer": mix, "state_rw": 2 * state,
+                                                    "tail_rw": 2 * tail, "kv_written": kv}
+
+
+def stage_bytes(geom, n_seq, T):
+    """Algorithmic bytes of each stage kind of kva_update_states, per call."""
+    gw = geom.gdn_width
+    g_mix = n_seq * T * geom.n_gdn * gw * 2
+    state = n_seq * geom.n_gdn * geom.gdn_n_v * geom.gdn_d_k * geom.gdn_d_v * 4
+    tail = n_seq * geom.n_gdn * (geom.conv_k - 1) * geom.gdn_conv_ch * 2
+    kv = n_seq * T * geom.n_attn * 2 * geom.attn_n_kv * geom.attn_d_h * 2
+    return {"gdn_prepare": g_mix + tail, "gdn_scan": 2 * state, "gdn_tail": 2 * tail,
+            "kv_write": 2 * kv}
+
+
+def run_state(args, rank, world, local_rank):
+    """The state-update stress workload: precomputed bf16 mixer inputs N(0,1) of 24
+    gated-DeltaNet + 8 attention layers for 8 independent sequences of 4096 tokens, run as
+    4 calls of 8 x 1024 tokens; DeltaNet states N(0, 0.1) carried; paged KV cache (pages of
+    256 tokens, shuffled page table).  One step = one call."""
+    import hybrid_deltanet_attention_kva_b200 as K
+    from hybrid_deltanet_attention_kva_b200 import multi
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    multi.init("nccl", timeout_s=120, device=dev)
+    wl = KI.workload(5)
+    geom, T, n_seq = wl.geom, wl.ubatches[0], wl.n_seq
+    n_ub = len(wl.ubatches)
+    seed = multi.rank_seed(wl.seed, rank)
+    mixers = [KI.make_mixer_inputs(geom, n_seq, T, seed + 10 + u, device="cuda") for u in range(n_ub)]
+    P = KI.make_layer_params(geom, seed + 1, device="cuda")
+    st = KI.make_states(geom, n_seq, seed + 2, std=wl.state_std, device="cuda")
+    pps = wl.max_pos // wl.page_size
+    pt = KI.make_page_table(n_seq, pps, seed + 3).to(dev)
+    shape = (n_seq * pps, geom.attn_n_kv, wl.page_size, geom.attn_d_h)
+    kc = [torch.zeros(shape, dtype=torch.bfloat16, device=dev) for _ in range(geom.n_attn)]
+    vc = [torch.zeros_like(k) for k in kc]
+    kv = K.KvCache(kc, vc, page_table=pt, page_size=wl.page_size, n_pages=n_seq * pps)
+    Wt = K.Weights(layer=P)
+    S, tail = st["state"], st["conv_tail"]
+    h = K.kva_init(K.make_dims(geom, T, n_seq, dtype=torch.bfloat16))
+    stream = torch.cuda.current_stream()
+
+    def step(i, mix=None):
+        u = i % n_ub
+        K.kva_update_states(h, mixers[u] if mix is None else mix, [u * T] * n_seq, Wt, S, tail, kv,
+                            stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert K.kva_get_device_status(h) == 0, "device status set during warm-up"
+    K.kva_profile_read(h)
+    clocks = Clocks(local_rank)
+    time.sleep(0.3)
+    multi.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    multi.barrier()
+    clk = clocks.stop()
+    ms = multi.max_over_ranks(e0.elapsed_time(e1), dev)
+    launches = int(sum(v["launches"] for v in K.kva_profile_read(h).values()))
+    status = K.kva_get_device_status(h)
+
+    n_prof = max(1, min(args.steps, 50))
+    K.kva_profile_enable(h, n_prof * 16 + 64)
+    for i in range(n_prof):
+        step(i)
+    torch.cuda.synchronize()
+    prof = K.kva_profile_read(h)
+    K.kva_profile_enable(h, 0)
+    status |= K.kva_get_device_status(h)
+
+    # end to end: each call's mixer inputs copied from pinned host memory inside the timed
+    # region, one state matrix read back
+    e2e = None
+    if not args.no_e2e:
+        host_mix = mixers[0].cpu().pin_memory()
+        dmix = torch.empty_like(mixers[0])
+        out_host = torch.empty(geom.gdn_d_v, geom.gdn_d_k).pin_memory()
+        steps_e2e = 5
+        torch.cuda.synchronize()
+        multi.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(steps_e2e):
+            dmix.copy_(host_mix, non_blocking=True)
+            step(i, dmix)
+            out_host.copy_(S[0, 0, 0], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        multi.barrier()
+        ems = multi.max_over_ranks(f0.elapsed_time(f1), dev)
+        e2e = {"value": world * steps_e2e * n_seq * T / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": host_mix.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 4,
+               "steps": steps_e2e,
+               "what": "kva_update_states through the binding; the call's mixer inputs copied from "
+                       "pinned host memory each step, one DeltaNet state matrix copied back"}
+    K.kva_free(h)
+    if rank != 0:
+        multi.finish()
+        return
+
+    flops, bytes_, parts = state_algorithmic(geom, n_seq, T)
+    peaks, src = load_peaks()
+    ms_step = ms / args.steps
+    t_roof = bytes_ / (peaks["hbm_gbs"] * 1e9)
+    sb = stage_bytes(geom, n_seq, T)
+    stages = {k: v["ms"] / n_prof for k, v in prof.items()}
+    top = max(sb, key=lambda k: stages.get(k, 0.0))
+    ach = sb[top] / (stages[top] / 1e3) / 1e9
+    line = {
+        "metric": "KVA state-update tokens/s on 1 B200 (8 sequences x 1024-token ubatch) and % of HBM roofline",
+        "value": world * args.steps * n_seq * T / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (bf16 N(0,1) mixer inputs, states N(0,0.1), seeded)",
+        "config": {"workload": "state updates alone (no projector): 24 gated-DeltaNet + 8 attention "
+                               "layers, 8 sequences x 4096 tokens as 4 calls of 8 x 1024, paged KV "
+                               "cache (256-token pages, shuffled page table)",
+                   "tokens_per_step": n_seq * T, "parallelism": f"independent sequences per GPU x{world}",
+                   "l2": "4.3 GB of mixer inputs per call exceed L2"},
+        "roofline": {"bound": "hbm", "kernel": top, "achieved": ach, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                     "bytes_per_launch_alg": sb[top], "avg_ms_per_step": stages[top],
+                     "peak_kind": f"{src} HBM copy bandwidth"},
+        "path_roofline": {"flops_alg": flops, "bytes_alg": bytes_, "bytes_parts": parts,
+                          "t_roof_ms": t_roof * 1e3, "frac": t_roof / (ms_step / 1e3),
+                          "peaks": f"{src}: {peaks['hbm_gbs']} GB/s"},
+        "stages_ms_per_step": stages,
+        "gpu_launches": launches, "device_status": status, "clocks": clk, "e2e": e2e,
+    }
     print(json.dumps(line), flush=True)
     multi.finish()
 
@@ -597,6 +774,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "state":
+        run_state(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

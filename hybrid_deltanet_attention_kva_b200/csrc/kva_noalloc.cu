@@ -34,27 +34,36 @@ static_assert(kKBytes % 256 == 0 && kVBytes % 256 == 0 && kGBytes % 256 == 0,
 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+// Device status bits (KVA_DEV_*) of the calls: a pipeline wait inside the scan that gave
+// up sets KVA_DEV_WAIT_TIMEOUT here.  Read and cleared by kva_gdn_layer_update_noalloc_status.
+static __device__ int g_status;
 
-// Device address of g_scratch per device.  In host code the symbol's name is
-// only a host-side stand-in, so the address must come from the runtime.
+// Device addresses of g_scratch and g_status per device.  In host code the symbols' names
+// are only host-side stand-ins, so the addresses must come from the runtime.  They stay
+// valid for the life of the device's primary context (a cudaDeviceReset invalidates them).
 constexpr int kMaxDevices = 64;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+int* g_status_ptr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mu;
 
-int scratch_for_current_device(void** out) {
+int symbols_for_current_device(void** scratch, int** status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KVA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p ||
+        cudaGetSymbolAddress(&q, g_status) != cudaSuccess || !q) {
       cudaGetLastError();
       return KVA_ERR_CUDA;
     }
+    g_status_ptr[dev] = static_cast<int*>(q);
     g_scratch_ptr[dev] = p;
   }
-  *out = g_scratch_ptr[dev];
+  *scratch = g_scratch_ptr[dev];
+  *status = g_status_ptr[dev];
   return KVA_OK;
 }
 
@@ -82,7 +91,8 @@ extern "C" int kva_gdn_layer_update_noalloc(const void* mixer_in, int64_t mixer_
   if (T == 0) return KVA_OK;
 
   void* base = nullptr;
-  int e = scratch_for_current_device(&base);
+  int* status = nullptr;
+  int e = symbols_for_current_device(&base, &status);
   if (e) return e;
   unsigned char* b = static_cast<unsigned char*>(base);
 
@@ -111,8 +121,29 @@ extern "C" int kva_gdn_layer_update_noalloc(const void* mixer_in, int64_t mixer_
     kva::gdn_chunk_split(b + kKBytes + kVBytes + kGBytes, 1, 1, n_v, T, &g.b1buf, &g.scbuf);
   }
   g.eps = eps;
+  g.err = status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((e = kva::launch_gdn_prepare(g, s))) return e;
   if ((e = kva::launch_gdn_tail(g, s))) return e;
   return kva::launch_gdn_scan(g, s);
+}
+
+extern "C" int kva_gdn_layer_update_noalloc_status(void* stream, int32_t* status) {
+  if (!status) return KVA_ERR_INVALID_ARG;
+  *status = 0;
+  void* base = nullptr;
+  int* word = nullptr;
+  int e = symbols_for_current_device(&base, &word);
+  if (e) return e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyAsync(&v, word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(word, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return KVA_ERR_CUDA;
+  }
+  *status = v;
+  return v ? KVA_ERR_DEVICE : KVA_OK;
 }

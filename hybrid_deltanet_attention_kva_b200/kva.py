@@ -123,6 +123,7 @@ def _load() -> C.CDLL:
         "kva_op_attention": (I32, [I32, P, I64, P, I64, I32, I32, I32, P]),
         "kva_op_gdn_scan": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "kva_gdn_layer_update_noalloc": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, F32, P]),
+        "kva_gdn_layer_update_noalloc_status": (I32, [P, C.POINTER(I32)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -137,7 +138,7 @@ EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update
             "kva_profile_enable", "kva_profile_read",
             "kva_op_rmsnorm", "kva_op_gemm", "kva_op_gemm_q8_0", "kva_op_gemm_q4_0", "kva_op_attention",
             "kva_op_gdn_scan",
-            "kva_gdn_layer_update_noalloc")
+            "kva_gdn_layer_update_noalloc", "kva_gdn_layer_update_noalloc_status")
 
 
 def lib() -> C.CDLL:
@@ -394,8 +395,33 @@ def kva_gdn_layer_update_noalloc(mixer_in: torch.Tensor, n_k: int, n_v: int, d: 
                                  state: torch.Tensor, conv_state: torch.Tensor, eps: float = 1e-6,
                                  stream=None) -> None:
     """One gated-DeltaNet layer's state update without any device allocation (see
-    include/kva_ops.h): for callers that may not allocate device memory."""
+    include/kva_ops.h): for callers that may not allocate device memory.
+
+    The entry point reads mixer_in and conv_state as bf16 and state as fp32, so other
+    formats or sizes are refused here before anything reaches the device."""
     T, ld = mixer_in.shape
+    C = 2 * n_k * d + n_v * d
+    if mixer_in.dtype != torch.bfloat16 or conv_state.dtype != torch.bfloat16:
+        raise ValueError("mixer_in and conv_state must be bf16")
+    if state.dtype != torch.float32 or any(t.dtype != torch.float32 for t in (conv_w, A_log, dt_bias)):
+        raise ValueError("state, conv_w, A_log and dt_bias must be fp32")
+    if mixer_in.stride(1) != 1 or ld < C + 2 * n_v:
+        raise ValueError(f"mixer_in must be row-major with at least {C + 2 * n_v} columns")
+    ld = mixer_in.stride(0)
+    for t, n, what in ((state, n_v * d * d, "state"), (conv_state, 3 * C, "conv_state"),
+                       (conv_w, 4 * C, "conv_w"), (A_log, n_v, "A_log"), (dt_bias, n_v, "dt_bias")):
+        if t.numel() != n or not t.is_contiguous():
+            raise ValueError(f"{what} must be a contiguous tensor of {n} values, got {tuple(t.shape)}")
     _check(_lib.kva_gdn_layer_update_noalloc(
         _ptr(mixer_in), ld, T, n_k, n_v, d, _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(state),
         _ptr(conv_state), float(eps), _stream(stream)), "kva_gdn_layer_update_noalloc")
+
+
+def kva_gdn_layer_update_noalloc_status(stream=None) -> int:
+    """Device status bits of kva_gdn_layer_update_noalloc calls since the last read (0 =
+    clean); synchronises the stream and clears the bits."""
+    st = C.c_int32(0)
+    rc = _lib.kva_gdn_layer_update_noalloc_status(_stream(stream), C.byref(st))
+    if rc not in (KVA_OK, KVA_ERR_DEVICE):
+        _check(rc, "kva_gdn_layer_update_noalloc_status")
+    return st.value

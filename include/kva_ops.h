@@ -116,16 +116,27 @@ int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state,
  *   mixer_in   bf16 [T, mixer_ld]: this layer's columns [q | k | v | a | b] from column 0
  *   conv_w     fp32 [C, 4], A_log / dt_bias fp32 [n_v]
  *   state      fp32 [n_v, d, d], conv_state bf16 [3, C]: read and updated in place
- * Sizes beyond the KVA_NOALLOC_* limits return KVA_ERR_TOO_LARGE before any launch.
- * The first call on a device looks up the array's device address (once per device,
- * with that device current); make that first call before any stream capture.
- * All calls share the one array: calls whose work overlaps on the GPU (different
- * streams, or different host threads) race on it and must be serialised by the
- * caller.  Returns kva_status. */
+ * mixer_in and conv_state are always bf16 (this call has no handle that would name
+ * another format).  Sizes beyond the KVA_NOALLOC_* limits return KVA_ERR_TOO_LARGE
+ * before any launch.  The first call on a device looks up the device addresses of the
+ * array and of a status word beside it (once per device, with that device current);
+ * make that first call before any stream capture.  The addresses are kept for the life
+ * of the device's primary context: do not use this entry point across a
+ * cudaDeviceReset.  All calls share the one array: calls whose work overlaps on the
+ * GPU (different streams, or different host threads) race on it and must be
+ * serialised by the caller.  A pipeline wait that gave up inside the scan sets
+ * KVA_DEV_WAIT_TIMEOUT in the status word (read it with
+ * kva_gdn_layer_update_noalloc_status).  Returns kva_status. */
 int kva_gdn_layer_update_noalloc(const void* mixer_in, int64_t mixer_ld, int32_t T, int32_t n_k,
                                  int32_t n_v, int32_t d, const float* conv_w, const float* A_log,
                                  const float* dt_bias, float* state, void* conv_state, float eps,
                                  void* stream);
+
+/* Device status bits (KVA_DEV_*) that kva_gdn_layer_update_noalloc calls on the current
+ * device have set since the last read.  Synchronises `stream`, stores the bits in *status
+ * (0 = clean), clears them, and returns KVA_ERR_DEVICE when bits were set.  Allocates
+ * nothing. */
+int kva_gdn_layer_update_noalloc_status(void* stream, int32_t* status);
 
 #ifdef __cplusplus
 }

@@ -171,7 +171,7 @@ def _to_dtype(W, dt):
 
 
 def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outliers=8,
-                 dt=torch.float16):
+                 dt=torch.float16, mixer=True):
     """Run consecutive ubatches of one sequence on the GPU; return GPU results + inputs."""
     W = _to_dtype(KI.make_projector_weights(geom, seed), dt)
     P = KI.make_layer_params(geom, seed + 1)
@@ -188,7 +188,7 @@ def _run_prefill(K, geom, ubatches, residual_dtype, seed, draft=False, n_outlier
     pos = 0
     try:
         for T in ubatches:
-            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda")
+            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda") if mixer else None
             do = (torch.empty(T, geom.n_draft_cols, dtype=dt, device="cuda")
                   if draft and geom.n_draft else None)
             K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wg, S, tail, caches.c, pos,
@@ -414,6 +414,78 @@ def test_prefill_full_size_sampled(K, cfg, dt):
             assert m.get("max_excess_over_rms", m["max_over_rms"]) <= tol_out, (name, m)
 
 
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_prefill_benched_configuration_every_layer(K, cfg):
+    """The call exactly as the benchmark makes it: fp16 operands, drafter outputs on and no
+    mixer copy (mixer_out = NULL changes the heads epilogue's control flow), r2 T=1024 and
+    r3 1024 + 512 with state, conv tail and caches carried.  Every DeltaNet layer's final
+    state and conv tail and every written row of every attention cache are compared with
+    the float64 oracle; the drafter outputs at 16 sampled rows per ubatch."""
+    import json
+    wl = KI.workload(cfg)
+    geom = wl.geom
+    dt = torch.float16
+    r = _run_prefill(K, geom, wl.ubatches, wl.residual_dtype, wl.seed, draft=True, dt=dt,
+                     mixer=False)
+    tol_out, tol_state = TOLS[dt]
+    Wh = r["W"].pop("W_heads")
+    Wn = R.weights_to_f64(r["W"])
+    Pn = {k: f64(v) for k, v in r["P"].items()}
+    res = f64(r["res"])
+    offs = geom.layer_offsets
+    zs, pos = [], 0
+    for T in wl.ubatches:
+        zs.append(R.projector_trunk(res[pos:pos + T], Wn, geom))
+        pos += T
+    metrics = {}
+    # drafter outputs at sampled rows of every ubatch
+    Wd = f64(Wh[geom.n_mix:geom.n_total])
+    for i, z in enumerate(zs):
+        rows = np.unique(np.linspace(0, z.shape[0] - 1, 16).astype(int))
+        metrics[f"drafter_{i}"] = _err(f64(r["drafts"][i])[rows], R.projector_heads(z[rows], Wd))
+    del Wd
+    # every gated-DeltaNet layer, carried across the ubatches in order
+    S_o = f64(r["st"]["state"][0])
+    tail_o = f64(r["st"]["conv_tail"][0])
+    state_rel = []
+    for gi, li in enumerate(geom.gdn_layers()):
+        Wl = f64(Wh[offs[li]:offs[li] + geom.gdn_width])
+        for z in zs:
+            pr = R.gdn_prepare(R.projector_heads(z, Wl), tail_o[gi], Pn["conv_w"][gi],
+                               Pn["A_log"][gi], Pn["dt_bias"][gi], geom)
+            tail_o[gi] = pr["tail"]
+            S_o[gi] = R.delta_scan_chunked(S_o[gi], pr["k"], pr["v"], pr["g"], pr["beta"])
+        num = np.sqrt(np.sum((f64(r["S"][gi]) - S_o[gi]) ** 2, axis=(-2, -1)))
+        den = np.sqrt(np.sum(S_o[gi] ** 2, axis=(-2, -1)))
+        state_rel.append(float((num / den).max()))
+        metrics[f"tail_{gi}"] = _err(r["tail"][gi], tail_o[gi])
+    metrics["state_rel_frob_max_per_layer"] = state_rel
+    # every attention layer, every written cache row
+    kc, vc, _, _ = r["caches"].oracle_views(0)
+    for ai, li in enumerate(geom.attn_layers()):
+        Wl = f64(Wh[offs[li]:offs[li] + geom.attn_width])
+        pos = 0
+        for z in zs:
+            T = z.shape[0]
+            Kx, Vx = R.attn_kv(R.projector_heads(z, Wl), Pn["k_norm_g"][ai], pos, geom)
+            kc[ai][:, pos:pos + T] = Kx.transpose(1, 0, 2)
+            vc[ai][:, pos:pos + T] = Vx.transpose(1, 0, 2)
+            pos += T
+        gk, gv = f64(r["caches"].k[ai][0]), f64(r["caches"].v[ai][0])
+        written = kc[ai] != SENT
+        np.testing.assert_array_equal(gk == SENT, ~written)
+        np.testing.assert_array_equal(gv == SENT, ~written)
+        assert written.sum() == geom.attn_n_kv * sum(wl.ubatches) * geom.attn_d_h
+        metrics[f"K_cache_{ai}"] = _err(gk[written], kc[ai][written], elem=BF16_ELEM)
+        metrics[f"V_cache_{ai}"] = _err(gv[written], vc[ai][written], elem=BF16_ELEM)
+    print("PARITY_METRICS_BENCHED", cfg, json.dumps(metrics))
+    for gi in range(geom.n_gdn):
+        assert state_rel[gi] <= tol_state, (f"state layer {gi}", state_rel[gi])
+    for name, m in metrics.items():
+        if isinstance(m, dict):
+            assert m.get("max_excess_over_rms", m["max_over_rms"]) <= tol_out, (name, m)
+
+
 # ------------------------------------------------------------------ quantized projector weights
 def _q8_projector(W, fmt="q8_0"):
     """Every projector matrix as q8_0 or q4_0 (the oracle's quantizer): (GPU weight dict with
@@ -465,7 +537,7 @@ def test_prefill_q8_0_projector_weights(K, geom, draft, fmt):
         Wt = K.Weights(proj=Wg, layer={k: v.cuda() for k, v in P.items()})
         pos = 0
         for T in splits:
-            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda")
+            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda") if mixer else None
             do = torch.empty(T, geom.n_draft_cols, dtype=dt, device="cuda") if draft else None
             K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wt, S, tail, caches.c, pos, draft_out=do,
                                  mixer_out=mo)

@@ -5,16 +5,20 @@ cache pool (or a plugin whose host program owns device memory) cannot create a
 kva_handle, because that calls cudaMalloc.  The allocation-free entry point keeps
 its scratch in a fixed array inside the library instead.  This test checks that it
 produces what the handle-based kva_update_states produces for the same layer, on
-two calls in a row (the second continues from the first call's state and conv tail),
-within the tolerances the other parity tests use.  It sits in a file collected last
-so a run that stops at the first failure has already run every other test.
+two calls in a row (the second continues from the first call's state and conv tail).
+Both run the same kernels on the same bf16 inputs with deterministic reductions, so the
+states and conv tails must be bitwise equal: a tolerance could hide a wrong offset into
+the shared scratch.  T = 256 is the largest ubatch the fixed scratch holds, and the r3
+layer (n_k * d = 2048, n_v * d = 6144) fills the key and value regions to their limits.
+The device status word of the entry point must stay clean after every call.  It sits in
+a file collected last so a run that stops at the first failure has already run every
+other test.
 """
 import numpy as np
 import pytest
 import torch
 
 import kva_inputs as KI
-from tests.parity import assert_state_close, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +30,7 @@ def K():
     return K
 
 
-@pytest.mark.parametrize("geom_name,T", [("r3", 200), ("tiny", 97)])
+@pytest.mark.parametrize("geom_name,T", [("r3", 200), ("r3", 256), ("tiny", 97), ("tiny", 256)])
 def test_noalloc_matches_handle_path_two_calls(K, geom_name, T):
     base = KI.GEOMETRIES[geom_name]
     # a stack with one gated-DeltaNet layer, so the handle path updates exactly that layer
@@ -52,7 +56,9 @@ def test_noalloc_matches_handle_path_two_calls(K, geom_name, T):
                                            conv_w, A_log, dt_bias, S_n, tail_n, geom.norm_eps)
             torch.cuda.synchronize()
             assert K.kva_get_device_status(h) == 0
-            assert_state_close(S_n, f64(S_h[0, 0]), what=f"no-alloc state, call {call}")
+            assert K.kva_gdn_layer_update_noalloc_status() == 0
+            assert torch.equal(S_n, S_h[0, 0]), (
+                f"state differs after call {call}: max |diff| {(S_n - S_h[0, 0]).abs().max().item()}")
             assert torch.equal(tail_n, tail_h[0, 0]), f"conv tail differs after call {call}"
     finally:
         K.kva_free(h)
@@ -70,3 +76,20 @@ def test_noalloc_refuses_sizes_beyond_its_scratch(K):
                                        P["A_log"][0].cuda(), P["dt_bias"][0].cuda(), S, tail)
     assert ei.value.status == K.KVA_ERR_TOO_LARGE
     assert bool((S == 0).all())                                 # nothing was launched
+
+
+def test_noalloc_binding_refuses_formats_it_would_misread(K):
+    geom = KI.with_changes(KI.TINY, layer_types=(KI.GDN,), n_draft=0)
+    P = KI.make_layer_params(geom, 1)
+    args = [P["conv_w"][0].cuda(), P["A_log"][0].cuda(), P["dt_bias"][0].cuda()]
+    d, n_k, n_v = geom.gdn_d_k, geom.gdn_n_k, geom.gdn_n_v
+    mix = torch.zeros(8, geom.gdn_width, dtype=torch.bfloat16, device="cuda")
+    S = torch.zeros(n_v, d, d, device="cuda")
+    tail = torch.zeros(3, geom.gdn_conv_ch, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):                             # an fp16 mixer would be read as bf16
+        K.kva_gdn_layer_update_noalloc(mix.half(), n_k, n_v, d, *args, S, tail)
+    with pytest.raises(ValueError):                             # a state one head short
+        K.kva_gdn_layer_update_noalloc(mix, n_k, n_v, d, *args, S[1:].contiguous(), tail)
+    with pytest.raises(ValueError):                             # a conv tail of 2 rows
+        K.kva_gdn_layer_update_noalloc(mix, n_k, n_v, d, *args, S, tail[:2].contiguous())
+    assert bool((S == 0).all())
