@@ -69,6 +69,7 @@ class Geometry:
     conv_k: int = 4
     rope_theta: float = 1.0e7
     norm_eps: float = 1.0e-6
+    attn_n_q: int = 24     # query heads of an attention layer (exact last-token pass only)
 
     # ---- derived sizes (bookkeeping only) ----
     @property
@@ -118,6 +119,14 @@ class Geometry:
     def n_total(self) -> int:
         return self.n_mix + self.n_draft_cols
 
+    def last_width(self, i: int) -> int:
+        """Columns of layer i's exact last-token inputs: the mixer columns of the layer, then
+        the output gate z (n_v * d_v) of a gated-DeltaNet layer, or q and its gate
+        (2 * n_q * d_h) of an attention layer."""
+        if self.layer_types[i] == GDN:
+            return self.gdn_width + self.gdn_n_v * self.gdn_d_v
+        return self.attn_width + 2 * self.attn_n_q * self.attn_d_h
+
     def gdn_layers(self) -> List[int]:
         return [i for i, t in enumerate(self.layer_types) if t == GDN]
 
@@ -153,7 +162,7 @@ R3 = Geometry(name="r3", hidden=5120, d_model=3072, n_heads=24, ffn=8448,
 TINY = Geometry(name="tiny", hidden=512, d_model=256, n_heads=2, ffn=704,
                 layer_types=(GDN, GDN, ATTN), gdn_n_k=2, gdn_n_v=4, gdn_d_k=64,
                 gdn_d_v=64, attn_n_kv=1, attn_d_h=128, rope_dims=32, window=0,
-                n_draft=0)
+                n_draft=0, attn_n_q=2)
 
 GEOMETRIES = {"tiny": TINY, "r2": R2, "r3": R3}
 
@@ -280,6 +289,26 @@ def make_mixer_inputs(geom: Geometry, n_seq: int, T: int, seed: int,
     """Precomputed mixer inputs bf16 [n_seq, T, n_mix], N(0,1)."""
     dr = Draw(seed, device)
     return dr.normal((n_seq, T, geom.n_mix), 1.0, dtype=torch.bfloat16)
+
+
+def make_last_token_inputs(geom: Geometry, layer: int, n_seq: int, seed: int,
+                           device: str = "cpu") -> torch.Tensor:
+    """Exact inputs of one late layer for the last token of n_seq sequences, bf16
+    [n_seq, last_width(layer)], N(0,1)."""
+    dr = Draw(seed, device)
+    return dr.normal((n_seq, geom.last_width(layer)), 1.0, dtype=torch.bfloat16)
+
+
+def make_last_token_params(geom: Geometry, seed: int, random_gains: bool = False,
+                           device: str = "cpu") -> Dict[str, torch.Tensor]:
+    """Gains of the exact last-token pass: the gated RMSNorm weight of each gated-DeltaNet
+    layer [n_gdn, d_v] and the q RMSNorm gain of each attention layer [n_attn, d_h]; 1, or
+    U(0.5, 1.5) with random_gains."""
+    dr = Draw(seed, device)
+    shapes = {"gdn_norm_w": (geom.n_gdn, geom.gdn_d_v), "q_norm_g": (geom.n_attn, geom.attn_d_h)}
+    if random_gains:
+        return {k: dr.uniform(v, 0.5, 1.5) for k, v in shapes.items()}
+    return {k: torch.ones(v, dtype=torch.float32, device=device) for k, v in shapes.items()}
 
 
 def make_page_table(n_seq: int, pages_per_seq: int, seed: int,

@@ -48,6 +48,17 @@ Readings where the pages are silent (each also stated where it is used):
   R16 q8_0 projector weights ([KVA] "Projector quantization"): each projector matrix
       W [N, K] as q8_0 blocks (R15's block rule) of 32 consecutive input values of a
       row; a weight is fp16(d) * code.
+  R18 exact last-token pass ([KVA] "What the hell?"): when it follows, the approximated
+      path covers tokens 0..T-2 of the ubatch (the projector is causal, so its predictions
+      for them do not depend on token T-1) and the last token enters each late layer's
+      state / cache through that layer's exact inputs, one layer at a time (each layer's
+      inputs come from the base model's projections of the previous layer's output).
+  R19 attention decode: q RMSNorm per head (gain q_norm) and RoPE at the token's
+      position like k; scale 1/sqrt(d_h); the output multiplied by sigmoid(gate).
+  R20 gated-DeltaNet decode readout: o_h = S_h q_hat (no extra scale; the gated RMSNorm
+      that follows makes a constant factor irrelevant), then RMSNorm(o_h) * w * silu(z_h).
+  R21 grouped queries: query head h reads KV head h // (n_q / n_kv) (24 over 4 in the
+      base model, [MLA] "What this is").
   R17 q4_0 projector weights (the same section's q4_0 row): blocks of 32 consecutive
       input values of a row; m = the block's value of largest magnitude (the first one
       on a tie), d = m / -8 (so m itself is code 0), code q = min(15, floor(x / d + 8.5))
@@ -472,6 +483,88 @@ def prefill_ubatch(residual: np.ndarray, W: Dict, geom, params: Dict, state, tai
     state, tail = update_states(Y, geom, params, state, tail, kcache, vcache, pos0,
                                 scan=scan, debug=debug, kv_rotate=kv_rotate)
     return Y, state, tail
+
+
+# ---------------------------------------------------------------------------
+# exact last-token pass ([KVA] "What the hell?": after the cheap state updates the engine
+# runs the last token of each ubatch through the late layers exactly, on top of the
+# approximated context).  One late layer's token mixer, given that layer's exact inputs
+# for the token (R18-R21); the projections around it belong to the base model.
+# ---------------------------------------------------------------------------
+def gdn_readout(S: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """o_h = S_h q_(h // (n_v / n_k)) per v head (R20): S [n_v, d_v, d_k], q [n_k, d_k]
+    -> [n_v, d_v].  The state read with a query, as the rank-1 writes v k^T store v at k."""
+    n_v = S.shape[0]
+    kmap = np.arange(n_v) // (n_v // q.shape[0])
+    return np.einsum("hij,hj->hi", S, q[kmap])
+
+
+def gated_rmsnorm(o: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = EPS) -> np.ndarray:
+    """Output gate of a gated-DeltaNet layer (R20): per v head RMSNorm(o_h) * w * silu(z_h).
+    o, z [n_v, d_v], w [d_v]."""
+    return rmsnorm(o, w, eps) * silu(np.asarray(z, dtype=np.float64))
+
+
+def gdn_decode(x: np.ndarray, z: np.ndarray, tail: np.ndarray, S: np.ndarray,
+               conv_w: np.ndarray, A_log: np.ndarray, dt_bias: np.ndarray,
+               norm_w: np.ndarray, geom):
+    """One token through a gated-DeltaNet layer's mixer (R18, R20).
+
+    x [gdn_width] the token's exact [q | k | v | a | b] (R4), z [n_v * d_v] its output gate
+    input.  The conv, norms, gates and state update are the prefill's own steps on a
+    one-token ubatch; then the state is read with q and the gated RMSNorm applied.
+    Returns (o [n_v * d_v], new state [n_v, d_v, d_k], new tail [K-1, C])."""
+    pr = gdn_prepare(np.asarray(x, dtype=np.float64)[None], tail, conv_w, A_log, dt_bias, geom)
+    S1 = delta_scan_sequential(S, pr["k"], pr["v"], pr["g"], pr["beta"])
+    o = gdn_readout(S1, pr["q"][0])
+    nv, dv = geom.gdn_n_v, geom.gdn_d_v
+    return gated_rmsnorm(o, np.asarray(z, dtype=np.float64).reshape(nv, dv), norm_w).reshape(-1), \
+        S1, pr["tail"]
+
+
+def gqa_decode_attention(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray) -> np.ndarray:
+    """Softmax attention of one query per head over n keys with grouped KV heads (R21):
+    q [n_q, d], Kc, Vc [n, n_kv, d]; query head h reads KV head h // (n_q / n_kv); scale
+    1/sqrt(d).  Returns [n_q, d]."""
+    n_q, d = q.shape
+    kmap = np.arange(n_q) // (n_q // Kc.shape[1])
+    out = np.empty((n_q, d))
+    for h in range(n_q):
+        s = Kc[:, kmap[h]] @ q[h] / math.sqrt(d)
+        p = np.exp(s - s.max())
+        out[h] = (p / p.sum()) @ Vc[:, kmap[h]]
+    return out
+
+
+def attn_decode(x: np.ndarray, k_gain: np.ndarray, q_gain: np.ndarray, kcache: np.ndarray,
+                vcache: np.ndarray, pos: int, geom, page_table: Optional[np.ndarray] = None,
+                page_size: int = 0) -> np.ndarray:
+    """One token at position pos through a full-attention layer's mixer (R18, R19, R21).
+
+    x [last_width] the token's exact [k | v | q | gate]: k and v as in the mixer (k RMSNorm
+    + RoPE, v as is) are written to the cache at pos (in place, like update_states); q gets
+    its own RMSNorm (gain q_gain) and the same RoPE at pos; the query attends to the
+    sequence's cache rows 0..pos (those the approximated path wrote and its own); the
+    result is multiplied by sigmoid(gate).  Returns o [n_q * d_h]."""
+    x = np.asarray(x, dtype=np.float64)
+    n_kv, d, n_q = geom.attn_n_kv, geom.attn_d_h, geom.attn_n_q
+    w = geom.attn_width
+    Kn, Vn = attn_kv(x[None, :w], k_gain, pos, geom)
+    slots = kv_slots(0, pos + 1, page_table, page_size)
+    if page_table is None:
+        kcache[:, pos, :] = Kn[0]
+        vcache[:, pos, :] = Vn[0]
+        Kc = kcache[:, slots, :].transpose(1, 0, 2)
+        Vc = vcache[:, slots, :].transpose(1, 0, 2)
+    else:
+        kcache[slots[-1] // page_size, :, slots[-1] % page_size, :] = Kn[0]
+        vcache[slots[-1] // page_size, :, slots[-1] % page_size, :] = Vn[0]
+        Kc = kcache[slots // page_size, :, slots % page_size, :]
+        Vc = vcache[slots // page_size, :, slots % page_size, :]
+    q = rmsnorm(x[w:w + n_q * d].reshape(n_q, d), q_gain)
+    q = rope_apply(q[None], np.array([pos]), geom.rope_dims, geom.rope_theta)[0]
+    gate = x[w + n_q * d:w + 2 * n_q * d].reshape(n_q, d)
+    return (gqa_decode_attention(q, Kc, Vc) * sigmoid(gate)).reshape(-1)
 
 
 def weights_to_f64(W) -> Dict:

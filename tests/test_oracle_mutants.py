@@ -118,7 +118,8 @@ def _chunked_no_decay_mask(S0, k, v, g, beta, chunk=64):
 R_orig = {name: getattr(R, name) for name in (
     "rope_apply", "rope_inv_freq", "causal_conv_silu", "delta_scan_sequential",
     "block_causal_attention", "rmsnorm", "gdn_gates", "delta_scan_chunked", "hadamard_rotate",
-    "q8_0_quantize", "projector_block", "projector_trunk")}
+    "q8_0_quantize", "projector_block", "projector_trunk", "gdn_readout", "gated_rmsnorm",
+    "gdn_decode", "gqa_decode_attention", "attn_decode", "rope_apply")}
 
 def _hadamard_unnormalised(x):
     # the +-1 Walsh-Hadamard matrix without the 1/sqrt(n) that makes it orthonormal
@@ -174,6 +175,68 @@ def _trunk_blocks_reversed(residual, W, geom):
     return R_orig["projector_trunk"](residual, dict(W, blocks=list(W["blocks"])[::-1]), geom)
 
 
+def _readout_gqa_modulo(S, q):
+    # v head h reads query head h % n_k
+    n_v = S.shape[0]
+    return np.einsum("hij,hj->hi", S, q[np.arange(n_v) % q.shape[0]])
+
+
+def _gated_norm_sigmoid(o, z, w, eps=R.EPS):
+    # sigmoid(z) as the gate instead of silu(z)
+    return R_orig["rmsnorm"](o, w, eps) * R.sigmoid(z)
+
+
+def _decode_reads_old_state(x, z, tail, S, conv_w, A_log, dt_bias, norm_w, geom):
+    # the readout taken from the state before the token's own write
+    o_new, S1, t1 = R_orig["gdn_decode"](x, z, tail, S, conv_w, A_log, dt_bias, norm_w, geom)
+    pr = R.gdn_prepare(np.asarray(x, dtype=np.float64)[None], tail, conv_w, A_log, dt_bias, geom)
+    o = R_orig["gdn_readout"](np.asarray(S, dtype=np.float64), pr["q"][0])
+    nv, dv = geom.gdn_n_v, geom.gdn_d_v
+    return R_orig["gated_rmsnorm"](o, np.asarray(z).reshape(nv, dv), norm_w).reshape(-1), S1, t1
+
+
+def _gqa_decode_modulo(q, Kc, Vc):
+    # query head h reads KV head h % n_kv
+    n_q = q.shape[0]
+    perm = np.arange(n_q) % Kc.shape[1]
+    out = np.empty_like(q)
+    for h in range(n_q):
+        s = Kc[:, perm[h]] @ q[h] / math.sqrt(q.shape[1])
+        p = np.exp(s - s.max())
+        out[h] = (p / p.sum()) @ Vc[:, perm[h]]
+    return out
+
+
+def _gqa_decode_no_scale(q, Kc, Vc):
+    return R_orig["gqa_decode_attention"](q * math.sqrt(q.shape[1]), Kc, Vc)
+
+
+def _attn_decode_gate_silu(x, k_gain, q_gain, kcache, vcache, pos, geom, page_table=None, page_size=0):
+    # silu(gate) instead of sigmoid(gate): undo the sigmoid and apply silu
+    o = R_orig["attn_decode"](x, k_gain, q_gain, kcache, vcache, pos, geom, page_table, page_size)
+    w, nqd = geom.attn_width, geom.attn_n_q * geom.attn_d_h
+    gate = np.asarray(x, dtype=np.float64)[w + nqd:w + 2 * nqd]
+    return o * gate
+
+
+def _attn_decode_q_unrotated(x, k_gain, q_gain, kcache, vcache, pos, geom, page_table=None, page_size=0):
+    # RoPE applied to k only: rope_apply leaves the one-row q (the call with a single
+    # position equal to pos and n_q heads) unrotated
+    real = R_orig["rope_apply"]
+
+    def rope_k_only(t, positions, rope_dims, theta):
+        t = np.asarray(t)
+        if t.shape[0] == 1 and t.shape[1] == geom.attn_n_q and geom.attn_n_q != geom.attn_n_kv:
+            return np.array(t, dtype=np.float64, copy=True)
+        return real(t, positions, rope_dims, theta)
+
+    R.rope_apply = rope_k_only
+    try:
+        return R_orig["attn_decode"](x, k_gain, q_gain, kcache, vcache, pos, geom, page_table, page_size)
+    finally:
+        R.rope_apply = real
+
+
 MUTANTS = [
     ("rope_apply", _rope_wrong_sign, [P.test_rope_equals_complex_rotation]),
     ("rope_apply", _rope_interleaved, [P.test_rope_equals_complex_rotation]),
@@ -198,6 +261,13 @@ MUTANTS = [
      [P.test_projector_chains_its_distinct_blocks_in_order_on_one_token]),
     ("projector_trunk", _trunk_blocks_reversed,
      [P.test_projector_chains_its_distinct_blocks_in_order_on_one_token]),
+    ("gdn_readout", _readout_gqa_modulo, [P.test_gdn_readout_returns_values_written_at_orthonormal_keys]),
+    ("gated_rmsnorm", _gated_norm_sigmoid, [P.test_gated_rmsnorm_closed_form]),
+    ("gdn_decode", _decode_reads_old_state, [P.test_gdn_decode_reads_the_value_it_just_wrote]),
+    ("gqa_decode_attention", _gqa_decode_modulo, [P.test_attn_decode_brute_force_loops]),
+    ("gqa_decode_attention", _gqa_decode_no_scale, [P.test_attn_decode_brute_force_loops]),
+    ("attn_decode", _attn_decode_gate_silu, [P.test_attn_decode_first_token_returns_its_value_times_the_gate]),
+    ("attn_decode", _attn_decode_q_unrotated, [P.test_attn_decode_depends_on_relative_positions_only]),
 ]
 
 

@@ -543,3 +543,197 @@ def test_q4_0_error_bound_and_range():
     mb = np.take_along_axis(back, first, axis=-1)[..., 0]
     assert np.all(np.abs(mb - m) <= store * (1 + 1e-9))
     np.testing.assert_array_equal(R.q4_0_unpack(R.q4_0_pack(c)), c)
+
+
+# ---------------------------------------------------------------- exact last-token pass
+def test_gdn_readout_returns_values_written_at_orthonormal_keys():
+    # a state holding rank-1 writes v_j k_j^T at orthonormal keys returns v_j when read with
+    # k_j; v head h belongs to key head h // (n_v / n_k)
+    n_k, n_v, d = 2, 4, 8
+    rng = np.random.default_rng(5)
+    Q = [np.linalg.qr(rng.standard_normal((d, d)))[0] for _ in range(n_k)]   # columns: keys
+    vals = rng.standard_normal((n_v, d, d))                                   # vals[h, j]: v_j
+    S = np.stack([sum(np.outer(vals[h, j], Q[h // 2][:, j]) for j in range(d)) for h in range(n_v)])
+    for j in range(d):
+        q = np.stack([Q[kh][:, j] for kh in range(n_k)])
+        np.testing.assert_allclose(R.gdn_readout(S, q), vals[:, j], rtol=1e-10, atol=1e-12)
+
+
+def test_gated_rmsnorm_closed_form():
+    o = np.array([[3.0, 4.0, 0.0, 0.0], [1.0, 1.0, 1.0, 1.0]])
+    z = np.array([[0.0, 2.0, -1.0, 40.0], [1.0, -3.0, 0.5, 0.0]])
+    w = np.array([1.0, 0.5, 2.0, 1.5])
+    rms0 = math.sqrt(25.0 / 4.0 + R.EPS)
+    rms1 = math.sqrt(1.0 + R.EPS)
+    sil = lambda t: t / (1.0 + math.exp(-t))
+    want = np.array([[3 / rms0 * 1.0 * sil(0.0), 4 / rms0 * 0.5 * sil(2.0), 0.0, 0.0],
+                     [1 / rms1 * 1.0 * sil(1.0), 1 / rms1 * 0.5 * sil(-3.0), 1 / rms1 * 2.0 * sil(0.5), 0.0]])
+    np.testing.assert_allclose(R.gated_rmsnorm(o, z, w), want, rtol=1e-12, atol=1e-15)
+
+
+def _tiny_decode_layer(seed=3):
+    geom = KI.TINY
+    P = {k: v.double().numpy() for k, v in KI.make_layer_params(geom, seed).items()}
+    L = {k: v.double().numpy() for k, v in KI.make_last_token_params(geom, seed + 1, random_gains=True).items()}
+    st = KI.make_states(geom, 1, seed + 2, std=0.3)
+    return geom, P, L, st["state"][0].double().numpy(), st["conv_tail"][0].double().numpy()
+
+
+def test_gdn_decode_state_and_tail_equal_a_one_token_ubatch():
+    # the decode's state update is the prefill's own update on a ubatch of one token
+    geom, P, L, S0, tail0 = _tiny_decode_layer()
+    x = RNG.standard_normal(geom.last_width(0))
+    gw = geom.gdn_width
+    o, S1, t1 = R.gdn_decode(x[:gw], x[gw:], tail0[0], S0[0], P["conv_w"][0], P["A_log"][0],
+                             P["dt_bias"][0], L["gdn_norm_w"][0], geom)
+    one = KI.with_changes(geom, layer_types=(KI.GDN,))
+    Pone = {"conv_w": P["conv_w"][:1], "A_log": P["A_log"][:1], "dt_bias": P["dt_bias"][:1],
+            "k_norm_g": np.zeros((0, geom.attn_d_h))}
+    S_u, t_u = R.update_states(x[None, :gw], one, Pone, S0[:1], tail0[:1], [], [], 0)
+    np.testing.assert_allclose(S1, S_u[0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(t1, t_u[0])
+    assert o.shape == (geom.gdn_n_v * geom.gdn_d_v,)
+
+
+def test_gdn_decode_reads_the_value_it_just_wrote():
+    # q = k (same inputs, tail rows and conv taps on the q and k channels), beta -> 1 and
+    # g -> 0: the delta rule writes v at k, so the read returns the token's own v after conv
+    # and SiLU, and the output is the gated RMSNorm of that v
+    geom, P, L, S0, tail0 = _tiny_decode_layer(seed=9)
+    nk = geom.gdn_n_k * geom.gdn_d_k
+    nv, dv = geom.gdn_n_v, geom.gdn_d_v
+    C = geom.gdn_conv_ch
+    x = RNG.standard_normal(geom.last_width(0))
+    x[:nk] = x[nk:2 * nk]                                  # q inputs = k inputs
+    x[C + nv:C + 2 * nv] = 60.0                            # b: beta = sigmoid(60) = 1 - 9e-27
+    A_log = np.full(nv, -80.0)                             # g = -exp(-80) softplus(.) ~ -2e-35
+    tail = tail0[0].copy()
+    tail[:, :nk] = tail[:, nk:2 * nk]
+    w = P["conv_w"][0].copy()
+    w[:nk] = w[nk:2 * nk]
+    gw = geom.gdn_width
+    o, S1, _ = R.gdn_decode(x[:gw], x[gw:], tail, S0[0], w, A_log, P["dt_bias"][0],
+                            L["gdn_norm_w"][0], geom)
+    ext = np.concatenate([tail, x[None, :C]], axis=0)
+    conv = sum(ext[j] * w[:, j] for j in range(4))
+    act = conv / (1.0 + np.exp(-conv))
+    v = act[2 * nk:].reshape(nv, dv)
+    k = act[nk:2 * nk].reshape(geom.gdn_n_k, -1)
+    k = k / np.sqrt(np.sum(k * k, axis=1, keepdims=True) + R.EPS)
+    # with q = k, beta = 1, g = 0 the read is S1 k = (1 - n) S0 k + n v, n = |k|^2 (1 up to
+    # the eps inside the L2 norm)
+    kv = k[np.arange(nv) // (nv // geom.gdn_n_k)]
+    n = np.sum(kv * kv, axis=1, keepdims=True)
+    v = (1.0 - n) * np.einsum("hij,hj->hi", S0[0], kv) + n * v
+    z = x[gw:].reshape(nv, dv)
+    want = v / np.sqrt(np.mean(v * v, axis=1, keepdims=True) + R.EPS) * L["gdn_norm_w"][0] \
+        * (z / (1.0 + np.exp(-z)))
+    np.testing.assert_allclose(o.reshape(nv, dv), want, rtol=1e-9, atol=1e-12)
+
+
+def _attn_setup(seed, pos, n_q=6, n_kv=2, d=32, rope=16):
+    geom = KI.with_changes(KI.TINY, attn_n_kv=n_kv, attn_d_h=d, rope_dims=rope, attn_n_q=n_q)
+    rng = np.random.default_rng(seed)
+    kc = rng.standard_normal((n_kv, pos + 4, d))
+    vc = rng.standard_normal((n_kv, pos + 4, d))
+    x = rng.standard_normal(geom.last_width(2))
+    kg = rng.uniform(0.5, 1.5, d)
+    qg = rng.uniform(0.5, 1.5, d)
+    return geom, kc, vc, x, kg, qg
+
+
+def test_attn_decode_first_token_returns_its_value_times_the_gate():
+    geom, kc, vc, x, kg, qg = _attn_setup(1, 0)
+    o = R.attn_decode(x, kg, qg, kc, vc, 0, geom).reshape(6, 32)
+    w = geom.attn_width
+    v = x[w // 2:w].reshape(2, 32)
+    gate = x[w + 6 * 32:].reshape(6, 32)
+    for h in range(6):
+        np.testing.assert_allclose(o[h], v[h // 3] / (1.0 + np.exp(-gate[h])), rtol=1e-12)
+
+
+def test_attn_decode_brute_force_loops():
+    # explicit loops: 2 x 2 rotations of the pairs (i, i + r/2), softmax over rows 0..pos,
+    # query head h on KV head h // 3
+    pos = 9
+    geom, kc, vc, x, kg, qg = _attn_setup(2, pos)
+    kc0, vc0 = kc.copy(), vc.copy()
+    o = R.attn_decode(x, kg, qg, kc, vc, pos, geom).reshape(6, 32)
+    d, r, w = 32, 16, geom.attn_width
+
+    def norm_rot(vec, g, p):
+        y = vec / math.sqrt(sum(t * t for t in vec) / d + R.EPS) * g
+        out = y.copy()
+        for i in range(r // 2):
+            a = p * geom.rope_theta ** (-2.0 * i / r)
+            out[i] = y[i] * math.cos(a) - y[i + r // 2] * math.sin(a)
+            out[i + r // 2] = y[i + r // 2] * math.cos(a) + y[i] * math.sin(a)
+        return out
+
+    knew = [norm_rot(x[hh * d:(hh + 1) * d], kg, pos) for hh in range(2)]
+    vnew = [x[w // 2 + hh * d:w // 2 + (hh + 1) * d] for hh in range(2)]
+    for hh in range(2):
+        np.testing.assert_allclose(kc[hh, pos], knew[hh], rtol=1e-12)      # written in place
+        np.testing.assert_array_equal(vc[hh, pos], vnew[hh])
+        np.testing.assert_array_equal(kc[hh, :pos], kc0[hh, :pos])         # nothing else moved
+    for h in range(6):
+        q = norm_rot(x[w + h * d:w + (h + 1) * d], qg, pos)
+        hh = h // 3
+        scores = [sum(q[i] * (knew[hh][i] if j == pos else kc0[hh, j, i]) for i in range(d)) / math.sqrt(d)
+                  for j in range(pos + 1)]
+        m = max(scores)
+        e = [math.exp(s - m) for s in scores]
+        want = sum(e[j] / sum(e) * (vnew[hh] if j == pos else vc0[hh, j]) for j in range(pos + 1))
+        gate = x[w + 6 * d + h * d:w + 6 * d + (h + 1) * d]
+        np.testing.assert_allclose(o[h], want / (1.0 + np.exp(-gate)), rtol=1e-10, atol=1e-12)
+
+
+def test_attn_decode_depends_on_relative_positions_only():
+    # cache rows written by the prefill's own k path at positions j = 0..pos-1; the score of
+    # row j is <R_pos q, R_j k_j> = Re sum_i conj(q_i) k_i e^{i (j - pos) w_i} over the
+    # rotated pairs (as complex numbers q_i + i q_(i+r/2)) plus the plain dot product of the
+    # other dims: only j - pos enters
+    pos = 7
+    geom, _, _, x, kg, qg = _attn_setup(3, pos)
+    d, r, w = 32, 16, geom.attn_width
+    raw = np.random.default_rng(4).standard_normal((pos, w))
+    kc = np.zeros((2, pos + 2, d))
+    vc = np.zeros_like(kc)
+    Kx, Vx = R.attn_kv(raw, kg, 0, geom)
+    kc[:, :pos] = Kx.transpose(1, 0, 2)
+    vc[:, :pos] = Vx.transpose(1, 0, 2)
+    o = R.attn_decode(x, kg, qg, kc, vc, pos, geom).reshape(6, d)
+    omega = geom.rope_theta ** (-2.0 * np.arange(r // 2) / r)
+    rows = np.concatenate([raw, x[None, :w]], axis=0)                # unrotated k of rows 0..pos
+    kn = rows[:, :w // 2].reshape(pos + 1, 2, d)
+    kn = kn / np.sqrt(np.mean(kn * kn, axis=-1, keepdims=True) + R.EPS) * kg
+    vv = rows[:, w // 2:].reshape(pos + 1, 2, d)
+    for h in range(6):
+        q = x[w + h * d:w + (h + 1) * d]
+        q = q / math.sqrt(np.mean(q * q) + R.EPS) * qg
+        qc = q[:r // 2] + 1j * q[r // 2:r]
+        kk = kn[:, h // 3]
+        kcx = kk[:, :r // 2] + 1j * kk[:, r // 2:r]
+        rel = np.arange(pos + 1)[:, None] - pos
+        sc = (np.real(np.sum(np.conj(qc)[None] * kcx * np.exp(1j * rel * omega[None]), axis=1))
+              + kk[:, r:] @ q[r:]) / math.sqrt(d)
+        p = np.exp(sc - sc.max())
+        want = (p / p.sum()) @ vv[:, h // 3]
+        gate = x[w + 6 * d + h * d:w + 6 * d + (h + 1) * d]
+        np.testing.assert_allclose(o[h], want / (1.0 + np.exp(-gate)), rtol=1e-9, atol=1e-12)
+
+
+def test_attn_decode_paged_equals_contiguous():
+    pos, ps = 20, 8
+    geom, kc, vc, x, kg, qg = _attn_setup(5, pos)
+    n_pages = 6
+    pt = np.array([4, 0, 5])                               # rows 0..23 on pages 4, 0, 5
+    kp = np.random.default_rng(6).standard_normal((n_pages, 2, ps, 32))
+    vp = np.random.default_rng(7).standard_normal((n_pages, 2, ps, 32))
+    for j in range(pos):
+        kp[pt[j // ps], :, j % ps] = kc[:, j]
+        vp[pt[j // ps], :, j % ps] = vc[:, j]
+    o_c = R.attn_decode(x, kg, qg, kc, vc, pos, geom)
+    o_p = R.attn_decode(x, kg, qg, kp, vp, pos, geom, page_table=pt, page_size=ps)
+    np.testing.assert_allclose(o_p, o_c, rtol=1e-12)
+    np.testing.assert_allclose(kp[pt[pos // ps], :, pos % ps], kc[:, pos], rtol=1e-12)
