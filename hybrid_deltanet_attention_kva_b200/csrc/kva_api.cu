@@ -38,6 +38,7 @@ struct kva_handle {
   __nv_bfloat16* kbuf = nullptr;  // [max_seq, n_gdn, max_T, n_k d_k]
   __nv_bfloat16* vbuf = nullptr;  // [max_seq, n_gdn, max_T, n_v d_v]
   float* gbuf = nullptr;          // [max_seq, n_gdn, 2, n_v, max_T]
+  float* dec_part = nullptr;      // last-token attention partials [kDecodeSlots, 8, d_h + 2]
   int* status = nullptr;          // device status word
   void* chunk = nullptr;          // per-chunk B1 and scalars of the 128-dimensional scan
   // heads GEMM with the state-update epilogue (kva_prefill_ubatch), when the dims allow it
@@ -75,7 +76,7 @@ int staged(kva_handle* h, int kind, cudaStream_t s, F&& launch) {
 namespace {
 
 struct Layout {
-  size_t off[15];
+  size_t off[16];
   size_t total;
 };
 
@@ -146,7 +147,7 @@ Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
   const size_t T = d->max_T, S = d->max_seq;
   const size_t dm = d->d_model;
   const size_t C = 2ull * d->gdn_n_k * d->gdn_d_k + (size_t)d->gdn_n_v * d->gdn_d_v;
-  size_t sz[14];
+  size_t sz[15];
   sz[0] = T * d->hidden * 2;                                          // u_in
   sz[1] = T * dm * 2;                                                 // u
   sz[2] = T * dm * 4;                                                 // x
@@ -166,9 +167,11 @@ Layout layout_of(const kva_dims* d, int ng, int64_t n_mix) {
   sz[11] = fz ? ng * nblk * kMixHaloRows * C * 2 : 0;                      // halo rows
   sz[12] = fz ? ng * 3 * C * 2 : 0;                                         // last rows
   sz[13] = fz ? fused_tiles(d, ng, na, &ndt) * sizeof(MixTile) : 0;         // tile table
+  // partial states of the last-token attention (sequence x KV head x split slots)
+  sz[14] = na ? (size_t)kDecodeSlots * kDecodeMaxGroup * (d->attn_d_h + 2) * 4 : 0;
   Layout L;
   size_t o = 0;
-  for (int i = 0; i < 14; ++i) {
+  for (int i = 0; i < 15; ++i) {
     L.off[i] = o;
     o += align_up(sz[i]);
   }
@@ -372,6 +375,7 @@ int kva_init(const kva_dims* dims, kva_handle** out) {
   h->gbuf = reinterpret_cast<float*>(b + L.off[8]);
   h->status = reinterpret_cast<int*>(b + L.off[9]);
   h->chunk = b + L.off[10];
+  h->dec_part = na ? reinterpret_cast<float*>(b + L.off[14]) : nullptr;
   h->fused = fused_ok(dims, ng, na);
   if (h->fused) {
     h->halo = b + L.off[11];
@@ -800,6 +804,120 @@ int kva_update_states(kva_handle* h, const void* mixer_in, int64_t mixer_ld, int
   e = update_states_impl(h, mixer_in, mixer_ld, n_seq, T, pos, w, state, conv_state, kv, debug_qkv,
                          debug_gb, s);
   if (!e) h->tokens += (int64_t)n_seq * T;
+  if (cur != h->device) cudaSetDevice(cur);
+  return e;
+}
+
+int kva_last_token_layer(kva_handle* h, int32_t layer, int32_t n_seq, const void* x, int64_t x_ld,
+                         const int64_t* pos, const kva_weights* w, const kva_last_params* lp,
+                         float* state, void* conv_state, const kva_kv_cache* kv, void* out,
+                         int32_t out_dtype, int64_t out_ld, void* stream) {
+  if (!h || !w || !lp) return KVA_ERR_INVALID_ARG;
+  const kva_dims& d = h->d;
+  if (layer < 0 || layer >= d.n_late || n_seq < 0) return KVA_ERR_INVALID_ARG;
+  if (n_seq > d.max_seq) return KVA_ERR_TOO_LARGE;
+  if (n_seq == 0) return KVA_OK;
+  if (!x || !pos || !out) return KVA_ERR_INVALID_ARG;
+  if (out_dtype != KVA_F32 && out_dtype != d.compute_dtype) return KVA_ERR_INVALID_ARG;
+  if (!a16(x) || x_ld % 8 || !a16(out) || out_ld % 4) return KVA_ERR_ALIGNMENT;
+  for (int i = 0; i < n_seq; ++i)
+    if (pos[i] < 0) return KVA_ERR_INVALID_ARG;
+  const bool gdn = d.layer_type[layer] == KVA_LAYER_GDN;
+  int li = 0;  // index among the layers of this type
+  for (int i = 0; i < layer; ++i) li += d.layer_type[i] == d.layer_type[layer];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return KVA_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return KVA_ERR_CUDA;
+  int e = KVA_OK;
+  if (gdn) {
+    const int nvdv = d.gdn_n_v * d.gdn_d_v;
+    if (x_ld < h->gdn_width + nvdv || out_ld < nvdv) e = KVA_ERR_INVALID_ARG;
+    else if (!w->conv_w || !w->A_log || !w->dt_bias || !lp->gdn_norm_w || !state || !conv_state)
+      e = KVA_ERR_INVALID_ARG;
+    else if (!a16(w->conv_w) || !a16(state) || !a16(conv_state)) e = KVA_ERR_ALIGNMENT;
+    if (!e) {
+      GdnDecodeLaunch g;
+      g.x = x;
+      g.x_ld = x_ld;
+      g.x_dtype = d.compute_dtype;
+      g.n_seq = n_seq;
+      g.n_k = d.gdn_n_k;
+      g.n_v = d.gdn_n_v;
+      g.d = d.gdn_d_k;
+      g.C = h->C;
+      g.conv_w = w->conv_w + (int64_t)li * h->C * 4;
+      g.A_log = w->A_log + (int64_t)li * d.gdn_n_v;
+      g.dt_bias = w->dt_bias + (int64_t)li * d.gdn_n_v;
+      g.norm_w = lp->gdn_norm_w + (int64_t)li * d.gdn_d_v;
+      const int64_t sstate = (int64_t)d.gdn_n_v * d.gdn_d_v * d.gdn_d_k;
+      g.state = state + (int64_t)li * sstate;
+      g.state_seq_stride = (int64_t)h->n_gdn * sstate;
+      g.conv_state = static_cast<uint16_t*>(conv_state) + (int64_t)li * 3 * h->C;
+      g.conv_seq_stride = (int64_t)h->n_gdn * 3 * h->C;
+      g.out = out;
+      g.out_ld = out_ld;
+      g.out_dtype = out_dtype;
+      g.eps = d.norm_eps;
+      h->last_stream = s;
+      e = staged(h, KVA_ST_LAST_TOKEN, s, [&] { return launch_gdn_decode(g, s); });
+      if (!e) ++h->launches[KVA_ST_LAST_TOKEN];  // two kernels
+    }
+  } else {
+    const int n_q = lp->attn_n_q, dh = d.attn_d_h;
+    if (n_q <= 0 || n_q % d.attn_n_kv || n_q / d.attn_n_kv > kDecodeMaxGroup) e = KVA_ERR_UNSUPPORTED;
+    else if (x_ld < h->attn_width + 2LL * n_q * dh || out_ld < (int64_t)n_q * dh) e = KVA_ERR_INVALID_ARG;
+    else if (!w->k_norm_g || !lp->q_norm_g) e = KVA_ERR_INVALID_ARG;
+    else if (!(e = check_cache(h, kv, n_seq, pos, 1)) && kv->dtype != KVA_BF16 && kv->dtype != KVA_F16)
+      e = KVA_ERR_UNSUPPORTED;
+    if (!e && (int64_t)n_seq * d.attn_n_kv > kDecodeSlots) e = KVA_ERR_UNSUPPORTED;
+    if (!e) {
+      AttnDecodeLaunch a;
+      a.x = x;
+      a.x_ld = x_ld;
+      a.x_dtype = d.compute_dtype;
+      a.n_seq = n_seq;
+      a.n_kv = d.attn_n_kv;
+      a.n_q = n_q;
+      a.G = n_q / d.attn_n_kv;
+      a.d_h = dh;
+      a.rope_dims = d.rope_dims;
+      for (int i = 0; i < d.rope_dims / 2 && i < 128; ++i)
+        a.inv_freq[i] = std::pow(d.rope_theta, -2.0 * i / d.rope_dims);
+      a.k_gain = w->k_norm_g + (int64_t)li * dh;
+      a.q_gain = lp->q_norm_g + (int64_t)li * dh;
+      int64_t max_rows = 0;
+      for (int i = 0; i < n_seq; ++i) {
+        a.pos[i] = pos[i];
+        if (pos[i] + 1 > max_rows) max_rows = pos[i] + 1;
+      }
+      a.kc = kv->k[li];
+      a.vc = kv->v[li];
+      a.layout = kv->layout;
+      a.max_pos = kv->max_pos;
+      a.page_size = kv->page_size;
+      a.n_pages = kv->n_pages;
+      a.pages_per_seq = kv->pages_per_seq;
+      a.page_table = kv->page_table;
+      a.cache_dtype = kv->dtype;
+      const int slots_per = kDecodeSlots / (n_seq * d.attn_n_kv);
+      a.n_split = attn_decode_splits(n_seq, d.attn_n_kv, max_rows, num_sms(), &a.rows_per_split);
+      if (a.n_split > slots_per) {  // fewer, longer splits so the partials fit the workspace
+        const int64_t tiles = (max_rows + 63) / 64;
+        a.rows_per_split = (tiles + slots_per - 1) / slots_per * 64;
+        a.n_split = (int)((max_rows + a.rows_per_split - 1) / a.rows_per_split);
+      }
+      a.part = h->dec_part;
+      a.out = out;
+      a.out_ld = out_ld;
+      a.out_dtype = out_dtype;
+      a.eps = d.norm_eps;
+      a.err = h->status;
+      h->last_stream = s;
+      e = staged(h, KVA_ST_LAST_TOKEN, s, [&] { return launch_attn_decode(a, s); });
+      if (!e) ++h->launches[KVA_ST_LAST_TOKEN];  // two kernels
+    }
+  }
   if (cur != h->device) cudaSetDevice(cur);
   return e;
 }

@@ -147,6 +147,60 @@ struct KvLaunch {
 int launch_kv_write(const KvLaunch& k, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
+// Exact last-token pass of one late layer (kva_last_token_layer).
+struct GdnDecodeLaunch {
+  const void* x = nullptr;        // 16-bit [n_seq, x_ld]: [q | k | v | a | b | z] of the token
+  int64_t x_ld = 0;
+  int x_dtype = KVA_BF16;         // also the conv tail's format
+  int n_seq = 0, n_k = 0, n_v = 0, d = 0, C = 0;
+  const float* conv_w = nullptr;  // this layer's [C, 4]
+  const float* A_log = nullptr;   // [n_v]
+  const float* dt_bias = nullptr; // [n_v]
+  const float* norm_w = nullptr;  // [d] gated RMSNorm weight
+  float* state = nullptr;         // this layer's [n_v, d, d] of sequence 0
+  int64_t state_seq_stride = 0;   // floats between sequences
+  void* conv_state = nullptr;     // this layer's [3, C] of sequence 0
+  int64_t conv_seq_stride = 0;    // elements between sequences
+  void* out = nullptr;            // [n_seq, out_ld]
+  int64_t out_ld = 0;
+  int out_dtype = KVA_BF16;       // KVA_F32 or x_dtype
+  float eps = 1e-6f;
+};
+int launch_gdn_decode(const GdnDecodeLaunch& g, cudaStream_t s);
+
+constexpr int kDecodeMaxSplit = 64;    // cache-row splits per (sequence, KV head)
+constexpr int kDecodeSlots = 2048;     // partial states (sequence x KV head x split) in the workspace
+constexpr int kDecodeMaxGroup = 8;     // query heads per KV head
+struct AttnDecodeLaunch {
+  const void* x = nullptr;        // 16-bit [n_seq, x_ld]: [k | v | q | gate] of the token
+  int64_t x_ld = 0;
+  int x_dtype = KVA_BF16;
+  int n_seq = 0, n_kv = 0, n_q = 0, G = 0, d_h = 0, rope_dims = 0;
+  double inv_freq[128] = {0};     // theta^(-2i / rope_dims) (fp64, host)
+  const float* k_gain = nullptr;  // this layer's [d_h]
+  const float* q_gain = nullptr;  // [d_h]
+  int64_t pos[kMaxSeqPos] = {0};  // position of each sequence's token
+  void* kc = nullptr;             // this layer's K and V caches
+  void* vc = nullptr;
+  int layout = KVA_KV_CONTIGUOUS;
+  int64_t max_pos = 0;
+  int page_size = 0, n_pages = 0, pages_per_seq = 0;
+  const int32_t* page_table = nullptr;
+  int cache_dtype = KVA_BF16;
+  int n_split = 1;
+  int64_t rows_per_split = 0;     // a multiple of the 64-row tile
+  float* part = nullptr;          // [n_seq, n_kv, n_split, G, d_h + 2] partial O, max, sum
+  void* out = nullptr;            // [n_seq, out_ld]
+  int64_t out_ld = 0;
+  int out_dtype = KVA_BF16;
+  float eps = 1e-6f;
+  int* err = nullptr;
+};
+// splits of the longest sequence's max_rows cache rows for n_seq x n_kv CTAs on `sms` SMs
+int attn_decode_splits(int n_seq, int n_kv, int64_t max_rows, int sms, int64_t* rows_per_split);
+int launch_attn_decode(const AttnDecodeLaunch& a, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
 // Heads GEMM with the state-update epilogue (the wide head GEMM writes the scan's
 // inputs, the gates and the KV-cache rows directly instead of the mixer).
 // The N dimension is tiled per layer segment: every tile lies inside one segment.

@@ -76,8 +76,12 @@ class KvaKvCache(C.Structure):
                 ("pages_per_seq", C.c_int32), ("page_table", C.c_void_p), ("dtype", C.c_int32)]
 
 
+class KvaLastParams(C.Structure):
+    _fields_ = [("attn_n_q", C.c_int32), ("gdn_norm_w", C.c_void_p), ("q_norm_g", C.c_void_p)]
+
+
 ST_NAMES = ("rmsnorm", "gemm_trunk", "attention", "gemm_heads", "gdn_prepare", "gdn_tail",
-            "gdn_scan", "kv_write")
+            "gdn_scan", "kv_write", "last_token")
 ST_COUNT = len(ST_NAMES)
 
 
@@ -106,6 +110,9 @@ def _load() -> C.CDLL:
                                      C.POINTER(KvaKvCache), I64, P, P, P]),
         "kva_update_states": (I32, [P, P, I64, I32, I32, C.POINTER(I64), C.POINTER(KvaWeights),
                                     P, P, C.POINTER(KvaKvCache), P, P, P]),
+        "kva_last_token_layer": (I32, [P, I32, I32, P, I64, C.POINTER(I64), C.POINTER(KvaWeights),
+                                       C.POINTER(KvaLastParams), P, P, C.POINTER(KvaKvCache), P, I32,
+                                       I64, P]),
         "kva_get_device_status": (I32, [P, C.POINTER(I32)]),
         "kva_stats": (I32, [P, C.POINTER(I64)]),
         "kva_heads_fused": (I32, [P, C.POINTER(I32)]),
@@ -134,6 +141,7 @@ def _load() -> C.CDLL:
 
 _lib = _load()
 EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update_states",
+            "kva_last_token_layer",
             "kva_get_device_status", "kva_stats", "kva_heads_fused", "kva_free", "kva_strerror",
             "kva_profile_enable", "kva_profile_read",
             "kva_op_rmsnorm", "kva_op_gemm", "kva_op_gemm_q8_0", "kva_op_gemm_q4_0", "kva_op_attention",
@@ -297,6 +305,37 @@ def kva_update_states(handle: int, mixer_in: torch.Tensor, pos: Sequence[int], w
         handle, _ptr(mixer_in), ld, n_seq, T, pos_arr, C.byref(weights.c), _ptr(state),
         _ptr(conv_state), C.byref(kv.c) if kv is not None else None, _ptr(debug_qkv),
         _ptr(debug_gb), _stream(stream)), "kva_update_states")
+
+
+class LastParams:
+    """kva_last_params: query heads of an attention layer, the gated RMSNorm weights of the
+    gated-DeltaNet layers [n_gdn, d_v] and the q RMSNorm gains of the attention layers
+    [n_attn, d_h] (fp32 device tensors)."""
+
+    def __init__(self, attn_n_q: int, gdn_norm_w: Optional[torch.Tensor] = None,
+                 q_norm_g: Optional[torch.Tensor] = None):
+        self._keep = [t for t in (gdn_norm_w, q_norm_g) if t is not None]
+        self.c = KvaLastParams()
+        self.c.attn_n_q = attn_n_q
+        self.c.gdn_norm_w = _ptr(gdn_norm_w)
+        self.c.q_norm_g = _ptr(q_norm_g)
+
+
+def kva_last_token_layer(handle: int, layer: int, x: torch.Tensor, pos: Sequence[int],
+                         weights: Weights, last: LastParams, state: Optional[torch.Tensor],
+                         conv_state: Optional[torch.Tensor], kv: Optional[KvCache], out: torch.Tensor,
+                         stream=None) -> None:
+    """The exact last-token pass through late layer `layer` for x.shape[0] sequences (see
+    include/kva.h): x [n_seq, >= layer's input width] in the handle's compute dtype, out
+    [n_seq, >= output width] fp32 or the compute dtype."""
+    n_seq = x.shape[0]
+    if x.stride(1) != 1 or out.stride(1) != 1:
+        raise ValueError("x and out must be row-major")
+    pos_arr = (C.c_int64 * max(1, n_seq))(*[int(p) for p in pos])
+    _check(_lib.kva_last_token_layer(
+        handle, layer, n_seq, _ptr(x), x.stride(0), pos_arr, C.byref(weights.c), C.byref(last.c),
+        _ptr(state), _ptr(conv_state), C.byref(kv.c) if kv is not None else None, _ptr(out),
+        _DT[out.dtype], out.stride(0), _stream(stream)), "kva_last_token_layer")
 
 
 def kva_get_device_status(handle: int) -> int:

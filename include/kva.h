@@ -209,6 +209,44 @@ int kva_update_states(kva_handle* h, const void* mixer_in, int64_t mixer_ld, int
                       void* conv_state, const kva_kv_cache* kv, void* debug_qkv,
                       void* debug_gb, void* stream);
 
+/* Parameters of the exact last-token pass that the projector path does not need. */
+typedef struct kva_last_params {
+  int32_t attn_n_q;          /* query heads of an attention layer: a multiple of attn_n_kv, at
+                                most 8 per KV head (24 over 4 in the model card's base model) */
+  const float* gdn_norm_w;   /* [n_gdn, d_v] weight of the gated RMSNorm at each gated-DeltaNet
+                                layer's output (device) */
+  const float* q_norm_g;     /* [n_attn, d_h] q RMSNorm gain of each attention layer (device) */
+} kva_last_params;
+
+/* The exact last-token pass through ONE late layer's token mixer, for n_seq sequences
+ * ("Qwen3.8-27B-KVA" model card, "What the hell?": after the cheap state updates the engine
+ * runs the last token of each ubatch through the late layers exactly, on top of the
+ * approximated context).  When this pass follows, kva_prefill_ubatch covers tokens
+ * 0..T-2 of the ubatch and the last token reaches each late layer's state / cache here,
+ * with that layer's exact inputs; the caller runs the layers in order, since each layer's
+ * inputs come from the base model's projections of the previous layer's output (those
+ * projections, the o-projection and the FFN are the caller's).
+ *   layer      index among the n_late late layers (0-based)
+ *   x          compute_dtype [n_seq, x_ld], the token's exact inputs of that layer:
+ *              gated-DeltaNet: [q | k | v | a | b] as in the mixer, then the output gate
+ *              z (n_v * d_v); attention: [k | v] as in the mixer, then q (n_q * d_h) and
+ *              its gate (n_q * d_h)
+ *   pos        HOST int64 [n_seq], the token's position (RoPE angle and cache row)
+ *   w          the late layers' parameters (conv_w, A_log, dt_bias, k_norm_g)
+ *   lp         the pass's own parameters (above)
+ *   state, conv_state, kv   as in kva_update_states (all layers; this layer's part is
+ *              read and updated: the state and conv tail take the token, the caches
+ *              get its K and V rows at pos)
+ *   out        [n_seq, out_ld] in out_dtype (KVA_F32 or compute_dtype): the mixer output,
+ *              n_v * d_v values o = RMSNorm(S q) * w * silu(z) per value head for a
+ *              gated-DeltaNet layer, n_q * d_h values softmax(q K^T / sqrt(d_h)) V *
+ *              sigmoid(gate) per query head over cache rows 0..pos for an attention layer
+ * KV caches must be KVA_BF16 or KVA_F16 (KVA_ERR_UNSUPPORTED for q8_0 caches). */
+int kva_last_token_layer(kva_handle* h, int32_t layer, int32_t n_seq, const void* x, int64_t x_ld,
+                         const int64_t* pos, const kva_weights* w, const kva_last_params* lp,
+                         float* state, void* conv_state, const kva_kv_cache* kv, void* out,
+                         int32_t out_dtype, int64_t out_ld, void* stream);
+
 /* Synchronise the handle's last stream, return the device status bits in
  * *status (0 = clean) and clear them.  Returns KVA_ERR_DEVICE when bits were set. */
 int kva_get_device_status(kva_handle* h, int32_t* status);
@@ -234,7 +272,8 @@ typedef enum kva_stage {
   KVA_ST_GDN_TAIL = 5,    /* conv tail shift */
   KVA_ST_GDN_SCAN = 6,    /* chunked gated delta-rule scan */
   KVA_ST_KV_WRITE = 7,    /* k norm + RoPE + KV cache write */
-  KVA_ST_COUNT = 8
+  KVA_ST_LAST_TOKEN = 8,  /* the exact last-token pass of a late layer */
+  KVA_ST_COUNT = 9
 } kva_stage;
 
 /* Device-time profile of the stages, summed since the last read. */

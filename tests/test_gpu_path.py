@@ -439,11 +439,12 @@ def test_prefill_benched_configuration_every_layer(K, cfg):
         pos += T
     metrics = {}
     # drafter outputs at sampled rows of every ubatch
-    Wd = f64(Wh[geom.n_mix:geom.n_total])
-    for i, z in enumerate(zs):
-        rows = np.unique(np.linspace(0, z.shape[0] - 1, 16).astype(int))
-        metrics[f"drafter_{i}"] = _err(f64(r["drafts"][i])[rows], R.projector_heads(z[rows], Wd))
-    del Wd
+    if geom.n_draft:
+        Wd = f64(Wh[geom.n_mix:geom.n_total])
+        for i, z in enumerate(zs):
+            rows = np.unique(np.linspace(0, z.shape[0] - 1, 16).astype(int))
+            metrics[f"drafter_{i}"] = _err(f64(r["drafts"][i])[rows], R.projector_heads(z[rows], Wd))
+        del Wd
     # every gated-DeltaNet layer, carried across the ubatches in order
     S_o = f64(r["st"]["state"][0])
     tail_o = f64(r["st"]["conv_tail"][0])
