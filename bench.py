@@ -62,7 +62,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kernel-case", default=None,
-                    choices=["heads", "heads_fused", "heads_q8", "heads_q4", "resid", "gdn", "attention"],
+                    choices=["heads", "heads_fused", "heads_q8", "heads_q4", "resid", "gdn", "attention",
+                             "last_token"],
                     help="run a small case of one hot kernel three times and exit (for ncu "
                          "captures; the GEMM cases then print their CUDA-event time)")
     return ap.parse_args()
@@ -668,7 +669,7 @@ def _time_case(case, fn, flops, reps=20):
     print(json.dumps({"case": case, "us_per_launch": round(us, 2), "tflops": round(flops / us * 1e-6, 1)}))
 
 
-def run_kernel_case(case):
+def run_kernel_case(case, kv_cache="bf16"):
     """Small cases of the hot kernels, each above L2 in size where the kernel streams HBM:
     heads   - the heads GEMM's CTA-pair kernel on M = 1024, K = 3072, N = 49 152 (302 MB of
               weights, 1/5.8 of the r3 head matrix)
@@ -680,8 +681,13 @@ def run_kernel_case(case):
     heads_fused - kva_prefill_ubatch with the first 8 r3 late layers (6 gated-DeltaNet, 2
               attention, no drafter): the heads GEMM with the state-update epilogue
     gdn     - kva_update_states on the first 8 r3 late layers (6 gated-DeltaNet, 2 attention),
-              T = 1024, every launch on the caller's stream
-    attention - one block-causal attention of the r3 trunk (T = 1024, 24 heads, window 1024)"""
+              T = 1024, every launch on the caller's stream (with --kv-cache q8_0 the caches
+              take Hadamard-rotated q8_0 rows)
+    attention - one block-causal attention of the r3 trunk (T = 1024, 24 heads, window 1024)
+    last_token - the exact last-token pass of one sequence through all 32 r3 late layers at
+              position 32767 (8 attention layers each reading 32768 cache rows of 4 KV heads,
+              24 gated-DeltaNet layers updating 48 states); prints the CUDA-event time of the
+              attention and DeltaNet layers and their HBM rate"""
     import hybrid_deltanet_attention_kva_b200 as K
     torch.manual_seed(0)
     if case == "heads":
@@ -744,8 +750,12 @@ def run_kernel_case(case):
         st = KI.make_states(geom, 1, 3, std=0.1)
         mix = KI.make_mixer_inputs(geom, 1, T_UB, 4, device="cuda").half()
         S, tail = st["state"].cuda(), st["conv_tail"].cuda().half()
-        kc = [torch.zeros(1, geom.attn_n_kv, 4096, geom.attn_d_h, dtype=torch.bfloat16, device="cuda")
-              for _ in range(geom.n_attn)]
+        if kv_cache == "q8_0":
+            kc = [torch.zeros(1, geom.attn_n_kv, 4096, geom.attn_d_h * 34 // 32, dtype=torch.uint8,
+                              device="cuda") for _ in range(geom.n_attn)]
+        else:
+            kc = [torch.zeros(1, geom.attn_n_kv, 4096, geom.attn_d_h, dtype=torch.bfloat16, device="cuda")
+                  for _ in range(geom.n_attn)]
         kv = K.KvCache(kc, [torch.zeros_like(k) for k in kc], max_pos=4096)
         Wt = K.Weights(layer={k: x.cuda() for k, x in P.items()})
         h = K.kva_init(K.make_dims(geom, T_UB, 1, dtype=torch.float16))
@@ -755,6 +765,9 @@ def run_kernel_case(case):
         torch.cuda.synchronize()
         K.kva_profile_read(h)
         K.kva_free(h)
+    elif case == "last_token":
+        run_last_token_case(K)
+        return
     else:
         T, heads = T_UB, KI.R3.n_heads
         qkv = torch.randn(T, 3 * heads * 128, device="cuda").half()
@@ -764,10 +777,71 @@ def run_kernel_case(case):
     torch.cuda.synchronize()
 
 
+def last_token_bytes(geom, pos):
+    """Bytes the exact last-token pass must move at position pos: every cache row 0..pos of
+    every attention layer read once (K and V), the token's rows written; every DeltaNet
+    state read and written, the conv tails read and written, the inputs read."""
+    rows = pos + 1
+    attn = geom.n_attn * 2 * geom.attn_n_kv * geom.attn_d_h * 2 * rows
+    state = geom.n_gdn * geom.gdn_n_v * geom.gdn_d_k * geom.gdn_d_v * 4 * 2
+    tail = geom.n_gdn * 3 * geom.gdn_conv_ch * 2 * 2
+    inputs = sum(geom.last_width(i) for i in range(geom.n_late)) * 2
+    return attn, state + tail + inputs
+
+
+def run_last_token_case(K):
+    geom = KI.with_changes(KI.R3, n_draft=0)
+    pos, reps = CACHE_POS - 1, 20
+    dt = torch.float16
+    P = KI.make_layer_params(geom, 71, device="cuda")
+    L = KI.make_last_token_params(geom, 72, device="cuda")
+    st = KI.make_states(geom, 1, 73, std=0.1, device="cuda")
+    S, tail = st["state"], st["conv_tail"].to(dt)
+    kc = [torch.randn(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h, device="cuda").to(torch.bfloat16)
+          for _ in range(geom.n_attn)]
+    vc = [torch.randn_like(k) for k in kc]
+    kv = K.KvCache(kc, vc, max_pos=CACHE_POS)
+    xs = [KI.make_last_token_inputs(geom, li, 1, 80 + li, device="cuda").to(dt) for li in range(geom.n_late)]
+    outs = [torch.empty(1, geom.attn_n_q * geom.attn_d_h if t == KI.ATTN else geom.gdn_n_v * geom.gdn_d_v,
+                        device="cuda", dtype=dt) for t in geom.layer_types]
+    h = K.kva_init(K.make_dims(geom, 16, 1, dtype=dt))
+    Wt = K.Weights(layer=P)
+    lp = K.LastParams(geom.attn_n_q, L["gdn_norm_w"], L["q_norm_g"])
+
+    def run(kind):
+        for li, t in enumerate(geom.layer_types):
+            if kind is None or t == kind:
+                K.kva_last_token_layer(h, li, xs[li], [pos], Wt, lp, S, tail, kv, outs[li])
+
+    res = {}
+    for kind, name in ((KI.ATTN, "attention"), (KI.GDN, "gated_deltanet"), (None, "all")):
+        for _ in range(3):
+            run(kind)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            run(kind)
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / reps
+    assert K.kva_get_device_status(h) == 0
+    K.kva_free(h)
+    ab, gb = last_token_bytes(geom, pos)
+    peaks, src = load_peaks()
+    print(json.dumps({"case": "last_token", "pos": pos, "us_per_pass": round(res["all"], 1),
+                      "attention_us": round(res["attention"], 1), "deltanet_us": round(res["gated_deltanet"], 1),
+                      "attention_gbs": round(ab / res["attention"] * 1e-3, 1),
+                      "deltanet_gbs": round(gb / res["gated_deltanet"] * 1e-3, 1),
+                      "pass_gbs": round((ab + gb) / res["all"] * 1e-3, 1),
+                      "hbm_peak_gbs": peaks["hbm_gbs"], "peak_kind": src,
+                      "attention_bytes": ab, "deltanet_bytes": gb}))
+
+
 def main():
     args = parse()
     if args.kernel_case:
-        run_kernel_case(args.kernel_case)
+        run_kernel_case(args.kernel_case, args.kv_cache)
         return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
