@@ -180,6 +180,22 @@ class Clocks:
                 "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- per-rank plan
+N_POOL = 4  # residual ubatches each rank cycles through
+
+
+def rank_residual_seeds(seed, rank):
+    """Seeds of the residual ubatches rank `rank` runs: every rank has its own independent
+    sequence (weak scaling, no data exchange)."""
+    from hybrid_deltanet_attention_kva_b200 import multi
+    return [multi.rank_seed(seed + 100 + i, rank) for i in range(N_POOL)]
+
+
+def job_throughput(world, steps, tokens_per_step, ms_max):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's device time."""
+    return world * steps * tokens_per_step / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import hybrid_deltanet_attention_kva_b200 as K
@@ -221,9 +237,8 @@ def run_ours(args, rank, world, local_rank):
     P = KI.make_layer_params(geom, seed + 1, device="cuda")
     st = KI.make_states(geom, 1, seed + 2, device="cuda")
     st["conv_tail"] = st["conv_tail"].to(dt)
-    n_pool = 4
-    res = [KI.make_residual(geom, T_UB, multi.rank_seed(seed + 100 + i, rank), device="cuda")
-           for i in range(n_pool)]
+    n_pool = N_POOL
+    res = [KI.make_residual(geom, T_UB, sd, device="cuda") for sd in rank_residual_seeds(seed, rank)]
     if args.kv_cache == "q8_0":  # rows of d_h / 32 blocks of 34 bytes
         kc = [torch.zeros(1, geom.attn_n_kv, CACHE_POS, geom.attn_d_h * 34 // 32, dtype=torch.uint8,
                           device=dev) for _ in range(geom.n_attn)]
@@ -338,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(f0.elapsed_time(f1))
-        e2e = {"value": world * steps_e2e * T_UB / (ems / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_throughput(world, steps_e2e, T_UB, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": res[0].numel() * 2,
                "d2h_bytes_per_step": out_host.numel() * 2 if draft is not None else 0,
                "steps": steps_e2e,
@@ -370,7 +385,7 @@ def run_ours(args, rank, world, local_rank):
     long_timed = ms / 1e3 >= LONG_LOOP_S
     line = {
         "metric": METRIC,
-        "value": world * args.steps * T_UB / (ms / 1e3),
+        "value": job_throughput(world, args.steps, T_UB, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -544,7 +559,7 @@ def run_state(args, rank, world, local_rank):
         torch.cuda.synchronize()
         multi.barrier()
         ems = multi.max_over_ranks(f0.elapsed_time(f1), dev)
-        e2e = {"value": world * steps_e2e * n_seq * T / (ems / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_throughput(world, steps_e2e, n_seq * T, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": host_mix.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 4,
                "steps": steps_e2e,
                "what": "kva_update_states through the binding; the call's mixer inputs copied from "
@@ -564,7 +579,7 @@ def run_state(args, rank, world, local_rank):
     ach = sb[top] / (stages[top] / 1e3) / 1e9
     line = {
         "metric": "KVA state-update tokens/s on 1 B200 (8 sequences x 1024-token ubatch) and % of HBM roofline",
-        "value": world * args.steps * n_seq * T / (ms / 1e3),
+        "value": job_throughput(world, args.steps, n_seq * T, ms),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (bf16 N(0,1) mixer inputs, states N(0,0.1), seeded)",

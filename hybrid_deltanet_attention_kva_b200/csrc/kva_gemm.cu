@@ -1,4 +1,5 @@
-// Persistent bf16 GEMM on the 5th-generation tensor cores (tcgen05 / TMEM),
+// Persistent 16-bit (fp16 or bf16 operands, fp32 accumulation) GEMM on the 5th-generation
+// tensor cores (tcgen05 / TMEM),
 // D = A * B^T with fused epilogues.  It serves every linear layer of the KVA
 // projector ("Qwen3.8-27B-KVA" model card, architecture: Linear{5120 -> d},
 // the q/k/v/o and SwiGLU projections of the 3 causal blocks, and the one wide
@@ -51,7 +52,7 @@ struct GemmParams {
   void* D1;
   int64_t ldd1;
   int64_t n_split;
-  int splits;  // K ranges per tile (ADD_F32 only; partial sums added atomically)
+  int splits;  // K ranges per tile (ADD_F32 only; each range's partial sum is added by a TMA reduce-add)
   int d_tma;   // CTA pairs: D written (ADD_F32: added) by TMA from staged chunks (tensor map mD)
   int b_const; // CTA pairs: the first stages' B tiles are loaded before griddepcontrol.wait
   int* err;

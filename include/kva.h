@@ -25,7 +25,9 @@
  *   - Matrices are row-major.  Weights are [out, in] (the `in` dim contiguous).
  *     bf16 means IEEE bfloat16 stored in 2 bytes.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
- *     the legacy default stream).  They never synchronise and never allocate.
+ *     the legacy default stream).  They never synchronise and never allocate (the per-step
+ *     test entry point kva_op_gdn_scan of kva_ops.h, which has no handle, is the one call
+ *     that takes stream-ordered scratch).
  *   - Every call returns a kva_status.  Arguments are validated on the host
  *     before anything is enqueued; on an error nothing is launched.  Errors that
  *     only the device can see (page-table entry out of range, an internal wait
