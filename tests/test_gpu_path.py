@@ -538,7 +538,7 @@ def test_prefill_q8_0_projector_weights(K, geom, draft, fmt):
         Wt = K.Weights(proj=Wg, layer={k: v.cuda() for k, v in P.items()})
         pos = 0
         for T in splits:
-            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda") if mixer else None
+            mo = torch.empty(T, geom.n_mix, dtype=dt, device="cuda")
             do = torch.empty(T, geom.n_draft_cols, dtype=dt, device="cuda") if draft else None
             K.kva_prefill_ubatch(h, res[pos:pos + T].cuda(), Wt, S, tail, caches.c, pos, draft_out=do,
                                  mixer_out=mo)
