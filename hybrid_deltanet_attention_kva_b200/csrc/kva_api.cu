@@ -861,7 +861,6 @@ int kva_last_token_layer(kva_handle* h, int32_t layer, int32_t n_seq, const void
       g.eps = d.norm_eps;
       h->last_stream = s;
       e = staged(h, KVA_ST_LAST_TOKEN, s, [&] { return launch_gdn_decode(g, s); });
-      if (!e) ++h->launches[KVA_ST_LAST_TOKEN];  // two kernels
     }
   } else {
     const int n_q = lp->attn_n_q, dh = d.attn_d_h;

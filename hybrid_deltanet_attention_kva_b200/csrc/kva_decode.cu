@@ -10,8 +10,10 @@
 //   g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), then per state row v
 //       S[v,:] <- e^g S[v,:] + beta (v_v - e^g S[v,:].k) k,   o_v = S[v,:].q
 //   (the delta rule of one token), each row read and written once as 512-byte warp
-//   vectors; then the gated RMSNorm o = RMSNorm(o) * w * silu(z).  A second kernel shifts
-//   the conv tail after every head has read it.
+//   vectors (all of a warp's rows in flight before the first is used); then the gated
+//   RMSNorm o = RMSNorm(o) * w * silu(z).  The value heads of one key head form a cluster:
+//   each block shifts its own value channels of the conv tail once it has read them, and
+//   block 0 shifts the shared q and k channels after the cluster barrier.
 // Full-attention layer (split-K flash decoding):
 //   every CTA forms the token's k (RMSNorm + RoPE) and its query group (the n_q / n_kv
 //   query heads that read one KV head, RMSNorm + RoPE) in shared memory; split 0 writes
@@ -39,6 +41,18 @@ constexpr int DEC_THREADS = 128;
 template <int D>
 __device__ __forceinline__ uint32_t dsw(int row, int col) {
   return static_cast<uint32_t>(row * D * 2 + ((((col >> 3) ^ (row & 7)) << 4) | ((col & 7) * 2)));
+}
+
+// byte offset of (row, col) in a K or V tile of 64 rows: with TMA, D / 64 boxes of
+// [64 rows][64 dims] in the 128-byte swizzle the copy engine writes; with cp.async, rows of
+// D values whose 16-byte chunks are XOR-swizzled by the row (dsw)
+template <int D, bool TMA>
+__device__ __forceinline__ uint32_t toff(int row, int col) {
+  if constexpr (TMA)
+    return static_cast<uint32_t>((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                                 (col & 7) * 2);
+  else
+    return dsw<D>(row, col);
 }
 
 // RoPE on this lane's EPL consecutive dims (dims lane * EPL + i): pairs (i, i + half)
@@ -86,8 +100,11 @@ __device__ __forceinline__ T from_f(float x) {
 // gated-DeltaNet layer
 // ============================================================================
 template <int D, typename TX, typename TO>
-__global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p) {
+__global__ void __launch_bounds__(256) gdn_decode_kernel(const GdnDecodeLaunch p) {
   constexpr int EPL = D / 32;
+  constexpr int NW = 8;
+  constexpr int RPW = D / NW;  // state rows per warp, all loaded before any is used
+  using V = typename std::conditional<EPL == 4, float4, float2>::type;
   __shared__ float qv[D], kv[D], vv[D], zz[D], ov[D];
   __shared__ float sc[4];
   griddep_wait_and_release();
@@ -96,11 +113,17 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
   const int n_k = p.n_k, n_v = p.n_v, C = p.C;
   const int kh = h / (n_v / n_k);
   const TX* x = static_cast<const TX*>(p.x) + s * p.x_ld;
-  const TX* tail = static_cast<const TX*>(p.conv_state) + s * p.conv_seq_stride;  // [3][C]
+  TX* tail = static_cast<TX*>(p.conv_state) + s * p.conv_seq_stride;  // [3][C]
   const float4* w4 = reinterpret_cast<const float4*>(p.conv_w);
+  float* S = p.state + s * p.state_seq_stride + static_cast<int64_t>(h) * D * D;
+
+  // this warp's state rows start streaming in before anything else
+  V rows[RPW];
+#pragma unroll
+  for (int j = 0; j < RPW; ++j) rows[j] = reinterpret_cast<const V*>(S + (warp * RPW + j) * D)[lane];
 
   // causal conv over [tail; x] (tap 3 = this token) + SiLU on the head's q, k, v channels
-  for (int c = tid; c < 3 * D; c += 128) {
+  for (int c = tid; c < 3 * D; c += 256) {
     const int part = c / D, i = c - part * D;
     const int ch = part == 0 ? kh * D + i : part == 1 ? n_k * D + kh * D + i : 2 * n_k * D + h * D + i;
     const float4 w = w4[ch];
@@ -109,7 +132,7 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
     const float act = a / (1.f + expf(-a));
     (part == 0 ? qv : part == 1 ? kv : vv)[i] = act;
   }
-  for (int i = tid; i < D; i += 128) zz[i] = to_f(x[C + 2 * n_v + h * D + i]);
+  for (int i = tid; i < D; i += 256) zz[i] = to_f(x[C + 2 * n_v + h * D + i]);
   if (tid == 0) {
     const float a = to_f(x[C + h]) + p.dt_bias[h];
     const float b = to_f(x[C + n_v + h]);
@@ -117,7 +140,28 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
     sc[0] = expf(-expf(p.A_log[h]) * sp);  // e^g
     sc[1] = 1.f / (1.f + expf(-b));        // beta
   }
-  __syncthreads();
+  __syncthreads();  // every read of the old conv tail by this block is done
+  // the new conv tail [rows 1, 2; x]: this head's value channels (read by this block only)
+  // now; the key head's q and k channels, which the cluster's other blocks read too, by
+  // block 0 of the cluster after the cluster barrier
+  {
+    const int c0 = 2 * n_k * D + h * D;
+    for (int i = tid; i < D; i += 256) {
+      const TX t1 = tail[C + c0 + i], t2 = tail[2 * C + c0 + i];
+      tail[c0 + i] = t1;
+      tail[C + c0 + i] = t2;
+      tail[2 * C + c0 + i] = x[c0 + i];
+    }
+  }
+  cluster_sync();
+  if (cluster_ctarank() == 0)
+    for (int i = tid; i < 2 * D; i += 256) {
+      const int c = i < D ? kh * D + i : n_k * D + kh * D + (i - D);
+      const TX t1 = tail[C + c], t2 = tail[2 * C + c];
+      tail[c] = t1;
+      tail[C + c] = t2;
+      tail[2 * C + c] = x[c];
+    }
   if (warp < 2) {  // L2 norms of q (warp 0) and k (warp 1)
     float* arr = warp == 0 ? qv : kv;
     float ss = 0.f;
@@ -130,7 +174,7 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
   }
   __syncthreads();
 
-  // state rows: this lane's EPL consecutive columns of each row of this warp's block
+  // the one-token delta rule on this lane's EPL consecutive columns of each row
   float kr[EPL], qr[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
@@ -138,33 +182,24 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
     qr[i] = qv[lane * EPL + i];
   }
   const float eg = sc[0], beta = sc[1];
-  float* S = p.state + s * p.state_seq_stride + static_cast<int64_t>(h) * D * D;
-  constexpr int RPW = D / 4;  // rows per warp
-  constexpr int RB = 4;       // rows in flight
-  using V = typename std::conditional<EPL == 4, float4, float2>::type;
-#pragma unroll 1
-  for (int r0 = warp * RPW; r0 < (warp + 1) * RPW; r0 += RB) {
-    V rows[RB];
 #pragma unroll
-    for (int j = 0; j < RB; ++j) rows[j] = reinterpret_cast<const V*>(S + (r0 + j) * D)[lane];
+  for (int j = 0; j < RPW; ++j) {
+    const int r = warp * RPW + j;
+    float* e = reinterpret_cast<float*>(&rows[j]);
+    float sk = 0.f;
 #pragma unroll
-    for (int j = 0; j < RB; ++j) {
-      float* e = reinterpret_cast<float*>(&rows[j]);
-      float sk = 0.f;
+    for (int i = 0; i < EPL; ++i) sk += e[i] * kr[i];
+    sk = warp_sum(sk);
+    const float coef = beta * (vv[r] - eg * sk);
+    float o = 0.f;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) sk += e[i] * kr[i];
-      sk = warp_sum(sk);
-      const float coef = beta * (vv[r0 + j] - eg * sk);
-      float o = 0.f;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        e[i] = eg * e[i] + coef * kr[i];
-        o += e[i] * qr[i];
-      }
-      o = warp_sum(o);
-      reinterpret_cast<V*>(S + (r0 + j) * D)[lane] = rows[j];
-      if (lane == 0) ov[r0 + j] = o;
+    for (int i = 0; i < EPL; ++i) {
+      e[i] = eg * e[i] + coef * kr[i];
+      o += e[i] * qr[i];
     }
+    o = warp_sum(o);
+    reinterpret_cast<V*>(S + r * D)[lane] = rows[j];
+    if (lane == 0) ov[r] = o;
   }
   __syncthreads();
   if (warp == 0) {
@@ -176,25 +211,11 @@ __global__ void __launch_bounds__(128) gdn_decode_kernel(const GdnDecodeLaunch p
   }
   __syncthreads();
   TO* out = static_cast<TO*>(p.out) + s * p.out_ld + h * D;
-  const float r = sc[2];
-  for (int i = tid; i < D; i += 128) {
+  const float rr = sc[2];
+  for (int i = tid; i < D; i += 256) {
     const float z = zz[i];
-    out[i] = from_f<TO>(ov[i] * r * p.norm_w[i] * (z / (1.f + expf(-z))));
+    out[i] = from_f<TO>(ov[i] * rr * p.norm_w[i] * (z / (1.f + expf(-z))));
   }
-}
-
-// the new conv tail [tail rows 1, 2; x], after every head has read the old one
-template <typename TX>
-__global__ void __launch_bounds__(256) gdn_decode_tail_kernel(const GdnDecodeLaunch p) {
-  griddep_wait_and_release();
-  const int c = blockIdx.x * 256 + threadIdx.x, s = blockIdx.y;
-  if (c >= p.C) return;
-  TX* t = static_cast<TX*>(p.conv_state) + s * p.conv_seq_stride;
-  const TX* x = static_cast<const TX*>(p.x) + s * p.x_ld;
-  const TX t1 = t[p.C + c], t2 = t[2 * p.C + c];
-  t[c] = t1;
-  t[p.C + c] = t2;
-  t[2 * p.C + c] = x[c];
 }
 
 // ============================================================================
@@ -208,36 +229,40 @@ struct DecSmem {
   static constexpr int Q = V + DEC_STAGES * TILE_BYTES;          // [16][D] query group
   static constexpr int KN = Q + 16 * D * 2;                      // the token's k row
   static constexpr int VN = KN + D * 2;                          // and v row
-  static constexpr int BYTES = VN + D * 2;
+  static constexpr int BAR = VN + D * 2;                         // [stage] tile landed (TMA path)
+  static constexpr int MISC = BAR + DEC_STAGES * 8;              // abort flag
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;                     // slack for 1024-byte alignment
   // after the row loop, per warp: m[8], l[8], O[8][D] fp32 (inside the K tiles)
   static constexpr int MERGE_WARP = (16 + 8 * D) * 4;
   static_assert(4 * MERGE_WARP <= DEC_STAGES * TILE_BYTES, "merge area fits the tiles");
 };
 
-// address of cache row j of (sequence s, KV head kvh), or nullptr for a page-table entry
-// out of range (which sets the device status word)
-template <typename TC>
-__device__ __forceinline__ const TC* dec_row(const AttnDecodeLaunch& p, const void* base, int s, int kvh,
-                                             int64_t j) {
+// element offset of cache row j of (sequence s, KV head kvh) in the K and the V array (the
+// same for both), or -1 for a page-table entry out of range (which sets the device status word)
+__device__ __forceinline__ int64_t dec_row(const AttnDecodeLaunch& p, int s, int kvh, int64_t j) {
   if (p.layout == KVA_KV_PAGED) {
     const int64_t pi = j / p.page_size;
     const int page = pi < p.pages_per_seq ? p.page_table[static_cast<int64_t>(s) * p.pages_per_seq + pi] : -1;
     if (page < 0 || page >= p.n_pages) {
       set_device_error(p.err, KVA_DEV_PAGE_OOB);
-      return nullptr;
+      return -1;
     }
-    return static_cast<const TC*>(base) +
-           ((static_cast<int64_t>(page) * p.n_kv + kvh) * p.page_size + j % p.page_size) * p.d_h;
+    return ((static_cast<int64_t>(page) * p.n_kv + kvh) * p.page_size + j % p.page_size) * p.d_h;
   }
-  return static_cast<const TC*>(base) + ((static_cast<int64_t>(s) * p.n_kv + kvh) * p.max_pos + j) * p.d_h;
+  return ((static_cast<int64_t>(s) * p.n_kv + kvh) * p.max_pos + j) * p.d_h;
 }
 
-template <int D, typename TX, typename TC>
-__global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDecodeLaunch p) {
+template <int D, typename TX, typename TC, bool TMA>
+__global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const __grid_constant__ CUtensorMap mKc,
+                                                                  const __grid_constant__ CUtensorMap mVc,
+                                                                  const AttnDecodeLaunch p) {
   using L = DecSmem<D>;
   constexpr int EPL = D / 32;
   constexpr int CH = D / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t dsm[];
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
   const int G = p.G;
@@ -249,7 +274,89 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
   TC* qsm = reinterpret_cast<TC*>(dsm + L::Q);
   TC* knew = reinterpret_cast<TC*>(dsm + L::KN);
   TC* vnew = reinterpret_cast<TC*>(dsm + L::VN);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + L::BAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + L::MISC);
+  if (TMA && tid == 0) {
+    for (int i = 0; i < DEC_STAGES; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&mKc);
+    tma_prefetch_desc(&mVc);
+  }
   griddep_wait_and_release();
+
+  // ---- the row ring: rows r_begin .. r_end - 1 in 64-row tiles; the first tiles are
+  // requested before anything else, this token's own row goes in from shared memory later
+  const int64_t n_rows = r_end > r_begin ? r_end - r_begin : 0;
+  const int n_tiles = static_cast<int>((n_rows + DEC_TILE - 1) / DEC_TILE);
+  int issued = 0, last_ok = -1;  // thread 0 (TMA path): tiles requested, last tile seen landed
+  auto issue = [&](int t) {
+    const int st = t % DEC_STAGES;
+    const uint32_t kb = sbase + L::K + st * L::TILE_BYTES, vb = sbase + L::V + st * L::TILE_BYTES;
+    const int64_t j0 = r_begin + static_cast<int64_t>(t) * DEC_TILE;
+    if constexpr (TMA) {  // thread 0: the tile's D / 64 boxes of K and of V
+      int64_t y = j0, z = static_cast<int64_t>(s) * p.n_kv + kvh;
+      if (p.layout == KVA_KV_PAGED) {  // a tile lies inside one page (page_size % 64 == 0)
+        const int64_t pi = j0 / p.page_size;
+        int page = pi < p.pages_per_seq ? p.page_table[static_cast<int64_t>(s) * p.pages_per_seq + pi] : -1;
+        if (page < 0 || page >= p.n_pages) {
+          set_device_error(p.err, KVA_DEV_PAGE_OOB);
+          page = 0;  // read a valid page; the result is flagged
+        }
+        y = j0 % p.page_size;
+        z = static_cast<int64_t>(page) * p.n_kv + kvh;
+      }
+      mbar_arrive_expect_tx(&full[st], 2 * L::TILE_BYTES);
+#pragma unroll
+      for (int q = 0; q < D / 64; ++q) {
+        tma_load_3d(dsm + L::K + st * L::TILE_BYTES + q * 8192, &mKc, &full[st], 64 * q,
+                    static_cast<int>(y), static_cast<int>(z), l2_policy_evict_first());
+        tma_load_3d(dsm + L::V + st * L::TILE_BYTES + q * 8192, &mVc, &full[st], 64 * q,
+                    static_cast<int>(y), static_cast<int>(z), l2_policy_evict_first());
+      }
+      issued = t + 1;
+    } else {
+      const int c = tid % CH;
+      for (int r = tid / CH; r < DEC_TILE; r += DEC_THREADS / CH) {
+        const int64_t j = j0 + r;
+        if (j == pos) continue;
+        const uint32_t off = dsw<D>(r, 8 * c);
+        const int64_t o = j < r_end ? dec_row(p, s, kvh, j) : -1;
+        cp_async16(kb + off, static_cast<const TC*>(p.kc) + (o >= 0 ? o + 8 * c : 0), o >= 0 ? 16u : 0u);
+        cp_async16(vb + off, static_cast<const TC*>(p.vc) + (o >= 0 ? o + 8 * c : 0), o >= 0 ? 16u : 0u);
+      }
+    }
+  };
+  // this token's own row from shared memory; with TMA also zero V rows past the split's end
+  // (the copy engine read whatever the cache holds there, and 0 x NaN would poison the sum)
+  auto put_pos = [&](int t) {
+    const int st = t % DEC_STAGES;
+    const int64_t j0 = r_begin + static_cast<int64_t>(t) * DEC_TILE;
+    const int64_t r = pos - j0;
+    if (r >= 0 && r < DEC_TILE)
+      for (int c = tid; c < CH; c += DEC_THREADS) {
+        const uint32_t off = toff<D, TMA>(static_cast<int>(r), 8 * c);
+        *reinterpret_cast<uint4*>(dsm + L::K + st * L::TILE_BYTES + off) = reinterpret_cast<const uint4*>(knew)[c];
+        *reinterpret_cast<uint4*>(dsm + L::V + st * L::TILE_BYTES + off) = reinterpret_cast<const uint4*>(vnew)[c];
+      }
+    if (TMA && j0 + DEC_TILE > r_end)
+      for (int i = tid; i < DEC_TILE * CH; i += DEC_THREADS) {
+        const int rr = i / CH, c = i - rr * CH;
+        if (j0 + rr >= r_end)
+          *reinterpret_cast<uint4*>(dsm + L::V + st * L::TILE_BYTES + toff<D, TMA>(rr, 8 * c)) =
+              make_uint4(0u, 0u, 0u, 0u);
+      }
+  };
+  if constexpr (TMA) {
+    if (tid == 0)
+      for (int t = 0; t < DEC_STAGES - 1 && t < n_tiles; ++t) issue(t);
+  } else {
+#pragma unroll
+    for (int t = 0; t < DEC_STAGES - 1; ++t) {
+      if (t < n_tiles) issue(t);
+      cp_async_commit();
+    }
+  }
 
   // ---- the token's k (RMSNorm + RoPE), v, and the query group (RMSNorm + RoPE)
   const TX* x = static_cast<const TX*>(p.x) + s * p.x_ld;
@@ -281,12 +388,11 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
   for (int i = tid; i < D; i += DEC_THREADS) vnew[i] = F16<TC>::from(to_f(x[p.n_kv * D + kvh * D + i]));
   __syncthreads();
   if (split == 0) {  // the token's K and V rows go to the cache (no CTA reads them back)
-    TC* kd = const_cast<TC*>(dec_row<TC>(p, p.kc, s, kvh, pos));
-    TC* vd = const_cast<TC*>(dec_row<TC>(p, p.vc, s, kvh, pos));
-    if (kd && vd)
+    const int64_t o = dec_row(p, s, kvh, pos);
+    if (o >= 0)
       for (int i = tid; i < CH; i += DEC_THREADS) {
-        reinterpret_cast<uint4*>(kd)[i] = reinterpret_cast<const uint4*>(knew)[i];
-        reinterpret_cast<uint4*>(vd)[i] = reinterpret_cast<const uint4*>(vnew)[i];
+        reinterpret_cast<uint4*>(static_cast<TC*>(p.kc) + o)[i] = reinterpret_cast<const uint4*>(knew)[i];
+        reinterpret_cast<uint4*>(static_cast<TC*>(p.vc) + o)[i] = reinterpret_cast<const uint4*>(vnew)[i];
       }
   }
 
@@ -298,31 +404,12 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
     qa2[kk] = *reinterpret_cast<const uint32_t*>(dsm + L::Q + dsw<D>(lane >> 2, 16 * kk + 8 + 2 * (lane & 3)));
   }
 
-  // ---- the row ring
-  const int64_t n_rows = r_end > r_begin ? r_end - r_begin : 0;
-  const int n_tiles = static_cast<int>((n_rows + DEC_TILE - 1) / DEC_TILE);
-  auto issue = [&](int t) {
-    const int st = t % DEC_STAGES;
-    const uint32_t kb = sbase + L::K + st * L::TILE_BYTES, vb = sbase + L::V + st * L::TILE_BYTES;
-    for (int i = tid; i < DEC_TILE * CH; i += DEC_THREADS) {
-      const int r = i / CH, c = i - r * CH;
-      const int64_t j = r_begin + static_cast<int64_t>(t) * DEC_TILE + r;
-      const uint32_t off = dsw<D>(r, 8 * c);
-      if (j == pos) {  // this token's own row, from shared memory
-        *reinterpret_cast<uint4*>(dsm + L::K + st * L::TILE_BYTES + off) = reinterpret_cast<const uint4*>(knew)[c];
-        *reinterpret_cast<uint4*>(dsm + L::V + st * L::TILE_BYTES + off) = reinterpret_cast<const uint4*>(vnew)[c];
-        continue;
-      }
-      const TC* ks = j < r_end ? dec_row<TC>(p, p.kc, s, kvh, j) : nullptr;
-      const TC* vs = j < r_end ? dec_row<TC>(p, p.vc, s, kvh, j) : nullptr;
-      cp_async16(kb + off, ks ? ks + 8 * c : static_cast<const TC*>(p.kc), ks ? 16u : 0u);
-      cp_async16(vb + off, vs ? vs + 8 * c : static_cast<const TC*>(p.vc), vs ? 16u : 0u);
-    }
-  };
+  // the cp.async tiles of the prologue hold every row but this token's (put_pos, below); TMA
+  // tiles get theirs once they have landed
+  if constexpr (!TMA) {
 #pragma unroll
-  for (int t = 0; t < DEC_STAGES - 1; ++t) {
-    if (t < n_tiles) issue(t);
-    cp_async_commit();
+    for (int t = 0; t < DEC_STAGES - 1; ++t)
+      if (t < n_tiles) put_pos(t);
   }
 
   const float kNegInf = -__int_as_float(0x7f800000);
@@ -335,11 +422,28 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
 
 #pragma unroll 1
   for (int t = 0; t < n_tiles; ++t) {
-    if (t + DEC_STAGES - 1 < n_tiles) issue(t + DEC_STAGES - 1);
-    cp_async_commit();
-    cp_async_wait<DEC_STAGES - 1>();
-    __syncthreads();
     const int st = t % DEC_STAGES;
+    if constexpr (TMA) {
+      if (tid == 0 && !*abort_flag && t + DEC_STAGES - 1 < n_tiles) issue(t + DEC_STAGES - 1);
+      if (!*abort_flag) {
+        if (mbar_wait(&full[st], (t / DEC_STAGES) & 1, abort_flag)) {
+          if (tid == 0) last_ok = t;
+        } else {
+          *abort_flag = 1;
+          set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+        }
+      }
+      put_pos(t);
+      fence_proxy_async_smem();  // generic writes into a tile the copy engine refills later
+    } else {
+      if (t + DEC_STAGES - 1 < n_tiles) {
+        issue(t + DEC_STAGES - 1);
+        put_pos(t + DEC_STAGES - 1);
+      }
+      cp_async_commit();
+      cp_async_wait<DEC_STAGES - 1>();
+    }
+    __syncthreads();
     const uint32_t kb = sbase + L::K + st * L::TILE_BYTES, vb = sbase + L::V + st * L::TILE_BYTES;
     const int rw = 16 * warp;  // this warp's first row of the tile
 
@@ -348,7 +452,7 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t b[4];
-      ldmatrix_x4(b, kb + dsw<D>(rw + (mi >> 1) * 8 + lr, 16 * kk + (mi & 1) * 8));
+      ldmatrix_x4(b, kb + toff<D, TMA>(rw + (mi >> 1) * 8 + lr, 16 * kk + (mi & 1) * 8));
       const uint32_t a[4] = {qa0[kk], 0u, qa2[kk], 0u};
       const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
       F16<TC>::mma(sacc[0], a, b0);
@@ -392,13 +496,21 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
       o[mt][2] *= al0;
       o[mt][3] *= al1;
       uint32_t a[4];
-      ldmatrix_x4_trans(a, vb + dsw<D>(rw + (mi >> 1) * 8 + lr, 16 * mt + (mi & 1) * 8));
+      ldmatrix_x4_trans(a, vb + toff<D, TMA>(rw + (mi >> 1) * 8 + lr, 16 * mt + (mi & 1) * 8));
       const uint32_t av[4] = {a[0], a[1], a[2], a[3]};
       F16<TC>::mma(o[mt], av, pb);
     }
     __syncthreads();  // the stage is free for the next issue
   }
-  cp_async_wait<0>();
+  if constexpr (TMA) {
+    // every tile this block requested has landed before its shared memory is reused
+    if (tid == 0)
+      for (int t = last_ok + 1; t < issued; ++t)
+        if (!mbar_wait_limit(&full[t % DEC_STAGES], (t / DEC_STAGES) & 1))
+          set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+  } else {
+    cp_async_wait<0>();
+  }
   __syncthreads();
 
   // ---- merge the four warps' states, then write this split's partial
@@ -444,51 +556,86 @@ __global__ void __launch_bounds__(DEC_THREADS) attn_decode_kernel(const AttnDeco
   }
 }
 
-// every query head: merge the splits, divide by the softmax sum, apply sigmoid(gate)
+// every query head: merge the splits, divide by the softmax sum, apply sigmoid(gate).  The
+// splits' maxima and sums are staged in shared memory first, so each thread's sum over the
+// splits is a run of independent loads.
 template <int D, typename TX, typename TO>
 __global__ void __launch_bounds__(D) attn_decode_combine_kernel(const AttnDecodeLaunch p) {
+  __shared__ float wsm[kDecodeMaxSplit];  // per split: weight 2^(m - M)
+  __shared__ float lsum;
   griddep_wait_and_release();
   const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
   const int G = p.G, kvh = h / G, g = h - kvh * G;
   const float kNegInf = -__int_as_float(0x7f800000);
-  const float* base = p.part + (static_cast<int64_t>(s) * p.n_kv + kvh) * p.n_split * G * (D + 2) + g * (D + 2);
+  const int64_t stride = static_cast<int64_t>(G) * (D + 2);
+  const float* base = p.part + (static_cast<int64_t>(s) * p.n_kv + kvh) * p.n_split * stride + g * (D + 2);
   const int64_t rows = p.pos[s] + 1;
   const int ns = static_cast<int>((rows + p.rows_per_split - 1) / p.rows_per_split);
-  float M = kNegInf;
-  for (int i = 0; i < ns; ++i) M = fmaxf(M, base[static_cast<int64_t>(i) * G * (D + 2) + D]);
-  float O = 0.f, Ls = 0.f;
-  for (int i = 0; i < ns; ++i) {
-    const float* b = base + static_cast<int64_t>(i) * G * (D + 2);
-    const float m = b[D];
-    const float f = m == kNegInf ? 0.f : exp2f(m - M);
-    O += f * b[d];
-    Ls += f * b[D + 1];
+  if (d < 32) {  // one warp: the maxima, the weights, the softmax sum
+    float M = kNegInf;
+    for (int i = d; i < ns; i += 32) M = fmaxf(M, base[i * stride + D]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int i = d; i < ns; i += 32) {
+      const float m = base[i * stride + D];
+      const float f = m == kNegInf ? 0.f : exp2f(m - M);
+      wsm[i] = f;
+      L += f * base[i * stride + D + 1];
+    }
+    L = warp_sum(L);
+    if (d == 0) lsum = L;
   }
+  __syncthreads();
+  float O = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < ns; ++i) O += wsm[i] * base[i * stride + d];
   const TX* x = static_cast<const TX*>(p.x) + s * p.x_ld;
   const float gate = to_f(x[2 * p.n_kv * D + p.n_q * D + h * D + d]);
   TO* out = static_cast<TO*>(p.out) + s * p.out_ld + h * D;
-  out[d] = from_f<TO>(O / Ls * (1.f / (1.f + expf(-gate))));
+  out[d] = from_f<TO>(O / lsum * (1.f / (1.f + expf(-gate))));
 }
 
 template <typename TX, typename TO>
 int launch_gdn_decode_t(const GdnDecodeLaunch& g, cudaStream_t s) {
-  cudaError_t r;
-  dim3 grid(g.n_v, g.n_seq);
-  if (g.d == 128) r = launch_pdl(gdn_decode_kernel<128, TX, TO>, grid, dim3(128), 0, s, g);
-  else r = launch_pdl(gdn_decode_kernel<64, TX, TO>, grid, dim3(128), 0, s, g);
-  if (r != cudaSuccess) return KVA_ERR_CUDA;
-  r = launch_pdl(gdn_decode_tail_kernel<TX>, dim3((g.C + 255) / 256, g.n_seq), dim3(256), 0, s, g);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g.n_v, g.n_seq);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = g.n_v / g.n_k;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t r = g.d == 128 ? cudaLaunchKernelEx(&cfg, gdn_decode_kernel<128, TX, TO>, g)
+                                   : cudaLaunchKernelEx(&cfg, gdn_decode_kernel<64, TX, TO>, g);
   return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
 }
 
 template <int D, typename TX, typename TC, typename TO>
 int launch_attn_decode_t(const AttnDecodeLaunch& a, cudaStream_t s) {
-  const size_t smem = DecSmem<D>::BYTES;
-  if (cudaFuncSetAttribute(attn_decode_kernel<D, TX, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  const size_t smem = DecSmem<D>::ALLOC;
+  // TMA boxes of 64 rows need the rows of a tile in one page (page_size % 64 == 0)
+  const bool tma = a.layout == KVA_KV_CONTIGUOUS || a.page_size % DEC_TILE == 0;
+  CUtensorMap mK{}, mV{};
+  if (tma) {
+    const int64_t rows = a.layout == KVA_KV_CONTIGUOUS ? a.max_pos : a.page_size;
+    const int64_t planes = a.layout == KVA_KV_CONTIGUOUS ? static_cast<int64_t>(a.n_seq) * a.n_kv
+                                                         : static_cast<int64_t>(a.n_pages) * a.n_kv;
+    const bool f16 = a.cache_dtype == KVA_F16;
+    if (!make_map_3d_16bit(&mK, a.kc, f16, D, rows, planes, 64, DEC_TILE) ||
+        !make_map_3d_16bit(&mV, a.vc, f16, D, rows, planes, 64, DEC_TILE))
+      return KVA_ERR_CUDA;
+  }
+  auto kern = tma ? attn_decode_kernel<D, TX, TC, true> : attn_decode_kernel<D, TX, TC, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
     return KVA_ERR_CUDA;
-  cudaError_t r = launch_pdl(attn_decode_kernel<D, TX, TC>, dim3(a.n_split, a.n_kv, a.n_seq),
-                             dim3(DEC_THREADS), smem, s, a);
+  cudaError_t r = launch_pdl(kern, dim3(a.n_split, a.n_kv, a.n_seq), dim3(DEC_THREADS), smem, s, mK, mV, a);
   if (r != cudaSuccess) return KVA_ERR_CUDA;
   r = launch_pdl(attn_decode_combine_kernel<D, TX, TO>, dim3(a.n_q, a.n_seq), dim3(D), 0, s, a);
   return r == cudaSuccess ? KVA_OK : KVA_ERR_CUDA;
@@ -507,6 +654,7 @@ int launch_attn_decode_tc(const AttnDecodeLaunch& a, cudaStream_t s) {
 int launch_gdn_decode(const GdnDecodeLaunch& g, cudaStream_t s) {
   if (g.n_seq == 0) return KVA_OK;
   if (g.d != 64 && g.d != 128) return KVA_ERR_UNSUPPORTED;
+  if (g.n_v % g.n_k || g.n_v / g.n_k > 8) return KVA_ERR_UNSUPPORTED;  // portable cluster size
   const bool xf = g.x_dtype == KVA_F16, of32 = g.out_dtype == KVA_F32;
   if (xf) return of32 ? launch_gdn_decode_t<__half, float>(g, s) : launch_gdn_decode_t<__half, __half>(g, s);
   return of32 ? launch_gdn_decode_t<__nv_bfloat16, float>(g, s)
@@ -515,7 +663,8 @@ int launch_gdn_decode(const GdnDecodeLaunch& g, cudaStream_t s) {
 
 int attn_decode_splits(int n_seq, int n_kv, int64_t max_rows, int sms, int64_t* rows_per_split) {
   const int64_t tiles = (max_rows + DEC_TILE - 1) / DEC_TILE;
-  int64_t want = (2LL * sms + static_cast<int64_t>(n_seq) * n_kv - 1) / (static_cast<int64_t>(n_seq) * n_kv);
+  // one CTA per SM (three 64-row stages fill its shared memory): one wave of equal splits
+  int64_t want = sms / (static_cast<int64_t>(n_seq) * n_kv);
   if (want > kDecodeMaxSplit) want = kDecodeMaxSplit;
   if (want > tiles) want = tiles;
   if (want < 1) want = 1;
@@ -528,6 +677,7 @@ int launch_attn_decode(const AttnDecodeLaunch& a, cudaStream_t s) {
   if (a.n_seq == 0) return KVA_OK;
   if (a.d_h != 128 && a.d_h != 256) return KVA_ERR_UNSUPPORTED;
   if (a.G < 1 || a.G > 8 || a.n_q != a.G * a.n_kv) return KVA_ERR_UNSUPPORTED;
+  if (a.n_split < 1 || a.n_split > kDecodeMaxSplit) return KVA_ERR_INVALID_ARG;
   const int epl = a.d_h / 32;
   if (a.rope_dims < 0 || a.rope_dims % 2 || a.rope_dims > a.d_h) return KVA_ERR_UNSUPPORTED;
   if (a.rope_dims > 0) {

@@ -58,13 +58,205 @@ __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 // ============================================================================
 // chunk preparation
 // ============================================================================
+constexpr int LDB = 16 * 16 + 8;  // diagonal-block stride of the fp32 copies (floats)
+
+// Shared-memory views of one chunk's preparation, worked by four warps (threads 0-127):
+// warp w owns the 16 rows [16 w, 16 w + 16) of K K^T and L.
+struct PrepView {
+  uint32_t kb;      // K tile: two 128B-swizzled [64][64] halves (shared address)
+  uint32_t sL;      // L below the diagonal blocks, Tm on them: [64][64] fp16, t64 layout
+  uint8_t* L;       // the same tile, generic pointer
+  uint8_t* B1;      // B1 tile [64][64] fp16, t64 layout; blocks above the diagonal stay zero
+  float* Ld;        // the 4 diagonal blocks of L in fp32, stride LDB
+  float* ab;        // decay factors a[64], b[1..3][64]
+  float* gam;       // cumulative decay gam[64]
+  float* dec;       // e^(gam_last - gam)[64]
+  const float* gs;  // raw g[64] (0 past T)
+  const float* bs;  // beta[64] (0 past T)
+};
+
+// (1) K K^T for the blocks on and below the diagonal: warp w, column tiles [0, 2 w + 2) of 8
+__device__ __forceinline__ void prep_kkt(const PrepView& v, float (&acc)[8][4], int warp, int lane) {
+  const int mi = lane >> 3, lr = lane & 7;
+  const int mt = warp;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < SD / 16; ++ks) {
+    uint32_t a[4];
+    ldmatrix_x4(a, v.kb + kv_off(mt * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1)));
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      if (jj > mt) continue;
+      uint32_t bb[4];
+      ldmatrix_x4(bb, v.kb + kv_off(jj * 16 + (mi >> 1) * 8 + lr, ks * 2 + (mi & 1)));
+      const uint32_t b0[2] = {bb[0], bb[1]}, b1[2] = {bb[2], bb[3]};
+      mma_f16_16816(acc[2 * jj], a, b0);
+      mma_f16_16816(acc[2 * jj + 1], a, b1);
+    }
+  }
+}
+
+// (2) cumulative decays (one warp); the chain's scalars {e^gam[64], e^gam_last, 0...} go to
+//     `scg` (SC_FLOATS floats, 8-byte aligned)
+__device__ __forceinline__ void prep_decays(const PrepView& v, float* scg, int lane) {
+  const float v0 = v.gs[2 * lane], v1 = v.gs[2 * lane + 1];
+  const float pair = v0 + v1;
+  float incl = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const float ex = incl - pair;
+  const float total = __shfl_sync(0xffffffffu, incl, 31);
+  const float ga = ex + v0, gb2 = ex + pair;
+  v.gam[2 * lane] = ga;
+  v.gam[2 * lane + 1] = gb2;
+  v.dec[2 * lane] = expf(total - ga);
+  v.dec[2 * lane + 1] = expf(total - gb2);
+  *reinterpret_cast<float2*>(scg + 2 * lane) = make_float2(expf(ga), expf(gb2));
+  if (lane < (SC_FLOATS - SCH) / 2)
+    *reinterpret_cast<float2*>(scg + SCH + 2 * lane) = make_float2(lane == 0 ? expf(total) : 0.f, 0.f);
+  // below the diagonal blocks e^(gam_t - gam_s) = a_t b_i(s) with the reference
+  // r_i = gam at the last token of block i - 1 (t in block i, s < 16 i): both
+  // factors are at most 1, so neither overflows however strong the decay
+  const int bi = lane >> 3;  // block of tokens 2 lane, 2 lane + 1
+  float ref[4];
+#pragma unroll
+  for (int i = 1; i < 4; ++i) ref[i] = __shfl_sync(0xffffffffu, gb2, 8 * i - 1);
+  ref[0] = 0.f;
+  float rb = ref[1];
+#pragma unroll
+  for (int i = 2; i < 4; ++i) rb = bi == i ? ref[i] : rb;
+  v.ab[2 * lane] = bi ? __expf(ga - rb) : 1.f;
+  v.ab[2 * lane + 1] = bi ? __expf(gb2 - rb) : 1.f;
+#pragma unroll
+  for (int i = 1; i < 4; ++i) {
+    const bool below = 2 * lane < 16 * i;
+    v.ab[SCH * i + 2 * lane] = below ? __expf(ref[i] - ga) : 0.f;
+    v.ab[SCH * i + 2 * lane + 1] = below ? __expf(ref[i] - gb2) : 0.f;
+  }
+}
+
+// (3) L = beta_t e^(gam_t - gam_s) k_t.k_s below the diagonal: fp32 copies of the diagonal
+//     blocks (direct exponentials), fp16 blocks below them (factored decays)
+__device__ __forceinline__ void prep_l(const PrepView& v, const float (&acc)[8][4], int warp, int lane) {
+  const int g = lane >> 2, cq = lane & 3, mt = warp;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int sb = j >> 1;
+    if (sb > mt) continue;
+    const int s0 = j * 8 + 2 * cq;
+    if (sb == mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = mt * 16 + g + (e >> 1) * 8;
+        const int s = s0 + (e & 1);
+        v.Ld[mt * LDB + (t & 15) * 16 + (s & 15)] =
+            s < t ? v.bs[t] * __expf(v.gam[t] - v.gam[s]) * acc[j][e] : 0.f;
+      }
+    } else {
+      const int t0 = mt * 16 + g;
+      const float r0 = v.bs[t0] * v.ab[t0], r1 = v.bs[t0 + 8] * v.ab[t0 + 8];
+      const float c0 = v.ab[SCH * mt + s0], c1 = v.ab[SCH * mt + s0 + 1];
+      *reinterpret_cast<uint32_t*>(v.L + t64_elem(t0, s0)) = pack_f16(r0 * c0 * acc[j][0], r0 * c1 * acc[j][1]);
+      *reinterpret_cast<uint32_t*>(v.L + t64_elem(t0 + 8, s0)) = pack_f16(r1 * c0 * acc[j][2], r1 * c1 * acc[j][3]);
+    }
+  }
+}
+
+// (4) diagonal blocks of Tm = (I + L)^-1 in fp32, one row per thread (threads 0-63): row r
+//     of (I + L_b)^-1 solves x (I + L_b) = e_r; going from the last column down, x_p is
+//     final when reached and is eliminated from every earlier column (the FMAs of one step
+//     are independent).  Tm's blocks go to L's diagonal, B1's to B1.
+__device__ __forceinline__ void prep_diag(const PrepView& v, int tid) {
+  const int blk = tid >> 4, r = tid & 15;
+  const float* Lb = v.Ld + blk * LDB;
+  float x[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) x[q] = q == r ? 1.f : 0.f;
+#pragma unroll
+  for (int q2 = 15; q2 >= 1; --q2) {
+    float lrow[16];
+#pragma unroll
+    for (int v4 = 0; v4 < (q2 + 3) / 4; ++v4) {
+      const float4 l4 = reinterpret_cast<const float4*>(Lb + q2 * 16)[v4];
+      lrow[4 * v4] = l4.x;
+      lrow[4 * v4 + 1] = l4.y;
+      lrow[4 * v4 + 2] = l4.z;
+      lrow[4 * v4 + 3] = l4.w;
+    }
+#pragma unroll
+    for (int q = 0; q < q2; ++q) x[q] = fmaf(-x[q2], lrow[q], x[q]);
+  }
+  const int t = blk * 16 + r;
+  const float dt = v.dec[t];
+  const float* bb = v.bs + blk * 16;
+  uint32_t tm[8], bv[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    tm[q] = pack_f16(x[2 * q], x[2 * q + 1]);
+    bv[q] = pack_f16(dt * x[2 * q] * bb[2 * q], dt * x[2 * q + 1] * bb[2 * q + 1]);
+  }
+  *reinterpret_cast<uint4*>(v.L + t64_off(t, 2 * blk)) = make_uint4(tm[0], tm[1], tm[2], tm[3]);
+  *reinterpret_cast<uint4*>(v.L + t64_off(t, 2 * blk + 1)) = make_uint4(tm[4], tm[5], tm[6], tm[7]);
+  *reinterpret_cast<uint4*>(v.B1 + t64_off(t, 2 * blk)) = make_uint4(bv[0], bv[1], bv[2], bv[3]);
+  *reinterpret_cast<uint4*>(v.B1 + t64_off(t, 2 * blk + 1)) = make_uint4(bv[4], bv[5], bv[6], bv[7]);
+}
+
+// (5) blocks below the diagonal by column block jb, 8 columns (half hf) per task:
+//     X_ij = -Tm_ii sum_{k=jb}^{i-1} L_ik X_k,jb,  B1_ij = diag(dec) X_ij diag(beta).
+//     Warps 0 and 1 take column block 0 (three block rows), warps 2 and 3 column blocks 1
+//     then 2 (two and one).
+__device__ __forceinline__ void prep_offdiag_task(const PrepView& v, int jb, int hf, int lane) {
+  const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, lr = lane & 7;
+  const int s0 = 16 * jb + 8 * hf;
+  const int s = s0 + 2 * cq;
+  const float b0s = v.bs[s], b1s = v.bs[s + 1];
+#pragma unroll
+  for (int jj = 0; jj < 3; ++jj) {
+    if (jj != jb) continue;
+    uint32_t xf[4][2];
+    ldmatrix_x2_trans(xf[jj], v.sL + t64_off(16 * jj + (mi & 1) * 8 + lr, s0 >> 3));
+#pragma unroll
+    for (int i = jj + 1; i < 4; ++i) {
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = jj; k < i; ++k) {
+        uint32_t a[4];
+        ldmatrix_x4(a, v.sL + t64_off(16 * i + (mi & 1) * 8 + lr, 2 * k + (mi >> 1)));
+        mma_f16_16816(y, a, xf[k]);
+      }
+      const uint32_t yb[2] = {movmatrix_trans(pack_f16(y[0], y[1])), movmatrix_trans(pack_f16(y[2], y[3]))};
+      uint32_t a[4];
+      ldmatrix_x4(a, v.sL + t64_off(16 * i + (mi & 1) * 8 + lr, 2 * i + (mi >> 1)));
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16_16816(x, a, yb);
+      const int ta = 16 * i + g, tb2 = ta + 8;
+      const float d0 = v.dec[ta], d1 = v.dec[tb2];
+      *reinterpret_cast<uint32_t*>(v.B1 + t64_elem(ta, s)) = pack_f16(-d0 * x[0] * b0s, -d0 * x[1] * b1s);
+      *reinterpret_cast<uint32_t*>(v.B1 + t64_elem(tb2, s)) = pack_f16(-d1 * x[2] * b0s, -d1 * x[3] * b1s);
+      xf[i][0] = movmatrix_trans(pack_f16(-x[0], -x[1]));
+      xf[i][1] = movmatrix_trans(pack_f16(-x[2], -x[3]));
+    }
+  }
+}
+__device__ __forceinline__ void prep_offdiag(const PrepView& v, int warp, int lane) {
+  if (warp < 2) {
+    prep_offdiag_task(v, 0, warp, lane);
+  } else {
+    prep_offdiag_task(v, 1, warp - 2, lane);
+    prep_offdiag_task(v, 2, warp - 2, lane);
+  }
+}
+
 struct Cp {
   static constexpr int THREADS = 128;
   static constexpr int K = 0;                      // K chunk tile, 16 KB
   static constexpr int L = K + SCH * SD * 2;       // L below the diagonal blocks, Tm on them
   static constexpr int B1 = L + SCH * SCH * 2;     // B1 staging tile
-  static constexpr int LDB = 16 * 16 + 8;          // diagonal-block stride (floats)
-  static constexpr int LD = B1 + SCH * SCH * 2;    // diagonal blocks of L, fp32
+  static constexpr int LD = B1 + SCH * SCH * 2;    // diagonal blocks of L, fp32 (stride LDB)
   static constexpr int AB = LD + 4 * LDB * 4;      // decay factors a[64], b[1..3][64]
   static constexpr int GAM = AB + 4 * SCH * 4;     // gam[64], decay[64]
   static constexpr int GB = GAM + 2 * SCH * 4;     // g[64], beta[64]
@@ -83,7 +275,6 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* kbar = reinterpret_cast<uint64_t*>(sm + Cp::BAR);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, lr = lane & 7;
   const int h = blockIdx.x, c = blockIdx.y;
   const int slot = (blockIdx.z / nl) * p.n_gdn + l0 + blockIdx.z % nl;  // layers [l0, l0 + nl)
   const int T = p.T, n_v = p.n_v;
@@ -126,182 +317,16 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
   // zero-filled); on a timeout the status is set and the block carries on
   if (!mbar_wait_limit(kbar, 0)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
 
-  // (1) K K^T for the blocks on and below the diagonal: warp w, column tiles
-  //     [0, 2 w + 2) of 8
-  const int mt = warp;
+  const PrepView v{kb, sL, sm + Cp::L, B1, Ld, ab, gam, dec, gs, bs};
   float acc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < SD / 16; ++ks) {
-    uint32_t a[4];
-    ldmatrix_x4(a, kb + kv_off(mt * 16 + (mi & 1) * 8 + lr, ks * 2 + (mi >> 1)));
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      if (jj > mt) continue;
-      uint32_t bb[4];
-      ldmatrix_x4(bb, kb + kv_off(jj * 16 + (mi >> 1) * 8 + lr, ks * 2 + (mi & 1)));
-      const uint32_t b0[2] = {bb[0], bb[1]}, b1[2] = {bb[2], bb[3]};
-      mma_f16_16816(acc[2 * jj], a, b0);
-      mma_f16_16816(acc[2 * jj + 1], a, b1);
-    }
-  }
-  // (2) cumulative decays (warp 0, the one with the fewest K K^T tiles); the
-  //     chain's scalars go straight to global memory
-  if (warp == 0) {
-    const float v0 = gs[2 * lane], v1 = gs[2 * lane + 1];
-    const float pair = v0 + v1;
-    float incl = pair;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const float ex = incl - pair;
-    const float total = __shfl_sync(0xffffffffu, incl, 31);
-    const float ga = ex + v0, gb2 = ex + pair;
-    gam[2 * lane] = ga;
-    gam[2 * lane + 1] = gb2;
-    dec[2 * lane] = expf(total - ga);
-    dec[2 * lane + 1] = expf(total - gb2);
-    float* scg = p.scbuf + (head * n_chunks + c) * SC_FLOATS;
-    *reinterpret_cast<float2*>(scg + 2 * lane) = make_float2(expf(ga), expf(gb2));
-    if (lane < (SC_FLOATS - SCH) / 2)
-      *reinterpret_cast<float2*>(scg + SCH + 2 * lane) =
-          make_float2(lane == 0 ? expf(total) : 0.f, 0.f);
-    // below the diagonal blocks e^(gam_t - gam_s) = a_t b_i(s) with the reference
-    // r_i = gam at the last token of block i - 1 (t in block i, s < 16 i): both
-    // factors are at most 1, so neither overflows however strong the decay
-    const int bi = lane >> 3;  // block of tokens 2 lane, 2 lane + 1
-    float ref[4];
-#pragma unroll
-    for (int i = 1; i < 4; ++i) ref[i] = __shfl_sync(0xffffffffu, gb2, 8 * i - 1);
-    ref[0] = 0.f;
-    float rb = ref[1];
-#pragma unroll
-    for (int i = 2; i < 4; ++i) rb = bi == i ? ref[i] : rb;
-    ab[2 * lane] = bi ? __expf(ga - rb) : 1.f;
-    ab[2 * lane + 1] = bi ? __expf(gb2 - rb) : 1.f;
-#pragma unroll
-    for (int i = 1; i < 4; ++i) {
-      const bool below = 2 * lane < 16 * i;
-      ab[SCH * i + 2 * lane] = below ? __expf(ref[i] - ga) : 0.f;
-      ab[SCH * i + 2 * lane + 1] = below ? __expf(ref[i] - gb2) : 0.f;
-    }
-  }
+  prep_kkt(v, acc, warp, lane);
+  if (warp == 0) prep_decays(v, p.scbuf + (head * n_chunks + c) * SC_FLOATS, lane);
   __syncthreads();
-  // (3) L = beta_t e^(gam_t - gam_s) k_t.k_s below the diagonal: fp32 copies of the
-  //     diagonal blocks (direct exponentials), fp16 blocks below them (factored decays)
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int sb = j >> 1;
-    if (sb > mt) continue;
-    const int s0 = j * 8 + 2 * cq;
-    if (sb == mt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = mt * 16 + g + (e >> 1) * 8;
-        const int s = s0 + (e & 1);
-        Ld[mt * Cp::LDB + (t & 15) * 16 + (s & 15)] =
-            s < t ? bs[t] * __expf(gam[t] - gam[s]) * acc[j][e] : 0.f;
-      }
-    } else {
-      const int t0 = mt * 16 + g;
-      const float r0 = bs[t0] * ab[t0], r1 = bs[t0 + 8] * ab[t0 + 8];
-      const float c0 = ab[SCH * mt + s0], c1 = ab[SCH * mt + s0 + 1];
-      *reinterpret_cast<uint32_t*>(sm + Cp::L + t64_elem(t0, s0)) =
-          pack_f16(r0 * c0 * acc[j][0], r0 * c1 * acc[j][1]);
-      *reinterpret_cast<uint32_t*>(sm + Cp::L + t64_elem(t0 + 8, s0)) =
-          pack_f16(r1 * c0 * acc[j][2], r1 * c1 * acc[j][3]);
-    }
-  }
+  prep_l(v, acc, warp, lane);
   __syncthreads();
-  // (4) diagonal blocks of Tm = (I + L)^-1 in fp32, one row per thread: row r of
-  //     (I + L_b)^-1 solves x (I + L_b) = e_r; going from the last column down, x_p
-  //     is final when reached and is eliminated from every earlier column (the FMAs
-  //     of one step are independent)
-  if (tid < 64) {
-    const int blk = tid >> 4, r = tid & 15;
-    const float* Lb = Ld + blk * Cp::LDB;
-    float x[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) x[q] = q == r ? 1.f : 0.f;
-#pragma unroll
-    for (int q2 = 15; q2 >= 1; --q2) {
-      float lrow[16];
-#pragma unroll
-      for (int v4 = 0; v4 < (q2 + 3) / 4; ++v4) {
-        const float4 l4 = reinterpret_cast<const float4*>(Lb + q2 * 16)[v4];
-        lrow[4 * v4] = l4.x;
-        lrow[4 * v4 + 1] = l4.y;
-        lrow[4 * v4 + 2] = l4.z;
-        lrow[4 * v4 + 3] = l4.w;
-      }
-#pragma unroll
-      for (int q = 0; q < q2; ++q) x[q] = fmaf(-x[q2], lrow[q], x[q]);
-    }
-    const int t = blk * 16 + r;
-    const float dt = dec[t];
-    const float* bb = bs + blk * 16;
-    uint32_t tm[8], bv[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      tm[q] = pack_f16(x[2 * q], x[2 * q + 1]);
-      bv[q] = pack_f16(dt * x[2 * q] * bb[2 * q], dt * x[2 * q + 1] * bb[2 * q + 1]);
-    }
-    *reinterpret_cast<uint4*>(sm + Cp::L + t64_off(t, 2 * blk)) =
-        make_uint4(tm[0], tm[1], tm[2], tm[3]);
-    *reinterpret_cast<uint4*>(sm + Cp::L + t64_off(t, 2 * blk + 1)) =
-        make_uint4(tm[4], tm[5], tm[6], tm[7]);
-    *reinterpret_cast<uint4*>(B1 + t64_off(t, 2 * blk)) = make_uint4(bv[0], bv[1], bv[2], bv[3]);
-    *reinterpret_cast<uint4*>(B1 + t64_off(t, 2 * blk + 1)) = make_uint4(bv[4], bv[5], bv[6], bv[7]);
-  }
+  if (tid < 64) prep_diag(v, tid);
   __syncthreads();
-  // (5) blocks below the diagonal by column block jb, 8 columns (half hf) per task:
-  //     X_ij = -Tm_ii sum_{k=jb}^{i-1} L_ik X_k,jb,  B1_ij = diag(dec) X_ij diag(beta).
-  //     Warps 0 and 1 take column block 0 (three block rows), warps 2 and 3 column
-  //     blocks 1 then 2 (two and one).
-  auto offdiag = [&](const int jb, const int hf) {
-    const int s0 = 16 * jb + 8 * hf;
-    const int s = s0 + 2 * cq;
-    const float b0s = bs[s], b1s = bs[s + 1];
-#pragma unroll
-    for (int jj = 0; jj < 3; ++jj) {
-      if (jj != jb) continue;
-      uint32_t xf[4][2];
-      ldmatrix_x2_trans(xf[jj], sL + t64_off(16 * jj + (mi & 1) * 8 + lr, s0 >> 3));
-#pragma unroll
-      for (int i = jj + 1; i < 4; ++i) {
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = jj; k < i; ++k) {
-          uint32_t a[4];
-          ldmatrix_x4(a, sL + t64_off(16 * i + (mi & 1) * 8 + lr, 2 * k + (mi >> 1)));
-          mma_f16_16816(y, a, xf[k]);
-        }
-        const uint32_t yb[2] = {movmatrix_trans(pack_f16(y[0], y[1])),
-                                movmatrix_trans(pack_f16(y[2], y[3]))};
-        uint32_t a[4];
-        ldmatrix_x4(a, sL + t64_off(16 * i + (mi & 1) * 8 + lr, 2 * i + (mi >> 1)));
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16_16816(x, a, yb);
-        const int ta = 16 * i + g, tb2 = ta + 8;
-        const float d0 = dec[ta], d1 = dec[tb2];
-        *reinterpret_cast<uint32_t*>(B1 + t64_elem(ta, s)) =
-            pack_f16(-d0 * x[0] * b0s, -d0 * x[1] * b1s);
-        *reinterpret_cast<uint32_t*>(B1 + t64_elem(tb2, s)) =
-            pack_f16(-d1 * x[2] * b0s, -d1 * x[3] * b1s);
-        xf[i][0] = movmatrix_trans(pack_f16(-x[0], -x[1]));
-        xf[i][1] = movmatrix_trans(pack_f16(-x[2], -x[3]));
-      }
-    }
-  };
-  if (warp < 2) {
-    offdiag(0, warp);
-  } else {
-    offdiag(1, warp - 2);
-    offdiag(2, warp - 2);
-  }
+  prep_offdiag(v, warp, lane);
   __syncthreads();
   // (6) B1 to global memory, row-major [64][64] (16-byte pieces, coalesced)
   uint8_t* dst = static_cast<uint8_t*>(p.b1buf) + (head * n_chunks + c) * B1_BYTES;

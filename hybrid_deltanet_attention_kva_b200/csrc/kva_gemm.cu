@@ -1480,8 +1480,8 @@ bool make_map_3d_16bit(void* map, const void* base, bool fp16, int64_t d0, int64
   return r == CUDA_SUCCESS;
 }
 
-// Split-K factor for the residual-add GEMMs (whose partial sums are added
-// atomically): the number of K ranges s in [1, 8] (each at least 4 K blocks) that
+// Split-K factor for the residual-add GEMMs (whose partial sums are added by TMA
+// reduce-adds): the number of K ranges s in [1, 8] (each at least 4 K blocks) that
 // minimises the waves of work items per unit of K work, ceil(tiles * s / slots) / s,
 // with a small charge per extra split for its atomic traffic.
 static int choose_splits(int tiles, int slots, int num_k) {
