@@ -1001,6 +1001,29 @@ int kva_op_gemm(int32_t dtype, const void* A, int64_t lda, const void* const* B,
   return launch_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
+int kva_test_gemm_wait_timeout(int32_t dtype, const void* A, const void* B, void* D, int32_t M,
+                               int32_t N, int32_t K, int32_t* err, void* stream) {
+  if (!A || !B || !D || !err) return KVA_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return KVA_ERR_INVALID_ARG;
+  GemmArgs a;
+  a.A = A;
+  a.lda = K;
+  a.B[0] = B;
+  a.b_mode = KVA_B_SINGLE;
+  a.ldb = K;
+  a.D = D;
+  a.ldd = N;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.epilogue = KVA_EPI_STORE_BF16;
+  a.block_n = 512;  // the CTA-pair kernel
+  a.err = err;
+  a.dtype = dtype;
+  a.stall_item1 = 1;  // the first work item
+  return launch_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
 static int op_gemm_quant(int wq, int32_t dtype, const void* A, int64_t lda, const void* const* Bq,
                          const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
                          int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream) {

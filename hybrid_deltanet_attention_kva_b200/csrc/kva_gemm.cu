@@ -56,6 +56,8 @@ struct GemmParams {
   int d_tma;   // CTA pairs: D written (ADD_F32: added) by TMA from staged chunks (tensor map mD)
   int b_const; // CTA pairs: the first stages' B tiles are loaded before griddepcontrol.wait
   int* err;
+  int stall_item1;  // CTA pairs, test of the failure path: 1 + the work item whose MMA issuer
+                    // first waits on a barrier that nothing arrives on (0: never)
 };
 
 template <typename T>
@@ -1020,6 +1022,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
   (void)mix_stage;
   uint8_t* red_stage = reinterpret_cast<uint8_t*>(bars) + 1024;  // 1024-byte aligned
   (void)red_stage;
+  uint64_t* stallbar = bars + 18;  // nothing arrives on it (p.stall_item1)
+  static_assert(2 * S + 5 <= 18, "the stall barrier's slot is free");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1032,6 +1036,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       mbar_init(&empty[i], 1);
       if (WQ) mbar_init(&rawfull[i], 1);
     }
+    mbar_init(stallbar, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 2 * 32 * Cfg::epi_warps(EPI));  // every epilogue thread of both CTAs
@@ -1218,6 +1223,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int it = cid; it < items && ok; it += ncl) {
+        if (p.stall_item1 == it + 1) {
+          // test of the failure path: a wait that runs out (about a millisecond), then the
+          // abort and drain below, as for any pipeline wait that gives up
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(stallbar, 0))
+            if (globaltimer_ns() - t0 > 1000000ull) break;
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -1586,6 +1600,7 @@ static int launch_pair(const GemmArgs& a, cudaStream_t s) {
   p.n_split = a.n_split;
   p.err = a.err;
   p.b_const = a.b_const ? 1 : 0;
+  p.stall_item1 = a.stall_item1;
   // residual adds by TMA reduction when D is a plain fp32 matrix the tensor map can describe
   CUtensorMap mD = mA;
   p.d_tma = 0;

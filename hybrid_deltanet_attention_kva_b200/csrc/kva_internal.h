@@ -68,6 +68,9 @@ struct GemmArgs {
                             //   codes (uint8 [rows, K / 2], two per byte); fp16 scales Bs[i]
   const void* Bs[3] = {nullptr, nullptr, nullptr};  //   [K / 32, rows]
   int64_t lds = 0;          // wq: row stride of Bs in scales (0: the matrix's rows)
+  int stall_item1 = 0;      // CTA pairs, test of the failure path (kva_test_gemm_wait_timeout):
+                            //   1 + the work item whose MMA issuer waits on a barrier that
+                            //   nothing arrives on until the wait runs out (0: never)
 };
 
 int num_sms();

@@ -130,6 +130,7 @@ def _load() -> C.CDLL:
         "kva_op_attention": (I32, [I32, P, I64, P, I64, I32, I32, I32, P]),
         "kva_op_gdn_scan": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "kva_gdn_layer_update_noalloc": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, F32, P]),
+        "kva_test_gemm_wait_timeout": (I32, [I32, P, P, P, I32, I32, I32, P, P]),
         "kva_gdn_layer_update_noalloc_status": (I32, [P, C.POINTER(I32)]),
     }
     for name, (res, args) in sig.items():
@@ -146,7 +147,8 @@ EXPORTED = ("kva_init", "kva_workspace_bytes", "kva_prefill_ubatch", "kva_update
             "kva_profile_enable", "kva_profile_read",
             "kva_op_rmsnorm", "kva_op_gemm", "kva_op_gemm_q8_0", "kva_op_gemm_q4_0", "kva_op_attention",
             "kva_op_gdn_scan",
-            "kva_gdn_layer_update_noalloc", "kva_gdn_layer_update_noalloc_status")
+            "kva_gdn_layer_update_noalloc", "kva_gdn_layer_update_noalloc_status",
+            "kva_test_gemm_wait_timeout")
 
 
 def lib() -> C.CDLL:
@@ -464,3 +466,13 @@ def kva_gdn_layer_update_noalloc_status(stream=None) -> int:
     if rc not in (KVA_OK, KVA_ERR_DEVICE):
         _check(rc, "kva_gdn_layer_update_noalloc_status")
     return st.value
+
+
+def kva_test_gemm_wait_timeout(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor, err: torch.Tensor,
+                               stream=None) -> None:
+    """The CTA-pair GEMM with one pipeline wait made to run out (see include/kva_ops.h): the
+    kernel must come back with KVA_DEV_WAIT_TIMEOUT in the device int `err`."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check(_lib.kva_test_gemm_wait_timeout(_DT[A.dtype], _ptr(A), _ptr(B), _ptr(D), M, N, K, _ptr(err),
+                                           _stream(stream)), "kva_test_gemm_wait_timeout")

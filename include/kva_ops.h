@@ -54,6 +54,17 @@ int kva_op_gemm_q4_0(int32_t dtype, const void* A, int64_t lda, const void* cons
                      const void* const* Bs, int32_t b_mode, int64_t seg_rows, void* D, int64_t ldd,
                      int32_t M, int32_t N, int32_t K, int32_t epilogue, int32_t* err, void* stream);
 
+/* Test of the failure path of the pipelined kernels; the method has no counterpart to it.
+ * Runs kva_op_gemm's CTA-pair kernel (epilogue KVA_EPI_STORE_BF16, A [M, K], B [N, K], D
+ * [M, N], all row-major with the K or N dimension contiguous) with the MMA issuer of the
+ * first work item waiting on a barrier that nothing arrives on.  That wait runs out after
+ * about a millisecond; the kernel then raises its abort flag, lets every copy and MMA it
+ * issued land, and returns with KVA_DEV_WAIT_TIMEOUT set in the device int *err.  D is left
+ * partly written.  Other blocks may wait out their own limit (2 s) before they see the
+ * abort, so the call can take a few seconds.  Same size rules as kva_op_gemm. */
+int kva_test_gemm_wait_timeout(int32_t dtype, const void* A, const void* B, void* D, int32_t M,
+                               int32_t N, int32_t K, int32_t* err, void* stream);
+
 /* RMSNorm of `rows` rows of width n ("Qwen3.8-27B-KVA" model card, architecture):
  * out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g, out [rows, ldo] in out_dtype (bf16 / fp16).
  * x is [rows, ldx] in x_dtype.  n, ldx, ldo multiples of 4; pointers 16-byte aligned. */

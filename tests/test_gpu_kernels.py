@@ -343,3 +343,25 @@ def test_gemm_q8_0_swiglu_and_segments(K, dt):
                        N=3 * seg, b_mode=K.B_SEGMENTS, seg_rows=seg)
     want2 = a @ np.concatenate([p[2] for p in parts]).T
     assert_rms_close(D2, want2, tol=Q8_TOL[dt], what="q8_0 segments", elem=BF16_ELEM)
+
+
+def test_pipeline_wait_that_runs_out_is_reported_and_the_next_call_is_clean(K):
+    """Failure detection without a GPU fault: the CTA-pair GEMM's MMA issuer waits on a barrier
+    that nothing arrives on; the wait gives up after about a millisecond, the kernel drains its
+    own copies and MMAs and returns with KVA_DEV_WAIT_TIMEOUT in its status word.  The context
+    stays usable: the same GEMM right after is correct and reports nothing."""
+    torch.manual_seed(3)
+    M, N, Kd = 256, 256, 256
+    A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+    B = (torch.randn(N, Kd, device="cuda") * 0.05).half()
+    D = torch.zeros(M, N, dtype=torch.half, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kva_test_gemm_wait_timeout(A, B, D, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & K.KVA_DEV_WAIT_TIMEOUT
+    err.zero_()
+    K.kva_op_gemm(A, [B], D, N=N, epilogue=K.EPI_STORE_BF16, block_n=512, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = (A.float() @ B.float().T)
+    assert torch.allclose(D.float(), want, rtol=2e-3, atol=2e-3)
