@@ -897,11 +897,14 @@ struct PairCfg {
   static constexpr int raw_bytes(int wq) { return wq == 1 ? RAW_BYTES : (wq == 2 ? RAW_BYTES_Q4 : 0); }
   static constexpr int raw_codes(int wq) { return wq == 1 ? RAW_CODES : RAW_CODES_Q4; }
   // producer warp, MMA warp, the epilogue warps (eight for the state-update epilogue), then
-  // for q8_0 weights eight converter warps (two per 32-row quarter, one per 32-value block)
-  static constexpr int CONV_WARPS = 8;
+  // for quantized weights the converter warps: teams of four that take the stages in turn,
+  // each warp one 32-row quarter of the B half.  Three teams where the registers allow (576
+  // threads at up to 112 registers), two with the SwiGLU epilogue's larger register need.
+  static constexpr int conv_teams(int epi) { return epi == EPI_SWIGLU_BF16 ? 2 : 3; }
+  static constexpr int conv_warps(int epi) { return 4 * conv_teams(epi); }
   static constexpr int epi_warps(int epi) { return epi == EPI_MIXER ? MIX_EPI_WARPS : 4; }
   static constexpr int threads(int epi, int wq = 0) {
-    return 64 + 32 * (epi_warps(epi) + (wq ? CONV_WARPS : 0));
+    return 64 + 32 * (epi_warps(epi) + (wq ? conv_warps(epi) : 0));
   }
 };
 
@@ -1032,7 +1035,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], WQ ? 1 + 2 * Cfg::CONV_WARPS : 1);  // WQ: + both CTAs' converter warps
+      // WQ: + one converter team's warps of both CTAs
+      mbar_init(&full[i], WQ ? 1 + 2 * 4 : 1);
       mbar_init(&empty[i], 1);
       if (WQ) mbar_init(&rawfull[i], 1);
     }
@@ -1277,30 +1281,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
     }
   } else if (WQ && warp >= 2 + Cfg::epi_warps(EPI)) {
     // ------------------------------------------------ q8_0 converters (both CTAs)
-    // converter warp c owns rows 32 (c & 3) .. + 31 of this CTA's B half and the stage's
-    // 32-value block c >> 2: once a stage's raw codes and scales have landed it writes its
-    // part of the 16-bit B tile; each warp then arrives on the leader's full barrier (its
-    // stores made visible to the tensor cores first)
+    // converter team t (warps 4 t .. 4 t + 3) takes the k-blocks whose running count is t
+    // modulo the team count, so the teams' stages are converted at the same time; warp c
+    // of a team owns rows 32 c .. 32 c + 31 of this CTA's B half.  Once a stage's raw codes
+    // and scales have landed the warp writes its rows of the 16-bit B tile and arrives on
+    // the leader's full barrier (its stores made visible to the tensor cores first)
     const int cw = warp - 2 - Cfg::epi_warps(EPI);
-    const int r = (cw & 3) * 32 + lane, hb = cw >> 2;
-    int stage = 0;
+    const int team = cw / 4, r = (cw & 3) * 32 + lane;
+    int stage = 0, cnt = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int it = cid; it < items && ok; it += ncl) {
       int kb0, kb1;
       k_range(it, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&rawfull[stage], phase, abort_flag));
-        if (!ok) break;
-        if constexpr (WQ == 2)
-          q4_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
-        else
-          q8_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (leader) mbar_arrive(&full[stage]);
-          else mbar_arrive_remote(mapa_shared(smem_u32(&full[stage]), 0));
+      for (int kb = kb0; kb < kb1; ++kb, ++cnt) {
+        if (cnt % Cfg::conv_teams(EPI) == team) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&rawfull[stage], phase, abort_flag));
+          if (!ok) break;
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            if constexpr (WQ == 2)
+              q4_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
+            else
+              q8_0_dequant_block<T>(sR + stage * RAWB, sB + stage * Cfg::B_BYTES, r, hb);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive(&full[stage]);
+            else mbar_arrive_remote(mapa_shared(smem_u32(&full[stage]), 0));
+          }
         }
         if (++stage == S) {
           stage = 0;
