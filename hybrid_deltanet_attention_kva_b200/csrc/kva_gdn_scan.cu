@@ -253,11 +253,11 @@ __device__ __forceinline__ void prep_offdiag(const PrepView& v, int warp, int la
 
 struct Cp {
   static constexpr int THREADS = 128;
-  static constexpr int K = 0;                      // K chunk tile, 16 KB
+  static constexpr int K = 0;                      // K chunk tile, 16 KB; once K K^T is formed its
+  static constexpr int B1 = K;                     //   space holds the B1 staging tile
+  static constexpr int LD = K + SCH * SCH * 2;     //   and the diagonal blocks of L, fp32 (stride LDB)
   static constexpr int L = K + SCH * SD * 2;       // L below the diagonal blocks, Tm on them
-  static constexpr int B1 = L + SCH * SCH * 2;     // B1 staging tile
-  static constexpr int LD = B1 + SCH * SCH * 2;    // diagonal blocks of L, fp32 (stride LDB)
-  static constexpr int AB = LD + 4 * LDB * 4;      // decay factors a[64], b[1..3][64]
+  static constexpr int AB = L + SCH * SCH * 2;     // decay factors a[64], b[1..3][64]
   static constexpr int GAM = AB + 4 * SCH * 4;     // gam[64], decay[64]
   static constexpr int GB = GAM + 2 * SCH * 4;     // g[64], beta[64]
   static constexpr int BAR = GB + 2 * SCH * 4;
@@ -268,6 +268,7 @@ struct Cp {
 // grid (value head, chunk, sequence x layer in [l0, l0 + nl)): the value heads that share a key head
 // are neighbours, so their K tile is read from L2.  4 warps; warp w owns the 16
 // rows [16 w, 16 w + 16) of K K^T and L.
+static_assert(Cp::LD + 4 * LDB * 4 <= Cp::L, "B1 and the diagonal blocks fit the K tile's space");
 __global__ void __launch_bounds__(Cp::THREADS, 6)
     gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap mK, const GdnLaunch p, int l0, int nl) {
   extern __shared__ uint8_t smem_raw[];
@@ -294,8 +295,7 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
   const uint32_t kb = smem_u32(sm + Cp::K);
   griddep_wait_and_release();  // K, g and beta come from the kernels before
 
-  // K rows of the chunk, raw g and beta (zero past T: identity steps); the B1
-  // staging tile starts from zero (its blocks above the diagonal stay zero)
+  // K rows of the chunk, raw g and beta (zero past T: identity steps)
   if (tid == 0) {
     mbar_init(kbar, 1);
     fence_mbar_init();
@@ -309,8 +309,6 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
     const float* src =
         p.gbuf + (static_cast<int64_t>(slot) * 2 * n_v + (tid < SCH ? 0 : n_v) + h) * T;
     gs[tid] = t < T ? src[t] : 0.f;
-    for (int i = tid; i < B1_BYTES / 16; i += Cp::THREADS)
-      reinterpret_cast<uint4*>(B1)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();  // the barrier is initialised before anyone waits on it
   // every thread waits for the K tile (the load always completes: rows past T are
@@ -321,7 +319,10 @@ __global__ void __launch_bounds__(Cp::THREADS, 6)
   float acc[8][4];
   prep_kkt(v, acc, warp, lane);
   if (warp == 0) prep_decays(v, p.scbuf + (head * n_chunks + c) * SC_FLOATS, lane);
-  __syncthreads();
+  __syncthreads();  // K is read: its space takes B1 (from zero: the blocks above the diagonal
+                    // stay zero) and the diagonal blocks of L
+  for (int i = tid; i < B1_BYTES / 16; i += Cp::THREADS)
+    reinterpret_cast<uint4*>(B1)[i] = make_uint4(0u, 0u, 0u, 0u);
   prep_l(v, acc, warp, lane);
   __syncthreads();
   if (tid < 64) prep_diag(v, tid);
