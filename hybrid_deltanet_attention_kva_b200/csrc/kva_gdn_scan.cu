@@ -269,7 +269,7 @@ struct Cp {
 // are neighbours, so their K tile is read from L2.  4 warps; warp w owns the 16
 // rows [16 w, 16 w + 16) of K K^T and L.
 static_assert(Cp::LD + 4 * LDB * 4 <= Cp::L, "B1 and the diagonal blocks fit the K tile's space");
-__global__ void __launch_bounds__(Cp::THREADS, 6)
+__global__ void __launch_bounds__(Cp::THREADS, 8)
     gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap mK, const GdnLaunch p, int l0, int nl) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
