@@ -122,15 +122,29 @@ __global__ void __launch_bounds__(256) gdn_decode_kernel(const GdnDecodeLaunch p
 #pragma unroll
   for (int j = 0; j < RPW; ++j) rows[j] = reinterpret_cast<const V*>(S + (warp * RPW + j) * D)[lane];
 
-  // causal conv over [tail; x] (tap 3 = this token) + SiLU on the head's q, k, v channels
-  for (int c = tid; c < 3 * D; c += 256) {
+  // causal conv over [tail; x] (tap 3 = this token) + SiLU on the head's q, k, v channels.
+  // Thread t takes channel t of [q | k] and, for t < D, channel t of v; the raw values it
+  // reads are also the new conv tail [rows 1, 2; x] of those channels, written below.
+  TX qk_keep[3], v_keep[3];
+  int qk_ch = -1, v_ch = -1;
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int c = tid + pass * 256;
+    if (c >= 3 * D) break;
     const int part = c / D, i = c - part * D;
     const int ch = part == 0 ? kh * D + i : part == 1 ? n_k * D + kh * D + i : 2 * n_k * D + h * D + i;
     const float4 w = w4[ch];
-    const float a = w.x * to_f(tail[ch]) + w.y * to_f(tail[C + ch]) + w.z * to_f(tail[2 * C + ch]) +
-                    w.w * to_f(x[ch]);
+    const TX t0 = tail[ch], t1 = tail[C + ch], t2 = tail[2 * C + ch], xc = x[ch];
+    const float a = w.x * to_f(t0) + w.y * to_f(t1) + w.z * to_f(t2) + w.w * to_f(xc);
     const float act = a / (1.f + expf(-a));
     (part == 0 ? qv : part == 1 ? kv : vv)[i] = act;
+    if (part == 2) {
+      v_ch = ch;
+      v_keep[0] = t1, v_keep[1] = t2, v_keep[2] = xc;
+    } else {
+      qk_ch = ch;
+      qk_keep[0] = t1, qk_keep[1] = t2, qk_keep[2] = xc;
+    }
   }
   for (int i = tid; i < D; i += 256) zz[i] = to_f(x[C + 2 * n_v + h * D + i]);
   if (tid == 0) {
@@ -140,28 +154,21 @@ __global__ void __launch_bounds__(256) gdn_decode_kernel(const GdnDecodeLaunch p
     sc[0] = expf(-expf(p.A_log[h]) * sp);  // e^g
     sc[1] = 1.f / (1.f + expf(-b));        // beta
   }
-  __syncthreads();  // every read of the old conv tail by this block is done
-  // the new conv tail [rows 1, 2; x]: this head's value channels (read by this block only)
-  // now; the key head's q and k channels, which the cluster's other blocks read too, by
-  // block 0 of the cluster after the cluster barrier
-  {
-    const int c0 = 2 * n_k * D + h * D;
-    for (int i = tid; i < D; i += 256) {
-      const TX t1 = tail[C + c0 + i], t2 = tail[2 * C + c0 + i];
-      tail[c0 + i] = t1;
-      tail[C + c0 + i] = t2;
-      tail[2 * C + c0 + i] = x[c0 + i];
-    }
+  // the new conv tail: this head's value channels (read by this block only) at once; the key
+  // head's q and k channels, which the cluster's other blocks read too, by block 0 of the
+  // cluster after the cluster barrier
+  if (v_ch >= 0) {
+    tail[v_ch] = v_keep[0];
+    tail[C + v_ch] = v_keep[1];
+    tail[2 * C + v_ch] = v_keep[2];
   }
+  __syncthreads();
   cluster_sync();
-  if (cluster_ctarank() == 0)
-    for (int i = tid; i < 2 * D; i += 256) {
-      const int c = i < D ? kh * D + i : n_k * D + kh * D + (i - D);
-      const TX t1 = tail[C + c], t2 = tail[2 * C + c];
-      tail[c] = t1;
-      tail[C + c] = t2;
-      tail[2 * C + c] = x[c];
-    }
+  if (cluster_ctarank() == 0 && qk_ch >= 0) {
+    tail[qk_ch] = qk_keep[0];
+    tail[C + qk_ch] = qk_keep[1];
+    tail[2 * C + qk_ch] = qk_keep[2];
+  }
   if (warp < 2) {  // L2 norms of q (warp 0) and k (warp 1)
     float* arr = warp == 0 ? qv : kv;
     float ss = 0.f;
