@@ -19,14 +19,16 @@
 // 2. gdn_scan_tc_kernel, one CTA per (sequence, layer, value head), two CTAs per
 //    SM: the state S (128 x 128 fp32) lives in tensor memory for the whole ubatch,
 //    TMEM lane v holding state row v.  Per chunk, eight warps (two per TMEM lane
-//    quarter, each owning half of the columns) and one issuing thread run
+//    quarter, each owning half of the columns) and one elected lane of warp 0 run
 //        pass 1: A <- fp16(S)                            (tcgen05.ld / st)
 //        MMA   : Y  = A K^T             | S <- e^gam_last S meanwhile
-//        pass 2: A <- fp16(-Y diag(e^gam))
-//        MMA   : D  = V^T B1^T + A B1^T                 (V^T as an MN-major operand)
+//        pass 2: A <- fp16(V^T - Y diag(e^gam))          (V rows read from shared memory)
+//        MMA   : D  = A B1^T
 //        pass 3: A <- fp16(D)
 //        MMA   : S += A K                                (K as an MN-major operand)
-//    K, V and B1 of the next chunk arrive by TMA while a chunk runs.  Every wait
+//    Rounding V^T - Y diag(e^gam) once (the chunk's corrected values before B1) keeps
+//    the round to four instructions.  K, V and B1 of the next chunk arrive by TMA,
+//    issued by one thread of warp 1 while the tensor cores form Y.  Every wait
 //    is bounded; on a timeout the block raises its abort flag, runs the remaining
 //    steps without waiting or issuing, drains its own copies and MMAs, and returns
 //    with the device status set.
@@ -347,6 +349,7 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_S = 0;    // state, fp32 128 x 128
 constexpr uint32_t COL_A = 128;  // 16-bit A operand (up to 128 x 128)
 constexpr uint32_t COL_Y = 192;  // Y, then D: fp32 128 x 64
+constexpr int kLoader = 32;      // the thread (warp 1) that issues the chunk loads
 
 struct Sc {
   static constexpr int KT = SCH * SD * 2;     // K or V chunk: two [64][64] 128B-swizzled halves
@@ -364,7 +367,6 @@ struct Sc {
 };
 
 constexpr uint32_t ID_Y = idesc_f16kind_f32_major(128, 64, 0, false, false);   // TMEM A, K-major B
-constexpr uint32_t ID_VB = idesc_f16kind_f32_major(128, 64, 0, true, false);   // MN-major A
 constexpr uint32_t ID_S = idesc_f16kind_f32_major(128, 128, 0, false, true);   // MN-major B
 
 __global__ void __launch_bounds__(NTHREADS, 2)
@@ -415,23 +417,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const uint32_t tY = tb + lrow + COL_Y + 32 * hc;  // this thread's 32 Y / D columns
   float* Sg = p.state + static_cast<int64_t>(head) * SD * SD + (32 * qd + lane) * SD + 64 * hc;
 
-#pragma unroll 1
-  for (int q = 0; q < 2; ++q) {
-    uint32_t r[32];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 v = reinterpret_cast<const float4*>(Sg + 32 * q)[j];
-      r[4 * j] = __float_as_uint(v.x);
-      r[4 * j + 1] = __float_as_uint(v.y);
-      r[4 * j + 2] = __float_as_uint(v.z);
-      r[4 * j + 3] = __float_as_uint(v.w);
-    }
-    tmem_st_32x32b_x32(tS + 32 * q, r);
-  }
-  tmem_st_wait();
-
   const uint64_t pol_k = l2_policy_evict_normal(), pol_v = l2_policy_evict_first();
-  int issued = 0;  // chunks whose operands were requested (thread 0)
+  int issued = 0;  // chunks whose operands were requested (the loader thread)
   auto load = [&](int c) {
     const int s = c & 1;
     uint64_t* bar = &full[s];
@@ -447,15 +434,23 @@ __global__ void __launch_bounds__(NTHREADS, 2)
               p.scbuf + (static_cast<int64_t>(head) * n_chunks + c) * SC_FLOATS, SC_FLOATS * 4, bar);
     issued = c + 1;
   };
-  auto prefetch = [&](int c) {
-    tma_prefetch_l2_3d(&mK, kh * SD, c * SCH, slot);
-    tma_prefetch_l2_3d(&mK, kh * SD + 64, c * SCH, slot);
-    tma_prefetch_l2_3d(&mV, h * SD, c * SCH, slot);
-    tma_prefetch_l2_3d(&mV, h * SD + 64, c * SCH, slot);
-    tma_prefetch_l2_3d(&mB, 0, c * SCH, head);
-  };
-  if (tid == 0) load(0);
+  // the first chunk's operands are requested before the state is read, so the two overlap
+  if (tid == kLoader) load(0);
   __syncwarp();
+#pragma unroll 1
+  for (int q = 0; q < 2; ++q) {
+    uint32_t r[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = reinterpret_cast<const float4*>(Sg + 32 * q)[j];
+      r[4 * j] = __float_as_uint(v.x);
+      r[4 * j + 1] = __float_as_uint(v.y);
+      r[4 * j + 2] = __float_as_uint(v.z);
+      r[4 * j + 3] = __float_as_uint(v.w);
+    }
+    tmem_st_32x32b_x32(tS + 32 * q, r);
+  }
+  tmem_st_wait();
 
   bool ok = true;
   for (int c = 0; c < n_chunks; ++c) {
@@ -464,13 +459,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (!*abort_flag) ok &= mbar_wait(&full[s], (c >> 1) & 1, abort_flag);
     if (c > 0 && !*abort_flag) ok &= mbar_wait(done, (c - 1) & 1, abort_flag);
     tc_fence_after();
-    // the slot of chunk c - 1 is free: the next chunk's operands go there
-    if (tid == 0 && !*abort_flag) {
-      if (c + 1 < n_chunks) load(c + 1);
-      if (c + 2 < n_chunks) prefetch(c + 2);
-    }
-    __syncwarp();
     const uint32_t kb = smem_u32(sm + Sc::K + s * Sc::KT);
+    const uint64_t dKk = sdesc_k_sw128(kb), dKm = sdesc_mn_sw128(kb, Sc::HALF);
 
     // pass 1: A <- fp16(S); the state values stay in registers for the rescale
     uint32_t r0[32], r1[32];
@@ -489,15 +479,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
-      if (!*abort_flag) {
+      if (elect_one() && !*abort_flag) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          umma_f16_ts(tb + COL_Y, tb + COL_A + 8 * j,
-                      sdesc_k_sw128(kb + (j >> 2) * Sc::HALF + (j & 3) * 32), ID_Y, j > 0);
+          umma_f16_ts(tb + COL_Y, tb + COL_A + 8 * j, dKk + (((j >> 2) * Sc::HALF + (j & 3) * 32) >> 4),
+                      ID_Y, j > 0);
         umma_commit(ybar);
       }
+    } else if (tid == kLoader && !*abort_flag && c + 1 < n_chunks) {
+      // the slot of chunk c - 1 is free (its MMAs completed before this chunk began, its
+      // scalars and V rows were read before the barrier above): the next chunk's operands
+      // go there while the tensor cores form Y (an L2 prefetch of the chunk after would put
+      // five more TMA instructions, about 90 cycles each, on this thread)
+      load(c + 1);
     }
     __syncwarp();
     // S <- e^gam_last S while the tensor cores form Y (those MMAs read only A and K)
@@ -514,34 +510,40 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (!*abort_flag) ok &= mbar_wait(ybar, c & 1, abort_flag);
     tc_fence_after();
 
-    // pass 2: A <- fp16(-Y diag(e^gam)), this thread's 32 columns
+    // pass 2: A <- fp16(V^T - Y diag(e^gam)), this thread's 32 columns (tokens); the
+    // thread's value row of V comes from the swizzled tile while Y is read
     {
-      uint32_t r[32], a[16];
+      uint32_t r[32], vp[16], a[16];
       tmem_ld_32x32b_x32(tY, r);
+      const uint8_t* vt = sm + Sc::V + s * Sc::KT;
+      const int vr = 32 * qd + lane;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = 32 * hc + 2 * j;
+        const uint32_t lo = *reinterpret_cast<const uint16_t*>(vt + kv_off(t, vr >> 3) + (vr & 7) * 2);
+        const uint32_t hi = *reinterpret_cast<const uint16_t*>(vt + kv_off(t + 1, vr >> 3) + (vr & 7) * 2);
+        vp[j] = lo | (hi << 16);
+      }
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float4 e = reinterpret_cast<const float4*>(sc + 32 * hc)[j];
-        a[2 * j] = pack_f16(-e.x * u2f(r[4 * j]), -e.y * u2f(r[4 * j + 1]));
-        a[2 * j + 1] = pack_f16(-e.z * u2f(r[4 * j + 2]), -e.w * u2f(r[4 * j + 3]));
+        const float2 v0 = F16<__half>::unpack(vp[2 * j]), v1 = F16<__half>::unpack(vp[2 * j + 1]);
+        a[2 * j] = pack_f16(v0.x - e.x * u2f(r[4 * j]), v0.y - e.y * u2f(r[4 * j + 1]));
+        a[2 * j + 1] = pack_f16(v1.x - e.z * u2f(r[4 * j + 2]), v1.y - e.w * u2f(r[4 * j + 3]));
       }
       tmem_st_32x32b_x16(tA + 16 * hc, a);
     }
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
-      if (!*abort_flag) {
-        const uint32_t vb = smem_u32(sm + Sc::V + s * Sc::KT);
-        const uint32_t bb = smem_u32(sm + Sc::B1 + s * B1_BYTES);
+      if (elect_one() && !*abort_flag) {
+        const uint64_t dB = sdesc_k_sw128(smem_u32(sm + Sc::B1 + s * B1_BYTES));
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          umma_f16_ss(tb + COL_Y, sdesc_mn_sw128(vb + j * 2048, Sc::HALF), sdesc_k_sw128(bb + j * 32),
-                      ID_VB, j > 0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          umma_f16_ts(tb + COL_Y, tb + COL_A + 8 * j, sdesc_k_sw128(bb + j * 32), ID_Y, 1);
+          umma_f16_ts(tb + COL_Y, tb + COL_A + 8 * j, dB + ((j * 32) >> 4), ID_Y, j > 0);
         umma_commit(dbar);
       }
     }
@@ -561,12 +563,12 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
-      if (!*abort_flag) {
+      if (elect_one() && !*abort_flag) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          umma_f16_ts(tb + COL_S, tb + COL_A + 8 * j, sdesc_mn_sw128(kb + j * 2048, Sc::HALF), ID_S, 1);
+          umma_f16_ts(tb + COL_S, tb + COL_A + 8 * j, dKm + ((j * 2048) >> 4), ID_S, 1);
         umma_commit(done);
       }
     }
@@ -588,15 +590,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       reinterpret_cast<float4*>(Sg + 32 * q)[j] =
           make_float4(u2f(r[4 * j]), u2f(r[4 * j + 1]), u2f(r[4 * j + 2]), u2f(r[4 * j + 3]));
   }
-  if (tid == 0) {
-    // every copy and MMA this block issued has landed before it exits
+  // every copy and MMA this block issued has landed before it exits
+  if (tid == kLoader) {
     for (int s = 0; s < 2; ++s)
       if (issued > s) {
         const int cl = s + 2 * ((issued - 1 - s) / 2);
         if (!mbar_wait_limit(&full[s], (cl >> 1) & 1)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
       }
-    umma_commit(drain);
-    if (!mbar_wait_limit(drain, 0)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+  }
+  if (warp == 0) {
+    if (elect_one()) {
+      umma_commit(drain);
+      if (!mbar_wait_limit(drain, 0)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -106,7 +106,7 @@ int kva_op_gdn_scan(const void* k, const void* v, const float* gb, float* state,
                     int32_t n_layers, int32_t T, int32_t n_k, int32_t n_v, int32_t d,
                     void* stream);
 
-/* Limits of kva_gdn_layer_update_noalloc's fixed scratch (about 6.6 MB per GPU). */
+/* Limits of kva_gdn_layer_update_noalloc's fixed scratch (about 6.5 MB per GPU). */
 #define KVA_NOALLOC_MAX_T 256    /* tokens per call */
 #define KVA_NOALLOC_MAX_QK 2048  /* n_k * d */
 #define KVA_NOALLOC_MAX_V 6144   /* n_v * d */
