@@ -168,25 +168,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
     }
   } else if (warp == 9) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------ MMA issuer
+      // (the warp runs the loop converged and one elected lane issues)
       constexpr uint32_t idS = idesc_f16kind_f32(ATT_BQ, ATT_BKV, F16<E>::umma_fmt);
       constexpr uint32_t idO = idesc_f16kind_f32_major(ATT_BQ, ATT_D, F16<E>::umma_fmt, false, true);
       const uint32_t sQ = smem_u32(sm);
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      const uint32_t issuer = elect_one();  // elected once: a commit tracks its own lane's MMAs
+      bool ok = mbar_wait_warp(bar_q, 0, abort_flag);
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(&fullK[s], (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&fullK[s], (j >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t sK = smem_u32(sm + ATT_OFF_K + s * ATT_TILE);
+        if (issuer) {
 #pragma unroll
-        for (int k = 0; k < ATT_D / 16; ++k) {  // 16 dims per MMA: half k / 4, 32 bytes each
-          const uint32_t off = (k >> 2) * ATT_HALF + (k & 3) * 32;
-          umma_f16_ss(tb + ATT_COL_S + s * 128, sdesc_k_sw128(sQ + off), sdesc_k_sw128(sK + off), idS,
-                      k > 0 ? 1u : 0u);
+          for (int k = 0; k < ATT_D / 16; ++k) {  // 16 dims per MMA: half k / 4, 32 bytes each
+            const uint32_t off = (k >> 2) * ATT_HALF + (k & 3) * 32;
+            umma_f16_ss(tb + ATT_COL_S + s * 128, sdesc_k_sw128(sQ + off), sdesc_k_sw128(sK + off), idS,
+                        k > 0 ? 1u : 0u);
+          }
+          umma_commit(&barS[s]);
+          umma_commit(&emptyK[s]);
         }
-        umma_commit(&barS[s]);
-        umma_commit(&emptyK[s]);
+        __syncwarp();
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -196,27 +201,33 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           ok = false;
           break;
         }
-        if (!mbar_wait(&barP[s], (j >> 1) & 1, abort_flag) ||
-            !mbar_wait(&fullV[s], (j >> 1) & 1, abort_flag)) {
+        if (!mbar_wait_warp(&barP[s], (j >> 1) & 1, abort_flag) ||
+            !mbar_wait_warp(&fullV[s], (j >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t sV = smem_u32(sm + ATT_OFF_V + s * ATT_TILE);
+        if (issuer) {
 #pragma unroll
-        for (int k = 0; k < ATT_BKV / 16; ++k)  // 16 keys per MMA: 8 columns of P, 16 rows of V
-          umma_f16_ts(tb + ATT_COL_O, tb + ATT_COL_P + s * 64 + k * 8,
-                      sdesc_mn_sw128(sV + k * 2048, ATT_HALF), idO, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(barO);
-        umma_commit(&emptyV[s]);
+          for (int k = 0; k < ATT_BKV / 16; ++k)  // 16 keys per MMA: 8 columns of P, 16 rows of V
+            umma_f16_ts(tb + ATT_COL_O, tb + ATT_COL_P + s * 64 + k * 8,
+                        sdesc_mn_sw128(sV + k * 2048, ATT_HALF), idO, (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit(barO);
+          umma_commit(&emptyV[s]);
+        }
+        __syncwarp();
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         *abort_flag = 1;
         set_device_error(err, KVA_DEV_WAIT_TIMEOUT);
       }
       // every MMA issued completes before TMEM is released
-      umma_commit(bar_drain);
-      mbar_wait_limit(bar_drain, 0);
+      if (issuer) {
+        umma_commit(bar_drain);
+        mbar_wait_limit(bar_drain, 0);
+      }
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------ softmax and output (warps 0-7)

@@ -97,6 +97,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// mbar_wait by every lane of a converged warp; the warp agrees on the outcome (a lane
+// that gave up makes the whole warp give up), so it stays converged for elect_one().
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait<kCluster>(bar, parity, abort_flag));
+}
+
 // Wait with the time limit only (for draining the block's own copies and MMAs
 // before it exits, whatever the abort flag says).
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity) {

@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   }
   tmem_st_wait();
 
+  // warp 0's issuing lane, elected once: a commit tracks only its own lane's MMAs
+  const uint32_t issuer = warp == 0 ? elect_one() : 0u;
   bool ok = true;
   for (int c = 0; c < n_chunks; ++c) {
     const int s = c & 1;
@@ -481,7 +483,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
-      if (elect_one() && !*abort_flag) {
+      if (issuer && !*abort_flag) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           umma_f16_ts(tb + COL_Y, tb + COL_A + 8 * j, dKk + (((j >> 2) * Sc::HALF + (j & 3) * 32) >> 4),
@@ -539,7 +541,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
-      if (elect_one() && !*abort_flag) {
+      if (issuer && !*abort_flag) {
         const uint64_t dB = sdesc_k_sw128(smem_u32(sm + Sc::B1 + s * B1_BYTES));
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
-      if (elect_one() && !*abort_flag) {
+      if (issuer && !*abort_flag) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           umma_f16_ts(tb + COL_S, tb + COL_A + 8 * j, dKm + ((j * 2048) >> 4), ID_S, 1);
@@ -599,7 +601,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
   }
   if (warp == 0) {
-    if (elect_one()) {
+    if (issuer) {
       umma_commit(drain);
       if (!mbar_wait_limit(drain, 0)) set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
     }

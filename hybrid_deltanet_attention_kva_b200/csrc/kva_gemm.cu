@@ -11,9 +11,9 @@
 //   warp 0      TMA producer: A tile [128 x 64] and this CTA's B tile per stage,
 //               128-byte swizzle, into a STAGES-deep shared-memory ring (the
 //               weights' first stages are requested before the PDL wait).
-//   warp 1      TMEM allocator + single-thread MMA issuer: 4 tcgen05.mma (K = 16)
-//               per stage into one of two TMEM accumulators, tcgen05.commit frees
-//               the stage.
+//   warp 1      TMEM allocator + MMA issuer (the warp waits converged, one elected
+//               lane issues): 4 tcgen05.mma (K = 16) per stage into one of two TMEM
+//               accumulators, tcgen05.commit frees the stage.
 //   warps 2..   epilogue, while the MMA warp accumulates the next tile in the other
 //               TMEM buffer: 16-bit stores and residual adds through per-warp
 //               shared staging and TMA (bulk stores / reduce-adds), SwiGLU, or the
@@ -292,16 +292,18 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------ MMA issuer
+      // (the warp runs the loop converged and one elected lane issues, as in the pair kernel)
       constexpr uint32_t idesc = idesc_f16kind_f32(Cfg::BM, BN, F16<T>::umma_fmt);
+      const uint32_t issuer = elect_one();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+        if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -310,39 +312,46 @@ __global__ void __launch_bounds__(192, 1)
         const int sp = (tile / num_m) % splits;
         const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
           const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+          if (issuer) {
 #pragma unroll
-          for (int j = 0; j < Cfg::BK / 16; ++j) {
-            umma_f16_ss(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
-                        idesc, (kb != kb0 || j != 0) ? 1u : 0u);
+            for (int j = 0; j < Cfg::BK / 16; ++j) {
+              umma_f16_ss(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
+                          idesc, (kb != kb0 || j != 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[stage]);
           }
-          umma_commit(&empty[stage]);
+          __syncwarp();
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if (issuer) umma_commit(&tfull[acc]);
+        __syncwarp();
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         *abort_flag = 1;
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
       }
-      // Drain: every MMA issued by this thread completes before TMEM is freed.
-      umma_commit(&tfull[acc]);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(&tfull[acc], acc_phase)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      // Drain: every MMA issued (by the issuing lane) completes before TMEM is freed.
+      if (issuer) {
+        umma_commit(&tfull[acc]);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&tfull[acc], acc_phase)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
       }
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------ epilogue warps 2..5
@@ -1218,9 +1227,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
+    if (leader) {
       // ------------------------------------------------ MMA issuer (leader only)
+      // The warp runs the loop converged and one elected lane issues: from a converged warp
+      // the operands stay in uniform registers and an MMA issues in about half the time it
+      // takes from a lone lane.  The lane is elected once: a commit only tracks the MMAs
+      // of the lane that issues it.
       constexpr uint32_t idesc = idesc_f16kind_f32(2 * Cfg::BM, BN, F16<T>::umma_fmt);
+      const uint32_t issuer = elect_one();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -1233,10 +1247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try_wait(stallbar, 0))
             if (globaltimer_ns() - t0 > 1000000ull) break;
+          __syncwarp();
           ok = false;
           break;
         }
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+        if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -1245,39 +1260,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::threads(EPI
         const int sp = (it / num_m) % splits;
         const int kb0 = sp * num_k / splits, kb1 = (sp + 1) * num_k / splits;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait<WQ != 0>(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait_warp<WQ != 0>(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
           const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+          if (issuer) {
 #pragma unroll
-          for (int j = 0; j < Cfg::BK / 16; ++j) {
-            umma_f16_ss_pair(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
-                             idesc, (kb != kb0 || j != 0) ? 1u : 0u);
+            for (int j = 0; j < Cfg::BK / 16; ++j) {
+              umma_f16_ss_pair(d_tmem, sdesc_k_sw128(a_base + 32 * j), sdesc_k_sw128(b_base + 32 * j),
+                               idesc, (kb != kb0 || j != 0) ? 1u : 0u);
+            }
+            umma_commit_pair(&empty[stage], 0x3);
           }
-          umma_commit_pair(&empty[stage], 0x3);
+          __syncwarp();
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit_pair(&tfull[acc], 0x3);
+        if (issuer) umma_commit_pair(&tfull[acc], 0x3);
+        __syncwarp();
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         *abort_flag = 1;
         set_device_error(p.err, KVA_DEV_WAIT_TIMEOUT);
       }
       // Drain: the pair's MMAs complete before either CTA releases TMEM or exits.
-      umma_commit_pair(&tfull[acc], 0x3);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(&tfull[acc], acc_phase)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (issuer) {
+        umma_commit_pair(&tfull[acc], 0x3);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&tfull[acc], acc_phase)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
       }
+      __syncwarp();
     }
   } else if (WQ && warp >= 2 + Cfg::epi_warps(EPI)) {
     // ------------------------------------------------ q8_0 converters (both CTAs)
