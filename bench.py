@@ -63,7 +63,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kernel-case", default=None,
                     choices=["heads", "heads_fused", "heads_q8", "heads_q4", "resid", "gdn", "attention",
-                             "last_token"],
+                             "last_token", "gemm_shapes"],
                     help="run a small case of one hot kernel three times and exit (for ncu "
                          "captures; the GEMM cases then print their CUDA-event time)")
     return ap.parse_args()
@@ -699,6 +699,9 @@ def run_kernel_case(case, kv_cache="bf16"):
               T = 1024, every launch on the caller's stream (with --kv-cache q8_0 the caches
               take Hadamard-rotated q8_0 rows)
     attention - one block-causal attention of the r3 trunk (T = 1024, 24 heads, window 1024)
+    gemm_shapes - the r3 path's GEMM shapes (M = 1024 tokens) through this library's pair GEMM
+              with a plain 16-bit store and, for comparison only, through torch.matmul (the
+              vendor library, which the path never calls): mean of 20 back-to-back launches
     last_token - the exact last-token pass of one sequence through all 32 r3 late layers at
               position 32767 (8 attention layers each reading 32768 cache rows of 4 KV heads,
               24 gated-DeltaNet layers updating 48 states); prints the CUDA-event time of the
@@ -783,6 +786,9 @@ def run_kernel_case(case, kv_cache="bf16"):
     elif case == "last_token":
         run_last_token_case(K)
         return
+    elif case == "gemm_shapes":
+        run_gemm_shapes_case(K)
+        return
     else:
         T, heads = T_UB, KI.R3.n_heads
         qkv = torch.randn(T, 3 * heads * 128, device="cuda").half()
@@ -790,6 +796,56 @@ def run_kernel_case(case, kv_cache="bf16"):
         for _ in range(3):
             K.kva_op_attention(qkv, out, heads, KI.R3.window)
     torch.cuda.synchronize()
+
+
+def run_gemm_shapes_case(K):
+    """Each r3 GEMM shape (M, K, N) once through kva_op_gemm (fp16 operands, fp16 store) and
+    once through torch.matmul, the mean CUDA-event time of 20 back-to-back launches (best of
+    three loops) each; one JSON line per shape.  The residual-add GEMMs of the path (input linear, o, down) run here with
+    the plain store, like the library call they are compared with."""
+    import hybrid_deltanet_attention_kva_b200 as KK
+    g = KI.R3
+    shapes = [("heads", g.d_model, g.n_total), ("qkv", g.d_model, 3 * g.n_heads * g.head_dim),
+              ("gate_up", g.d_model, 2 * g.ffn), ("o", g.n_heads * g.head_dim, g.d_model),
+              ("down", g.ffn, g.d_model), ("input", g.hidden, g.d_model)]
+
+    def best(fn, reps=20):
+        # the mean of `reps` back-to-back launches (so the host's launch work overlaps the
+        # device), best of three such loops
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t = 1e30
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t = min(t, e0.elapsed_time(e1) * 1e3 / reps)
+        return t
+
+    M = T_UB
+    for name, Kd, N in shapes:
+        A = (torch.randn(M, Kd, device="cuda") * 0.5).half()
+        B = (torch.randn(N, Kd, device="cuda") * 0.02).half()
+        D = torch.empty(M, N, dtype=torch.half, device="cuda")
+        ours = best(lambda: KK.kva_op_gemm(A, [B], D, N=N, epilogue=KK.EPI_STORE_BF16))
+        lib = best(lambda: torch.matmul(A, B.t(), out=D))
+        fl = 2.0 * M * N * Kd
+        line = {"case": "gemm_shapes", "gemm": name, "M": M, "K": Kd, "N": N,
+                "us": round(ours, 1), "tflops": round(fl / ours * 1e-6, 1),
+                "library_us": round(lib, 1), "library_tflops": round(fl / lib * 1e-6, 1)}
+        if N == g.d_model:
+            # the path runs these with split K, partial sums reduce-added into the fp32 stream
+            R = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+            add = best(lambda: KK.kva_op_gemm(A, [B], R, N=N, epilogue=KK.EPI_ADD_F32))
+            line.update({"residual_add_us": round(add, 1), "residual_add_tflops": round(fl / add * 1e-6, 1)})
+            del R
+        print(json.dumps(line))
+        del A, B, D
+        torch.cuda.empty_cache()
 
 
 def last_token_bytes(geom, pos):
