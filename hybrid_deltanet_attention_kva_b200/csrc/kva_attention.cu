@@ -12,7 +12,7 @@
 //   warp 8   TMA producer: Q once, then 128-key K and V tiles into two stages each
 //            (128-byte swizzle; K and V have their own full / empty barriers, so the
 //            next K tile is loaded as soon as its S product has read the stage)
-//   warp 9   one thread issues the MMAs: S_j = Q K_j^T (both operands K-major in
+//   warp 9   waits converged, one elected lane issues the MMAs: S_j = Q K_j^T (both operands K-major in
 //            shared memory) into TMEM buffer j % 2, and O += P_j V_j with P_j read
 //            from TMEM and V_j as an MN-major shared-memory operand
 //   warps 0-7  two threads per query row (TMEM lane = row; warps w and w + 4 take

@@ -785,7 +785,7 @@ __device__ __forceinline__ void epilogue_mixer(const MixParams& mp, uint32_t tme
 // The same pipeline on a pair of CTAs (a cluster of 2) sharing one 256 x 256 tile
 // through tcgen05.mma.cta_group::2: each CTA loads its 128 rows of A and its 128 rows
 // of B (B rows 0-127 of the tile in the leader, 128-255 in the peer), the leader's
-// single thread issues M = 256 MMAs that read both CTAs' operands, and each CTA's
+// elected issuing lane issues M = 256 MMAs that read both CTAs' operands, and each CTA's
 // TMEM receives its own 128 rows of the accumulator.  Per CTA this halves the B
 // bytes that the tensor core reads from shared memory per MMA, the limit of the
 // one-CTA 128 x 256 tile.  TMA loads of both CTAs complete on the leader's barrier
