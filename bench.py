@@ -104,6 +104,18 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def code_hash(path):
+    """sha256 prefix of a C++/CUDA source with its comments and blank lines taken out, so that
+    an edit of the comments alone does not retire a measurement taken on the same code."""
+    import re
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    body = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(body.encode()).hexdigest()[:16]
+
+
 def heads_traffic(geom_name, fused):
     """dram bytes per launch of the heads GEMM (with the state-update epilogue when `fused`)
     from the committed ncu summary, or None when the summary is missing or the GEMM source
@@ -113,15 +125,14 @@ def heads_traffic(geom_name, fused):
     src = os.path.join(ROOT, "hybrid_deltanet_attention_kva_b200", "csrc", "kva_gemm.cu")
     if not os.path.exists(path):
         return None
-    with open(src, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    h = code_hash(src)
     vals = {}
     with open(path) as f:
         for line in f:
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel source sha256 prefix") != h:
+    if vals.get("kernel code sha256 prefix") != h:
         return None
     try:
         return float(vals["traffic bytes per launch (full size)"])
