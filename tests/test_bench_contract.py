@@ -63,3 +63,18 @@ def test_algorithmic_work_from_the_parameter_counts():
         assert 0 <= got_b - approx_bytes < 5e-3 * approx_bytes, (g.name, got_b, approx_bytes)
     f3, b3 = bench.algorithmic(KI.R3)
     assert round(f3 / 1e12, 3) == 2.632 and round(b3 / 1e9, 2) == 2.72
+
+
+def test_traffic_gate_hash_ignores_comments_only(tmp_path):
+    """The heads GEMM's DRAM traffic is reported only while the GEMM's code matches the code
+    it was captured on: an edit of comments or blank lines keeps the hash, an edit of code
+    changes it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    base = "int f(int x) {\n  return x + 1;  // add one\n}\n"
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text(base)
+    b.write_text("/* header\n   lines */\n" + base.replace("// add one", "// a different note") + "\n\n")
+    c.write_text(base.replace("x + 1", "x + 2"))
+    assert bench.code_hash(str(a)) == bench.code_hash(str(b))
+    assert bench.code_hash(str(a)) != bench.code_hash(str(c))
