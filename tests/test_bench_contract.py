@@ -78,3 +78,27 @@ def test_traffic_gate_hash_ignores_comments_only(tmp_path):
     c.write_text(base.replace("x + 1", "x + 2"))
     assert bench.code_hash(str(a)) == bench.code_hash(str(b))
     assert bench.code_hash(str(a)) != bench.code_hash(str(c))
+
+
+def test_state_workload_and_last_token_accounting():
+    """The HBM rooflines of the state-only workload and of the last-token pass rest on these
+    byte counts; each is checked against its r3 value worked out from the model card's shapes
+    (24 gated-DeltaNet layers of 48 value heads, 128 x 128 fp32 states, 10 240 conv channels,
+    8 attention layers of 4 KV heads of 256, mixer rows of 264 448 16-bit values)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    g = KI.R3
+    # 8 sequences x 1024 tokens
+    mixer = 8 * 1024 * 264448 * 2
+    states = 8 * 24 * 48 * 128 * 128 * 4 * 2        # read and written
+    tails = 8 * 24 * 3 * 10240 * 2 * 2              # read and written
+    kv = 8 * 1024 * 8 * 2 * 4 * 256 * 2             # K and V rows written
+    flops, nbytes, parts = bench.state_algorithmic(g, 8, 1024)
+    assert nbytes == mixer + states + tails + kv
+    assert abs(nbytes / 1e9 - 5.83) < 0.01         # the survey's 5.83 GB per call
+    assert flops == 8 * 1024 * 24 * 48 * 4 * 128 * 128
+    assert parts["kv_written"] == kv and parts["state_rw"] == states
+    # last token at position 32767: all 32768 rows of K and V of every attention layer
+    attn, rest = bench.last_token_bytes(g, 32767)
+    assert attn == 8 * 2 * 4 * 256 * 2 * 32768 == 2 ** 30
+    assert rest >= 24 * 48 * 128 * 128 * 4 * 2     # at least the states read and written
