@@ -76,9 +76,9 @@ def geometry(name):
 
 
 def algorithmic(geom, T=T_UB):
-    """FLOPs and HBM bytes the method must spend on one ubatch (see the accounting
-    in the design notes): every linear 2*params*T, causal attention over unmasked
-    pairs, the recurrence 4*d_k*d_v per token per v head; bytes = weights once,
+    """FLOPs and HBM bytes the method must spend on one ubatch: every linear
+    2*params*T, causal attention over unmasked pairs, the recurrence 4*d_k*d_v per
+    token per v head (the chunked form's extra products are not counted); bytes = weights once,
     residual in, state read+write, conv tail, KV rows written, drafter outputs."""
     d, H, F = geom.d_model, geom.hidden, geom.ffn
     lin = H * d + geom.n_blocks * (4 * d * d + 3 * d * F) + geom.n_total * d
@@ -463,7 +463,7 @@ STATE_SEQ = 8
 
 
 def state_algorithmic(geom, n_seq, T):
-    """Bytes one kva_update_states call must move (HBM-bound; see the design notes): the
+    """Bytes one kva_update_states call must move (the workload is HBM-bound): the
     mixer inputs read once, every DeltaNet state read and written, the conv tails read and
     written, the K/V rows written; FLOPs of the recurrence 4*d_k*d_v per token per v head."""
     mix = n_seq * T * geom.n_mix * 2

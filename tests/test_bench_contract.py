@@ -95,7 +95,7 @@ def test_state_workload_and_last_token_accounting():
     kv = 8 * 1024 * 8 * 2 * 4 * 256 * 2             # K and V rows written
     flops, nbytes, parts = bench.state_algorithmic(g, 8, 1024)
     assert nbytes == mixer + states + tails + kv
-    assert abs(nbytes / 1e9 - 5.83) < 0.01         # the survey's 5.83 GB per call
+    assert abs(nbytes / 1e9 - 5.83) < 0.01         # 5.83 GB per call
     assert flops == 8 * 1024 * 24 * 48 * 4 * 128 * 128
     assert parts["kv_written"] == kv and parts["state_rw"] == states
     # last token at position 32767: all 32768 rows of K and V of every attention layer
